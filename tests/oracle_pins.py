@@ -1,0 +1,318 @@
+"""Pins for the fp64 oracle: checks that tie it to something other than itself.
+
+Each ``check_*`` takes an ``oracle.OracleLib`` and raises ``AssertionError`` on
+a mismatch. ``test_oracle_pins.py`` runs them against the oracle as built;
+``test_oracle_mutants.py`` runs them against copies of ``oracle.c`` with one
+planted mistake each and expects every copy to fail at least one check.
+
+The pins are: hand-worked closed forms (``golden/hand_worked.json``), the
+rank characterisation of top-k evaluated in exact rational arithmetic on tiny
+inputs, fp32 -> bf16 rounding by an independent library routine, and
+invariants that any correct implementation satisfies (unit norms, scaling by
+powers of two, permutation of the corpus, prefix property of top-k, 1/tau
+scaling, masks that exclude nothing, duplicate queries).
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "hand_worked.json")
+
+
+def golden() -> dict:
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+def pack_bits(excluded: np.ndarray) -> np.ndarray:
+    """Pack a boolean [n] array into uint32 words, bit (j & 31) of word j >> 5."""
+    n = excluded.shape[0]
+    words = np.zeros((n + 31) // 32, dtype=np.uint32)
+    for j in np.nonzero(excluded)[0]:
+        words[j >> 5] |= np.uint32(1) << np.uint32(j & 31)
+    return words
+
+
+def _as_float(x):
+    return -math.inf if x == "-inf" else float(x)
+
+
+def bf16_bits_via_torch(values_f32: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 (nearest-even) by torch's own conversion, as uint16 bits."""
+    t = torch.from_numpy(np.ascontiguousarray(values_f32, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def bf16_value(bits: int) -> float:
+    return float(np.array([bits << 16], dtype=np.uint32).view(np.float32)[0])
+
+
+# ---------------------------------------------------------------------------
+
+
+def check_bf16_rounding(o):
+    # closed forms
+    assert o.bf16_from_double(0.6) == 0x3F1A
+    assert o.bf16_from_double(0.8) == 0x3F4D
+    assert o.bf16_from_double(0.1) == 0x3DCD
+    assert o.bf16_from_double(1.0) == 0x3F80
+    assert o.bf16_from_double(-2.0) == 0xC000
+    assert o.bf16_from_double(0.0) == 0x0000
+    assert o.bf16_from_double(-0.0) == 0x8000
+    # ties to even: 1 + 2^-8 lies halfway between 1 and 1 + 2^-7 -> 1 (even)
+    assert o.bf16_from_double(1.0 + 2.0 ** -8) == 0x3F80
+    # 1 + 3*2^-8 lies halfway between 1 + 2^-7 (odd) and 1 + 2^-6 (even) -> 1 + 2^-6
+    assert o.bf16_from_double(1.0 + 3 * 2.0 ** -8) == 0x3F82
+    # just above a tie rounds up
+    assert o.bf16_from_double(1.0 + 2.0 ** -8 + 2.0 ** -30) == 0x3F81
+    # subnormal: 2^-130 is exactly representable (bf16 subnormal quantum 2^-133)
+    assert o.bf16_from_double(2.0 ** -130) == 0x0008
+    # independent route: for fp32-representable values, one rounding to bf16
+    # must agree with torch's fp32 -> bf16 conversion
+    rng = np.random.default_rng(7)
+    vals = np.concatenate([
+        rng.standard_normal(4000).astype(np.float32),
+        (rng.standard_normal(2000) * 1e-3).astype(np.float32),
+        (rng.integers(-2 ** 15, 2 ** 15, 2000) * 2.0 ** -20).astype(np.float32),
+    ])
+    ref = bf16_bits_via_torch(vals)
+    mine = np.array([o.bf16_from_double(float(v)) for v in vals], dtype=np.uint16)
+    assert np.array_equal(mine, ref), "bf16 rounding disagrees with torch's fp32->bf16"
+
+
+def check_h1_normalize(o):
+    g = golden()["H1_normalize"]
+    rows = np.array(g["rows"], dtype=np.float32)
+    out_bf = o.normalize(rows, "bf16")
+    assert np.array_equal(out_bf, np.array(g["expected_bf16_bits"], dtype=np.uint16)), out_bf
+    out_f = o.normalize(rows, "f32")
+    exp_f = np.array(g["expected_f64"], dtype=np.float64)
+    assert np.allclose(out_f, exp_f, rtol=2e-7, atol=0), (out_f, exp_f)
+    norms = o.row_norms(rows)
+    assert np.allclose(norms, [5.0, 1e-6, 1e-6, 5.0], rtol=1e-7), norms
+
+
+def check_normalize_invariants(o):
+    rng = np.random.default_rng(11)
+    for d in (16, 48, 128, 256):
+        x = rng.standard_normal((64, d)).astype(np.float32)
+        x[3] = 0.0
+        x[5] *= 1e-9  # below the norm floor
+        y = o.normalize(x, "f32").astype(np.float64)
+        big = (x.astype(np.float64) ** 2).sum(1) >= 1e-12
+        # unit length where the floor is not active
+        assert np.allclose(np.linalg.norm(y[big], axis=1), 1.0, atol=1e-6)
+        # below the floor: divided by exactly 1e-6
+        assert np.allclose(y[~big], x[~big].astype(np.float64) * 1e6, rtol=1e-6, atol=1e-30)
+        # scaling a row by a power of two changes nothing (above the floor)
+        for s in (-3, 5):
+            xs = (x * np.float32(2.0 ** s)).astype(np.float32)
+            keep = big & ((xs.astype(np.float64) ** 2).sum(1) >= 1e-12)
+            assert np.array_equal(o.normalize(xs, "f32")[keep], o.normalize(x, "f32")[keep])
+            assert np.array_equal(o.normalize(xs, "bf16")[keep], o.normalize(x, "bf16")[keep])
+        # flipping the sign of a row flips its output; permuting coordinates permutes it
+        assert np.array_equal(o.normalize(-x, "f32"), -o.normalize(x, "f32"))
+        perm = rng.permutation(d)
+        assert np.array_equal(o.normalize(x[:, perm], "f32"), o.normalize(x, "f32")[:, perm])
+        # direction is kept: y_i * x_j == y_j * x_i
+        xd = x[big].astype(np.float64)
+        cross = y[big][:, :, None] * xd[:, None, :] - y[big][:, None, :] * xd[:, :, None]
+        assert np.abs(cross).max() < 1e-5 * np.abs(xd).max()
+        # row norms: |a e_i| = |a|; scaling by powers of two
+        assert np.allclose(o.row_norms(np.eye(d, dtype=np.float32) * -3.0), 3.0)
+        nrm = o.row_norms(x)
+        assert np.allclose(o.row_norms(x * np.float32(4.0))[big], 4.0 * nrm[big], rtol=1e-12)
+    # bf16 input: the same invariants hold for bf16-stored raw rows
+    xb = bf16_bits_via_torch(rng.standard_normal((32, 64)).astype(np.float32)).reshape(32, 64)
+    yb = o.normalize(xb, "f32").astype(np.float64)
+    assert np.allclose(np.linalg.norm(yb, axis=1), 1.0, atol=1e-6)
+
+
+def check_h2_topk(o):
+    g = golden()["H2_topk"]
+    V = np.array(g["corpus"], dtype=np.float32)
+    u = np.array([g["query"]], dtype=np.float32)
+    for case in g["cases"]:
+        excl = np.zeros(V.shape[0], dtype=bool)
+        excl[case["exclude"]] = True
+        mask = pack_bits(excl) if case["exclude"] else None
+        ids, scores = o.topk(u, V, case["k"], tau=case["tau"], exclude=mask)
+        assert ids[0].tolist() == case["ids"], (case, ids)
+        assert np.array_equal(scores[0], np.array([_as_float(s) for s in case["scores"]])), (case, scores)
+
+
+def check_h3_fused(o):
+    g = golden()["H3_fused"]
+    V = np.array(g["corpus_raw"], dtype=np.float32)
+    u = np.array([g["query"]], dtype=np.float32)
+    norms = o.row_norms(V)
+    assert np.allclose(norms, g["norms"], rtol=1e-9), norms
+    for case in g["cases"]:
+        ids, scores = o.topk(u, V, case["k"], tau=case["tau"], norms=norms)
+        assert ids[0].tolist() == case["ids"], (case, ids)
+        assert np.allclose(scores[0], case["scores"], rtol=1e-7, atol=0), (case, scores)
+
+
+def check_exact_rational(o):
+    """Rank characterisation in exact arithmetic: the entry at rank r has
+    exactly r eligible candidates better than it (higher score, or equal score
+    and lower id), and its score is the exact dot product over tau."""
+    rng = np.random.default_rng(3)
+    for trial in range(60):
+        n = int(rng.integers(1, 40))
+        d = int(rng.integers(1, 6))
+        b = 3
+        k = int(rng.integers(1, n + 4))
+        V = (rng.integers(-4, 5, size=(n, d)) / 4.0).astype(np.float32)
+        Q = (rng.integers(-4, 5, size=(b, d)) / 4.0).astype(np.float32)
+        tau = float(rng.choice([1.0, 0.5, 0.25, 2.0]))
+        excl = rng.random(n) < (0.25 if trial % 2 else 0.0)
+        mask = pack_bits(excl) if excl.any() else None
+        ids, scores = o.topk(Q, V, k, tau=tau, exclude=mask)
+        for qi in range(b):
+            exact = [sum(Fraction(float(Q[qi, i])) * Fraction(float(V[j, i])) for i in range(d))
+                     / Fraction(tau) for j in range(n)]
+            eligible = [j for j in range(n) if not excl[j]]
+            got = ids[qi].tolist()
+            for r in range(k):
+                if r >= len(eligible):
+                    assert got[r] == -1 and scores[qi, r] == -math.inf, (trial, qi, r)
+                    continue
+                j = got[r]
+                assert 0 <= j < n and not excl[j], (trial, qi, r, j)
+                assert Fraction(float(scores[qi, r])) == exact[j], (trial, qi, r)
+                better = sum(1 for i in eligible
+                             if exact[i] > exact[j] or (exact[i] == exact[j] and i < j))
+                assert better == r, (trial, qi, r, better)
+            assert len(set(x for x in got if x >= 0)) == min(k, len(eligible))
+
+
+def check_invariants(o):
+    rng = np.random.default_rng(5)
+    n, d, b, k = 300, 32, 6, 20
+    V = o.normalize(rng.standard_normal((n, d)).astype(np.float32), "f32")
+    Q = o.normalize(rng.standard_normal((b, d)).astype(np.float32), "f32")
+    ids, scores = o.topk(Q, V, k)
+    # corpus permutation: ids map through the permutation, scores are unchanged
+    perm = rng.permutation(n)
+    ids_p, scores_p = o.topk(Q, V[perm], k)
+    assert np.array_equal(perm[ids_p], ids)
+    assert np.array_equal(scores_p, scores)
+    # top-k is the prefix of top-(k+1)
+    ids1, scores1 = o.topk(Q, V, k + 1)
+    assert np.array_equal(ids1[:, :k], ids) and np.array_equal(scores1[:, :k], scores)
+    # scores are non-increasing
+    assert (np.diff(scores, axis=1) <= 0).all()
+    # tau = 0.25: same ids, scores times 4 exactly
+    ids_t, scores_t = o.topk(Q, V, k, tau=0.25)
+    assert np.array_equal(ids_t, ids) and np.array_equal(scores_t, 4.0 * scores)
+    # a mask that excludes nothing equals no mask
+    ids_m, scores_m = o.topk(Q, V, k, exclude=np.zeros((n + 31) // 32, dtype=np.uint32))
+    assert np.array_equal(ids_m, ids) and np.array_equal(scores_m, scores)
+    # excluding each query's best candidate removes it and shifts the rest up
+    for qi in range(b):
+        excl = np.zeros(n, dtype=bool)
+        excl[ids[qi, 0]] = True
+        ids_x, _ = o.topk(Q[qi:qi + 1], V, k, exclude=pack_bits(excl))
+        assert np.array_equal(ids_x[0, :k - 1], ids[qi, 1:])
+    # excluded candidates never appear
+    excl = rng.random(n) < 0.5
+    ids_e, _ = o.topk(Q, V, k, exclude=pack_bits(excl))
+    assert not excl[ids_e[ids_e >= 0]].any()
+    # duplicate queries give identical rows; a query's row does not depend on the batch
+    Qd = np.concatenate([Q, Q[:2]])
+    ids_d, scores_d = o.topk(Qd, V, k)
+    assert np.array_equal(ids_d[b:], ids[:2]) and np.array_equal(scores_d[b:], scores[:2])
+    ids_s, scores_s = o.topk(Q[3:4], V, k)
+    assert np.array_equal(ids_s[0], ids[3]) and np.array_equal(scores_s[0], scores[3])
+    # k > n pads with (-1, -inf)
+    ids_big, scores_big = o.topk(Q[:1], V[:5], 8)
+    assert (ids_big[0, 5:] == -1).all() and np.isneginf(scores_big[0, 5:]).all()
+    assert sorted(ids_big[0, :5].tolist()) == list(range(5))
+    # fused norms: scaling a raw row by a power of two leaves its fused score unchanged
+    raw = rng.standard_normal((n, d)).astype(np.float32)
+    scale = (2.0 ** rng.integers(-4, 5, size=(n, 1))).astype(np.float32)
+    ids_f, sc_f = o.topk(Q, raw, k, norms=o.row_norms(raw))
+    ids_g, sc_g = o.topk(Q, raw * scale, k, norms=o.row_norms(raw * scale))
+    assert np.array_equal(ids_f, ids_g) and np.array_equal(sc_f, sc_g)
+
+
+def check_ties(o):
+    # all rows identical: every score ties, ids come out 0..k-1
+    row = np.array([[0.25, -0.5, 0.75, 0.125]], dtype=np.float32)
+    V = np.repeat(row, 1000, axis=0)
+    Q = np.array([[1.0, 1.0, 1.0, 1.0], [-1.0, 0.5, 0.0, 2.0]], dtype=np.float32)
+    ids, scores = o.topk(Q, V, 300)
+    assert (ids == np.arange(300)[None, :]).all()
+    assert (scores == scores[:, :1]).all()
+    # identity corpus: query e_t scores 1 at t and 0 elsewhere
+    d = 24
+    E = np.eye(d, dtype=np.float32)
+    for t in (0, 7, 23):
+        ids, scores = o.topk(E[t:t + 1], E, 6)
+        expect = [t] + [j for j in range(d) if j != t][:5]
+        assert ids[0].tolist() == expect, (t, ids)
+        assert scores[0].tolist() == [1.0, 0, 0, 0, 0, 0]
+
+
+def check_scores_for(o):
+    rng = np.random.default_rng(9)
+    V = rng.standard_normal((50, 8)).astype(np.float32)
+    Q = rng.standard_normal((2, 8)).astype(np.float32)
+    norms = o.row_norms(V)
+    ids, scores = o.topk(Q, V, 10, tau=0.5, norms=norms)
+    for qi in range(2):
+        s = o.scores_for(Q, qi, V, ids[qi], tau=0.5, norms=norms)
+        assert np.array_equal(s, scores[qi])
+    # closed form: e_0 against the H2 corpus
+    g = golden()["H2_topk"]
+    s = o.scores_for(np.array([g["query"]], dtype=np.float32), 0,
+                     np.array(g["corpus"], dtype=np.float32), [0, 1, 2, 3, 4, 5])
+    assert s.tolist() == [0.5, 1.0, 0.5, -1.0, 0.0, 0.75]
+
+
+def check_bf16_inputs(o):
+    """bf16-stored inputs: the closed forms of H1/H2/H3 hold when the rows and
+    queries are handed over as bf16 (all values there are exact in bf16)."""
+    g1 = golden()["H1_normalize"]
+    rows = np.array(g1["rows"], dtype=np.float32)[[0, 1, 3]]
+    rows_bf = bf16_bits_via_torch(rows).reshape(rows.shape)
+    assert np.array_equal(o.normalize(rows_bf, "bf16"),
+                          np.array(g1["expected_bf16_bits"], dtype=np.uint16)[[0, 1, 3]])
+    assert np.allclose(o.row_norms(rows_bf), [5.0, 1e-6, 5.0], rtol=1e-12)
+    g2 = golden()["H2_topk"]
+    V = bf16_bits_via_torch(np.array(g2["corpus"], dtype=np.float32)).reshape(6, 4)
+    u = bf16_bits_via_torch(np.array([g2["query"]], dtype=np.float32)).reshape(1, 4)
+    for case in g2["cases"]:
+        excl = np.zeros(6, dtype=bool)
+        excl[case["exclude"]] = True
+        ids, scores = o.topk(u, V, case["k"], tau=case["tau"],
+                             exclude=pack_bits(excl) if case["exclude"] else None)
+        assert ids[0].tolist() == case["ids"], (case, ids)
+        assert np.array_equal(scores[0], np.array([_as_float(s) for s in case["scores"]]))
+    g3 = golden()["H3_fused"]
+    raw = np.array(g3["corpus_raw"], dtype=np.float32)[:6]
+    raw_bf = bf16_bits_via_torch(raw).reshape(raw.shape)
+    ids, scores = o.topk(u, raw_bf, 3, norms=o.row_norms(raw_bf))
+    assert ids[0].tolist() == [1, 5, 0]
+    assert np.allclose(scores[0], [1.0, 0.8017837257372732, 0.5], rtol=1e-12)
+
+
+ALL_CHECKS = [
+    check_bf16_rounding,
+    check_bf16_inputs,
+    check_h1_normalize,
+    check_normalize_invariants,
+    check_h2_topk,
+    check_h3_fused,
+    check_exact_rational,
+    check_invariants,
+    check_ties,
+    check_scores_for,
+]

@@ -1,0 +1,52 @@
+"""Planted mistakes: each copy of oracle.c below carries one plausible bug
+(a dropped term, a wrong sign, index or operand, a misplaced floor, a broken
+tie rule or rounding). Every copy must fail at least one pin; a copy that
+passes them all would show a gap in the pins. CPU only; the copies are built
+in a temporary directory and never touch the real oracle."""
+import os
+
+import pytest
+
+import oracle
+import oracle_pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+
+MUTANTS = {
+    "dropped_square": ("ss += x * x;", "ss += x;"),
+    "eps_added_to_norm": ("sqrt(ss > ORACLE_EPS ? ss : ORACLE_EPS)", "(sqrt(ss) + ORACLE_EPS)"),
+    "eps_floor_ignored": ("ss > ORACLE_EPS ? ss : ORACLE_EPS", "ss"),
+    "multiply_by_norm": ("x / norm", "x * norm"),
+    "ascending_sort": ("if (a->s > b->s)\n        return -1;\n    if (a->s < b->s)\n        return 1;",
+                       "if (a->s > b->s)\n        return 1;\n    if (a->s < b->s)\n        return -1;"),
+    "higher_id_wins_ties": ("if (a->id < b->id)\n        return -1;\n    if (a->id > b->id)\n        return 1;",
+                            "if (a->id < b->id)\n        return 1;\n    if (a->id > b->id)\n        return -1;"),
+    "tau_multiplies": ("return dot / tau;", "return dot * tau;"),
+    "fused_norm_multiplies": ("dot = dot / norms[j];", "dot = dot * norms[j];"),
+    "mask_bit_index": ("(j & 31)", "(j & 15)"),
+    "mask_word_index": ("exclude[j >> 5]", "exclude[j >> 6]"),
+    "query_coordinates_reversed": ("load_elem(q, q_dtype, qrow * (int64_t)d + i)",
+                                   "load_elem(q, q_dtype, qrow * (int64_t)d + (d - 1 - i))"),
+    "id_after_compaction": ("pairs[m].id = j;", "pairs[m].id = m;"),
+    "bf16_truncates": ("rint(ax / quantum)", "floor(ax / quantum)"),
+    "bf16_one_bit_short": ("ldexp(1.0, lead - 7)", "ldexp(1.0, lead - 6)"),
+    "bf16_load_shift": ("(uint32_t)h << 16", "(uint32_t)h << 15"),
+    "pad_score_zero": ("out_scores[qi * k + r] = -INFINITY;", "out_scores[qi * k + r] = 0.0;"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation anchor for {name} not found"
+    path_c = tmp_path / f"{name}.c"
+    path_c.write_text(src.replace(old, new))
+    lib = oracle.OracleLib(oracle.build(force=True, src=str(path_c), out=str(tmp_path / f"{name}.so")))
+    failures = []
+    for check in oracle_pins.ALL_CHECKS:
+        try:
+            check(lib)
+        except AssertionError:
+            failures.append(check.__name__)
+    assert failures, f"planted mistake {name!r} passed every pin"
