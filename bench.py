@@ -1,0 +1,425 @@
+"""Benchmark: exact top-k inner-product search on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is the whole hot path over one batch: L2-normalise the raw corpus
+(and the raw queries), score every query against every candidate, filter and
+select the exact top-k. Inputs are seeded synthetic data (``workloads.py``)
+resident in HBM before timing starts. The default workload is the streaming
+single-query case (N = 1,000,000, d = 128, B = 1, k = 100).
+
+Multi-GPU (torchrun, one process per GPU): every rank runs an independent
+replica of the workload on its own queries - the path has no exchange step,
+so there is no collective in the data path; the value is the total over ranks
+(weak scaling), timed as the max over ranks.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime as dt
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "query-candidate scores/sec (exact top-k)"
+UNIT = "scores/s"
+DEFAULT_WORKLOAD = "stream_b1"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work of one step
+# ---------------------------------------------------------------------------
+def elem_bytes(name):
+    return {"f32": 4, "bf16": 2}[name]
+
+
+def work_model(w: W.Workload, plan: dict):
+    s_in = elem_bytes(w.raw_dtype)
+    if w.store == "raw":
+        k1_bytes = w.n * w.d * s_in + w.n * 4
+        s_corpus = s_in
+    else:
+        s_out = elem_bytes(w.store)
+        k1_bytes = w.n * w.d * (s_in + s_out)
+        s_corpus = s_out
+    rows_scanned = sum(plan["rows"])
+    per_row = w.d * s_corpus + (4 if w.store == "raw" else 0)
+    score_bytes = rows_scanned * per_row + (w.n // 8 if w.masked else 0)
+    score_flops = 2.0 * w.b * w.d * rows_scanned
+    return {"k1_bytes": k1_bytes, "score_bytes": score_bytes, "score_flops": score_flops,
+            "rows_scanned": rows_scanned}
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self, t0: float, t1: float):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for rec in csv.reader(f):
+                if len(rec) < 10:
+                    continue
+                try:
+                    ts = dt.datetime.strptime(rec[0].strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    rows.append((ts, float(rec[2]), float(rec[3]), [r.strip() for r in rec[6:10]]))
+                except Exception:
+                    continue
+        os.unlink(self.path)
+        inside = [r for r in rows if t0 - 0.05 <= r[0] <= t1 + 0.05] or rows
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i in range(4) if r[3][i].lower().startswith("active")})
+        return {"sm_mhz": float(np.median([r[1] for r in inside])), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":  # host-only arm: no process group, rank 0 works alone
+        return world, rank, local
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    if world > 1:
+        import torch.distributed as tdist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        tdist.init_process_group(backend, timeout=dt.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as tdist
+        tdist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as tdist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample of the workload
+# ---------------------------------------------------------------------------
+def oracle_sample_run(w: W.Workload, raw_c_np, raw_q_np, excl_np, n_s: int, b_s: int):
+    import oracle
+    corpus = raw_c_np[:n_s]
+    qs = raw_q_np[:b_s]
+    excl = None if excl_np is None else excl_np[: (n_s + 31) // 32]
+    t0 = time.perf_counter()
+    if w.store == "raw":
+        norms = oracle.row_norms(corpus)
+        stored = corpus
+    else:
+        norms = None
+        stored = oracle.normalize(corpus, w.store)
+    qn = oracle.normalize(qs, w.query_dtype)
+    oracle.topk(qn, stored, min(w.k, n_s), tau=float(np.float32(w.tau)), norms=norms, exclude=excl)
+    return time.perf_counter() - t0
+
+
+def oracle_sample_size(w: W.Workload, raw_c_np, raw_q_np, excl_np, seconds: float):
+    """Pick (n_s, b_s) so that one oracle run takes about `seconds`."""
+    import oracle
+    threads = oracle.max_threads()
+    b_s = min(w.b, max(1, threads))
+    n_s = min(w.n, 20_000)
+    t = oracle_sample_run(w, raw_c_np, raw_q_np, excl_np, n_s, b_s)
+    while n_s < w.n and t < seconds / 4:
+        n_s = min(w.n, n_s * 4)
+        t = oracle_sample_run(w, raw_c_np, raw_q_np, excl_np, n_s, b_s)
+    if t > 0 and n_s < w.n:
+        n_s = int(min(w.n, max(1000, n_s * seconds / t)))
+    return n_s, b_s, threads
+
+
+def cpu_baseline(w: W.Workload, raw_c, raw_q, excl, seconds=12.0):
+    raw_c_np = W.to_numpy_rows(raw_c)
+    raw_q_np = raw_q.detach().cpu().numpy()
+    excl_np = None if excl is None else excl.cpu().numpy().view(np.uint32)
+    n_s, b_s, threads = oracle_sample_size(w, raw_c_np, raw_q_np, excl_np, seconds)
+    t = oracle_sample_run(w, raw_c_np, raw_q_np, excl_np, n_s, b_s)
+    return {"value": b_s * n_s / t, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{b_s} queries x first {n_s} candidates of {w.name} (normalise + score + full sort), "
+                      f"one run of {t:.2f} s"}
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
+def run_ours(args, world, rank, local):
+    import exact_inner_product_b200 as tt
+
+    w = W.workload(args.workload)
+    if world > 1:  # each rank: its own queries (independent replica)
+        w = W.workload(args.workload, seed=w.seed + 7919 * rank)
+    dev = torch.device("cuda", local)
+    raw_c = W.corpus(w, dev)
+    raw_q = W.queries(w, dev)
+    excl = W.exclusion_bits(w, dev)
+    if w.store == "raw":
+        prepared = torch.empty((w.n,), dtype=torch.float32, device=dev)
+        mode = tt.TT_NORM_FUSED
+    else:
+        prepared = torch.empty((w.n, w.d), dtype=torch.float32 if w.store == "f32" else torch.bfloat16,
+                               device=dev)
+        mode = tt.TT_NORM_STORE
+    qn = torch.empty((w.b, w.d), dtype=torch.float32 if w.query_dtype == "f32" else torch.bfloat16,
+                     device=dev)
+    out_ids = torch.empty((w.b, w.k), dtype=torch.int32, device=dev)
+    out_scores = torch.empty((w.b, w.k), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    ev_k1 = []
+
+    def step(record_k1=False):
+        if record_k1:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        index = tt.tt_normalize_candidates(raw_c, prepared, mode)
+        if record_k1:
+            e1.record(stream)
+            ev_k1.append((e0, e1))
+        tt.tt_normalize_candidates(raw_q, qn, tt.TT_NORM_STORE, make_index=False)
+        tt.tt_score_topk(index, qn, w.k, tau=w.tau, exclude=excl, out_ids=out_ids, out_scores=out_scores)
+        return index
+
+    for _ in range(args.warmup):
+        last_index = step()
+    stats = tt.tt_last_stats(last_index)
+    plan = tt.tt_plan(w.n, w.k)
+    torch.cuda.synchronize(dev)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    launches0 = tt.tt_launch_count()
+    tt.tt_profile_begin()
+    t_wall0 = time.time()
+    e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for _ in range(args.steps):
+        step(record_k1=True)
+    e_stop.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    barrier(world)
+    prof = tt.tt_profile_end()
+    launches = tt.tt_launch_count() - launches0
+    clk = clocks.stop(t_wall0, t_wall1)
+    ms_total = e_start.elapsed_time(e_stop)
+    ms_total = max_over_ranks(ms_total, world)
+    ms_step = ms_total / args.steps
+
+    value = world * w.b * w.n / (ms_step / 1e3)
+    qps = world * w.b / (ms_step / 1e3)
+
+    # ---- roofline of the dominant kernel ----
+    peaks, peak_src = load_peaks()
+    work = work_model(w, plan)
+    k1_ms = sum(a.elapsed_time(b) for a, b in ev_k1) / max(1, len(ev_k1))
+    score_kind = "tensor" if stats["path"] == 2 else "stream"
+    score_ms = prof[score_kind]["ms"] / args.steps
+    if k1_ms >= score_ms:
+        dom = {"kernel": "k1_normalize (corpus)", "bound": "hbm", "ms": k1_ms, "bytes": work["k1_bytes"],
+               "launches_per_step": 1}
+    else:
+        t_flops = work["score_flops"] / (peaks["bf16_tflops_sustained"] * 1e12)
+        t_bytes = work["score_bytes"] / (peaks["hbm_gbs"] * 1e9)
+        bound = "tensor" if (stats["path"] == 2 and t_flops > t_bytes) else "hbm"
+        dom = {"kernel": f"k{2 if score_kind == 'stream' else 3}_{score_kind} (all levels)", "bound": bound,
+               "ms": score_ms, "bytes": work["score_bytes"], "flops": work["score_flops"],
+               "launches_per_step": prof[score_kind]["launches"] / args.steps}
+    if dom["bound"] == "hbm":
+        achieved = dom["bytes"] / (dom["ms"] / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None}
+    else:
+        achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_tflops_sustained"],
+                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops_sustained"], 4), "traffic": None}
+    roof["kernel"] = dom["kernel"]
+    roof["peak_source"] = peak_src + (" (sustained bf16)" if roof["bound"] == "tensor" else " (copy)")
+    roof["kernel_ms"] = round(dom["ms"], 5)
+
+    kernels = {k: {"ms_per_step": round(v["ms"] / args.steps, 5), "launches_per_step": v["launches"] / args.steps}
+               for k, v in prof.items() if v["launches"]}
+    kernels["k1_normalize_corpus"] = {"ms_per_step": round(k1_ms, 5), "launches_per_step": 1}
+
+    # ---- end to end through the public API, host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        host_c = raw_c.cpu().pin_memory()
+        host_q = raw_q.cpu().pin_memory()
+        host_x = excl.cpu().pin_memory() if excl is not None else None
+        e2e_steps = max(3, min(args.steps, args.e2e_steps))
+        tt.search(host_c, host_q, w.k, tau=w.tau, exclude=host_x, store_dtype=prepared.dtype,
+                  query_dtype=qn.dtype, fused=w.store == "raw")
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            tt.search(host_c, host_q, w.k, tau=w.tau, exclude=host_x, store_dtype=prepared.dtype,
+                      query_dtype=qn.dtype, fused=w.store == "raw")
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(a.elapsed_time(b_) / e2e_steps, world)
+        h2d = host_c.numel() * host_c.element_size() + host_q.numel() * host_q.element_size() + \
+            (host_x.numel() * 4 if host_x is not None else 0)
+        e2e = {"value": world * w.b * w.n / (e2e_ms / 1e3), "unit": UNIT, "ms_per_step": round(e2e_ms, 4),
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(w.b * w.k * 8), "steps": e2e_steps}
+        del host_c, host_q
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.store != "f32" else "f32",
+        "data": "synthetic (seeded, workloads.py)",
+        "config": {"workload": w.name, "n": w.n, "d": w.d, "b": w.b, "k": w.k, "tau": w.tau,
+                   "corpus_raw": w.raw_dtype, "corpus_store": w.store, "queries": w.query_dtype,
+                   "mask_rate": w.mask_rate, "l2": "inputs larger than L2 (raw corpus "
+                   f"{w.n * w.d * elem_bytes(w.raw_dtype) / 1e6:.0f} MB > 126 MB)",
+                   "path": "tensor-core" if stats["path"] == 2 else "streaming", "levels": plan["rows"],
+                   "parallelism": f"replicas x{world}"},
+        "topk_queries_per_s": qps,
+        "roofline": roof,
+        "kernels": kernels,
+        "clocks": clk,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, raw_c, raw_q, excl, seconds=args.cpu_seconds)
+    return line
+
+
+def run_reference(args, world, rank):
+    """The fp64 oracle as the reference arm, on this host's cores."""
+    if rank != 0:
+        return None
+    import oracle
+    w = W.workload(args.workload)
+    raw_c = W.corpus(w, "cpu")
+    raw_q = W.queries(w, "cpu")
+    excl = W.exclusion_bits(w, "cpu")
+    raw_c_np = W.to_numpy_rows(raw_c)
+    raw_q_np = raw_q.numpy()
+    excl_np = None if excl is None else excl.numpy().view(np.uint32)
+    budget = max(0.05, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    n_s, b_s, threads = oracle_sample_size(w, raw_c_np, raw_q_np, excl_np, budget)
+    for _ in range(args.warmup):
+        oracle_sample_run(w, raw_c_np, raw_q_np, excl_np, n_s, b_s)
+    t = 0.0
+    for _ in range(args.steps):
+        t += oracle_sample_run(w, raw_c_np, raw_q_np, excl_np, n_s, b_s)
+    ms = t / args.steps * 1e3
+    value = b_s * n_s / (ms / 1e3)
+    sample = (f"each step: {b_s} queries x first {n_s} candidates of {w.name} "
+              "(fp64 normalise + score + full sort)")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, workloads.py)",
+            "config": {"workload": w.name, "n": w.n, "d": w.d, "b": w.b, "k": w.k},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, world, rank)
+        else:
+            line = run_ours(args, world, rank, local)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1 and args.impl == "ours":
+            import torch.distributed as tdist
+            tdist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

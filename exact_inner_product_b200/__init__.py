@@ -1,0 +1,297 @@
+"""Exact top-k inner-product search on B200: Python binding of ``libtt.so``.
+
+Thin ctypes layer over the C ABI declared in ``include/tt.h``: every function
+here only marshals arguments (tensor pointers, sizes, the current CUDA stream)
+and raises ``TTError`` on a non-OK status. All computation runs in the CUDA
+kernels of the library. PyTorch supplies device memory and streams.
+
+    import exact_inner_product_b200 as tt
+    index = tt.tt_normalize_candidates(raw_corpus, torch.empty_like(raw_corpus, dtype=torch.bfloat16))
+    ids, scores = tt.tt_score_topk(index, queries, k=100)
+
+There is no fallback: if ``libtt.so`` has not been built, importing this
+package raises ``ImportError``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtt.so")
+
+TT_OK = 0
+TT_ERR_INVALID_ARG = 1
+TT_ERR_UNSUPPORTED = 2
+TT_ERR_CUDA = 3
+TT_ERR_NO_MEMORY = 4
+TT_ERR_TIMEOUT = 5
+TT_ERR_INTERNAL = 6
+
+TT_F32 = 0
+TT_BF16 = 1
+TT_NORM_STORE = 0
+TT_NORM_FUSED = 1
+TT_MAX_D = 512
+TT_MAX_K = 2048
+
+KIND_NAMES = ("normalize", "cast", "stream", "tensor", "select", "aux")
+TT_NUM_KINDS = len(KIND_NAMES)
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m exact_inner_product_b200.build` "
+        "(there is no CPU fallback)")
+
+
+class tt_options(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int32), ("rank_scale_pct", ctypes.c_int32),
+                ("force_levels", ctypes.c_int32), ("cap", ctypes.c_int32)]
+
+
+class tt_stats(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int32), ("levels", ctypes.c_int32), ("rescans", ctypes.c_int32),
+                ("launches", ctypes.c_int32), ("level_rows", ctypes.c_int64 * 4),
+                ("level_stride", ctypes.c_int64 * 4), ("cap", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+_lib = ctypes.CDLL(LIB_PATH)
+_vp, _i32, _i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+
+
+def _sig(name, res, args):
+    f = getattr(_lib, name)
+    f.restype = res
+    f.argtypes = args
+    return f
+
+
+_sig("tt_normalize_candidates", ctypes.c_int, [_vp, ctypes.c_int, _i64, _i32, _vp, ctypes.c_int, _i32, _vp,
+                                               ctypes.POINTER(_vp)])
+_sig("tt_index_wrap", ctypes.c_int, [_vp, ctypes.c_int, _i64, _i32, _vp, ctypes.POINTER(_vp)])
+_sig("tt_score_topk", ctypes.c_int, [_vp, _vp, ctypes.c_int, _i32, _vp, ctypes.c_float, _i32, _vp, _vp,
+                                     _vp])
+_sig("tt_score_topk_ex", ctypes.c_int, [_vp, _vp, ctypes.c_int, _i32, _vp, ctypes.c_float, _i32, _vp,
+                                        _vp, _vp, ctypes.POINTER(tt_options)])
+_sig("tt_last_stats", ctypes.c_int, [_vp, ctypes.POINTER(tt_stats)])
+_sig("tt_plan", ctypes.c_int, [_i64, _i32, ctypes.POINTER(tt_options), ctypes.POINTER(_i32),
+                               ctypes.POINTER(_i64), ctypes.POINTER(_i64), ctypes.POINTER(_i32),
+                               ctypes.POINTER(_i32)])
+_sig("tt_free", None, [_vp])
+_sig("tt_launch_count", _i64, [])
+_sig("tt_profile_begin", ctypes.c_int, [])
+_sig("tt_profile_end", ctypes.c_int, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64)])
+_sig("tt_status_string", ctypes.c_char_p, [ctypes.c_int])
+_sig("tt_last_error", ctypes.c_char_p, [])
+_sig("tt_version", ctypes.c_char_p, [])
+
+EXPORTED = ("tt_normalize_candidates", "tt_index_wrap", "tt_score_topk", "tt_score_topk_ex",
+            "tt_last_stats", "tt_plan", "tt_free", "tt_launch_count", "tt_profile_begin",
+            "tt_profile_end", "tt_status_string", "tt_last_error", "tt_version")
+
+
+class TTError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        name = _lib.tt_status_string(status).decode()
+        detail = _lib.tt_last_error().decode()
+        super().__init__(f"{where}: {name}" + (f" ({detail})" if detail else ""))
+
+
+def _check(status: int, where: str) -> None:
+    if status != TT_OK:
+        raise TTError(status, where)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return TT_F32
+    if t.dtype == torch.bfloat16:
+        return TT_BF16
+    raise TypeError(f"tensors must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _options(path=0, rank_scale_pct=0, force_levels=0, cap=0):
+    return tt_options(int(path), int(rank_scale_pct), int(force_levels), int(cap))
+
+
+class Index:
+    """A prepared corpus (handle from the C library). Keeps the tensors it
+    refers to alive; releases the handle (``tt_free``) when collected."""
+
+    def __init__(self, handle: int, rows: torch.Tensor, inv_norm: torch.Tensor | None, n: int, d: int):
+        self.handle = ctypes.c_void_p(handle)
+        self.rows = rows
+        self.inv_norm = inv_norm
+        self.n = n
+        self.d = d
+
+    def free(self) -> None:
+        if self.handle is not None and self.handle.value:
+            _lib.tt_free(self.handle)
+        self.handle = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+def tt_normalize_candidates(x: torch.Tensor, out: torch.Tensor, mode: int = TT_NORM_STORE,
+                            stream=None, make_index: bool = True) -> Index | None:
+    """Row-wise L2 normalisation (``tt_normalize_candidates``).
+
+    ``x``: [n, d] float32/bfloat16 on the GPU. ``mode=TT_NORM_STORE``: ``out``
+    is [n, d] (float32 or bfloat16) and receives the normalised rows.
+    ``mode=TT_NORM_FUSED``: ``out`` is [n] float32 and receives 1/norm; the
+    index then scores the raw rows. Returns an ``Index`` (or None when
+    ``make_index`` is False, e.g. for normalising queries)."""
+    if x.dim() != 2 or not x.is_contiguous() or not out.is_contiguous():
+        raise ValueError("x must be a contiguous [n, d] tensor and out contiguous")
+    n, d = x.shape
+    handle = ctypes.c_void_p()
+    st = _lib.tt_normalize_candidates(_ptr(x), _dtype(x), n, d, _ptr(out),
+                                      _dtype(out), int(mode), _stream(stream),
+                                      ctypes.byref(handle) if make_index else None)
+    _check(st, "tt_normalize_candidates")
+    if not make_index:
+        return None
+    if mode == TT_NORM_STORE:
+        return Index(handle.value, out, None, n, d)
+    return Index(handle.value, x, out, n, d)
+
+
+def tt_index_wrap(rows: torch.Tensor, inv_norm: torch.Tensor | None = None) -> Index:
+    """Handle over an already prepared corpus (``tt_index_wrap``)."""
+    if rows.dim() != 2 or not rows.is_contiguous():
+        raise ValueError("rows must be a contiguous [n, d] tensor")
+    n, d = rows.shape
+    handle = ctypes.c_void_p()
+    _check(_lib.tt_index_wrap(_ptr(rows), _dtype(rows), n, d, _ptr(inv_norm), ctypes.byref(handle)),
+           "tt_index_wrap")
+    return Index(handle.value, rows, inv_norm, n, d)
+
+
+def tt_score_topk(index: Index, queries: torch.Tensor, k: int, tau: float = 1.0,
+                  exclude: torch.Tensor | None = None, out_ids: torch.Tensor | None = None,
+                  out_scores: torch.Tensor | None = None, stream=None, **options):
+    """Exact top-k by inner product (``tt_score_topk`` / ``tt_score_topk_ex``).
+
+    ``queries``: [b, d] float32/bfloat16 on the GPU. ``exclude``: packed
+    exclusion bits, int32 tensor of ceil(n/32) words (bit j&31 of word j>>5).
+    Returns ``(ids int32 [b,k], scores float32 [b,k])``. Keyword options
+    (``path``, ``rank_scale_pct``, ``force_levels``, ``cap``) go to
+    ``tt_score_topk_ex``."""
+    if queries.dim() != 2 or not queries.is_contiguous():
+        raise ValueError("queries must be a contiguous [b, d] tensor")
+    b, d = queries.shape
+    if d != index.d:
+        raise ValueError(f"queries have d={d}, index has d={index.d}")
+    dev = queries.device
+    if out_ids is None:
+        out_ids = torch.empty((b, k), dtype=torch.int32, device=dev)
+    if out_scores is None:
+        out_scores = torch.empty((b, k), dtype=torch.float32, device=dev)
+    if exclude is not None and (exclude.dtype not in (torch.int32,) or not exclude.is_contiguous()):
+        raise TypeError("exclude must be a contiguous int32 tensor of packed bits")
+    if options:
+        opt = _options(**options)
+        st = _lib.tt_score_topk_ex(index.handle, _ptr(queries), _dtype(queries), b, _ptr(exclude),
+                                   float(tau), int(k), _ptr(out_ids), _ptr(out_scores), _stream(stream),
+                                   ctypes.byref(opt))
+    else:
+        st = _lib.tt_score_topk(index.handle, _ptr(queries), _dtype(queries), b, _ptr(exclude),
+                                float(tau), int(k), _ptr(out_ids), _ptr(out_scores), _stream(stream))
+    _check(st, "tt_score_topk")
+    return out_ids, out_scores
+
+
+def tt_free(index: Index) -> None:
+    index.free()
+
+
+def tt_last_stats(index: Index) -> dict:
+    s = tt_stats()
+    _check(_lib.tt_last_stats(index.handle, ctypes.byref(s)), "tt_last_stats")
+    return {"path": s.path, "levels": s.levels, "rescans": s.rescans, "launches": s.launches,
+            "level_rows": list(s.level_rows[:s.levels]), "level_stride": list(s.level_stride[:s.levels]),
+            "cap": s.cap}
+
+
+def tt_plan(n: int, k: int, **options) -> dict:
+    levels, cap = _i32(), _i32()
+    rows, strides, ranks = (_i64 * 4)(), (_i64 * 4)(), (_i32 * 4)()
+    opt = _options(**options)
+    _check(_lib.tt_plan(int(n), int(k), ctypes.byref(opt), ctypes.byref(levels), rows, strides, ranks,
+                        ctypes.byref(cap)), "tt_plan")
+    L = levels.value
+    return {"levels": L, "rows": list(rows[:L]), "strides": list(strides[:L]), "ranks": list(ranks[:L]),
+            "cap": cap.value}
+
+
+def tt_launch_count() -> int:
+    return int(_lib.tt_launch_count())
+
+
+def tt_profile_begin() -> None:
+    _check(_lib.tt_profile_begin(), "tt_profile_begin")
+
+
+def tt_profile_end() -> dict:
+    ms = (ctypes.c_double * TT_NUM_KINDS)()
+    cnt = (_i64 * TT_NUM_KINDS)()
+    _check(_lib.tt_profile_end(ms, cnt), "tt_profile_end")
+    return {name: {"ms": ms[i], "launches": cnt[i]} for i, name in enumerate(KIND_NAMES)}
+
+
+def tt_version() -> str:
+    return _lib.tt_version().decode()
+
+
+def search(corpus: torch.Tensor, queries: torch.Tensor, k: int, tau: float = 1.0,
+           exclude: torch.Tensor | None = None, store_dtype=torch.bfloat16,
+           query_dtype=None, fused: bool = False, device="cuda"):
+    """End-to-end call from host tensors: copy the raw corpus and queries to
+    the GPU, normalise both, score, and copy ``(ids, scores)`` back.
+
+    ``corpus`` [n, d] and ``queries`` [b, d] are CPU tensors (pinned memory
+    makes the copies asynchronous). ``fused`` keeps the corpus raw and folds
+    the norms into the scores. ``query_dtype`` defaults to float32 for small
+    batches (b <= 8) and bfloat16 otherwise."""
+    n, d = corpus.shape
+    b = queries.shape[0]
+    dc = corpus.to(device, non_blocking=True)
+    dq = queries.to(device, non_blocking=True)
+    dx = exclude.to(device, non_blocking=True) if exclude is not None else None
+    if fused:
+        inv = torch.empty((n,), dtype=torch.float32, device=device)
+        index = tt_normalize_candidates(dc, inv, TT_NORM_FUSED)
+    else:
+        rows = torch.empty((n, d), dtype=store_dtype, device=device)
+        index = tt_normalize_candidates(dc, rows, TT_NORM_STORE)
+    if query_dtype is None:
+        query_dtype = torch.float32 if b <= 8 else torch.bfloat16
+    qn = torch.empty((b, d), dtype=query_dtype, device=device)
+    tt_normalize_candidates(dq, qn, TT_NORM_STORE, make_index=False)
+    ids, scores = tt_score_topk(index, qn, k, tau=tau, exclude=dx)
+    out_ids = torch.empty((b, k), dtype=torch.int32, pin_memory=True)
+    out_scores = torch.empty((b, k), dtype=torch.float32, pin_memory=True)
+    out_ids.copy_(ids, non_blocking=True)
+    out_scores.copy_(scores, non_blocking=True)
+    torch.cuda.current_stream().synchronize()
+    index.free()
+    return out_ids, out_scores

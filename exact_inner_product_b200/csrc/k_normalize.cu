@@ -1,0 +1,224 @@
+// k_normalize.cu - K1: row-wise L2 normalisation of a corpus (or of a batch
+// of queries), and the fp32 -> bf16 query cast.
+//
+// norm_j = sqrt(max(sum_i v_ji^2, 1e-12)), out_ji = v_ji / norm_j
+// (x-algorithm recsys_two_tower_model.py, `_l2_normalize_candidates`; the
+// user vector gets the same treatment in `RecsysTwoTowerModel.__call__`).
+//
+// HBM-bound: every row is read once with 16-byte loads and written once with
+// 16-byte (or 8-byte) stores. L lanes of a warp share one row (L = 32 for
+// rows of >= 512 bytes), each lane keeping up to 4 chunks in registers, and
+// each warp works on two row groups at a time to keep enough bytes in
+// flight. fp32 arithmetic with IEEE sqrt and division; the result is rounded
+// to the output type to nearest-even.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tt_device.cuh"
+#include "tt_internal.h"
+
+namespace tt {
+namespace {
+
+constexpr int K1_THREADS = 256;
+
+template <typename T>
+struct Elem;
+template <>
+struct Elem<float> {
+    static constexpr int per_chunk = 4;
+    __device__ static void unpack(const uint4& c, float* x) {
+        x[0] = __uint_as_float(c.x);
+        x[1] = __uint_as_float(c.y);
+        x[2] = __uint_as_float(c.z);
+        x[3] = __uint_as_float(c.w);
+    }
+};
+template <>
+struct Elem<__nv_bfloat16> {
+    static constexpr int per_chunk = 8;
+    __device__ static void unpack(const uint4& c, float* x) {
+        const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            x[2 * i] = __uint_as_float(w[i] << 16);
+            x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+};
+
+// Streaming 16-byte load (read once). Not the read-only path: `out` may
+// alias `in`.
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+    return __ldcs(reinterpret_cast<const uint4*>(p));
+}
+
+// Store the normalised values of one input chunk (E elements) to out, at
+// element offset `e0` of the row.
+template <typename Tout, int E>
+__device__ __forceinline__ void store_chunk(Tout* row_out, int e0, const float* y);
+
+template <>
+__device__ __forceinline__ void store_chunk<float, 4>(float* row_out, int e0, const float* y) {
+    *reinterpret_cast<float4*>(row_out + e0) = make_float4(y[0], y[1], y[2], y[3]);
+}
+template <>
+__device__ __forceinline__ void store_chunk<float, 8>(float* row_out, int e0, const float* y) {
+    *reinterpret_cast<float4*>(row_out + e0) = make_float4(y[0], y[1], y[2], y[3]);
+    *reinterpret_cast<float4*>(row_out + e0 + 4) = make_float4(y[4], y[5], y[6], y[7]);
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+template <>
+__device__ __forceinline__ void store_chunk<__nv_bfloat16, 4>(__nv_bfloat16* row_out, int e0,
+                                                             const float* y) {
+    *reinterpret_cast<uint2*>(row_out + e0) =
+        make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
+}
+template <>
+__device__ __forceinline__ void store_chunk<__nv_bfloat16, 8>(__nv_bfloat16* row_out, int e0,
+                                                             const float* y) {
+    *reinterpret_cast<uint4*>(row_out + e0) =
+        make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                   pack_bf16x2(y[6], y[7]));
+}
+
+// MODE 0: out rows = v / norm (Tout). MODE 1: inv_norm[j] = 1 / norm.
+// L lanes per row, CPL 16-byte chunks per lane (d * elem <= 2048 bytes).
+template <typename Tin, typename Tout, int MODE, int L, int CPL>
+__global__ void __launch_bounds__(K1_THREADS)
+    k1_normalize(const Tin* in, int64_t n, int d, Tout* out,
+                 float* __restrict__ inv_norm) {
+    constexpr int E = Elem<Tin>::per_chunk;
+    constexpr int ROWS_PER_GROUP = 32 / L;
+    const int chunks = d / E;
+    const int lane = threadIdx.x & 31;
+    const int sub = lane % L;
+    const int grp = lane / L;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t step = nwarps * (2 * ROWS_PER_GROUP);
+
+    for (int64_t base = warp * (2 * ROWS_PER_GROUP); base < n; base += step) {
+        int64_t row[2] = {base + grp, base + ROWS_PER_GROUP + grp};
+        uint4 raw[2][CPL];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                const int c = sub + i * L;
+                if (row[u] < n && c < chunks)
+                    raw[u][i] = ld_stream(in + row[u] * d + (int64_t)c * E);
+                else
+                    raw[u][i] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+        float ss[2] = {0.f, 0.f};
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                float x[E];
+                Elem<Tin>::unpack(raw[u][i], x);
+#pragma unroll
+                for (int e = 0; e < E; ++e) ss[u] = fmaf(x[e], x[e], ss[u]);
+            }
+        }
+#pragma unroll
+        for (int off = L / 2; off > 0; off >>= 1) {
+            ss[0] += __shfl_xor_sync(0xFFFFFFFFu, ss[0], off);
+            ss[1] += __shfl_xor_sync(0xFFFFFFFFu, ss[1], off);
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            if (row[u] >= n) continue;
+            const float norm = __fsqrt_rn(fmaxf(ss[u], 1e-12f));
+            if (MODE == 1) {
+                if (sub == 0) inv_norm[row[u]] = __fdiv_rn(1.0f, norm);
+            } else {
+#pragma unroll
+                for (int i = 0; i < CPL; ++i) {
+                    const int c = sub + i * L;
+                    if (c < chunks) {
+                        float x[E], y[E];
+                        Elem<Tin>::unpack(raw[u][i], x);
+#pragma unroll
+                        for (int e = 0; e < E; ++e) y[e] = __fdiv_rn(x[e], norm);
+                        store_chunk<Tout, E>(out + row[u] * d, c * E, y);
+                    }
+                }
+            }
+        }
+    }
+}
+
+__global__ void k0_cast_bf16(const float4* __restrict__ in, int64_t count4, uint2* __restrict__ out) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count4;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const float4 v = in[i];
+        out[i] = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+    }
+}
+
+template <typename Tin, typename Tout, int MODE>
+cudaError_t dispatch_lanes(const void* in, int64_t n, int d, void* out, cudaStream_t s) {
+    constexpr int E = Elem<Tin>::per_chunk;
+    const int chunks = d / E;
+    int L = 32;
+    while (L > chunks) L >>= 1;
+    const int rows_per_block = (K1_THREADS / 32) * 2 * (32 / L);
+    int64_t blocks = (n + rows_per_block - 1) / rows_per_block;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t max_blocks = (int64_t)sms * (2048 / K1_THREADS);
+    if (blocks > max_blocks) blocks = max_blocks;
+    if (blocks < 1) blocks = 1;
+    const Tin* pin = static_cast<const Tin*>(in);
+    Tout* pout = MODE == 0 ? static_cast<Tout*>(out) : nullptr;
+    float* pinv = MODE == 1 ? static_cast<float*>(out) : nullptr;
+    note_launch_begin(TT_KIND_NORMALIZE, s);
+    const int cpl = (chunks + L - 1) / L;
+    const dim3 g((unsigned)blocks), t(K1_THREADS);
+    if (L == 32 && cpl == 1) k1_normalize<Tin, Tout, MODE, 32, 1><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
+    else if (L == 32 && cpl == 2) k1_normalize<Tin, Tout, MODE, 32, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
+    else if (L == 32) k1_normalize<Tin, Tout, MODE, 32, 4><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
+    else if (L == 16) k1_normalize<Tin, Tout, MODE, 16, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
+    else if (L == 8) k1_normalize<Tin, Tout, MODE, 8, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
+    else if (L == 4) k1_normalize<Tin, Tout, MODE, 4, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
+    else k1_normalize<Tin, Tout, MODE, 2, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
+    note_launch_end(TT_KIND_NORMALIZE, s);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_normalize(const void* in, int in_dtype, int64_t n, int d, void* out,
+                             int out_dtype, int mode, cudaStream_t s) {
+    if (n == 0) return cudaSuccess;
+    if (in_dtype == TT_F32) {
+        if (mode == TT_NORM_FUSED) return dispatch_lanes<float, float, 1>(in, n, d, out, s);
+        if (out_dtype == TT_F32) return dispatch_lanes<float, float, 0>(in, n, d, out, s);
+        return dispatch_lanes<float, __nv_bfloat16, 0>(in, n, d, out, s);
+    }
+    if (mode == TT_NORM_FUSED) return dispatch_lanes<__nv_bfloat16, float, 1>(in, n, d, out, s);
+    if (out_dtype == TT_F32) return dispatch_lanes<__nv_bfloat16, float, 0>(in, n, d, out, s);
+    return dispatch_lanes<__nv_bfloat16, __nv_bfloat16, 0>(in, n, d, out, s);
+}
+
+cudaError_t launch_cast_bf16(const float* in, int64_t count, __nv_bfloat16* out, cudaStream_t s) {
+    const int64_t count4 = count / 4;  // count is a multiple of 16 (d % 16 == 0)
+    if (count4 == 0) return cudaSuccess;
+    int64_t blocks = (count4 + 255) / 256;
+    if (blocks > 4096) blocks = 4096;
+    note_launch_begin(TT_KIND_CAST, s);
+    k0_cast_bf16<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(in), count4,
+                                                  reinterpret_cast<uint2*>(out));
+    note_launch_end(TT_KIND_CAST, s);
+    return cudaGetLastError();
+}
+
+}  // namespace tt

@@ -1,0 +1,286 @@
+// k_select.cu - K4: per-query selection over the candidate keys kept by a
+// scoring pass, plus the small bookkeeping kernels.
+//
+// One CTA per query. The r-th largest key is found by a most-significant-
+// digit radix select over the 64-bit keys (digits of 11/11/10/11/11/10
+// bits, a 2048-bin shared-memory histogram per digit), so its cost depends
+// only on the number of kept keys, not on how they are ordered. Keys are
+// distinct (the low word encodes the candidate id), so exactly r keys are
+// >= the r-th largest.
+//
+// Threshold mode: the next level's filter key is (r-th largest) - 1, so a
+// later pass keeps every key >= it.
+// Final mode: the kept keys >= the k-th largest are gathered, sorted
+// descending with a shared-memory bitonic sort and written as (id, score);
+// positions past the number of eligible candidates get (-1, -inf). The
+// result is exact when the pass kept every key above its threshold
+// (count <= cap) and either found at least k of them or had no threshold;
+// otherwise the query is flagged for a rescan with a corrected threshold.
+// (Order: score descending, ties by ascending id - mhtirogla.ai Two-tower
+// retrieval, Code, Towers::top_k; padding replaces the bf16.min fill of
+// recsys_two_tower_model.py `mask_and_top_k`.)
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tt_device.cuh"
+#include "tt_internal.h"
+
+namespace tt {
+namespace {
+
+constexpr int K4_THREADS = 256;
+constexpr int K4_SORT_MAX = 2048;  // >= TT_MAX_K
+constexpr int K4_BINS = 2048;
+
+struct K4Smem {
+    uint32_t hist[K4_BINS];
+    uint32_t part[K4_THREADS];
+    uint32_t above[K4_THREADS];
+    uint64_t sorted[K4_SORT_MAX];
+    uint64_t found_prefix;
+    uint32_t found_remaining;
+    uint32_t n_collected;
+};
+
+// r-th largest (1-based) of n distinct keys; 1 <= r <= n. Block-wide.
+__device__ uint64_t block_kth_largest(const uint64_t* __restrict__ keys, int n, int r, K4Smem& sm) {
+    const int tid = threadIdx.x;
+    // digits, most significant first: widths 11, 11, 10, 11, 11, 10
+    uint64_t prefix = 0, mask = 0;
+    uint32_t remaining = (uint32_t)r;
+    int shift = 64;
+#pragma unroll 1
+    for (int pass = 0; pass < 6; ++pass) {
+        const int w = (pass == 2 || pass == 5) ? 10 : 11;
+        shift -= w;
+        const int nb = 1 << w;
+        for (int i = tid; i < nb; i += K4_THREADS) sm.hist[i] = 0;
+        __syncthreads();
+        for (int i = tid; i < n; i += K4_THREADS) {
+            const uint64_t key = keys[i];
+            if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & (uint64_t)(nb - 1)], 1u);
+        }
+        __syncthreads();
+        // Thread t owns bins [t*per, (t+1)*per); above[t] = count in higher bins.
+        const int per = nb / K4_THREADS;
+        uint32_t local = 0;
+        for (int i = 0; i < per; ++i) local += sm.hist[tid * per + i];
+        sm.part[tid] = local;
+        __syncthreads();
+        if (tid < 32) {
+            uint32_t s = 0;
+            for (int i = 0; i < 8; ++i) s += sm.part[tid * 8 + i];
+            // suffix sum over lanes: sum of lanes > tid
+            uint32_t incl = s;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const uint32_t v = __shfl_down_sync(0xFFFFFFFFu, incl, off);
+                if (tid + off < 32) incl += v;
+            }
+            uint32_t run = incl - s;  // lanes above this one
+            for (int i = 7; i >= 0; --i) {
+                sm.above[tid * 8 + i] = run;
+                run += sm.part[tid * 8 + i];
+            }
+        }
+        __syncthreads();
+        const uint32_t above = sm.above[tid];
+        if (above < remaining && remaining <= above + local) {
+            uint32_t run = above;
+            for (int i = per - 1; i >= 0; --i) {
+                const uint32_t c = sm.hist[tid * per + i];
+                if (remaining <= run + c) {
+                    sm.found_prefix = (uint64_t)(tid * per + i);
+                    sm.found_remaining = remaining - run;
+                    break;
+                }
+                run += c;
+            }
+        }
+        __syncthreads();
+        prefix |= sm.found_prefix << shift;
+        mask |= (uint64_t)(nb - 1) << shift;
+        remaining = sm.found_remaining;
+        __syncthreads();
+    }
+    return prefix;
+}
+
+__global__ void __launch_bounds__(K4_THREADS)
+    k4_select_threshold(const uint64_t* __restrict__ keys, uint32_t* __restrict__ count, int cap,
+                        int r, uint64_t* __restrict__ theta_next, float* __restrict__ thf_next) {
+    __shared__ K4Smem sm;
+    const int q = blockIdx.x;
+    const uint32_t c = count[q];
+    const int n = c < (uint32_t)cap ? (int)c : cap;
+    uint64_t th = KEY_MIN;
+    if (n >= r && r > 0) th = block_kth_largest(keys + (int64_t)q * cap, n, r, sm) - 1;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        theta_next[q] = th;
+        thf_next[q] = key_floor(th);
+        count[q] = 0;
+    }
+}
+
+__global__ void __launch_bounds__(K4_THREADS)
+    k4_select_final(const uint64_t* __restrict__ keys, uint32_t* __restrict__ count, int cap, int k,
+                    uint64_t* __restrict__ theta, float* __restrict__ thf, int32_t* __restrict__ status,
+                    int* __restrict__ flags, int repair, int32_t* __restrict__ out_ids,
+                    float* __restrict__ out_scores) {
+    __shared__ K4Smem sm;
+    const int q = blockIdx.x;
+    const int tid = threadIdx.x;
+    if (repair && status[q] == 0) return;  // block-uniform
+    const uint32_t c = count[q];
+    const int n = c < (uint32_t)cap ? (int)c : cap;
+    const uint64_t th = theta[q];
+    const uint64_t* qkeys = keys + (int64_t)q * cap;
+    const bool exact = (c <= (uint32_t)cap) && (c >= (uint32_t)k || th == KEY_MIN);
+    if (exact) {
+        const int r = n < k ? n : k;
+        if (r > 0) {
+            const uint64_t kth = block_kth_largest(qkeys, n, r, sm);
+            if (tid == 0) sm.n_collected = 0;
+            __syncthreads();
+            for (int i = tid; i < n; i += K4_THREADS) {
+                const uint64_t key = qkeys[i];
+                if (key >= kth) sm.sorted[atomicAdd(&sm.n_collected, 1u)] = key;
+            }
+            __syncthreads();
+            int P = 1;
+            while (P < r) P <<= 1;
+            for (int i = r + tid; i < P; i += K4_THREADS) sm.sorted[i] = KEY_MIN;
+            __syncthreads();
+            // bitonic sort, descending
+            for (int size = 2; size <= P; size <<= 1) {
+                for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                    for (int i = tid; i < P; i += K4_THREADS) {
+                        const int j = i ^ stride;
+                        if (j > i) {
+                            const uint64_t x = sm.sorted[i], y = sm.sorted[j];
+                            const bool desc = (i & size) == 0;
+                            if (desc ? (x < y) : (x > y)) {
+                                sm.sorted[i] = y;
+                                sm.sorted[j] = x;
+                            }
+                        }
+                    }
+                    __syncthreads();
+                }
+            }
+        }
+        for (int i = tid; i < k; i += K4_THREADS) {
+            int32_t id = -1;
+            float sc = -INFINITY;
+            if (i < r) {
+                id = (int32_t)key_id(sm.sorted[i]);
+                sc = key_score(sm.sorted[i]);
+            }
+            out_ids[(int64_t)q * k + i] = id;
+            out_scores[(int64_t)q * k + i] = sc;
+        }
+        if (tid == 0) status[q] = 0;
+    } else {
+        uint64_t th_new = KEY_MIN;
+        if (c > (uint32_t)cap && n >= k) th_new = block_kth_largest(qkeys, n, k, sm) - 1;
+        if (tid == 0) {
+            theta[q] = th_new;
+            thf[q] = key_floor(th_new);
+            status[q] = 1;
+            atomicOr(flags, 1);
+        }
+    }
+    __syncthreads();
+    if (tid == 0) count[q] = 0;
+}
+
+__global__ void k4_init(uint32_t* count, uint64_t* theta, float* thf, uint64_t th0, int b, int b_pad,
+                        int* flags) {
+    const float f0 = key_floor(th0), fmax = key_floor(KEY_MAX);
+    for (int q = blockIdx.x * blockDim.x + threadIdx.x; q < b_pad; q += gridDim.x * blockDim.x) {
+        if (q < b) {
+            count[q] = 0;
+            theta[q] = th0;
+            thf[q] = f0;
+        } else {
+            theta[q] = KEY_MAX;
+            thf[q] = fmax;
+        }
+    }
+    if (blockIdx.x == 0 && threadIdx.x < 2) flags[threadIdx.x] = 0;
+}
+
+__global__ void k4_prepare_repair(uint64_t* theta, float* thf, const int32_t* status, int b, int* flags) {
+    const float fmax = key_floor(KEY_MAX);
+    for (int q = blockIdx.x * blockDim.x + threadIdx.x; q < b; q += gridDim.x * blockDim.x) {
+        if (status[q] == 0) {
+            theta[q] = KEY_MAX;
+            thf[q] = fmax;
+        }
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) flags[0] = 0;
+}
+
+__global__ void k4_pad(int32_t* out_ids, float* out_scores, int64_t count) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        out_ids[i] = -1;
+        out_scores[i] = -INFINITY;
+    }
+}
+
+unsigned small_grid(int64_t n) {
+    int64_t g = (n + 255) / 256;
+    if (g < 1) g = 1;
+    if (g > 1024) g = 1024;
+    return (unsigned)g;
+}
+
+}  // namespace
+
+cudaError_t launch_init(uint32_t* count, uint64_t* theta, float* thf, uint64_t theta_value, int b,
+                        int b_pad, int* flags, cudaStream_t s) {
+    note_launch_begin(TT_KIND_AUX, s);
+    k4_init<<<small_grid(b_pad), 256, 0, s>>>(count, theta, thf, theta_value, b, b_pad, flags);
+    note_launch_end(TT_KIND_AUX, s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select_threshold(const uint64_t* keys, uint32_t* count, int cap, int b, int r,
+                                    uint64_t* theta_next, float* thf_next, cudaStream_t s) {
+    if (b == 0) return cudaSuccess;
+    note_launch_begin(TT_KIND_SELECT, s);
+    k4_select_threshold<<<b, K4_THREADS, 0, s>>>(keys, count, cap, r, theta_next, thf_next);
+    note_launch_end(TT_KIND_SELECT, s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_select_final(const uint64_t* keys, uint32_t* count, int cap, int b, int k,
+                                uint64_t* theta, float* thf, int32_t* status, int* flags,
+                                int repair, int32_t* out_ids, float* out_scores, cudaStream_t s) {
+    if (b == 0) return cudaSuccess;
+    note_launch_begin(TT_KIND_SELECT, s);
+    k4_select_final<<<b, K4_THREADS, 0, s>>>(keys, count, cap, k, theta, thf, status, flags, repair,
+                                             out_ids, out_scores);
+    note_launch_end(TT_KIND_SELECT, s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_prepare_repair(uint64_t* theta, float* thf, const int32_t* status, int b,
+                                  int* flags, cudaStream_t s) {
+    note_launch_begin(TT_KIND_AUX, s);
+    k4_prepare_repair<<<small_grid(b), 256, 0, s>>>(theta, thf, status, b, flags);
+    note_launch_end(TT_KIND_AUX, s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pad(int32_t* out_ids, float* out_scores, int64_t count, cudaStream_t s) {
+    if (count == 0) return cudaSuccess;
+    note_launch_begin(TT_KIND_AUX, s);
+    k4_pad<<<small_grid(count), 256, 0, s>>>(out_ids, out_scores, count);
+    note_launch_end(TT_KIND_AUX, s);
+    return cudaGetLastError();
+}
+
+}  // namespace tt

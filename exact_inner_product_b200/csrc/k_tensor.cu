@@ -1,0 +1,355 @@
+// k_tensor.cu - K3: batched scorer on the 5th-generation tensor cores.
+//
+// For a batch of queries the scores S = V . U^T form a dense contraction
+// (recsys_two_tower_model.py `forward` / `compute_top_k`:
+// matmul(user.astype(bf16), post_embeddings.T)). This kernel computes it
+// tile by tile with tcgen05 MMAs (bf16 operands in shared memory, fp32
+// accumulators in tensor memory) and never writes the score matrix: the
+// epilogue reads each accumulator tile from TMEM, applies the per-candidate
+// scale and the exclusion mask and keeps only candidates whose key beats the
+// query's threshold (the same filter as the streaming scorer).
+//
+// Layout of one MMA: M = 128 corpus rows (TMEM lanes), N = NQ <= 256
+// queries (TMEM columns), K = 16. A query tile (NQ x d, bf16) stays resident
+// in shared memory for a whole work unit; corpus tiles stream through a ring
+// of 16 KB stages (128 rows x 64 elements, 128-byte swizzle). Two TMEM
+// accumulators (columns 0 and 256) let the epilogue drain tile t while the
+// tensor cores work on tile t + 1.
+//
+// Warp roles (320 threads): warp 0 issues TMA loads, warp 1 allocates TMEM
+// and issues MMAs (one thread), warps 2..9 are the epilogue: warp w reads
+// TMEM lanes 32*(w%4)..+31 (its 32 corpus rows) and one half of the columns.
+//
+// Work units: (query tile, corpus chunk) with the query tile varying
+// fastest, so the CTAs that run at the same time read the same corpus
+// chunks and share them through L2.
+//
+// Every wait is bounded; on expiry the kernel records an error code,
+// waits (bounded) for its own copies and MMAs in flight, frees TMEM and
+// returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tt_device.cuh"
+#include "tt_internal.h"
+
+namespace tt {
+namespace {
+
+constexpr int K3_M = 128;                  // corpus rows per tile
+constexpr int K3_KC = 64;                  // bf16 elements per 128-byte swizzle row
+constexpr int K3_STAGE_BYTES = K3_M * 128; // one K chunk of a corpus tile
+constexpr int K3_MAX_STAGES = 12;
+constexpr int K3_EPI_WARPS = 8;
+constexpr int K3_THREADS = 32 * (2 + K3_EPI_WARPS);
+constexpr int K3_TMEM_COLS = 512;
+constexpr int K3_ACC_COLS = 256;
+constexpr int K3_MAX_NQ = 256;
+constexpr int K3_SMEM_BUDGET = 227 * 1024;
+
+struct K3Ctl {
+    uint64_t full[K3_MAX_STAGES];
+    uint64_t empty[K3_MAX_STAGES];
+    uint64_t qfull, qempty;
+    uint64_t tfull[2], tempty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+struct K3Params {
+    PassArgs a;
+    int nq;          // queries per tile (multiple of 16, <= 256)
+    int q_tiles;     // ceil(b / nq)
+    int kchunks;     // ceil(d / 64)
+    int stages;
+    int64_t tiles;   // corpus tiles of 128 rows in this level
+    int chunks;      // corpus chunks (units = q_tiles * chunks)
+    uint32_t idesc;
+};
+
+__device__ __forceinline__ void unit_range(const K3Params& p, int u, int* qt, int64_t* t0,
+                                           int64_t* t1) {
+    *qt = u % p.q_tiles;
+    const int ch = u / p.q_tiles;
+    *t0 = p.tiles * ch / p.chunks;
+    *t1 = p.tiles * (ch + 1) / p.chunks;
+}
+
+__global__ void __launch_bounds__(K3_THREADS, 1)
+    k3_tensor(const __grid_constant__ CUtensorMap tm_rows, const __grid_constant__ CUtensorMap tm_q,
+              const K3Params p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int q_chunk_bytes = p.nq * 128;
+    uint8_t* qsm = smem;                                           // [kchunks][nq x 128 B]
+    uint8_t* ring = smem + (size_t)p.kchunks * q_chunk_bytes;      // [stages][16 KB]
+    K3Ctl* ctl = reinterpret_cast<K3Ctl*>(ring + (size_t)p.stages * K3_STAGE_BYTES);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int n_units = p.q_tiles * p.chunks;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < p.stages; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->empty[s], 1);
+        }
+        mbar_init(&ctl->qfull, 1);
+        mbar_init(&ctl->qempty, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&ctl->tfull[b], 1);
+            mbar_init(&ctl->tempty[b], K3_EPI_WARPS);
+        }
+        mbar_init(&ctl->drain, 1);
+        ctl->abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&ctl->tmem_base, K3_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = ctl->tmem_base;
+    volatile int* abort = &ctl->abort;
+
+    if (warp == 0) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_rows);
+            tma_prefetch_desc(&tm_q);
+            uint32_t it = 0;
+            int uc = 0, q_issued = -1;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++uc) {
+                int qt;
+                int64_t t0, t1;
+                unit_range(p, u, &qt, &t0, &t1);
+                if (!mbar_wait(&ctl->qempty, (uc & 1) ^ 1, abort)) { ok = false; break; }
+                q_issued = uc;
+                mbar_arrive_expect_tx(&ctl->qfull, (uint32_t)(p.kchunks * q_chunk_bytes));
+                for (int kc = 0; kc < p.kchunks; ++kc)
+                    tma_load_2d(qsm + (size_t)kc * q_chunk_bytes, &tm_q, &ctl->qfull, kc * K3_KC,
+                                qt * p.nq);
+                for (int64_t t = t0; ok && t < t1; ++t) {
+                    for (int kc = 0; kc < p.kchunks; ++kc, ++it) {
+                        const int s = it % p.stages;
+                        if (!mbar_wait(&ctl->empty[s], ((it / p.stages) & 1) ^ 1, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&ctl->full[s], K3_STAGE_BYTES);
+                        tma_load_2d(ring + (size_t)s * K3_STAGE_BYTES, &tm_rows, &ctl->full[s],
+                                    kc * K3_KC, (int32_t)(t * K3_M));
+                    }
+                }
+            }
+            if (!ok) {
+                atomicExch(p.a.err, ERR_TIMEOUT_TMA);
+                *abort = 1;
+            }
+            // Every issued load must land before the block may exit.
+            const uint32_t first = it > (uint32_t)p.stages ? it - p.stages : 0;
+            for (uint32_t j = first; j < it; ++j)
+                mbar_wait(&ctl->full[j % p.stages], (j / p.stages) & 1, nullptr);
+            if (q_issued >= 0) mbar_wait(&ctl->qfull, q_issued & 1, nullptr);
+        }
+    } else if (warp == 1) {
+        // ------------------------------ MMA issuer ------------------------------
+        if (lane == 0) {
+            uint32_t it = 0, tc = 0;
+            int uc = 0;
+            bool ok = true;
+            const uint32_t qbase = smem_u32(qsm);
+            const uint32_t rbase = smem_u32(ring);
+            for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x, ++uc) {
+                int qt;
+                int64_t t0, t1;
+                unit_range(p, u, &qt, &t0, &t1);
+                if (!mbar_wait(&ctl->qfull, uc & 1, abort)) { ok = false; break; }
+                tc_fence_after();
+                for (int64_t t = t0; ok && t < t1; ++t, ++tc) {
+                    const int buf = tc & 1;
+                    if (!mbar_wait(&ctl->tempty[buf], ((tc >> 1) & 1) ^ 1, abort)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem_base + (uint32_t)(buf * K3_ACC_COLS);
+                    for (int kc = 0; kc < p.kchunks; ++kc, ++it) {
+                        const int s = it % p.stages;
+                        if (!mbar_wait(&ctl->full[s], (it / p.stages) & 1, abort)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t a_addr = rbase + (uint32_t)(s * K3_STAGE_BYTES);
+                        const uint32_t b_addr = qbase + (uint32_t)(kc * q_chunk_bytes);
+#pragma unroll
+                        for (int kk = 0; kk < K3_KC / 16; ++kk) {
+                            umma_bf16(d_tmem, umma_desc_kmajor_sw128(a_addr + kk * 32),
+                                      umma_desc_kmajor_sw128(b_addr + kk * 32), p.idesc,
+                                      (kc | kk) != 0 ? 1u : 0u);
+                        }
+                        umma_commit(&ctl->empty[s]);  // stage free once these MMAs finish
+                    }
+                    if (ok) umma_commit(&ctl->tfull[buf]);  // accumulator ready
+                }
+                if (ok) umma_commit(&ctl->qempty);  // query tile free after this unit
+            }
+            if (!ok) {
+                atomicExch(p.a.err, ERR_TIMEOUT_MMA);
+                *abort = 1;
+            }
+            // Wait for every MMA issued by this thread before TMEM is freed.
+            umma_commit(&ctl->drain);
+            mbar_wait(&ctl->drain, 0, nullptr);
+        }
+    } else {
+        // ------------------------------ epilogue ------------------------------
+        const int ew = warp - 2;
+        const int quarter = warp & 3;        // TMEM lane quarter this warp may access
+        const int half = ew >> 2;            // which interleaved half of the 32-column chunks
+        const int row_in_tile = quarter * 32 + lane;
+        const int nchunk32 = (p.nq + 31) / 32;
+        const PassArgs& a = p.a;
+        uint32_t tc = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
+            int qt;
+            int64_t t0, t1;
+            unit_range(p, u, &qt, &t0, &t1);
+            // Thresholds of this unit's queries (padded past b with +inf /
+            // KEY_MAX, so out-of-range columns never pass).
+            const float* thf_unit = a.thf + (int64_t)qt * p.nq;
+            const uint64_t* th_unit = a.theta + (int64_t)qt * p.nq;
+            for (int64_t t = t0; t < t1; ++t, ++tc) {
+                const int buf = tc & 1;
+                // per-row data, fetched before waiting for the accumulator
+                const int64_t j = t * K3_M + row_in_tile;
+                const bool valid = j < a.n_rows;
+                const int64_t id = j * a.stride;
+                bool row_ok = valid;
+                float c = a.inv_tau;
+                if (valid) {
+                    if (a.exclude) row_ok = !((a.exclude[id >> 5] >> (id & 31)) & 1u);
+                    if (a.inv_norm) c = a.inv_norm[id] * a.inv_tau;
+                }
+                if (!mbar_wait(&ctl->tfull[buf], (tc >> 1) & 1, abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int ch = half; ch < nchunk32; ch += 2) {
+                    const int col0 = ch * 32;
+                    float v[32];
+                    tmem_ld_32cols(tmem_base + ((uint32_t)(quarter * 32) << 16) +
+                                       (uint32_t)(buf * K3_ACC_COLS + col0),
+                                   v);
+                    tmem_ld_wait();
+                    bool any = false;
+                    const float4* th4 = reinterpret_cast<const float4*>(thf_unit + col0);
+#pragma unroll
+                    for (int i4 = 0; i4 < 8; ++i4) {
+                            const float4 th = __ldg(th4 + i4);
+                        any |= v[4 * i4 + 0] * c >= th.x;
+                        any |= v[4 * i4 + 1] * c >= th.y;
+                        any |= v[4 * i4 + 2] * c >= th.z;
+                        any |= v[4 * i4 + 3] * c >= th.w;
+                    }
+                    any = any && row_ok;
+                    if (__any_sync(0xFFFFFFFFu, any)) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const float sc = v[i] * c;
+                            const uint64_t key = make_key(sc, (uint32_t)id);
+                            const bool keep = row_ok && key > __ldg(th_unit + col0 + i);
+                            const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, keep);
+                            if (ballot) {
+                                const int q = qt * p.nq + col0 + i;
+                                const int leader = __ffs(ballot) - 1;
+                                uint32_t base = 0;
+                                if (lane == leader) base = atomicAdd(a.count + q, (uint32_t)__popc(ballot));
+                                base = __shfl_sync(0xFFFFFFFFu, base, leader);
+                                if (keep) {
+                                    const uint32_t slot = base + __popc(ballot & lanemask_lt());
+                                    if (slot < (uint32_t)a.cap) a.keys[(int64_t)q * a.cap + slot] = key;
+                                }
+                            }
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->tempty[buf]);
+            }
+        }
+        if (!ok) {
+            atomicExch(a.err, ERR_TIMEOUT_EPI);
+            *abort = 1;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, K3_TMEM_COLS);
+    }
+}
+
+}  // namespace
+
+int tensor_pass_smem_bytes(int d, int nq) {
+    const int kchunks = (d + K3_KC - 1) / K3_KC;
+    const int q_bytes = kchunks * nq * 128;
+    const int fixed = 1024 + q_bytes + (int)sizeof(K3Ctl);
+    int stages = (K3_SMEM_BUDGET - fixed) / K3_STAGE_BYTES;
+    if (stages > K3_MAX_STAGES) stages = K3_MAX_STAGES;
+    if (stages < 2) return -1;
+    return fixed + stages * K3_STAGE_BYTES;
+}
+
+int tensor_pass_max_nq(int d) {
+    for (int nq = K3_MAX_NQ; nq >= 16; nq -= 16)
+        if (tensor_pass_smem_bytes(d, nq) > 0 && tensor_pass_smem_bytes(d, nq) <= K3_SMEM_BUDGET &&
+            ((d + K3_KC - 1) / K3_KC) * nq * 128 <= 128 * 1024)
+            return nq;
+    return 0;
+}
+
+cudaError_t launch_tensor_pass(const PassArgs& a, const CUtensorMap& tm_rows,
+                               const CUtensorMap& tm_queries, int nq, cudaStream_t s,
+                               int sm_count) {
+    if (a.n_rows == 0 || a.b == 0) return cudaSuccess;
+    K3Params p;
+    p.a = a;
+    p.nq = nq;
+    p.q_tiles = (a.b + nq - 1) / nq;
+    p.kchunks = (a.d + K3_KC - 1) / K3_KC;
+    const int smem = tensor_pass_smem_bytes(a.d, nq);
+    if (smem <= 0) return cudaErrorInvalidValue;
+    const int fixed = 1024 + p.kchunks * nq * 128 + (int)sizeof(K3Ctl);
+    p.stages = (smem - fixed) / K3_STAGE_BYTES;
+    p.tiles = (a.n_rows + K3_M - 1) / K3_M;
+    // Corpus chunks: make q_tiles * chunks a multiple of the SM count when
+    // possible (every CTA gets the same number of units), with at least one
+    // tile per chunk.
+    int chunks = 0;
+    for (int w = 1; w <= 8 && chunks == 0; ++w)
+        if (((int64_t)sm_count * w) % p.q_tiles == 0) chunks = (int)((int64_t)sm_count * w / p.q_tiles);
+    if (chunks == 0) chunks = (sm_count * 4 + p.q_tiles - 1) / p.q_tiles;
+    if (chunks < 1) chunks = 1;
+    if (chunks > p.tiles) chunks = (int)p.tiles;
+    p.chunks = chunks;
+    p.idesc = umma_idesc_bf16(K3_M, nq);
+    const int n_units = p.q_tiles * p.chunks;
+    const int grid = n_units < sm_count ? n_units : sm_count;
+    cudaError_t e = cudaFuncSetAttribute(k3_tensor, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    note_launch_begin(TT_KIND_TENSOR, s);
+    k3_tensor<<<grid, K3_THREADS, smem, s>>>(tm_rows, tm_queries, p);
+    note_launch_end(TT_KIND_TENSOR, s);
+    return cudaGetLastError();
+}
+
+}  // namespace tt

@@ -1,0 +1,704 @@
+// tt_api.cu - the C ABI: argument validation, the scan plan, kernel
+// orchestration, tensor maps, launch accounting and event timing.
+//
+// How tt_score_topk stays exact without ever materialising the score matrix:
+// each scoring pass keeps, per query, only candidates whose key (score, id)
+// beats a threshold key theta, and the final selection checks that the pass
+// kept everything it had to. Thresholds are estimated on coarser levels of
+// the corpus (every 64th row, every 4096th row, ...): the r-th best key of a
+// level, taken with r about 3k/64, predicts a filter that keeps about 3k
+// candidates of the next finer level. The deepest level is small enough to
+// keep every key (no threshold). A query's final pass is exact when it kept
+// at least k keys (so every member of the true top-k beat the threshold) and
+// its buffer did not overflow; if either fails - which the estimate makes
+// rare but never impossible - the query is rescanned with a threshold that
+// is correct by construction (the k-th best kept key, or none).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+#include <vector>
+
+#include "../../include/tt.h"
+#include "tt_device.cuh"
+#include "tt_internal.h"
+
+#define TT_VERSION_STRING "tt 0.1.0 (sm_100a)"
+
+struct tt_index {
+    const void* rows;
+    tt_dtype dtype;
+    int64_t n;
+    int32_t d;
+    const float* inv_norm;
+    int device;
+    // scratch (device), grown on demand
+    void* scratch;
+    size_t scratch_bytes;
+    int* h_flags;  // pinned, 2 ints: [0] rescan needed, [1] device error code
+    tt_stats last;
+};
+
+namespace tt {
+
+// ---------------------------------------------------------------------------
+// errors
+// ---------------------------------------------------------------------------
+static thread_local char g_last_error[256] = {0};
+
+static tt_status cuda_fail(cudaError_t e, const char* what) {
+    snprintf(g_last_error, sizeof g_last_error, "%s: %s", what, cudaGetErrorString(e));
+    return e == cudaErrorMemoryAllocation ? TT_ERR_NO_MEMORY : TT_ERR_CUDA;
+}
+
+#define TT_CUDA(call, what)                          \
+    do {                                             \
+        cudaError_t _e = (call);                     \
+        if (_e != cudaSuccess) return cuda_fail(_e, what); \
+    } while (0)
+
+// ---------------------------------------------------------------------------
+// launch accounting and event timing
+// ---------------------------------------------------------------------------
+static std::atomic<int64_t> g_launches{0};
+static std::mutex g_prof_mu;
+static bool g_prof_on = false;
+struct ProfRec {
+    int kind;
+    cudaEvent_t start, stop;
+};
+static std::vector<ProfRec> g_prof_recs;
+static std::vector<cudaEvent_t> g_event_pool;
+static cudaEvent_t g_pending_start = nullptr;
+
+static cudaEvent_t pool_event() {
+    if (!g_event_pool.empty()) {
+        cudaEvent_t e = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+void note_launch_begin(int kind, cudaStream_t s) {
+    (void)kind;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    std::lock_guard<std::mutex> lock(g_prof_mu);
+    if (!g_prof_on) return;
+    g_pending_start = pool_event();
+    if (g_pending_start) cudaEventRecord(g_pending_start, s);
+}
+
+void note_launch_end(int kind, cudaStream_t s) {
+    std::lock_guard<std::mutex> lock(g_prof_mu);
+    if (!g_prof_on || !g_pending_start) return;
+    cudaEvent_t stop = pool_event();
+    if (!stop) return;
+    cudaEventRecord(stop, s);
+    g_prof_recs.push_back({kind, g_pending_start, stop});
+    g_pending_start = nullptr;
+}
+
+// ---------------------------------------------------------------------------
+// tensor maps
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+static bool encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                      uint64_t rows, uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_rows,
+                      CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) {
+        snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled unavailable");
+        return false;
+    }
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {pitch_bytes};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+        return false;
+    }
+    return true;
+}
+
+bool stream_pass_tensor_map(const PassArgs& a, CUtensorMap* tm, int* nbox, int* row_pitch,
+                            bool* sw) {
+    const int elem = a.dtype == TT_F32 ? 4 : 2;
+    const int row_bytes = a.d * elem;
+    const CUtensorMapDataType dt =
+        a.dtype == TT_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const uint64_t pitch = (uint64_t)a.stride * (uint64_t)row_bytes;
+    if (row_bytes >= 128) {
+        *sw = true;
+        *nbox = (row_bytes + 127) / 128;
+        *row_pitch = *nbox * 128;
+        return encode_2d(tm, dt, a.rows, (uint64_t)a.d, (uint64_t)a.n_rows, pitch, 128 / elem, 32,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+    *sw = false;
+    *nbox = 1;
+    *row_pitch = row_bytes;
+    return encode_2d(tm, dt, a.rows, (uint64_t)a.d, (uint64_t)a.n_rows, pitch, (uint32_t)a.d, 32,
+                     CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+bool bf16_tile_tensor_map(const void* base, int64_t rows, int d, int64_t row_pitch_elems,
+                          int box_rows, CUtensorMap* tm) {
+    return encode_2d(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, (uint64_t)d, (uint64_t)rows,
+                     (uint64_t)row_pitch_elems * 2u, 64, (uint32_t)box_rows,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// ---------------------------------------------------------------------------
+// validation helpers
+// ---------------------------------------------------------------------------
+static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+static bool valid_dtype(int dt) { return dt == TT_F32 || dt == TT_BF16; }
+
+static tt_status check_d(int32_t d) {
+    if (d <= 0) return TT_ERR_INVALID_ARG;
+    if (d % 16 != 0 || d > TT_MAX_D) return TT_ERR_UNSUPPORTED;
+    return TT_OK;
+}
+
+// The pointer must be device (or managed) memory of the current device.
+static tt_status check_device_ptr(const void* p, const char* what) {
+    if (p == nullptr) return TT_OK;
+    cudaPointerAttributes attr;
+    cudaError_t e = cudaPointerGetAttributes(&attr, p);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        snprintf(g_last_error, sizeof g_last_error, "%s: %s", what, cudaGetErrorString(e));
+        return TT_ERR_CUDA;
+    }
+    if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged) {
+        snprintf(g_last_error, sizeof g_last_error, "%s is not device memory", what);
+        return TT_ERR_INVALID_ARG;
+    }
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (attr.device != dev) {
+        snprintf(g_last_error, sizeof g_last_error, "%s lives on device %d, current is %d", what,
+                 attr.device, dev);
+        return TT_ERR_INVALID_ARG;
+    }
+    return TT_OK;
+}
+
+static int sm_count_current() {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+// ---------------------------------------------------------------------------
+// scan plan
+// ---------------------------------------------------------------------------
+constexpr int STRIDE_RATIO = 64;
+constexpr int DEFAULT_CAP = 16384;
+constexpr int MIN_RANK = 32;
+constexpr int MAX_LEVELS = 4;
+constexpr int MAX_RESCANS = 64;
+
+struct Plan {
+    int levels;
+    int64_t stride[MAX_LEVELS];
+    int64_t rows[MAX_LEVELS];
+    int rank[MAX_LEVELS];  // rank[i] (i >= 1): r-th best key of level i sets theta of level i-1
+    int cap;
+};
+
+static tt_status make_plan(int64_t n, int32_t k, const tt_options* opt, Plan* p) {
+    int cap = (opt && opt->cap) ? opt->cap : DEFAULT_CAP;
+    if (cap < 256 || cap > DEFAULT_CAP || (cap & (cap - 1)) != 0) return TT_ERR_INVALID_ARG;
+    if (cap < 2 * k) return TT_ERR_INVALID_ARG;
+    const int scale = (opt && opt->rank_scale_pct) ? opt->rank_scale_pct : 100;
+    if (scale < 1 || scale > 10000) return TT_ERR_INVALID_ARG;
+    const int forced = opt ? opt->force_levels : 0;
+    if (forced < 0 || forced > MAX_LEVELS) return TT_ERR_INVALID_ARG;
+    p->cap = cap;
+    int L = 0;
+    int64_t s = 1;
+    if (forced > 0) {
+        L = forced - 1;
+        for (int i = 0; i < L; ++i) s *= STRIDE_RATIO;
+        while (L > 0 && s >= n) {  // keep at least two rows at the deepest level
+            s /= STRIDE_RATIO;
+            --L;
+        }
+    } else {
+        while ((n + s - 1) / s > cap && L < MAX_LEVELS - 1) {
+            s *= STRIDE_RATIO;
+            ++L;
+        }
+    }
+    p->levels = L + 1;
+    int64_t st = 1;
+    int need = k;  // rank needed at the finer level
+    p->rank[0] = k;
+    for (int i = 0; i <= L; ++i) {
+        p->stride[i] = st;
+        p->rows[i] = n > 0 ? (n + st - 1) / st : 0;
+        if (i >= 1) {
+            int64_t r = (3 * (int64_t)need + STRIDE_RATIO - 1) / STRIDE_RATIO;
+            if (r < MIN_RANK) r = MIN_RANK;
+            r = r * scale / 100;
+            if (r < 1) r = 1;
+            p->rank[i] = (int)r;
+            need = (int)r;
+        }
+        st *= STRIDE_RATIO;
+    }
+    return TT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// scratch
+// ---------------------------------------------------------------------------
+struct Scratch {
+    uint64_t* keys;
+    uint32_t* count;
+    uint64_t* theta;
+    float* thf;
+    int32_t* status;
+    int* flags;
+    __nv_bfloat16* qcast;
+};
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+static tt_status get_scratch(tt_index* ix, int b, int b_pad, int cap, int d, bool need_qcast,
+                             Scratch* out) {
+    size_t off = 0;
+    const size_t o_keys = off;
+    off = align_up(off + (size_t)b * cap * 8, 256);
+    const size_t o_count = off;
+    off = align_up(off + (size_t)b_pad * 4, 256);
+    const size_t o_theta = off;
+    off = align_up(off + (size_t)b_pad * 8, 256);
+    const size_t o_thf = off;
+    off = align_up(off + (size_t)b_pad * 4, 256);
+    const size_t o_status = off;
+    off = align_up(off + (size_t)b_pad * 4, 256);
+    const size_t o_flags = off;
+    off = align_up(off + 64, 256);
+    const size_t o_q = off;
+    off = align_up(off + (need_qcast ? (size_t)b * d * 2 : 0), 256);
+    if (off > ix->scratch_bytes) {
+        if (ix->scratch) {
+            cudaFree(ix->scratch);
+            ix->scratch = nullptr;
+            ix->scratch_bytes = 0;
+        }
+        const size_t want = off + off / 4;
+        cudaError_t e = cudaMalloc(&ix->scratch, want);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            ix->scratch = nullptr;
+            return cuda_fail(e, "scratch allocation");
+        }
+        ix->scratch_bytes = want;
+    }
+    uint8_t* base = static_cast<uint8_t*>(ix->scratch);
+    out->keys = reinterpret_cast<uint64_t*>(base + o_keys);
+    out->count = reinterpret_cast<uint32_t*>(base + o_count);
+    out->theta = reinterpret_cast<uint64_t*>(base + o_theta);
+    out->thf = reinterpret_cast<float*>(base + o_thf);
+    out->status = reinterpret_cast<int32_t*>(base + o_status);
+    out->flags = reinterpret_cast<int*>(base + o_flags);
+    out->qcast = need_qcast ? reinterpret_cast<__nv_bfloat16*>(base + o_q) : nullptr;
+    if (!ix->h_flags) {
+        cudaError_t e = cudaMallocHost(&ix->h_flags, 2 * sizeof(int));
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            ix->h_flags = nullptr;
+            return cuda_fail(e, "pinned flag allocation");
+        }
+    }
+    return TT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// one scoring pass over level i
+// ---------------------------------------------------------------------------
+struct PathCfg {
+    int path;           // 1 stream, 2 tensor
+    int nq;             // tensor path: queries per tile
+    const void* queries;
+    int q_dtype;
+    CUtensorMap tm_q;
+};
+
+static tt_status run_pass(const tt_index* ix, const PathCfg& pc, const Plan& plan, int level,
+                          const Scratch& sc, const uint32_t* exclude, float inv_tau, int b,
+                          cudaStream_t s, int sms) {
+    PassArgs a;
+    a.rows = ix->rows;
+    a.dtype = ix->dtype;
+    a.n_rows = plan.rows[level];
+    a.stride = plan.stride[level];
+    a.d = ix->d;
+    a.inv_norm = ix->inv_norm;
+    a.exclude = exclude;
+    a.inv_tau = inv_tau;
+    a.queries = pc.queries;
+    a.q_dtype = pc.q_dtype;
+    a.b = b;
+    a.theta = sc.theta;
+    a.thf = sc.thf;
+    a.count = sc.count;
+    a.keys = sc.keys;
+    a.cap = plan.cap;
+    a.err = sc.flags + 1;
+    cudaError_t e;
+    if (pc.path == 2) {
+        CUtensorMap tm_rows;
+        if (!bf16_tile_tensor_map(ix->rows, a.n_rows, ix->d, a.stride * ix->d, 128, &tm_rows))
+            return TT_ERR_CUDA;
+        e = launch_tensor_pass(a, tm_rows, pc.tm_q, pc.nq, s, sms);
+    } else {
+        e = launch_stream_pass(a, s, sms);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, pc.path == 2 ? "tensor pass" : "stream pass");
+    return TT_OK;
+}
+
+}  // namespace tt
+
+using namespace tt;
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* tt_version(void) { return TT_VERSION_STRING; }
+
+const char* tt_status_string(tt_status st) {
+    switch (st) {
+        case TT_OK: return "TT_OK";
+        case TT_ERR_INVALID_ARG: return "TT_ERR_INVALID_ARG";
+        case TT_ERR_UNSUPPORTED: return "TT_ERR_UNSUPPORTED";
+        case TT_ERR_CUDA: return "TT_ERR_CUDA";
+        case TT_ERR_NO_MEMORY: return "TT_ERR_NO_MEMORY";
+        case TT_ERR_TIMEOUT: return "TT_ERR_TIMEOUT";
+        case TT_ERR_INTERNAL: return "TT_ERR_INTERNAL";
+    }
+    return "TT_ERR_UNKNOWN";
+}
+
+const char* tt_last_error(void) { return g_last_error; }
+
+int64_t tt_launch_count(void) { return g_launches.load(); }
+
+tt_status tt_profile_begin(void) {
+    std::lock_guard<std::mutex> lock(g_prof_mu);
+    for (auto& r : g_prof_recs) {
+        g_event_pool.push_back(r.start);
+        g_event_pool.push_back(r.stop);
+    }
+    g_prof_recs.clear();
+    g_prof_on = true;
+    return TT_OK;
+}
+
+tt_status tt_profile_end(double* ms_per_kind, int64_t* launches_per_kind) {
+    std::lock_guard<std::mutex> lock(g_prof_mu);
+    g_prof_on = false;
+    double ms[TT_NUM_KINDS] = {0};
+    int64_t cnt[TT_NUM_KINDS] = {0};
+    tt_status st = TT_OK;
+    for (auto& r : g_prof_recs) {
+        float t = 0.f;
+        cudaError_t e = cudaEventSynchronize(r.stop);
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&t, r.start, r.stop);
+        if (e != cudaSuccess) {
+            st = cuda_fail(e, "profile event");
+            continue;
+        }
+        if (r.kind >= 0 && r.kind < TT_NUM_KINDS) {
+            ms[r.kind] += t;
+            cnt[r.kind] += 1;
+        }
+    }
+    for (auto& r : g_prof_recs) {
+        g_event_pool.push_back(r.start);
+        g_event_pool.push_back(r.stop);
+    }
+    g_prof_recs.clear();
+    for (int i = 0; i < TT_NUM_KINDS; ++i) {
+        if (ms_per_kind) ms_per_kind[i] = ms[i];
+        if (launches_per_kind) launches_per_kind[i] = cnt[i];
+    }
+    return st;
+}
+
+tt_status tt_plan(int64_t n, int32_t k, const tt_options* options, int32_t* levels,
+                  int64_t* rows, int64_t* strides, int32_t* ranks, int32_t* cap) {
+    if (n < 0 || n > TT_MAX_N) return TT_ERR_INVALID_ARG;
+    if (k <= 0) return TT_ERR_INVALID_ARG;
+    if (k > TT_MAX_K) return TT_ERR_UNSUPPORTED;
+    Plan p;
+    tt_status st = make_plan(n, k, options, &p);
+    if (st != TT_OK) return st;
+    if (levels) *levels = p.levels;
+    if (cap) *cap = p.cap;
+    for (int i = 0; i < p.levels; ++i) {
+        if (rows) rows[i] = p.rows[i];
+        if (strides) strides[i] = p.stride[i];
+        if (ranks) ranks[i] = p.rank[i];
+    }
+    return TT_OK;
+}
+
+static tt_status new_index(const void* rows, tt_dtype dtype, int64_t n, int32_t d,
+                           const float* inv_norm, tt_index** index_out) {
+    tt_index* ix = new (std::nothrow) tt_index;
+    if (!ix) return TT_ERR_NO_MEMORY;
+    memset(ix, 0, sizeof *ix);
+    ix->rows = rows;
+    ix->dtype = dtype;
+    ix->n = n;
+    ix->d = d;
+    ix->inv_norm = inv_norm;
+    cudaGetDevice(&ix->device);
+    *index_out = ix;
+    return TT_OK;
+}
+
+tt_status tt_normalize_candidates(const void* in, tt_dtype in_dtype, int64_t n, int32_t d,
+                                  void* out, tt_dtype out_dtype, int32_t mode, void* stream,
+                                  tt_index** index_out) {
+    // host-side checks first: nothing touches the device before they pass
+    if (index_out) *index_out = nullptr;
+    if (n < 0) return TT_ERR_INVALID_ARG;
+    if (n > TT_MAX_N) return TT_ERR_UNSUPPORTED;
+    tt_status st = check_d(d);
+    if (st != TT_OK) return st;
+    if (!valid_dtype(in_dtype) || !valid_dtype(out_dtype)) return TT_ERR_INVALID_ARG;
+    if (mode != TT_NORM_STORE && mode != TT_NORM_FUSED) return TT_ERR_INVALID_ARG;
+    if (n > 0 && (in == nullptr || out == nullptr)) return TT_ERR_INVALID_ARG;
+    if (!aligned(in, 16) || !aligned(out, 16)) return TT_ERR_INVALID_ARG;
+    if (n > 0) {
+        if ((st = check_device_ptr(in, "in")) != TT_OK) return st;
+        if ((st = check_device_ptr(out, "out")) != TT_OK) return st;
+        cudaError_t e = launch_normalize(in, in_dtype, n, d, out, out_dtype, mode,
+                                         static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "normalize");
+    }
+    if (index_out) {
+        if (mode == TT_NORM_STORE)
+            return new_index(out, out_dtype, n, d, nullptr, index_out);
+        return new_index(in, in_dtype, n, d, static_cast<const float*>(out), index_out);
+    }
+    return TT_OK;
+}
+
+tt_status tt_index_wrap(const void* rows, tt_dtype dtype, int64_t n, int32_t d,
+                        const float* inv_norm, tt_index** index_out) {
+    if (!index_out) return TT_ERR_INVALID_ARG;
+    *index_out = nullptr;
+    if (n < 0) return TT_ERR_INVALID_ARG;
+    if (n > TT_MAX_N) return TT_ERR_UNSUPPORTED;
+    tt_status st = check_d(d);
+    if (st != TT_OK) return st;
+    if (!valid_dtype(dtype)) return TT_ERR_INVALID_ARG;
+    if (n > 0 && rows == nullptr) return TT_ERR_INVALID_ARG;
+    if (!aligned(rows, 16) || !aligned(inv_norm, 4)) return TT_ERR_INVALID_ARG;
+    if (n > 0) {
+        if ((st = check_device_ptr(rows, "rows")) != TT_OK) return st;
+        if ((st = check_device_ptr(inv_norm, "inv_norm")) != TT_OK) return st;
+    }
+    return new_index(rows, dtype, n, d, inv_norm, index_out);
+}
+
+void tt_free(tt_index* index) {
+    if (!index) return;
+    if (index->scratch) cudaFree(index->scratch);
+    if (index->h_flags) cudaFreeHost(index->h_flags);
+    delete index;
+}
+
+tt_status tt_last_stats(const tt_index* index, tt_stats* out) {
+    if (!index || !out) return TT_ERR_INVALID_ARG;
+    *out = index->last;
+    return TT_OK;
+}
+
+tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtype, int32_t b,
+                           const uint32_t* exclude_bits, float tau, int32_t k, int32_t* out_ids,
+                           float* out_scores, void* stream, const tt_options* options) {
+    // ---------------- host-side validation (no device calls) ----------------
+    if (!index) return TT_ERR_INVALID_ARG;
+    if (b < 0) return TT_ERR_INVALID_ARG;
+    if (k <= 0) return TT_ERR_INVALID_ARG;
+    if (k > TT_MAX_K) return TT_ERR_UNSUPPORTED;
+    if (!(tau > 0.0f) || !isfinite(tau)) return TT_ERR_INVALID_ARG;
+    if (!valid_dtype(q_dtype)) return TT_ERR_INVALID_ARG;
+    if (b > 0 && (queries == nullptr || out_ids == nullptr || out_scores == nullptr))
+        return TT_ERR_INVALID_ARG;
+    if (!aligned(queries, 16) || !aligned(out_ids, 4) || !aligned(out_scores, 4) ||
+        !aligned(exclude_bits, 4))
+        return TT_ERR_INVALID_ARG;
+    const int path_req = options ? options->path : 0;
+    if (path_req < 0 || path_req > 2) return TT_ERR_INVALID_ARG;
+    Plan plan;
+    tt_status st = make_plan(index->n, k, options, &plan);
+    if (st != TT_OK) return st;
+    if (index->dtype == TT_F32 && index->d > 256) return TT_ERR_UNSUPPORTED;
+    const bool tc_possible = index->dtype == TT_BF16 && index->d >= 64 && tensor_pass_max_nq(index->d) > 0;
+    int path = path_req;
+    if (path == 0) path = (tc_possible && b > 8) ? 2 : 1;
+    if (path == 2 && !tc_possible) return TT_ERR_UNSUPPORTED;
+    if (b == 0) return TT_OK;
+
+    // ---------------- device checks ----------------
+    if ((st = check_device_ptr(queries, "queries")) != TT_OK) return st;
+    if ((st = check_device_ptr(out_ids, "out_ids")) != TT_OK) return st;
+    if ((st = check_device_ptr(out_scores, "out_scores")) != TT_OK) return st;
+    if ((st = check_device_ptr(exclude_bits, "exclude_bits")) != TT_OK) return st;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev != index->device) {
+        snprintf(g_last_error, sizeof g_last_error, "index was made on device %d, current is %d",
+                 index->device, dev);
+        return TT_ERR_INVALID_ARG;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t launches0 = g_launches.load();
+    tt_stats stats;
+    memset(&stats, 0, sizeof stats);
+    stats.path = path;
+    stats.levels = plan.levels;
+    stats.cap = plan.cap;
+    for (int i = 0; i < plan.levels; ++i) {
+        stats.level_rows[i] = plan.rows[i];
+        stats.level_stride[i] = plan.stride[i];
+    }
+
+    if (index->n == 0) {
+        cudaError_t e = launch_pad(out_ids, out_scores, (int64_t)b * k, s);
+        if (e != cudaSuccess) return cuda_fail(e, "pad");
+        stats.launches = (int)(g_launches.load() - launches0);
+        index->last = stats;
+        return TT_OK;
+    }
+
+    // Query tiling of the tensor-core path (decided before the scratch layout:
+    // threshold arrays are padded to whole query tiles plus one 32-column chunk).
+    int nq = 0, q_tiles = 1;
+    if (path == 2) {
+        const int max_nq = tensor_pass_max_nq(index->d);
+        q_tiles = (b + max_nq - 1) / max_nq;
+        nq = (b + q_tiles - 1) / q_tiles;
+        nq = (nq + 15) / 16 * 16;
+        if (nq > max_nq) nq = max_nq;
+    }
+    const int b_pad = (path == 2 ? q_tiles * nq : b) + 64;
+    const bool need_qcast = path == 2 && q_dtype == TT_F32;
+    Scratch sc;
+    if ((st = get_scratch(index, b, b_pad, plan.cap, index->d, need_qcast, &sc)) != TT_OK) return st;
+    const int sms = sm_count_current();
+    const float inv_tau = 1.0f / tau;
+
+    PathCfg pc;
+    memset(&pc, 0, sizeof pc);
+    pc.path = path;
+    pc.queries = queries;
+    pc.q_dtype = q_dtype;
+    if (path == 2) {
+        if (need_qcast) {
+            cudaError_t e = launch_cast_bf16(static_cast<const float*>(queries), (int64_t)b * index->d,
+                                             sc.qcast, s);
+            if (e != cudaSuccess) return cuda_fail(e, "query cast");
+            pc.queries = sc.qcast;
+            pc.q_dtype = TT_BF16;
+        }
+        pc.nq = nq;
+        if (!bf16_tile_tensor_map(pc.queries, b, index->d, index->d, nq, &pc.tm_q)) return TT_ERR_CUDA;
+    }
+
+    cudaError_t e = launch_init(sc.count, sc.theta, sc.thf, KEY_MIN, b, b_pad, sc.flags, s);
+    if (e != cudaSuccess) return cuda_fail(e, "init");
+    for (int lv = plan.levels - 1; lv >= 0; --lv) {
+        if ((st = run_pass(index, pc, plan, lv, sc, exclude_bits, inv_tau, b, s, sms)) != TT_OK) return st;
+        if (lv > 0)
+            e = launch_select_threshold(sc.keys, sc.count, plan.cap, b, plan.rank[lv], sc.theta,
+                                        sc.thf, s);
+        else
+            e = launch_select_final(sc.keys, sc.count, plan.cap, b, k, sc.theta, sc.thf, sc.status,
+                                    sc.flags, 0, out_ids, out_scores, s);
+        if (e != cudaSuccess) return cuda_fail(e, "select");
+    }
+    int rescans = 0;
+    while (true) {
+        TT_CUDA(cudaMemcpyAsync(index->h_flags, sc.flags, 2 * sizeof(int), cudaMemcpyDeviceToHost, s),
+                "flag readback");
+        TT_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+        if (index->h_flags[1] != 0) {
+            snprintf(g_last_error, sizeof g_last_error, "device wait expired (code %d)",
+                     index->h_flags[1]);
+            stats.rescans = rescans;
+            stats.launches = (int)(g_launches.load() - launches0);
+            index->last = stats;
+            return TT_ERR_TIMEOUT;
+        }
+        if (index->h_flags[0] == 0) break;
+        if (rescans >= MAX_RESCANS) {
+            snprintf(g_last_error, sizeof g_last_error, "exactness check not met after %d rescans",
+                     rescans);
+            return TT_ERR_INTERNAL;
+        }
+        e = launch_prepare_repair(sc.theta, sc.thf, sc.status, b, sc.flags, s);
+        if (e != cudaSuccess) return cuda_fail(e, "prepare rescan");
+        if ((st = run_pass(index, pc, plan, 0, sc, exclude_bits, inv_tau, b, s, sms)) != TT_OK) return st;
+        e = launch_select_final(sc.keys, sc.count, plan.cap, b, k, sc.theta, sc.thf, sc.status,
+                                sc.flags, 1, out_ids, out_scores, s);
+        if (e != cudaSuccess) return cuda_fail(e, "select");
+        ++rescans;
+    }
+    stats.rescans = rescans;
+    stats.launches = (int)(g_launches.load() - launches0);
+    index->last = stats;
+    return TT_OK;
+}
+
+tt_status tt_score_topk(tt_index* index, const void* queries, tt_dtype q_dtype, int32_t b,
+                        const uint32_t* exclude_bits, float tau, int32_t k, int32_t* out_ids,
+                        float* out_scores, void* stream) {
+    return tt_score_topk_ex(index, queries, q_dtype, b, exclude_bits, tau, k, out_ids, out_scores,
+                            stream, nullptr);
+}
+
+}  // extern "C"

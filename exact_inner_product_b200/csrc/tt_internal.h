@@ -1,0 +1,84 @@
+// tt_internal.h - host-side interfaces between the C-ABI layer (tt_api.cu)
+// and the kernel launchers (k_*.cu). Not part of the public ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/tt.h"
+
+namespace tt {
+
+// One scoring pass over one level of the corpus: level row j is corpus row
+// j * stride, for j < n_rows. Survivors (key > theta[q]) are appended to
+// keys[q * cap + slot], slot = atomicAdd(count[q], 1); slots >= cap are
+// counted but not stored.
+struct PassArgs {
+    const void* rows;          // corpus [n, d] (level rows are a strided view)
+    int dtype;                 // TT_F32 / TT_BF16 (corpus)
+    int64_t n_rows;            // rows in this level
+    int64_t stride;            // corpus rows between consecutive level rows
+    int d;
+    const float* inv_norm;     // [n] or null
+    const uint32_t* exclude;   // [ceil(n/32)] or null
+    float inv_tau;
+    const void* queries;       // [b, d]
+    int q_dtype;
+    int b;
+    const uint64_t* theta;     // [b_pad] threshold keys (KEY_MAX past b)
+    const float* thf;          // [b_pad] key_floor(theta), +inf past b
+    uint32_t* count;           // [b]
+    uint64_t* keys;            // [b * cap]
+    int cap;
+    int* err;                  // device error word
+};
+
+// Kernel launch bookkeeping (counts and optional event timing).
+void note_launch_begin(int kind, cudaStream_t s);
+void note_launch_end(int kind, cudaStream_t s);
+
+// Launchers. Each returns cudaSuccess or the launch error.
+cudaError_t launch_normalize(const void* in, int in_dtype, int64_t n, int d, void* out,
+                             int out_dtype, int mode, cudaStream_t s);
+cudaError_t launch_cast_bf16(const float* in, int64_t count, __nv_bfloat16* out, cudaStream_t s);
+cudaError_t launch_stream_pass(const PassArgs& a, cudaStream_t s, int sm_count);
+cudaError_t launch_tensor_pass(const PassArgs& a, const CUtensorMap& tm_rows,
+                               const CUtensorMap& tm_queries, int nq_tile, cudaStream_t s,
+                               int sm_count);
+// count[0..b) = 0; theta/thf[0..b) = theta_value; [b, b_pad) = KEY_MAX / +inf;
+// flags[0..2) = 0.
+cudaError_t launch_init(uint32_t* count, uint64_t* theta, float* thf, uint64_t theta_value, int b,
+                        int b_pad, int* flags, cudaStream_t s);
+// Threshold mode: theta_next[q] = (r-th best kept key) - 1, or KEY_MIN when
+// fewer than r keys were kept; counts reset to 0.
+cudaError_t launch_select_threshold(const uint64_t* keys, uint32_t* count, int cap, int b, int r,
+                                    uint64_t* theta_next, float* thf_next, cudaStream_t s);
+// Final mode: writes the sorted top-k (ids, scores) of queries whose pass was
+// exact; otherwise marks status[q] = 1, sets flags[0] and leaves the next
+// threshold in theta[q]. In a repair round (repair != 0) queries whose
+// status is 0 are skipped.
+cudaError_t launch_select_final(const uint64_t* keys, uint32_t* count, int cap, int b, int k,
+                                uint64_t* theta, float* thf, int32_t* status, int* flags,
+                                int repair, int32_t* out_ids, float* out_scores, cudaStream_t s);
+// Before a repair round: theta[q] = KEY_MAX where status[q] == 0; flags[0] = 0.
+cudaError_t launch_prepare_repair(uint64_t* theta, float* thf, const int32_t* status, int b,
+                                  int* flags, cudaStream_t s);
+
+// Tensor maps (built on the host through the driver entry point).
+// Streaming pass: rows of the level as a 2-D tensor {d, n_rows} with row
+// pitch stride*d*elem; 32-row boxes of 128 swizzled bytes (rows >= 128 B) or
+// of the whole unswizzled row.
+bool stream_pass_tensor_map(const PassArgs& a, CUtensorMap* tm, int* nbox, int* row_pitch,
+                            bool* sw);
+// Tensor-core pass: bf16 boxes of 64 elements x box_rows rows, 128-byte swizzle.
+bool bf16_tile_tensor_map(const void* base, int64_t rows, int d, int64_t row_pitch_elems,
+                          int box_rows, CUtensorMap* tm);
+cudaError_t launch_pad(int32_t* out_ids, float* out_scores, int64_t count, cudaStream_t s);
+
+// Shared-memory bytes the tensor-core pass needs for a given d and query tile.
+int tensor_pass_smem_bytes(int d, int nq_tile);
+int tensor_pass_max_nq(int d);
+
+}  // namespace tt

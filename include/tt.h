@@ -1,0 +1,230 @@
+/*
+ * tt.h - exact top-k maximum-inner-product search on NVIDIA B200 (sm_100a).
+ *
+ * The retrieval step of a two-tower recommender: L2-normalise the candidate
+ * corpus once, then for every user (query) vector return the k candidates
+ * with the largest dot product, exactly (brute force, no approximation).
+ *
+ *   x-algorithm recsys_two_tower_model.py:
+ *     `_l2_normalize_candidates`  v / sqrt(max(sum v^2, 1e-12))
+ *     `forward` / `compute_top_k`  scores = user . post_embeddings^T
+ *     `forward` / `mask_and_top_k` excluded candidates never win; sorted top-k
+ *   Two-Tower Retrieval at Industrial Scale, TwoTower.score: u @ v.t() / tau
+ *   mhtirogla.ai Two-tower retrieval, Code, Towers::top_k: score every item,
+ *     stable sort descending (lower index first on equal scores), take k.
+ *
+ * Conventions for every entry point:
+ *   - Data pointers are DEVICE pointers (cudaMalloc'd or torch CUDA tensors)
+ *     owned by the caller, 16-byte aligned, rows contiguous (row-major
+ *     [rows, d], row stride d elements). Host pointers are rejected with
+ *     TT_ERR_INVALID_ARG.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). Work is enqueued on it in order.
+ *   - Arguments are validated on the host before any device work; a rejected
+ *     call has no side effects.
+ *   - Errors are reported as tt_status values only; nothing aborts the process.
+ *   - bf16 means IEEE binary32 truncated to its upper 16 bits (bfloat16);
+ *     conversions to bf16 round to nearest, ties to even.
+ */
+#ifndef TT_H
+#define TT_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TT_API __attribute__((visibility("default")))
+#else
+#define TT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum tt_status {
+    TT_OK = 0,
+    TT_ERR_INVALID_ARG = 1, /* null, host or misaligned pointer; negative size; bad tau; ... */
+    TT_ERR_UNSUPPORTED = 2, /* well-formed but outside the kernels' range (see limits below) */
+    TT_ERR_CUDA = 3,        /* a CUDA call failed; tt_last_error() has the message */
+    TT_ERR_NO_MEMORY = 4,   /* device or pinned-host allocation failed */
+    TT_ERR_TIMEOUT = 5,     /* a bounded device-side wait expired; outputs are not valid */
+    TT_ERR_INTERNAL = 6     /* the exactness check could not be satisfied (not expected) */
+} tt_status;
+
+typedef enum tt_dtype { TT_F32 = 0, TT_BF16 = 1 } tt_dtype;
+
+/* How tt_normalize_candidates prepares the corpus. */
+typedef enum tt_norm_mode {
+    TT_NORM_STORE = 0, /* write normalised rows v_j / norm_j to `out` ([n,d], out_dtype) */
+    TT_NORM_FUSED = 1  /* keep rows raw; write inv_norm_j = 1 / norm_j to `out` ([n] f32);
+                          scores are multiplied by inv_norm_j inside the scorer */
+} tt_norm_mode;
+
+/* Limits. */
+#define TT_MAX_D 512        /* d must be a multiple of 16 and at most 512 (f32 corpus: 256) */
+#define TT_MAX_K 2048       /* k at most 2048 */
+#define TT_MAX_N 2147483647 /* candidate ids are int32: n < 2^31 */
+
+/* Opaque handle describing a prepared corpus. Owned by the library; release
+ * with tt_free. It refers to, but does not own, the caller's corpus buffers,
+ * which must stay alive and unchanged while the handle is used. It also owns
+ * the device scratch memory of tt_score_topk (grown on demand). A handle must
+ * not be used from two host threads at once. */
+typedef struct tt_index tt_index;
+
+/*
+ * tt_normalize_candidates - row-wise L2 normalisation of a corpus.
+ *
+ *   norm_j = sqrt(max(sum_i v_ji^2, 1e-12))      (fp32 arithmetic)
+ *   TT_NORM_STORE: out[j,i] = v_ji / norm_j, rounded to out_dtype
+ *   TT_NORM_FUSED: out[j]   = 1 / norm_j (f32); `in` is left as is
+ *
+ * (recsys_two_tower_model.py `_l2_normalize_candidates`; the same formula
+ * normalises the user vector in `RecsysTwoTowerModel.__call__`, so this call
+ * also serves to normalise a batch of queries.)
+ *
+ * in        device [n, d] rows, in_dtype (TT_F32 or TT_BF16)
+ * n         rows, 0 <= n < 2^31 (n = 0 is allowed: nothing to do)
+ * d         row width, multiple of 16, 16 <= d <= 512
+ * out       device buffer: [n, d] out_dtype (STORE) or [n] f32 (FUSED). For
+ *           STORE it may alias `in` when the dtypes match.
+ * out_dtype TT_F32 or TT_BF16 (ignored for FUSED)
+ * mode      tt_norm_mode
+ * stream    cudaStream_t
+ * index_out optional: if not NULL, receives a new handle over the prepared
+ *           corpus (STORE: rows = out; FUSED: rows = in, inv_norm = out),
+ *           which the caller releases with tt_free. If NULL, only the
+ *           normalisation is enqueued (e.g. for queries).
+ */
+TT_API tt_status tt_normalize_candidates(const void* in, tt_dtype in_dtype, int64_t n, int32_t d,
+                                  void* out, tt_dtype out_dtype, int32_t mode, void* stream,
+                                  tt_index** index_out);
+
+/*
+ * tt_index_wrap - a handle over a corpus that is already prepared (rows
+ * normalised and stored, or raw rows plus their f32 inv_norm), e.g. loaded
+ * from a checkpoint. No device work. rows: device [n, d] dtype; inv_norm:
+ * device [n] f32 or NULL. Limits as for tt_normalize_candidates.
+ */
+TT_API tt_status tt_index_wrap(const void* rows, tt_dtype dtype, int64_t n, int32_t d,
+                        const float* inv_norm, tt_index** index_out);
+
+/*
+ * tt_score_topk - exact top-k by inner product for a batch of queries.
+ *
+ *   s_bj = fl(dot_bj * c_j),  c_j = fl(inv_norm_j * fl(1/tau))  (inv_norm_j = 1
+ *          unless the handle was prepared with TT_NORM_FUSED)
+ *   dot_bj = sum_i q_bi * v_ji with fp32 accumulation
+ *   For each query: the k eligible candidates with the largest s_bj, sorted by
+ *   s descending; equal scores are ordered by ascending id. Candidates whose
+ *   exclusion bit is set never appear. When fewer than k candidates are
+ *   eligible, the remaining slots hold id -1 and score -INFINITY.
+ *
+ * (recsys_two_tower_model.py `forward`: compute_top_k, mask_and_top_k,
+ *  local_top_k with k_actual = min(k, N); TwoTower.score divides by tau.)
+ *
+ * The result is exact: the kernels keep fp32 scores and select by a total
+ * order on (score, id), and the call verifies on the device that no
+ * candidate of the true top-k was filtered out, rescanning when needed.
+ *
+ * index        handle from tt_normalize_candidates or tt_index_wrap
+ * queries      device [b, d], q_dtype. Queries are used as given (normalise
+ *              them first if the model expects unit vectors). On the tensor-
+ *              core path an f32 query batch is rounded to bf16 first; an f32
+ *              corpus or b <= 8 keeps f32 queries exactly.
+ * q_dtype      TT_F32 or TT_BF16
+ * b            number of queries, b >= 0 (b = 0: nothing to do)
+ * exclude_bits device uint32 words, ceil(n/32) of them, or NULL for none.
+ *              Bit (j & 31) of word (j >> 5) set = candidate j excluded.
+ * tau          temperature, finite and > 0 (1 = plain inner product)
+ * k            1 <= k <= 2048
+ * out_ids      device [b, k] int32
+ * out_scores   device [b, k] f32
+ * stream       cudaStream_t
+ *
+ * The call returns once the results are complete on `stream` (it
+ * synchronises with the stream to read the device-side exactness check).
+ * TT_ERR_TIMEOUT: a device-side wait gave up; outputs undefined.
+ */
+TT_API tt_status tt_score_topk(tt_index* index, const void* queries, tt_dtype q_dtype, int32_t b,
+                        const uint32_t* exclude_bits, float tau, int32_t k, int32_t* out_ids,
+                        float* out_scores, void* stream);
+
+/* Path selection and test hooks for tt_score_topk_ex. Zero-initialise, then
+ * set fields; tt_score_topk uses all zeros. */
+typedef struct tt_options {
+    int32_t path;           /* 0 auto; 1 CUDA-core streaming scorer; 2 tensor-core scorer */
+    int32_t rank_scale_pct; /* 0 = 100. Scales the ranks used to set the estimated
+                               thresholds (test hook: < 100 provokes rescans) */
+    int32_t force_levels;   /* 0 auto; > 0 = number of levels (1 = single pass) */
+    int32_t cap;            /* 0 auto (16384); candidate buffer per query, power of 2,
+                               256..16384 (test hook: small values provoke overflow) */
+} tt_options;
+
+TT_API tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtype, int32_t b,
+                           const uint32_t* exclude_bits, float tau, int32_t k, int32_t* out_ids,
+                           float* out_scores, void* stream, const tt_options* options);
+
+/* What the last tt_score_topk on a handle did. */
+typedef struct tt_stats {
+    int32_t path;            /* 1 streaming, 2 tensor core */
+    int32_t levels;          /* scoring passes in the plan (1 = single pass) */
+    int32_t rescans;         /* extra full passes made to restore exactness */
+    int32_t launches;        /* kernels launched by the call */
+    int64_t level_rows[4];   /* rows scanned per level, finest first */
+    int64_t level_stride[4]; /* corpus-row stride per level */
+    int32_t cap;             /* candidate buffer per query */
+    int32_t reserved;
+} tt_stats;
+
+TT_API tt_status tt_last_stats(const tt_index* index, tt_stats* out);
+
+/*
+ * tt_plan - the scan plan tt_score_topk would use for a corpus of n rows and
+ * a given k (host only, no device work). Level 0 is the whole corpus; level i
+ * scans every (64^i)-th row. The deepest level keeps every key; the r-th best
+ * key of level i (ranks[i], i >= 1) sets the filter threshold of level i-1.
+ * Arrays receive up to 4 entries. Any output pointer may be NULL.
+ * Errors as tt_score_topk for n, k and options.
+ */
+TT_API tt_status tt_plan(int64_t n, int32_t k, const tt_options* options, int32_t* levels, int64_t* rows,
+                  int64_t* strides, int32_t* ranks, int32_t* cap);
+
+/* Release a handle and its scratch memory. NULL is a no-op. Must not be
+ * called while work using the handle is still running on a stream. */
+TT_API void tt_free(tt_index* index);
+
+/* Kernel-launch accounting and event timing (library-wide). Kinds: */
+#define TT_KIND_NORMALIZE 0
+#define TT_KIND_CAST 1
+#define TT_KIND_STREAM 2
+#define TT_KIND_TENSOR 3
+#define TT_KIND_SELECT 4
+#define TT_KIND_AUX 5
+#define TT_NUM_KINDS 6
+
+/* Total kernels this library has launched in the process. */
+TT_API int64_t tt_launch_count(void);
+
+/* Start recording a CUDA event pair around every subsequent launch, on the
+ * launch stream. */
+TT_API tt_status tt_profile_begin(void);
+
+/* Stop recording, wait for the recorded events, and return per kind the
+ * summed device time (ms) and the number of launches since tt_profile_begin.
+ * Either array may be NULL; each has TT_NUM_KINDS entries. */
+TT_API tt_status tt_profile_end(double* ms_per_kind, int64_t* launches_per_kind);
+
+/* Human-readable name of a status, and the last CUDA error text seen by the
+ * calling thread (empty if none). */
+TT_API const char* tt_status_string(tt_status status);
+TT_API const char* tt_last_error(void);
+
+/* Library version string. */
+TT_API const char* tt_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TT_H */
