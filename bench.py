@@ -214,12 +214,18 @@ def cpu_baseline(w: W.Workload, raw_c, raw_q, excl, seconds=12.0):
 # ---------------------------------------------------------------------------
 # our implementation
 # ---------------------------------------------------------------------------
+def workload_from_args(args) -> W.Workload:
+    """The named workload, resized by --n/--b/--k (smaller cases for profiling)."""
+    over = {key: getattr(args, key) for key in ("n", "b", "k") if getattr(args, key)}
+    return W.workload(args.workload, **over)
+
+
 def run_ours(args, world, rank, local):
     import exact_inner_product_b200 as tt
 
-    w = W.workload(args.workload)
+    w = workload_from_args(args)
     if world > 1:  # each rank: its own queries (independent replica)
-        w = W.workload(args.workload, seed=w.seed + 7919 * rank)
+        w = W.workload(w.name, n=w.n, b=w.b, k=w.k, seed=w.seed + 7919 * rank)
     dev = torch.device("cuda", local)
     raw_c = W.corpus(w, dev)
     raw_q = W.queries(w, dev)
@@ -367,7 +373,7 @@ def run_reference(args, world, rank):
     if rank != 0:
         return None
     import oracle
-    w = W.workload(args.workload)
+    w = workload_from_args(args)
     raw_c = W.corpus(w, "cpu")
     raw_q = W.queries(w, "cpu")
     excl = W.exclusion_bits(w, "cpu")
@@ -400,6 +406,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--n", type=int, default=0, help="override the workload's corpus size")
+    ap.add_argument("--b", type=int, default=0, help="override the workload's batch size")
+    ap.add_argument("--k", type=int, default=0, help="override the workload's k")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
