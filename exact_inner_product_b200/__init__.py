@@ -80,6 +80,8 @@ _sig("tt_last_stats", ctypes.c_int, [_vp, ctypes.POINTER(tt_stats)])
 _sig("tt_plan", ctypes.c_int, [_i64, _i32, ctypes.POINTER(tt_options), ctypes.POINTER(_i32),
                                ctypes.POINTER(_i64), ctypes.POINTER(_i64), ctypes.POINTER(_i32),
                                ctypes.POINTER(_i32)])
+_sig("tt_score_topk_noalloc", ctypes.c_int, [_vp, ctypes.c_int, _i64, _i32, _vp, _vp, ctypes.c_int, _i32,
+                                             _vp, ctypes.c_float, _i32, _vp, _vp, _vp])
 _sig("tt_free", None, [_vp])
 _sig("tt_launch_count", _i64, [])
 _sig("tt_profile_begin", ctypes.c_int, [])
@@ -89,6 +91,7 @@ _sig("tt_last_error", ctypes.c_char_p, [])
 _sig("tt_version", ctypes.c_char_p, [])
 
 EXPORTED = ("tt_normalize_candidates", "tt_index_wrap", "tt_score_topk", "tt_score_topk_ex",
+            "tt_score_topk_noalloc",
             "tt_last_stats", "tt_plan", "tt_free", "tt_launch_count", "tt_profile_begin",
             "tt_profile_end", "tt_status_string", "tt_last_error", "tt_version")
 
@@ -217,6 +220,31 @@ def tt_score_topk(index: Index, queries: torch.Tensor, k: int, tau: float = 1.0,
         st = _lib.tt_score_topk(index.handle, _ptr(queries), _dtype(queries), b, _ptr(exclude),
                                 float(tau), int(k), _ptr(out_ids), _ptr(out_scores), _stream(stream))
     _check(st, "tt_score_topk")
+    return out_ids, out_scores
+
+
+def tt_score_topk_noalloc(rows: torch.Tensor, queries: torch.Tensor, k: int, tau: float = 1.0,
+                          inv_norm: torch.Tensor | None = None, exclude: torch.Tensor | None = None,
+                          out_ids: torch.Tensor | None = None, out_scores: torch.Tensor | None = None,
+                          stream=None):
+    """``tt_score_topk`` for callers that must not allocate device memory
+    (``tt_score_topk_noalloc``): the library works in a fixed array reserved
+    on each GPU, so this call makes no allocation of its own. ``rows`` is the
+    prepared corpus (normalised rows, or raw rows with ``inv_norm``). Output
+    tensors are allocated here only when not given; pass them in to keep the
+    whole call allocation-free. At most about 255 queries per call."""
+    if rows.dim() != 2 or queries.dim() != 2 or not rows.is_contiguous() or not queries.is_contiguous():
+        raise ValueError("rows and queries must be contiguous 2-D tensors")
+    n, d = rows.shape
+    b = queries.shape[0]
+    if out_ids is None:
+        out_ids = torch.empty((b, k), dtype=torch.int32, device=queries.device)
+    if out_scores is None:
+        out_scores = torch.empty((b, k), dtype=torch.float32, device=queries.device)
+    st = _lib.tt_score_topk_noalloc(_ptr(rows), _dtype(rows), n, d, _ptr(inv_norm), _ptr(queries),
+                                    _dtype(queries), b, _ptr(exclude), float(tau), int(k), _ptr(out_ids),
+                                    _ptr(out_scores), _stream(stream))
+    _check(st, "tt_score_topk_noalloc")
     return out_ids, out_scores
 
 

@@ -56,6 +56,10 @@ static tt_status cuda_fail(cudaError_t e, const char* what) {
     return e == cudaErrorMemoryAllocation ? TT_ERR_NO_MEMORY : TT_ERR_CUDA;
 }
 
+void set_last_error_message(const char* msg) {
+    snprintf(g_last_error, sizeof g_last_error, "%s", msg);
+}
+
 #define TT_CUDA(call, what)                          \
     do {                                             \
         cudaError_t _e = (call);                     \

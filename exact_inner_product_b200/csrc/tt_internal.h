@@ -35,6 +35,9 @@ struct PassArgs {
     int* err;                  // device error word
 };
 
+// Set the text tt_last_error() returns on the calling thread.
+void set_last_error_message(const char* msg);
+
 // Kernel launch bookkeeping (counts and optional event timing).
 void note_launch_begin(int kind, cudaStream_t s);
 void note_launch_end(int kind, cudaStream_t s);

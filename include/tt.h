@@ -194,6 +194,44 @@ TT_API tt_status tt_plan(int64_t n, int32_t k, const tt_options* options, int32_
  * called while work using the handle is still running on a stream. */
 TT_API void tt_free(tt_index* index);
 
+/*
+ * tt_score_topk_noalloc - tt_score_topk for callers that must not allocate
+ * device memory while they run. (Not a step of the method: the pages have no
+ * counterpart; it only changes where the work buffers live.)
+ *
+ * Who needs it: a process that reserved the GPU's memory up front (a serving
+ * process with its own memory pool, where a late cudaMalloc fails or
+ * fragments the pool), or a latency-bound loop in which cudaMalloc/cudaFree
+ * would stall all work on the device. tt_score_topk keeps its buffers in the
+ * index handle and grows them with cudaMalloc; this entry point calls no
+ * allocator at all (no cudaMalloc, cudaFree, pinned host memory or handle):
+ * its work buffers are one fixed array of TT_NOALLOC_SCRATCH_BYTES that the
+ * library declares in device memory, reserved on every GPU where the library
+ * is loaded until the process exits.
+ *
+ * Arguments: the corpus directly (rows: device [n, d] dtype; inv_norm:
+ * device [n] f32 for a raw corpus, else NULL), then as tt_score_topk. Result
+ * and exactness as tt_score_topk.
+ *
+ * Limits and rules:
+ *   - b is limited by the array: about 128 KiB of work memory per query, so
+ *     up to 255 queries per call; larger b is rejected with
+ *     TT_ERR_UNSUPPORTED (tt_last_error() says how much was needed);
+ *   - every call on a GPU uses the same array: calls that overlap on the GPU
+ *     (two streams or two host threads at once) race and corrupt each other's
+ *     results, so callers must serialise them;
+ *   - the array keeps the previous call's contents; each call resets what it
+ *     relies on before use;
+ *   - the first call on each GPU looks up the array's device address with
+ *     that GPU current; make this first call before any stream capture.
+ */
+#define TT_NOALLOC_SCRATCH_BYTES (32 * 1024 * 1024)
+
+TT_API tt_status tt_score_topk_noalloc(const void* rows, tt_dtype dtype, int64_t n, int32_t d,
+                                       const float* inv_norm, const void* queries, tt_dtype q_dtype,
+                                       int32_t b, const uint32_t* exclude_bits, float tau, int32_t k,
+                                       int32_t* out_ids, float* out_scores, void* stream);
+
 /* Kernel-launch accounting and event timing (library-wide). Kinds: */
 #define TT_KIND_NORMALIZE 0
 #define TT_KIND_CAST 1

@@ -1,0 +1,76 @@
+"""tt_score_topk_noalloc, the entry point for callers that must not allocate
+device memory while they run (for instance a serving process whose memory
+pool reserved the GPU at start-up, where a late cudaMalloc would fail or
+stall the device). It works in a fixed array the library reserves on each
+GPU instead of buffers grown with cudaMalloc.
+
+The test calls it through the C ABI, twice in a row on the same inputs (the
+array keeps the first call's leftovers, which the second call must not see),
+and checks both results against the regular tt_score_topk within the score
+tolerance of the other parity tests. It sits in a file of its own that
+pytest collects last, and passes alone in a fresh process as well as after
+the other tests.
+"""
+import ctypes
+import math
+
+import pytest
+import torch
+
+import parity
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+tt = pytest.importorskip("exact_inner_product_b200")
+
+
+def _noalloc(rows, inv, q, k, tau, excl, ids, scores):
+    return tt._lib.tt_score_topk_noalloc(
+        ctypes.c_void_p(rows.data_ptr()), tt._dtype(rows), rows.shape[0], rows.shape[1],
+        None if inv is None else ctypes.c_void_p(inv.data_ptr()), ctypes.c_void_p(q.data_ptr()),
+        tt._dtype(q), q.shape[0], None if excl is None else ctypes.c_void_p(excl.data_ptr()),
+        float(tau), int(k), ctypes.c_void_p(ids.data_ptr()), ctypes.c_void_p(scores.data_ptr()),
+        ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+
+CASES = [
+    ("small_batch", {"n": 150_001, "b": 40, "k": 300}),      # tensor-core scorer
+    ("stream_b1", {"n": 120_003, "k": 100}),                  # streaming scorer, fp32 query
+    ("masked_fused", {"n": 60_013, "b": 33, "k": 64}),        # raw corpus + norms, mask
+]
+
+
+@pytest.mark.parametrize("name,over", CASES, ids=[c[0] for c in CASES])
+def test_noalloc_matches_regular_entry_point(name, over):
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    w = W.workload(name, **over)
+    raw_c = W.corpus(w, "cuda")
+    raw_q = W.queries(w, "cuda")
+    excl = W.exclusion_bits(w, "cuda")
+    index, qn = parity.gpu_prepare(w, raw_c, raw_q)
+    ref_ids, ref_scores = tt.tt_score_topk(index, qn, w.k, tau=w.tau, exclude=excl)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        ids = torch.full((w.b, w.k), -7, dtype=torch.int32, device="cuda")
+        scores = torch.full((w.b, w.k), math.nan, dtype=torch.float32, device="cuda")
+        st = _noalloc(index.rows, index.inv_norm, qn, w.k, w.tau, excl, ids, scores)
+        assert st == tt.TT_OK, tt._lib.tt_last_error().decode()
+        torch.cuda.synchronize()
+        assert torch.equal(ids, ref_ids)
+        pad = torch.isinf(ref_scores)
+        assert torch.equal(pad, torch.isinf(scores))
+        assert (scores[~pad] - ref_scores[~pad]).abs().max().item() <= w.tolerance
+
+
+def test_noalloc_rejects_batches_beyond_its_array():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    rows = torch.nn.functional.normalize(torch.randn(1000, 64, device="cuda"), dim=1).to(torch.bfloat16)
+    q = torch.randn(1000, 64, device="cuda").to(torch.bfloat16)
+    ids = torch.empty((1000, 10), dtype=torch.int32, device="cuda")
+    scores = torch.empty((1000, 10), dtype=torch.float32, device="cuda")
+    st = _noalloc(rows, None, q, 10, 1.0, None, ids, scores)
+    assert st == tt.TT_ERR_UNSUPPORTED
+    assert "bytes" in tt._lib.tt_last_error().decode()
