@@ -8,8 +8,8 @@
 // HBM-bound: every row is read once with 16-byte loads and written once with
 // 16-byte (or 8-byte) stores. L lanes of a warp share one row (L = 32 for
 // rows of >= 512 bytes), each lane keeping up to 4 chunks in registers, and
-// each warp works on two row groups at a time to keep enough bytes in
-// flight. fp32 arithmetic with IEEE sqrt and division; the result is rounded
+// each warp works on two to four row groups at a time to keep enough bytes
+// in flight. fp32 arithmetic with IEEE sqrt and division; the result is rounded
 // to the output type to nearest-even.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -87,8 +87,9 @@ __device__ __forceinline__ void store_chunk<__nv_bfloat16, 8>(__nv_bfloat16* row
 }
 
 // MODE 0: out rows = v / norm (Tout). MODE 1: inv_norm[j] = 1 / norm.
-// L lanes per row, CPL 16-byte chunks per lane (d * elem <= 2048 bytes).
-template <typename Tin, typename Tout, int MODE, int L, int CPL>
+// L lanes per row, CPL 16-byte chunks per lane (d * elem <= 2048 bytes),
+// U row groups per warp in flight at once.
+template <typename Tin, typename Tout, int MODE, int L, int CPL, int U>
 __global__ void __launch_bounds__(K1_THREADS)
     k1_normalize(const Tin* in, int64_t n, int d, Tout* out,
                  float* __restrict__ inv_norm) {
@@ -100,13 +101,15 @@ __global__ void __launch_bounds__(K1_THREADS)
     const int grp = lane / L;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    const int64_t step = nwarps * (2 * ROWS_PER_GROUP);
+    const int64_t step = nwarps * (U * ROWS_PER_GROUP);
 
-    for (int64_t base = warp * (2 * ROWS_PER_GROUP); base < n; base += step) {
-        int64_t row[2] = {base + grp, base + ROWS_PER_GROUP + grp};
-        uint4 raw[2][CPL];
+    for (int64_t base = warp * (U * ROWS_PER_GROUP); base < n; base += step) {
+        int64_t row[U];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < U; ++u) row[u] = base + u * ROWS_PER_GROUP + grp;
+        uint4 raw[U][CPL];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
 #pragma unroll
             for (int i = 0; i < CPL; ++i) {
                 const int c = sub + i * L;
@@ -116,9 +119,10 @@ __global__ void __launch_bounds__(K1_THREADS)
                     raw[u][i] = make_uint4(0u, 0u, 0u, 0u);
             }
         }
-        float ss[2] = {0.f, 0.f};
+        float ss[U];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < U; ++u) {
+            ss[u] = 0.f;
 #pragma unroll
             for (int i = 0; i < CPL; ++i) {
                 float x[E];
@@ -129,11 +133,11 @@ __global__ void __launch_bounds__(K1_THREADS)
         }
 #pragma unroll
         for (int off = L / 2; off > 0; off >>= 1) {
-            ss[0] += __shfl_xor_sync(0xFFFFFFFFu, ss[0], off);
-            ss[1] += __shfl_xor_sync(0xFFFFFFFFu, ss[1], off);
+#pragma unroll
+            for (int u = 0; u < U; ++u) ss[u] += __shfl_xor_sync(0xFFFFFFFFu, ss[u], off);
         }
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < U; ++u) {
             if (row[u] >= n) continue;
             const float norm = __fsqrt_rn(fmaxf(ss[u], 1e-12f));
             if (MODE == 1) {
@@ -169,7 +173,9 @@ cudaError_t dispatch_lanes(const void* in, int64_t n, int d, void* out, cudaStre
     const int chunks = d / E;
     int L = 32;
     while (L > chunks) L >>= 1;
-    const int rows_per_block = (K1_THREADS / 32) * 2 * (32 / L);
+    const int cpl = (chunks + L - 1) / L;
+    const int unroll = (L == 32 && cpl == 1) ? 4 : 2;
+    const int rows_per_block = (K1_THREADS / 32) * unroll * (32 / L);
     int64_t blocks = (n + rows_per_block - 1) / rows_per_block;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -181,15 +187,14 @@ cudaError_t dispatch_lanes(const void* in, int64_t n, int d, void* out, cudaStre
     Tout* pout = MODE == 0 ? static_cast<Tout*>(out) : nullptr;
     float* pinv = MODE == 1 ? static_cast<float*>(out) : nullptr;
     note_launch_begin(TT_KIND_NORMALIZE, s);
-    const int cpl = (chunks + L - 1) / L;
     const dim3 g((unsigned)blocks), t(K1_THREADS);
-    if (L == 32 && cpl == 1) k1_normalize<Tin, Tout, MODE, 32, 1><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
-    else if (L == 32 && cpl == 2) k1_normalize<Tin, Tout, MODE, 32, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
-    else if (L == 32) k1_normalize<Tin, Tout, MODE, 32, 4><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
-    else if (L == 16) k1_normalize<Tin, Tout, MODE, 16, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
-    else if (L == 8) k1_normalize<Tin, Tout, MODE, 8, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
-    else if (L == 4) k1_normalize<Tin, Tout, MODE, 4, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
-    else k1_normalize<Tin, Tout, MODE, 2, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
+    if (L == 32 && cpl == 1) k1_normalize<Tin, Tout, MODE, 32, 1, 4><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
+    else if (L == 32 && cpl == 2) k1_normalize<Tin, Tout, MODE, 32, 2, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
+    else if (L == 32) k1_normalize<Tin, Tout, MODE, 32, 4, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
+    else if (L == 16) k1_normalize<Tin, Tout, MODE, 16, 2, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
+    else if (L == 8) k1_normalize<Tin, Tout, MODE, 8, 2, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
+    else if (L == 4) k1_normalize<Tin, Tout, MODE, 4, 2, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
+    else k1_normalize<Tin, Tout, MODE, 2, 2, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
     note_launch_end(TT_KIND_NORMALIZE, s);
     return cudaGetLastError();
 }

@@ -1,10 +1,12 @@
 // k_select.cu - K4: per-query selection over the candidate keys kept by a
 // scoring pass, plus the small bookkeeping kernels.
 //
-// One CTA per query. The r-th largest key is found by a most-significant-
-// digit radix select over the 64-bit keys (digits of 11/11/10/11/11/10
-// bits, a 2048-bin shared-memory histogram per digit), so its cost depends
-// only on the number of kept keys, not on how they are ordered. Keys are
+// One CTA per query; the kept keys are staged in shared memory when they fit.
+// The r-th largest key is found by a most-significant-digit radix select over
+// the 64-bit keys (digits of 11/11/10/11/11/10 bits, a 2048-bin shared-memory
+// histogram per digit) until at most 256 keys share the selected prefix;
+// those are ranked directly. Its cost depends only on the number of kept
+// keys, not on how they are ordered. Keys are
 // distinct (the low word encodes the candidate id), so exactly r keys are
 // >= the r-th largest.
 //
@@ -31,6 +33,7 @@ namespace {
 constexpr int K4_THREADS = 256;
 constexpr int K4_SORT_MAX = 2048;  // >= TT_MAX_K
 constexpr int K4_BINS = 2048;
+constexpr int K4_SMEM_KEYS = 4096;  // kept keys copied to shared memory when they fit
 
 struct K4Smem {
     uint32_t hist[K4_BINS];
@@ -39,11 +42,24 @@ struct K4Smem {
     uint64_t sorted[K4_SORT_MAX];
     uint64_t found_prefix;
     uint32_t found_remaining;
+    uint32_t found_count;
     uint32_t n_collected;
+    uint64_t result;
+    uint64_t keys[K4_SMEM_KEYS];
 };
 
+// The query's kept keys: copied to shared memory when they fit, else read in place.
+__device__ const uint64_t* stage_keys(const uint64_t* __restrict__ g, int n, K4Smem& sm) {
+    if (n > K4_SMEM_KEYS) return g;
+    for (int i = threadIdx.x; i < n; i += K4_THREADS) sm.keys[i] = g[i];
+    __syncthreads();
+    return sm.keys;
+}
+
 // r-th largest (1-based) of n distinct keys; 1 <= r <= n. Block-wide.
-__device__ uint64_t block_kth_largest(const uint64_t* __restrict__ keys, int n, int r, K4Smem& sm) {
+// Radix passes narrow the candidates to a digit prefix; once at most
+// K4_THREADS keys share the prefix they are gathered and ranked directly.
+__device__ uint64_t block_kth_largest(const uint64_t* keys, int n, int r, K4Smem& sm) {
     const int tid = threadIdx.x;
     // digits, most significant first: widths 11, 11, 10, 11, 11, 10
     uint64_t prefix = 0, mask = 0;
@@ -92,6 +108,7 @@ __device__ uint64_t block_kth_largest(const uint64_t* __restrict__ keys, int n, 
                 if (remaining <= run + c) {
                     sm.found_prefix = (uint64_t)(tid * per + i);
                     sm.found_remaining = remaining - run;
+                    sm.found_count = c;
                     break;
                 }
                 run += c;
@@ -101,7 +118,26 @@ __device__ uint64_t block_kth_largest(const uint64_t* __restrict__ keys, int n, 
         prefix |= sm.found_prefix << shift;
         mask |= (uint64_t)(nb - 1) << shift;
         remaining = sm.found_remaining;
+        const uint32_t count = sm.found_count;
         __syncthreads();
+        if (count <= (uint32_t)K4_THREADS) {
+            // gather the keys with this prefix and rank them by counting
+            if (tid == 0) sm.n_collected = 0;
+            __syncthreads();
+            for (int i = tid; i < n; i += K4_THREADS) {
+                const uint64_t key = keys[i];
+                if ((key & mask) == prefix) sm.sorted[atomicAdd(&sm.n_collected, 1u)] = key;
+            }
+            __syncthreads();
+            if (tid < (int)count) {
+                const uint64_t mine = sm.sorted[tid];
+                uint32_t above_me = 0;
+                for (uint32_t j = 0; j < count; ++j) above_me += sm.sorted[j] > mine;
+                if (above_me == remaining - 1) sm.result = mine;
+            }
+            __syncthreads();
+            return sm.result;
+        }
     }
     return prefix;
 }
@@ -109,12 +145,16 @@ __device__ uint64_t block_kth_largest(const uint64_t* __restrict__ keys, int n, 
 __global__ void __launch_bounds__(K4_THREADS)
     k4_select_threshold(const uint64_t* __restrict__ keys, uint32_t* __restrict__ count, int cap,
                         int r, uint64_t* __restrict__ theta_next, float* __restrict__ thf_next) {
-    __shared__ K4Smem sm;
+    extern __shared__ __align__(16) uint8_t k4_smem_raw[];
+    K4Smem& sm = *reinterpret_cast<K4Smem*>(k4_smem_raw);
     const int q = blockIdx.x;
     const uint32_t c = count[q];
     const int n = c < (uint32_t)cap ? (int)c : cap;
     uint64_t th = KEY_MIN;
-    if (n >= r && r > 0) th = block_kth_largest(keys + (int64_t)q * cap, n, r, sm) - 1;
+    if (n >= r && r > 0) {
+        const uint64_t* qkeys = stage_keys(keys + (int64_t)q * cap, n, sm);
+        th = block_kth_largest(qkeys, n, r, sm) - 1;
+    }
     __syncthreads();
     if (threadIdx.x == 0) {
         theta_next[q] = th;
@@ -128,14 +168,15 @@ __global__ void __launch_bounds__(K4_THREADS)
                     uint64_t* __restrict__ theta, float* __restrict__ thf, int32_t* __restrict__ status,
                     int* __restrict__ flags, int repair, int32_t* __restrict__ out_ids,
                     float* __restrict__ out_scores) {
-    __shared__ K4Smem sm;
+    extern __shared__ __align__(16) uint8_t k4_smem_raw[];
+    K4Smem& sm = *reinterpret_cast<K4Smem*>(k4_smem_raw);
     const int q = blockIdx.x;
     const int tid = threadIdx.x;
     if (repair && status[q] == 0) return;  // block-uniform
     const uint32_t c = count[q];
     const int n = c < (uint32_t)cap ? (int)c : cap;
     const uint64_t th = theta[q];
-    const uint64_t* qkeys = keys + (int64_t)q * cap;
+    const uint64_t* qkeys = stage_keys(keys + (int64_t)q * cap, n, sm);
     const bool exact = (c <= (uint32_t)cap) && (c >= (uint32_t)k || th == KEY_MIN);
     if (exact) {
         const int r = n < k ? n : k;
@@ -250,8 +291,10 @@ cudaError_t launch_init(uint32_t* count, uint64_t* theta, float* thf, uint64_t t
 cudaError_t launch_select_threshold(const uint64_t* keys, uint32_t* count, int cap, int b, int r,
                                     uint64_t* theta_next, float* thf_next, cudaStream_t s) {
     if (b == 0) return cudaSuccess;
+    const int smem = (int)sizeof(K4Smem);
+    cudaFuncSetAttribute(k4_select_threshold, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     note_launch_begin(TT_KIND_SELECT, s);
-    k4_select_threshold<<<b, K4_THREADS, 0, s>>>(keys, count, cap, r, theta_next, thf_next);
+    k4_select_threshold<<<b, K4_THREADS, smem, s>>>(keys, count, cap, r, theta_next, thf_next);
     note_launch_end(TT_KIND_SELECT, s);
     return cudaGetLastError();
 }
@@ -260,9 +303,11 @@ cudaError_t launch_select_final(const uint64_t* keys, uint32_t* count, int cap, 
                                 uint64_t* theta, float* thf, int32_t* status, int* flags,
                                 int repair, int32_t* out_ids, float* out_scores, cudaStream_t s) {
     if (b == 0) return cudaSuccess;
+    const int smem = (int)sizeof(K4Smem);
+    cudaFuncSetAttribute(k4_select_final, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     note_launch_begin(TT_KIND_SELECT, s);
-    k4_select_final<<<b, K4_THREADS, 0, s>>>(keys, count, cap, k, theta, thf, status, flags, repair,
-                                             out_ids, out_scores);
+    k4_select_final<<<b, K4_THREADS, smem, s>>>(keys, count, cap, k, theta, thf, status, flags, repair,
+                                                out_ids, out_scores);
     note_launch_end(TT_KIND_SELECT, s);
     return cudaGetLastError();
 }

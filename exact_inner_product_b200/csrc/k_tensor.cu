@@ -49,6 +49,8 @@ constexpr int K3_ACC_COLS = 256;
 constexpr int K3_MAX_NQ = 256;
 constexpr int K3_SMEM_BUDGET = 227 * 1024;
 
+constexpr int K3_WARP_COLS = K3_MAX_NQ / 2;  // columns one epilogue warp covers at most
+
 struct K3Ctl {
     uint64_t full[K3_MAX_STAGES];
     uint64_t empty[K3_MAX_STAGES];
@@ -57,11 +59,13 @@ struct K3Ctl {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
+    // per epilogue warp: fast-path thresholds of its columns for the current unit
+    float th_fast[K3_EPI_WARPS][K3_WARP_COLS];
 };
 
 struct K3Params {
     PassArgs a;
-    int nq;          // queries per tile (multiple of 16, <= 256)
+    int nq;          // queries per tile (multiple of 32, <= 256)
     int q_tiles;     // ceil(b / nq)
     int kchunks;     // ceil(d / 64)
     int stages;
@@ -69,6 +73,28 @@ struct K3Params {
     int chunks;      // corpus chunks (units = q_tiles * chunks)
     uint32_t idesc;
 };
+
+struct Cols32 {
+    float x[32];
+};
+
+// x[i] for a run-time i, from registers (no local memory): pick the group of
+// eight first, then halve; few values are live at any time.
+__device__ __forceinline__ float select32(const Cols32& c, int i) {
+    const int g = i >> 3;
+    float a[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const float lo = (g & 1) ? c.x[8 + k] : c.x[k];
+        const float hi = (g & 1) ? c.x[24 + k] : c.x[16 + k];
+        a[k] = (g & 2) ? hi : lo;
+    }
+    const int j = i & 7;
+    const float b0 = (j & 4) ? a[4] : a[0], b1 = (j & 4) ? a[5] : a[1];
+    const float b2 = (j & 4) ? a[6] : a[2], b3 = (j & 4) ? a[7] : a[3];
+    const float c0 = (j & 2) ? b2 : b0, c1 = (j & 2) ? b3 : b1;
+    return (j & 1) ? c1 : c0;
+}
 
 __device__ __forceinline__ void unit_range(const K3Params& p, int u, int* qt, int64_t* t0,
                                            int64_t* t1) {
@@ -206,22 +232,42 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
         }
     } else {
         // ------------------------------ epilogue ------------------------------
+        // Warp w reads TMEM lanes 32*(w%4).. (its 32 corpus rows) and the
+        // 32-column chunks half, half+2, half+4, half+6 of the query tile.
         const int ew = warp - 2;
-        const int quarter = warp & 3;        // TMEM lane quarter this warp may access
-        const int half = ew >> 2;            // which interleaved half of the 32-column chunks
+        const int quarter = warp & 3;
+        const int half = ew >> 2;
         const int row_in_tile = quarter * 32 + lane;
-        const int nchunk32 = (p.nq + 31) / 32;
+        const int nchunk32 = p.nq / 32;  // nq is a multiple of 32
         const PassArgs& a = p.a;
+        // With no per-row norms the score scale c is the same for every row,
+        // and the fast test compares the raw accumulator with th / c, lowered
+        // by a relative 2^-20 so that fl(v * c) >= th implies v >= th_fast
+        // (the exact test follows on the rare hits).
+        const bool uniform_c = a.inv_norm == nullptr;
+        float* th_fast = ctl->th_fast[ew];
         uint32_t tc = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
             int qt;
             int64_t t0, t1;
             unit_range(p, u, &qt, &t0, &t1);
-            // Thresholds of this unit's queries (padded past b with +inf /
-            // KEY_MAX, so out-of-range columns never pass).
             const float* thf_unit = a.thf + (int64_t)qt * p.nq;
             const uint64_t* th_unit = a.theta + (int64_t)qt * p.nq;
+            __syncwarp();
+            for (int j = lane; j < K3_WARP_COLS; j += 32) {
+                const int ch = half + 2 * (j >> 5);
+                float t = INFINITY;
+                if (ch < nchunk32) {
+                    t = __ldg(thf_unit + ch * 32 + (j & 31));
+                    if (uniform_c && t != INFINITY && t != -INFINITY) {
+                        const float r = t / a.inv_tau;
+                        t = r - fabsf(r) * 0x1p-20f - 1e-30f;
+                    }
+                }
+                th_fast[j] = t;
+            }
+            __syncwarp();
             for (int64_t t = t0; t < t1; ++t, ++tc) {
                 const int buf = tc & 1;
                 // per-row data, fetched before waiting for the accumulator
@@ -239,48 +285,74 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                for (int ch = half; ch < nchunk32; ch += 2) {
-                    const int col0 = ch * 32;
-                    float v[32];
-                    tmem_ld_32cols(tmem_base + ((uint32_t)(quarter * 32) << 16) +
-                                       (uint32_t)(buf * K3_ACC_COLS + col0),
-                                   v);
+                const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * K3_ACC_COLS);
+                // this warp's chunks (up to 4 x 32 columns), two in flight per wait
+                // (four would not fit the 168 registers a thread has here); a warp
+                // whose half of the tile is empty releases the accumulator at once
+                if (half >= nchunk32) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ctl->tempty[buf]);
+                }
+#pragma unroll
+                for (int pair = 0; pair < 2; ++pair) {
+                    const int cja = 2 * pair, cjb = 2 * pair + 1;
+                    if (half + 2 * cja >= nchunk32) break;  // warp-uniform
+                    const bool has_b = half + 2 * cjb < nchunk32;
+                    Cols32 v[2];
+                    tmem_ld_32cols(tbase + (uint32_t)((half + 2 * cja) * 32), v[0].x);
+                    if (has_b) tmem_ld_32cols(tbase + (uint32_t)((half + 2 * cjb) * 32), v[1].x);
                     tmem_ld_wait();
-                    bool any = false;
-                    const float4* th4 = reinterpret_cast<const float4*>(thf_unit + col0);
-#pragma unroll
-                    for (int i4 = 0; i4 < 8; ++i4) {
-                            const float4 th = __ldg(th4 + i4);
-                        any |= v[4 * i4 + 0] * c >= th.x;
-                        any |= v[4 * i4 + 1] * c >= th.y;
-                        any |= v[4 * i4 + 2] * c >= th.z;
-                        any |= v[4 * i4 + 3] * c >= th.w;
+                    const bool last = pair == 1 || half + 2 * (cjb + 1) >= nchunk32;
+                    if (last) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&ctl->tempty[buf]);  // values are in registers now
                     }
-                    any = any && row_ok;
-                    if (__any_sync(0xFFFFFFFFu, any)) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const float sc = v[i] * c;
-                            const uint64_t key = make_key(sc, (uint32_t)id);
-                            const bool keep = row_ok && key > __ldg(th_unit + col0 + i);
-                            const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, keep);
-                            if (ballot) {
-                                const int q = qt * p.nq + col0 + i;
-                                const int leader = __ffs(ballot) - 1;
-                                uint32_t base = 0;
-                                if (lane == leader) base = atomicAdd(a.count + q, (uint32_t)__popc(ballot));
-                                base = __shfl_sync(0xFFFFFFFFu, base, leader);
-                                if (keep) {
-                                    const uint32_t slot = base + __popc(ballot & lanemask_lt());
+                    for (int h = 0; h < 2; ++h) {
+                        const int cj = cja + h;
+                        if (h == 1 && !has_b) break;
+                        const float4* t4 = reinterpret_cast<const float4*>(th_fast + cj * 32);
+                        // four independent or-chains keep the compare latency short
+                        bool h0 = false, h1 = false, h2 = false, h3 = false;
+#pragma unroll
+                        for (int i4 = 0; i4 < 8; ++i4) {
+                            const float4 tf = t4[i4];
+                            if (uniform_c) {
+                                h0 |= v[h].x[4 * i4 + 0] >= tf.x;
+                                h1 |= v[h].x[4 * i4 + 1] >= tf.y;
+                                h2 |= v[h].x[4 * i4 + 2] >= tf.z;
+                                h3 |= v[h].x[4 * i4 + 3] >= tf.w;
+                            } else {
+                                h0 |= v[h].x[4 * i4 + 0] * c >= tf.x;
+                                h1 |= v[h].x[4 * i4 + 1] * c >= tf.y;
+                                h2 |= v[h].x[4 * i4 + 2] * c >= tf.z;
+                                h3 |= v[h].x[4 * i4 + 3] * c >= tf.w;
+                            }
+                        }
+                        // Rare: only the lanes concerned find the passing columns
+                        // and append those whose exact key beats the threshold key.
+                        if ((h0 | h1 | h2 | h3) && row_ok) {
+                            const int col0 = (half + 2 * cj) * 32;
+                            const float cf = uniform_c ? 1.0f : c;
+                            uint32_t m = 0;
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                m |= (v[h].x[i] * cf >= th_fast[cj * 32 + i]) ? (1u << i) : 0u;
+                            while (m) {
+                                const int i = __ffs(m) - 1;
+                                m &= m - 1;
+                                const uint64_t key = make_key(select32(v[h], i) * c, (uint32_t)id);
+                                if (key > __ldg(th_unit + col0 + i)) {
+                                    const int q = qt * p.nq + col0 + i;
+                                    const uint32_t slot = atomicAdd(a.count + q, 1u);
                                     if (slot < (uint32_t)a.cap) a.keys[(int64_t)q * a.cap + slot] = key;
                                 }
                             }
                         }
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&ctl->tempty[buf]);
             }
         }
         if (!ok) {
@@ -310,7 +382,7 @@ int tensor_pass_smem_bytes(int d, int nq) {
 }
 
 int tensor_pass_max_nq(int d) {
-    for (int nq = K3_MAX_NQ; nq >= 16; nq -= 16)
+    for (int nq = K3_MAX_NQ; nq >= 32; nq -= 32)
         if (tensor_pass_smem_bytes(d, nq) > 0 && tensor_pass_smem_bytes(d, nq) <= K3_SMEM_BUDGET &&
             ((d + K3_KC - 1) / K3_KC) * nq * 128 <= 128 * 1024)
             return nq;

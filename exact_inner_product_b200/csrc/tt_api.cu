@@ -154,27 +154,6 @@ static bool encode_2d(CUtensorMap* tm, CUtensorMapDataType dt, const void* base,
     return true;
 }
 
-bool stream_pass_tensor_map(const PassArgs& a, CUtensorMap* tm, int* nbox, int* row_pitch,
-                            bool* sw) {
-    const int elem = a.dtype == TT_F32 ? 4 : 2;
-    const int row_bytes = a.d * elem;
-    const CUtensorMapDataType dt =
-        a.dtype == TT_F32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-    const uint64_t pitch = (uint64_t)a.stride * (uint64_t)row_bytes;
-    if (row_bytes >= 128) {
-        *sw = true;
-        *nbox = (row_bytes + 127) / 128;
-        *row_pitch = *nbox * 128;
-        return encode_2d(tm, dt, a.rows, (uint64_t)a.d, (uint64_t)a.n_rows, pitch, 128 / elem, 32,
-                         CU_TENSOR_MAP_SWIZZLE_128B);
-    }
-    *sw = false;
-    *nbox = 1;
-    *row_pitch = row_bytes;
-    return encode_2d(tm, dt, a.rows, (uint64_t)a.d, (uint64_t)a.n_rows, pitch, (uint32_t)a.d, 32,
-                     CU_TENSOR_MAP_SWIZZLE_NONE);
-}
-
 bool bf16_tile_tensor_map(const void* base, int64_t rows, int d, int64_t row_pitch_elems,
                           int box_rows, CUtensorMap* tm) {
     return encode_2d(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, (uint64_t)d, (uint64_t)rows,
@@ -302,6 +281,64 @@ struct Scratch {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Scratch blocks released by tt_free are kept here (per device) and handed
+// to later handles, so that short-lived handles do not cudaMalloc/cudaFree on
+// every call (cudaFree waits for the whole device). Blocks stay with the
+// process until it exits.
+struct PooledBlock {
+    int device;
+    void* ptr;
+    size_t bytes;
+};
+static std::mutex g_pool_mu;
+static std::vector<PooledBlock> g_pool;
+
+static void* pool_take(int device, size_t need, size_t* got) {
+    std::lock_guard<std::mutex> lock(g_pool_mu);
+    int best = -1;
+    for (int i = 0; i < (int)g_pool.size(); ++i)
+        if (g_pool[i].device == device && g_pool[i].bytes >= need &&
+            (best < 0 || g_pool[i].bytes < g_pool[best].bytes))
+            best = i;
+    if (best < 0) return nullptr;
+    void* p = g_pool[best].ptr;
+    *got = g_pool[best].bytes;
+    g_pool.erase(g_pool.begin() + best);
+    return p;
+}
+
+static void pool_give(int device, void* ptr, size_t bytes) {
+    if (!ptr) return;
+    std::lock_guard<std::mutex> lock(g_pool_mu);
+    g_pool.push_back({device, ptr, bytes});
+}
+
+// Pinned host words for reading back the exactness flags, reused the same way.
+static std::vector<int*> g_pinned_pool;
+
+static int* pinned_take() {
+    {
+        std::lock_guard<std::mutex> lock(g_pool_mu);
+        if (!g_pinned_pool.empty()) {
+            int* p = g_pinned_pool.back();
+            g_pinned_pool.pop_back();
+            return p;
+        }
+    }
+    int* p = nullptr;
+    if (cudaMallocHost(&p, 2 * sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    return p;
+}
+
+static void pinned_give(int* p) {
+    if (!p) return;
+    std::lock_guard<std::mutex> lock(g_pool_mu);
+    g_pinned_pool.push_back(p);
+}
+
 static tt_status get_scratch(tt_index* ix, int b, int b_pad, int cap, int d, bool need_qcast,
                              Scratch* out) {
     size_t off = 0;
@@ -321,18 +358,23 @@ static tt_status get_scratch(tt_index* ix, int b, int b_pad, int cap, int d, boo
     off = align_up(off + (need_qcast ? (size_t)b * d * 2 : 0), 256);
     if (off > ix->scratch_bytes) {
         if (ix->scratch) {
-            cudaFree(ix->scratch);
+            // the old block may still be read by work queued on the stream
+            pool_give(ix->device, ix->scratch, ix->scratch_bytes);
             ix->scratch = nullptr;
             ix->scratch_bytes = 0;
         }
-        const size_t want = off + off / 4;
-        cudaError_t e = cudaMalloc(&ix->scratch, want);
-        if (e != cudaSuccess) {
-            cudaGetLastError();
-            ix->scratch = nullptr;
-            return cuda_fail(e, "scratch allocation");
+        size_t got = 0;
+        void* p = pool_take(ix->device, off, &got);
+        if (!p) {
+            got = off + off / 4;
+            cudaError_t e = cudaMalloc(&p, got);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                return cuda_fail(e, "scratch allocation");
+            }
         }
-        ix->scratch_bytes = want;
+        ix->scratch = p;
+        ix->scratch_bytes = got;
     }
     uint8_t* base = static_cast<uint8_t*>(ix->scratch);
     out->keys = reinterpret_cast<uint64_t*>(base + o_keys);
@@ -343,11 +385,10 @@ static tt_status get_scratch(tt_index* ix, int b, int b_pad, int cap, int d, boo
     out->flags = reinterpret_cast<int*>(base + o_flags);
     out->qcast = need_qcast ? reinterpret_cast<__nv_bfloat16*>(base + o_q) : nullptr;
     if (!ix->h_flags) {
-        cudaError_t e = cudaMallocHost(&ix->h_flags, 2 * sizeof(int));
-        if (e != cudaSuccess) {
-            cudaGetLastError();
-            ix->h_flags = nullptr;
-            return cuda_fail(e, "pinned flag allocation");
+        ix->h_flags = pinned_take();
+        if (!ix->h_flags) {
+            snprintf(g_last_error, sizeof g_last_error, "pinned flag allocation failed");
+            return TT_ERR_NO_MEMORY;
         }
     }
     return TT_OK;
@@ -549,8 +590,8 @@ tt_status tt_index_wrap(const void* rows, tt_dtype dtype, int64_t n, int32_t d,
 
 void tt_free(tt_index* index) {
     if (!index) return;
-    if (index->scratch) cudaFree(index->scratch);
-    if (index->h_flags) cudaFreeHost(index->h_flags);
+    pool_give(index->device, index->scratch, index->scratch_bytes);
+    pinned_give(index->h_flags);
     delete index;
 }
 
@@ -626,7 +667,7 @@ tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtyp
         const int max_nq = tensor_pass_max_nq(index->d);
         q_tiles = (b + max_nq - 1) / max_nq;
         nq = (b + q_tiles - 1) / q_tiles;
-        nq = (nq + 15) / 16 * 16;
+        nq = (nq + 31) / 32 * 32;  // whole 32-column chunks: no chunk reads past the tile
         if (nq > max_nq) nq = max_nq;
     }
     const int b_pad = (path == 2 ? q_tiles * nq : b) + 64;

@@ -70,11 +70,6 @@ cudaError_t launch_prepare_repair(uint64_t* theta, float* thf, const int32_t* st
                                   int* flags, cudaStream_t s);
 
 // Tensor maps (built on the host through the driver entry point).
-// Streaming pass: rows of the level as a 2-D tensor {d, n_rows} with row
-// pitch stride*d*elem; 32-row boxes of 128 swizzled bytes (rows >= 128 B) or
-// of the whole unswizzled row.
-bool stream_pass_tensor_map(const PassArgs& a, CUtensorMap* tm, int* nbox, int* row_pitch,
-                            bool* sw);
 // Tensor-core pass: bf16 boxes of 64 elements x box_rows rows, 128-byte swizzle.
 bool bf16_tile_tensor_map(const void* base, int64_t rows, int d, int64_t row_pitch_elems,
                           int box_rows, CUtensorMap* tm);

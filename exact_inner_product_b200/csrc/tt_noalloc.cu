@@ -120,7 +120,7 @@ tt_status tt_score_topk_noalloc(const void* rows, tt_dtype dtype, int64_t n, int
     if (path == 2) {
         const int max_nq = tensor_pass_max_nq(d);
         q_tiles = (b + max_nq - 1) / max_nq;
-        nq = ((b + q_tiles - 1) / q_tiles + 15) / 16 * 16;
+        nq = ((b + q_tiles - 1) / q_tiles + 31) / 32 * 32;  // whole 32-column chunks
         if (nq > max_nq) nq = max_nq;
     }
     const int b_pad = (path == 2 ? q_tiles * nq : b) + 64;

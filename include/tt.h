@@ -190,8 +190,10 @@ TT_API tt_status tt_last_stats(const tt_index* index, tt_stats* out);
 TT_API tt_status tt_plan(int64_t n, int32_t k, const tt_options* options, int32_t* levels, int64_t* rows,
                   int64_t* strides, int32_t* ranks, int32_t* cap);
 
-/* Release a handle and its scratch memory. NULL is a no-op. Must not be
- * called while work using the handle is still running on a stream. */
+/* Release a handle. Its scratch memory returns to a per-device pool that
+ * later handles reuse (it is not returned to CUDA before the process exits).
+ * NULL is a no-op. Must not be called while work using the handle is still
+ * running on a stream. */
 TT_API void tt_free(tt_index* index);
 
 /*
