@@ -210,6 +210,7 @@ static int sm_count_current() {
 // ---------------------------------------------------------------------------
 constexpr int STRIDE_RATIO = 64;
 constexpr int DEFAULT_CAP = 16384;
+constexpr int MAX_DEEPEST_ROWS = 4096;  // the deepest level keeps every key
 constexpr int MIN_RANK = 32;
 constexpr int MAX_LEVELS = 4;
 constexpr int MAX_RESCANS = 64;
@@ -241,7 +242,8 @@ static tt_status make_plan(int64_t n, int32_t k, const tt_options* opt, Plan* p)
             --L;
         }
     } else {
-        while ((n + s - 1) / s > cap && L < MAX_LEVELS - 1) {
+        const int64_t deepest = cap < MAX_DEEPEST_ROWS ? cap : MAX_DEEPEST_ROWS;
+        while ((n + s - 1) / s > deepest && L < MAX_LEVELS - 1) {
             s *= STRIDE_RATIO;
             ++L;
         }

@@ -15,7 +15,9 @@ Comparison rule (tol = the workload's score tolerance), per query:
  4. at every rank whose neighbouring oracle gaps both exceed tol, the id
     equals the oracle's id at that rank;
  5. every returned id has s_oracle(j) >= s_(k) - tol;
- 6. where the GPU's own scores tie exactly, ids ascend.
+ 6. where the GPU's own scores tie exactly, ids ascend;
+ 7. every oracle top-k member whose score exceeds the k-th score by more
+    than tol is returned (it cannot be displaced by rounding).
 """
 from __future__ import annotations
 
@@ -118,6 +120,10 @@ def compare(gpu_ids: np.ndarray, gpu_scores: np.ndarray, side: OracleSide, k: in
             continue
         kth = os_[nv - 1]
         assert (so >= kth - tol).all(), "a returned candidate is not near the top-k"
+        sure = oi[:nv][os_[:nv] > kth + tol]
+        missing = set(sure.tolist()) - set(vid.tolist())
+        assert not missing, (r_i, "oracle top-k members missing", sorted(missing)[:5])
+        stats["sure_checked"] = stats.get("sure_checked", 0) + len(sure)
         nxt = os_[nv] if nv < len(os_) else -math.inf
         if kth - nxt > tol:
             assert set(vid.tolist()) == set(oi[:nv].tolist()), (r_i, "top-k set differs")

@@ -118,7 +118,7 @@ def test_plan_levels():
     for n, k in ((400, 10), (10 ** 6, 100), (10 ** 7, 500), (5 * 10 ** 7, 1000), (2 * 10 ** 7, 256),
                  (2 ** 31 - 1, 2048), (1, 1), (0, 7)):
         p = tt.tt_plan(n, k)
-        assert p["rows"][-1] <= p["cap"] or p["levels"] == 4
+        assert p["rows"][-1] <= 4096 or p["levels"] == 4
         assert p["rows"][0] == n
         for i, (r, s) in enumerate(zip(p["rows"], p["strides"])):
             assert s == 64 ** i
@@ -130,12 +130,13 @@ def test_plan_levels():
             assert p["ranks"][i] * 64 >= 3 * need
             assert p["ranks"][i] * 64 <= p["cap"] // 2
     assert tt.tt_plan(400, 10)["levels"] == 1
-    assert tt.tt_plan(10 ** 6, 100) == {"levels": 2, "rows": [10 ** 6, 15625], "strides": [1, 64],
-                                        "ranks": [100, 32], "cap": 16384}
-    assert tt.tt_plan(5 * 10 ** 7, 1000)["ranks"] == [1000, 47, 32]
+    assert tt.tt_plan(10 ** 6, 100) == {"levels": 3, "rows": [10 ** 6, 15625, 245], "strides": [1, 64, 4096],
+                                        "ranks": [100, 32, 32], "cap": 16384}
+    assert tt.tt_plan(5 * 10 ** 7, 1000)["ranks"] == [1000, 47, 32, 32]
+    assert tt.tt_plan(4096, 10)["levels"] == 1 and tt.tt_plan(4097, 10)["levels"] == 2
     assert tt.tt_plan(10 ** 6, 100, force_levels=1)["levels"] == 1
     assert tt.tt_plan(10 ** 6, 100, force_levels=3)["levels"] == 3
-    assert tt.tt_plan(10 ** 6, 100, rank_scale_pct=50)["ranks"] == [100, 16]
+    assert tt.tt_plan(10 ** 6, 100, rank_scale_pct=50)["ranks"] == [100, 16, 16]
     with pytest.raises(tt.TTError):
         tt.tt_plan(10, 0)
     with pytest.raises(tt.TTError):
