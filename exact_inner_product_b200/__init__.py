@@ -42,7 +42,7 @@ TT_NUM_KINDS = len(KIND_NAMES)
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
-        f"{LIB_PATH} is missing: build it with `python -m exact_inner_product_b200.build` "
+        f"{LIB_PATH} is missing: build it with `python exact_inner_product_b200/build.py` "
         "(there is no CPU fallback)")
 
 
@@ -86,6 +86,8 @@ _sig("tt_free", None, [_vp])
 _sig("tt_launch_count", _i64, [])
 _sig("tt_profile_begin", ctypes.c_int, [])
 _sig("tt_profile_end", ctypes.c_int, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_i64)])
+_sig("tt_profile_launches", ctypes.c_int, [ctypes.POINTER(_i32), ctypes.POINTER(ctypes.c_double), _i32,
+                                           ctypes.POINTER(_i32)])
 _sig("tt_status_string", ctypes.c_char_p, [ctypes.c_int])
 _sig("tt_last_error", ctypes.c_char_p, [])
 _sig("tt_version", ctypes.c_char_p, [])
@@ -93,7 +95,7 @@ _sig("tt_version", ctypes.c_char_p, [])
 EXPORTED = ("tt_normalize_candidates", "tt_index_wrap", "tt_score_topk", "tt_score_topk_ex",
             "tt_score_topk_noalloc",
             "tt_last_stats", "tt_plan", "tt_free", "tt_launch_count", "tt_profile_begin",
-            "tt_profile_end", "tt_status_string", "tt_last_error", "tt_version")
+            "tt_profile_end", "tt_profile_launches", "tt_status_string", "tt_last_error", "tt_version")
 
 
 class TTError(RuntimeError):
@@ -284,6 +286,15 @@ def tt_profile_end() -> dict:
     cnt = (_i64 * TT_NUM_KINDS)()
     _check(_lib.tt_profile_end(ms, cnt), "tt_profile_end")
     return {name: {"ms": ms[i], "launches": cnt[i]} for i, name in enumerate(KIND_NAMES)}
+
+
+def tt_profile_launches(max_records: int = 4096) -> list:
+    """Launches recorded since tt_profile_begin: [(kind name, device ms), ...]."""
+    kinds = (_i32 * max_records)()
+    ms = (ctypes.c_double * max_records)()
+    n = _i32()
+    _check(_lib.tt_profile_launches(kinds, ms, max_records, ctypes.byref(n)), "tt_profile_launches")
+    return [(KIND_NAMES[kinds[i]], ms[i]) for i in range(n.value)]
 
 
 def tt_version() -> str:

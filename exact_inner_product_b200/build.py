@@ -1,6 +1,6 @@
 """Build libtt.so (the CUDA library behind include/tt.h) in place, for sm_100a.
 
-    python -m exact_inner_product_b200.build
+    python exact_inner_product_b200/build.py   (or __graft_entry__.build())
 
 Compiles every .cu file under csrc/ with nvcc into one shared library next to
 this file; the CUDA runtime is linked statically so the library only needs

@@ -480,6 +480,23 @@ tt_status tt_profile_begin(void) {
     return TT_OK;
 }
 
+tt_status tt_profile_launches(int32_t* kinds, double* ms, int32_t max_records, int32_t* n_records) {
+    std::lock_guard<std::mutex> lock(g_prof_mu);
+    int32_t n = 0;
+    for (auto& r : g_prof_recs) {
+        if (n >= max_records) break;
+        float t = 0.f;
+        cudaError_t e = cudaEventSynchronize(r.stop);
+        if (e == cudaSuccess) e = cudaEventElapsedTime(&t, r.start, r.stop);
+        if (e != cudaSuccess) return cuda_fail(e, "profile event");
+        if (kinds) kinds[n] = r.kind;
+        if (ms) ms[n] = t;
+        ++n;
+    }
+    if (n_records) *n_records = n;
+    return TT_OK;
+}
+
 tt_status tt_profile_end(double* ms_per_kind, int64_t* launches_per_kind) {
     std::lock_guard<std::mutex> lock(g_prof_mu);
     g_prof_on = false;

@@ -239,6 +239,18 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int m, int n) {
            | ((uint32_t)(m >> 4) << 24);      // M / 16
 }
 
+// Register rebalancing between warp groups (all four warps of a group must
+// execute it). The launch gives every thread the same budget; a group that
+// needs few registers gives some back so that another may take more.
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ uint32_t lanemask_lt() {
     uint32_t m;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));

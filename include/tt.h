@@ -255,6 +255,12 @@ TT_API tt_status tt_profile_begin(void);
  * Either array may be NULL; each has TT_NUM_KINDS entries. */
 TT_API tt_status tt_profile_end(double* ms_per_kind, int64_t* launches_per_kind);
 
+/* While recording (between tt_profile_begin and tt_profile_end): the launches
+ * recorded so far, in order, as (kind, device ms), waiting for their events.
+ * At most max_records are written; *n_records receives the number written. */
+TT_API tt_status tt_profile_launches(int32_t* kinds, double* ms, int32_t max_records,
+                                     int32_t* n_records);
+
 /* Human-readable name of a status, and the last CUDA error text seen by the
  * calling thread (empty if none). */
 TT_API const char* tt_status_string(tt_status status);
