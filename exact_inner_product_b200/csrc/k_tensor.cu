@@ -59,8 +59,10 @@ struct K3Ctl {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
-    // per epilogue warp: fast-path thresholds of its columns for the current unit
+    // per epilogue warp: fast-path thresholds and exact threshold keys of its
+    // columns for the current unit
     float th_fast[K3_EPI_WARPS][K3_WARP_COLS];
+    uint64_t th_key[K3_EPI_WARPS][K3_WARP_COLS];
 };
 
 struct K3Params {
@@ -246,6 +248,7 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
         // (the exact test follows on the rare hits).
         const bool uniform_c = a.inv_norm == nullptr;
         float* th_fast = ctl->th_fast[ew];
+        uint64_t* th_key = ctl->th_key[ew];
         uint32_t tc = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
@@ -258,6 +261,7 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
             for (int j = lane; j < K3_WARP_COLS; j += 32) {
                 const int ch = half + 2 * (j >> 5);
                 float t = INFINITY;
+                th_key[j] = ch < nchunk32 ? __ldg(th_unit + ch * 32 + (j & 31)) : KEY_MAX;
                 if (ch < nchunk32) {
                     t = __ldg(thf_unit + ch * 32 + (j & 31));
                     if (uniform_c && t != INFINITY && t != -INFINITY) {
@@ -344,7 +348,7 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
                                 const int i = __ffs(m) - 1;
                                 m &= m - 1;
                                 const uint64_t key = make_key(select32(v[h], i) * c, (uint32_t)id);
-                                if (key > __ldg(th_unit + col0 + i)) {
+                                if (key > th_key[cj * 32 + i]) {
                                     const int q = qt * p.nq + col0 + i;
                                     const uint32_t slot = atomicAdd(a.count + q, 1u);
                                     if (slot < (uint32_t)a.cap) a.keys[(int64_t)q * a.cap + slot] = key;
