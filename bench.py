@@ -41,6 +41,7 @@ METRIC = "query-candidate scores/sec (exact top-k)"
 UNIT = "scores/s"
 DEFAULT_WORKLOAD = "stream_b1"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PATH_NAMES = {1: "streaming", 2: "tensor-core", 3: "tensor-core (SM pairs)"}
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per unit of work
@@ -287,7 +288,8 @@ def run_ours(args, world, rank, local):
             e1.record(stream)
             ev_k1.append((e0, e1))
         tt.tt_normalize_candidates(raw_q, qn, tt.TT_NORM_STORE, make_index=False)
-        tt.tt_score_topk(index, qn, w.k, tau=w.tau, exclude=excl, out_ids=out_ids, out_scores=out_scores)
+        tt.tt_score_topk(index, qn, w.k, tau=w.tau, exclude=excl, out_ids=out_ids, out_scores=out_scores,
+                         path=args.path)
         return index
 
     for _ in range(args.warmup):
@@ -326,7 +328,8 @@ def run_ours(args, world, rank, local):
     peaks, peak_src = load_peaks()
     work = work_model(w, plan)
     k1_ms = sum(a.elapsed_time(b) for a, b in ev_k1) / max(1, len(ev_k1))
-    score_kind = "tensor" if stats["path"] == 2 else "stream"
+    score_kind = "tensor" if stats["path"] >= 2 else "stream"
+    score_kernel = {1: "k2_stream", 2: "k3_tensor", 3: "k3_pair"}[stats["path"]]
     score_ms = prof[score_kind]["ms"] / args.steps
     if k1_ms >= score_ms:
         dom = {"kernel": "k1_normalize (corpus)", "bound": "hbm", "ms": k1_ms, "bytes": work["k1_bytes"],
@@ -334,8 +337,8 @@ def run_ours(args, world, rank, local):
     else:
         t_flops = work["score_flops"] / (peaks["bf16_tflops_sustained"] * 1e12)
         t_bytes = work["score_bytes"] / (peaks["hbm_gbs"] * 1e9)
-        bound = "tensor" if (stats["path"] == 2 and t_flops > t_bytes) else "hbm"
-        dom = {"kernel": f"k{2 if score_kind == 'stream' else 3}_{score_kind} (all levels)", "bound": bound,
+        bound = "tensor" if (stats["path"] >= 2 and t_flops > t_bytes) else "hbm"
+        dom = {"kernel": f"{score_kernel} (all levels)", "bound": bound,
                "ms": score_ms, "bytes": work["score_bytes"], "flops": work["score_flops"],
                "launches_per_step": prof[score_kind]["launches"] / args.steps}
     if dom["bound"] == "hbm":
@@ -349,8 +352,7 @@ def run_ours(args, world, rank, local):
     if dom["kernel"].startswith("k1"):
         roof["traffic"] = recorded_traffic("k1_normalize", w.name, w.n)
     else:
-        roof["traffic"] = recorded_traffic("k3_tensor" if score_kind == "tensor" else "k2_stream", w.name,
-                                           work["rows_scanned"])
+        roof["traffic"] = recorded_traffic(score_kernel, w.name, work["rows_scanned"])
     roof["kernel"] = dom["kernel"]
     roof["peak_source"] = peak_src + (" (sustained bf16)" if roof["bound"] == "tensor" else " (copy)")
     roof["kernel_ms"] = round(dom["ms"], 5)
@@ -393,7 +395,7 @@ def run_ours(args, world, rank, local):
                    "corpus_raw": w.raw_dtype, "corpus_store": w.store, "queries": w.query_dtype,
                    "mask_rate": w.mask_rate, "l2": "inputs larger than L2 (raw corpus "
                    f"{w.n * w.d * elem_bytes(w.raw_dtype) / 1e6:.0f} MB > 126 MB)",
-                   "path": "tensor-core" if stats["path"] == 2 else "streaming", "levels": plan["rows"],
+                   "path": PATH_NAMES[stats["path"]], "levels": plan["rows"],
                    "parallelism": f"replicas x{world}"},
         "topk_queries_per_s": qps,
         "roofline": roof,
@@ -448,6 +450,8 @@ def main():
     ap.add_argument("--n", type=int, default=0, help="override the workload's corpus size")
     ap.add_argument("--b", type=int, default=0, help="override the workload's batch size")
     ap.add_argument("--k", type=int, default=0, help="override the workload's k")
+    ap.add_argument("--path", type=int, default=0, choices=[0, 1, 2, 3],
+                    help="scorer: 0 auto, 1 streaming, 2 tensor-core, 3 tensor-core on SM pairs")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")

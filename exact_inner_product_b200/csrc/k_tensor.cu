@@ -30,6 +30,7 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <stddef.h>
 #include <stdint.h>
 
 #include "tt_device.cuh"
@@ -61,9 +62,10 @@ struct K3Ctl {
     int abort;
     // per epilogue warp: fast-path thresholds and exact threshold keys of its
     // columns for the current unit
-    float th_fast[K3_EPI_WARPS][K3_WARP_COLS];
+    alignas(16) float th_fast[K3_EPI_WARPS][K3_WARP_COLS];  // read as float4
     uint64_t th_key[K3_EPI_WARPS][K3_WARP_COLS];
 };
+static_assert(offsetof(K3Ctl, th_fast) % 16 == 0, "float4 reads of th_fast need 16-byte alignment");
 
 struct K3Params {
     PassArgs a;
@@ -75,28 +77,6 @@ struct K3Params {
     int chunks;      // corpus chunks (units = q_tiles * chunks)
     uint32_t idesc;
 };
-
-struct Cols32 {
-    float x[32];
-};
-
-// x[i] for a run-time i, from registers (no local memory): pick the group of
-// eight first, then halve; few values are live at any time.
-__device__ __forceinline__ float select32(const Cols32& c, int i) {
-    const int g = i >> 3;
-    float a[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-        const float lo = (g & 1) ? c.x[8 + k] : c.x[k];
-        const float hi = (g & 1) ? c.x[24 + k] : c.x[16 + k];
-        a[k] = (g & 2) ? hi : lo;
-    }
-    const int j = i & 7;
-    const float b0 = (j & 4) ? a[4] : a[0], b1 = (j & 4) ? a[5] : a[1];
-    const float b2 = (j & 4) ? a[6] : a[2], b3 = (j & 4) ? a[7] : a[3];
-    const float c0 = (j & 2) ? b2 : b0, c1 = (j & 2) ? b3 : b1;
-    return (j & 1) ? c1 : c0;
-}
 
 __device__ __forceinline__ void unit_range(const K3Params& p, int u, int* qt, int64_t* t0,
                                            int64_t* t1) {

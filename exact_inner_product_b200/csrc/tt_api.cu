@@ -214,6 +214,14 @@ constexpr int MAX_DEEPEST_ROWS = 4096;  // the deepest level keeps every key
 constexpr int MIN_RANK = 32;
 constexpr int MAX_LEVELS = 4;
 constexpr int MAX_RESCANS = 64;
+// Batches at least this large, on a corpus stored normalised, go to the
+// tensor-core kernel on SM pairs (queries in tiles of 256 on TMEM lanes);
+// the rest to the single-SM kernel (queries in tiles of up to 256 on TMEM
+// columns, multiples of 32). Measured on B200 (level-0 pass): 50M x 128
+// stored rows, 1024 queries: 13.3 ms on pairs vs 14.6 ms single-SM; 20M x
+// 256 raw rows with per-row norms, 4096 queries: 41.3 ms vs 36.4 ms, so
+// corpora with per-row norms stay on the single-SM kernel.
+constexpr int PAIR_MIN_BATCH = 256;
 
 struct Plan {
     int levels;
@@ -400,7 +408,7 @@ static tt_status get_scratch(tt_index* ix, int b, int b_pad, int cap, int d, boo
 // one scoring pass over level i
 // ---------------------------------------------------------------------------
 struct PathCfg {
-    int path;           // 1 stream, 2 tensor
+    int path;           // 1 stream, 2 tensor, 3 tensor on SM pairs
     int nq;             // tensor path: queries per tile
     const void* queries;
     int q_dtype;
@@ -434,10 +442,15 @@ static tt_status run_pass(const tt_index* ix, const PathCfg& pc, const Plan& pla
         if (!bf16_tile_tensor_map(ix->rows, a.n_rows, ix->d, a.stride * ix->d, 128, &tm_rows))
             return TT_ERR_CUDA;
         e = launch_tensor_pass(a, tm_rows, pc.tm_q, pc.nq, s, sms);
+    } else if (pc.path == 3) {
+        CUtensorMap tm_rows;
+        if (!bf16_tile_tensor_map(ix->rows, a.n_rows, ix->d, a.stride * ix->d, 128, &tm_rows))
+            return TT_ERR_CUDA;
+        e = launch_tensor_pair_pass(a, tm_rows, pc.tm_q, s, sms);
     } else {
         e = launch_stream_pass(a, s, sms);
     }
-    if (e != cudaSuccess) return cuda_fail(e, pc.path == 2 ? "tensor pass" : "stream pass");
+    if (e != cudaSuccess) return cuda_fail(e, pc.path == 1 ? "stream pass" : "tensor pass");
     return TT_OK;
 }
 
@@ -636,15 +649,21 @@ tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtyp
         !aligned(exclude_bits, 4))
         return TT_ERR_INVALID_ARG;
     const int path_req = options ? options->path : 0;
-    if (path_req < 0 || path_req > 2) return TT_ERR_INVALID_ARG;
+    if (path_req < 0 || path_req > 3) return TT_ERR_INVALID_ARG;
     Plan plan;
     tt_status st = make_plan(index->n, k, options, &plan);
     if (st != TT_OK) return st;
     if (index->dtype == TT_F32 && index->d > 256) return TT_ERR_UNSUPPORTED;
     const bool tc_possible = index->dtype == TT_BF16 && index->d >= 64 && tensor_pass_max_nq(index->d) > 0;
+    const bool pair_possible = index->dtype == TT_BF16 && index->d >= 64 && tensor_pair_smem_bytes(index->d) > 0;
     int path = path_req;
-    if (path == 0) path = (tc_possible && b > 8) ? 2 : 1;
+    if (path == 0) {
+        path = 1;
+        if (tc_possible && b > 8) path = 2;
+        if (pair_possible && b >= PAIR_MIN_BATCH && index->inv_norm == nullptr) path = 3;
+    }
     if (path == 2 && !tc_possible) return TT_ERR_UNSUPPORTED;
+    if (path == 3 && !pair_possible) return TT_ERR_UNSUPPORTED;
     if (b == 0) return TT_OK;
 
     // ---------------- device checks ----------------
@@ -689,8 +708,9 @@ tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtyp
         nq = (nq + 31) / 32 * 32;  // whole 32-column chunks: no chunk reads past the tile
         if (nq > max_nq) nq = max_nq;
     }
-    const int b_pad = (path == 2 ? q_tiles * nq : b) + 64;
-    const bool need_qcast = path == 2 && q_dtype == TT_F32;
+    if (path == 3) q_tiles = (b + 255) / 256;
+    const int b_pad = (path == 2 ? q_tiles * nq : path == 3 ? q_tiles * 256 : b) + 64;
+    const bool need_qcast = path >= 2 && q_dtype == TT_F32;
     Scratch sc;
     if ((st = get_scratch(index, b, b_pad, plan.cap, index->d, need_qcast, &sc)) != TT_OK) return st;
     const int sms = sm_count_current();
@@ -701,7 +721,7 @@ tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtyp
     pc.path = path;
     pc.queries = queries;
     pc.q_dtype = q_dtype;
-    if (path == 2) {
+    if (path >= 2) {
         if (need_qcast) {
             cudaError_t e = launch_cast_bf16(static_cast<const float*>(queries), (int64_t)b * index->d,
                                              sc.qcast, s);
@@ -709,8 +729,10 @@ tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtyp
             pc.queries = sc.qcast;
             pc.q_dtype = TT_BF16;
         }
-        pc.nq = nq;
-        if (!bf16_tile_tensor_map(pc.queries, b, index->d, index->d, nq, &pc.tm_q)) return TT_ERR_CUDA;
+        pc.nq = path == 2 ? nq : 256;
+        // single-CTA kernel: boxes of nq queries; pairs: each CTA loads 128
+        if (!bf16_tile_tensor_map(pc.queries, b, index->d, index->d, path == 2 ? nq : 128, &pc.tm_q))
+            return TT_ERR_CUDA;
     }
 
     cudaError_t e = launch_init(sc.count, sc.theta, sc.thf, KEY_MIN, b, b_pad, sc.flags, s);

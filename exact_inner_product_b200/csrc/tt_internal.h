@@ -50,6 +50,10 @@ cudaError_t launch_stream_pass(const PassArgs& a, cudaStream_t s, int sm_count);
 cudaError_t launch_tensor_pass(const PassArgs& a, const CUtensorMap& tm_rows,
                                const CUtensorMap& tm_queries, int nq_tile, cudaStream_t s,
                                int sm_count);
+// Tensor-core pass on SM pairs (b >= 1; queries in tiles of 256, tm_queries
+// with boxes of 128 rows).
+cudaError_t launch_tensor_pair_pass(const PassArgs& a, const CUtensorMap& tm_rows,
+                                    const CUtensorMap& tm_queries, cudaStream_t s, int sm_count);
 // count[0..b) = 0; theta/thf[0..b) = theta_value; [b, b_pad) = KEY_MAX / +inf;
 // flags[0..2) = 0.
 cudaError_t launch_init(uint32_t* count, uint64_t* theta, float* thf, uint64_t theta_value, int b,
@@ -78,5 +82,6 @@ cudaError_t launch_pad(int32_t* out_ids, float* out_scores, int64_t count, cudaS
 // Shared-memory bytes the tensor-core pass needs for a given d and query tile.
 int tensor_pass_smem_bytes(int d, int nq_tile);
 int tensor_pass_max_nq(int d);
+int tensor_pair_smem_bytes(int d);  // -1 when d does not fit
 
 }  // namespace tt

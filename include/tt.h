@@ -153,7 +153,8 @@ TT_API tt_status tt_score_topk(tt_index* index, const void* queries, tt_dtype q_
 /* Path selection and test hooks for tt_score_topk_ex. Zero-initialise, then
  * set fields; tt_score_topk uses all zeros. */
 typedef struct tt_options {
-    int32_t path;           /* 0 auto; 1 CUDA-core streaming scorer; 2 tensor-core scorer */
+    int32_t path;           /* 0 auto; 1 CUDA-core streaming scorer; 2 tensor-core scorer
+                               (one SM per tile); 3 tensor-core scorer on SM pairs */
     int32_t rank_scale_pct; /* 0 = 100. Scales the ranks used to set the estimated
                                thresholds (test hook: < 100 provokes rescans) */
     int32_t force_levels;   /* 0 auto; > 0 = number of levels (1 = single pass) */
@@ -167,7 +168,7 @@ TT_API tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype
 
 /* What the last tt_score_topk on a handle did. */
 typedef struct tt_stats {
-    int32_t path;            /* 1 streaming, 2 tensor core */
+    int32_t path;            /* 1 streaming, 2 tensor core, 3 tensor core on SM pairs */
     int32_t levels;          /* scoring passes in the plan (1 = single pass) */
     int32_t rescans;         /* extra full passes made to restore exactness */
     int32_t launches;        /* kernels launched by the call */

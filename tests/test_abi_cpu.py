@@ -103,7 +103,10 @@ def test_host_validation_rejects_before_any_device_call():
     opt = tt.tt_options(2, 0, 0, 0)
     assert lib.tt_score_topk_ex(ixf, fake, 0, 4, None, 1.0, 10, ids, sc, None, ctypes.byref(opt)) \
         == tt.TT_ERR_UNSUPPORTED
-    bad = tt.tt_options(3, 0, 0, 0)
+    opt3 = tt.tt_options(3, 0, 0, 0)
+    assert lib.tt_score_topk_ex(ixf, fake, 0, 4, None, 1.0, 10, ids, sc, None, ctypes.byref(opt3)) \
+        == tt.TT_ERR_UNSUPPORTED
+    bad = tt.tt_options(4, 0, 0, 0)
     assert lib.tt_score_topk_ex(ixf, fake, 0, 4, None, 1.0, 10, ids, sc, None, ctypes.byref(bad)) \
         == tt.TT_ERR_INVALID_ARG
     lib.tt_free(ixf)

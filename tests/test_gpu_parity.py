@@ -1,8 +1,8 @@
 """CUDA path vs the fp64 oracle on seeded inputs (GPU).
 
 Sizes are small enough for the oracle to finish in seconds, yet span several
-tiles (32-row streaming tiles, 128-row tensor-core tiles, 256-query tiles)
-with ragged tails. Each case calls the library through its C ABI.
+tiles (32-row streaming tiles, 128-row tensor-core tiles, 256-query tiles,
+256-row tiles of the SM-pair kernel) with ragged tails. Each case calls the library through its C ABI.
 """
 import numpy as np
 import pytest
@@ -29,7 +29,8 @@ CASES = [
     ("stream_b1", {"n": 150_001, "b": 5, "k": 64}, 1),
     ("small_batch", {"n": 300_077}, 2),
     ("small_batch", {"n": 100_003, "b": 9, "k": 17}, 2),
-    ("large_batch", {"n": 400_005, "b": 300, "k": 1000, "oracle_queries": 12}, 2),
+    ("large_batch", {"n": 400_005, "b": 300, "k": 1000, "oracle_queries": 12}, 3),
+    ("large_batch", {"n": 250_001, "b": 200, "k": 300, "oracle_queries": 12}, 2),
     ("masked_fused", {"n": 200_099, "b": 520, "oracle_queries": 12}, 2),
     ("masked_fused", {"n": 120_031, "b": 3, "k": 256}, 1),
 ]
@@ -44,12 +45,23 @@ def test_parity_scaled(name, over, path):
     assert res["max_abs_err"] <= w.tolerance
 
 
-@pytest.mark.parametrize("path", [1, 2])
-def test_both_scorers_agree_with_oracle(path):
+@pytest.mark.parametrize("path", [1, 2, 3])
+def test_every_scorer_agrees_with_oracle(path):
     _cuda()
     w = W.workload("small_batch", n=70_001, b=40, k=100, tau=1.0)
     res, st = parity.run_case(w, path=path)
     assert st["path"] == path
+
+
+def test_pair_kernel_with_norms_and_mask():
+    """The SM-pair kernel on a raw corpus with per-row norms, tau and an
+    exclusion mask (the automatic choice sends such corpora to the single-SM
+    kernel, so it is forced here)."""
+    _cuda()
+    w = W.workload("masked_fused", n=200_099, b=520, oracle_queries=12)
+    res, st = parity.run_case(w, path=3)
+    assert st["path"] == 3
+    assert res["max_abs_err"] <= w.tolerance
 
 
 def test_normalize_matches_oracle():
@@ -91,14 +103,14 @@ def _pad16(a):
     return out
 
 
-@pytest.mark.parametrize("path", [1, 2])
+@pytest.mark.parametrize("path", [1, 2, 3])
 def test_hand_worked_h2(path):
     """The hand-worked d=4 example (zero-padded to d=16) through both scorers."""
     _cuda()
     import oracle_pins
     g = oracle_pins.golden()["H2_topk"]
     V = _pad16(g["corpus"])
-    if path == 2:  # tensor cores need a bf16 corpus with d >= 64
+    if path >= 2:  # tensor cores need a bf16 corpus with d >= 64
         V = np.pad(V, ((0, 0), (0, 48)))
     dtype = torch.float32 if path == 1 else torch.bfloat16
     index, rows = _index_from_rows(V, dtype)
@@ -118,13 +130,13 @@ def test_hand_worked_h2(path):
 
 
 def test_ties_across_tiles():
-    """All rows identical: every score ties; ids must be 0..k-1 on both paths."""
+    """All rows identical: every score ties; ids must be 0..k-1 on every path."""
     _cuda()
     n, d = 70_000, 64
     row = torch.randn(1, d)
     rows = (row / row.norm()).repeat(n, 1).to("cuda", torch.bfloat16).contiguous()
     index = tt.tt_index_wrap(rows)
-    for path, b in ((1, 2), (2, 40)):
+    for path, b in ((1, 2), (2, 40), (3, 300)):
         q = torch.randn(b, d, device="cuda").to(torch.bfloat16)
         ids, scores = tt.tt_score_topk(index, q, 700, path=path)
         assert (ids.cpu() == torch.arange(700, dtype=torch.int32)[None, :]).all()
@@ -137,7 +149,7 @@ def test_identity_corpus():
     E = torch.eye(d)
     index, rows = _index_from_rows(E.numpy(), torch.bfloat16)
     q = E[[0, 7, 63] * 4].to("cuda", torch.bfloat16).contiguous()
-    for path in (1, 2):
+    for path in (1, 2, 3):
         ids, scores = tt.tt_score_topk(index, q, 6, path=path)
         for r, t in enumerate([0, 7, 63] * 4):
             assert ids[r].tolist() == [t] + [j for j in range(d) if j != t][:5]
@@ -165,9 +177,9 @@ def test_edge_cases():
     empty = tt.tt_index_wrap(torch.empty((0, d), dtype=torch.bfloat16, device="cuda"))
     ids, scores = tt.tt_score_topk(empty, q, 3)
     assert (ids == -1).all() and torch.isinf(scores).all()
-    # a tiny corpus below one tile, on both paths
+    # a tiny corpus below one tile, on every path
     small = tt.tt_index_wrap(rows[:7].contiguous())
-    for path in (1, 2):
+    for path in (1, 2, 3):
         ids, _ = tt.tt_score_topk(small, q, 3, path=path)
         s = (q.float() @ rows[:7].float().T)
         ref = torch.sort(s, dim=1, descending=True, stable=True).indices[:, :3].to(torch.int32)
@@ -175,7 +187,8 @@ def test_edge_cases():
 
 
 @pytest.mark.parametrize("opts", [{"rank_scale_pct": 3}, {"cap": 256, "force_levels": 2},
-                                  {"force_levels": 1}, {"force_levels": 4}])
+                                  {"force_levels": 1}, {"force_levels": 4},
+                                  {"rank_scale_pct": 3, "path": 3}, {"cap": 256, "path": 3}])
 def test_rescans_stay_exact(opts):
     """Thresholds deliberately mis-estimated (tiny ranks, tiny buffers): the
     exactness check must trigger rescans and the answer must not change."""
@@ -197,10 +210,15 @@ def test_repeat_runs_are_bitwise_identical():
     for _ in range(3):
         again = tt.tt_score_topk(index, qn, w.k)
         assert torch.equal(first[0], again[0]) and torch.equal(first[1], again[1])
-    # batch invariance: a query's result does not depend on the rest of the batch
+    assert tt.tt_last_stats(index)["path"] == 3
+    # batch invariance: a query's result does not depend on the rest of the
+    # batch, nor on which tensor-core kernel the batch size selects
     sub = tt.tt_score_topk(index, qn[5:6].repeat(20, 1).contiguous(), w.k)
+    assert tt.tt_last_stats(index)["path"] == 2
     assert torch.equal(sub[0][0], first[0][5])
     assert torch.equal(sub[1][0], first[1][5])
+    single = tt.tt_score_topk(index, qn, w.k, path=2)
+    assert torch.equal(single[0], first[0]) and torch.equal(single[1], first[1])
 
 
 def test_rejects_host_pointers_and_bad_args():

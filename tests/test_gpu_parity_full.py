@@ -24,7 +24,7 @@ def test_full_size_parity(name):
     oracle.set_threads(oracle.max_threads())
     w = W.workload(name)
     res, st = parity.run_case(w)
-    expect_path = 1 if (w.store == "f32" or w.b <= 8) else 2
+    expect_path = 1 if (w.store == "f32" or w.b <= 8) else 2 if (w.b < 256 or w.store == "raw") else 3
     assert st["path"] == expect_path
     assert res["queries"] == len(W.oracle_query_ids(w))
     assert res["max_abs_err"] <= w.tolerance
