@@ -47,12 +47,23 @@ PATH_NAMES = {1: "streaming", 2: "tensor-core", 3: "tensor-core (SM pairs)"}
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per unit of work
 # from ncu captures of a kernel, with the sha256 of the kernel's source file at
 # capture time; `traffic` is reported only while that file is unchanged. Units:
-# K1 bytes per corpus row; K3 bytes per corpus row of one level-0 pass.
+# K1 bytes per corpus row; K3 bytes per level row scanned (level-0 capture,
+# applied to every level of a step, like `achieved`).
 TRAFFIC = {
     # ncu --set full -k regex:k1_normalize -s 5 -c 1 on `python bench.py --steps 50 --warmup 3
     # --no-e2e --no-cpu-baseline`: 512.016 MB read + 201.165 MB written for 1,000,000 rows
     ("k1_normalize", "stream_b1"): {"bytes_per_row": 713.181, "src": "exact_inner_product_b200/csrc/k_normalize.cu",
                                     "sha": "6d3e520d16da8b6d042167b6dd9594cc512d14f3cc131115f5cdfec93e963db7"},
+    # ncu --set full -k regex:k3_pair -s 5 -c 1 on `python bench.py --workload large_batch --n 4000000
+    # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 1587.723 MB read
+    # + 27.798 MB written; scaled to the full corpus by rows scanned
+    ("k3_pair", "large_batch"): {"bytes_per_row": 403.880, "src": "exact_inner_product_b200/csrc/k_tensor_pair.cu",
+                                 "sha": "43e2c4b1ce6837870992c30a53efa9ec8d8dfb0ced721048ba161508dce63734"},
+    # ncu --set full -k regex:k3_tensor -s 5 -c 1 on `python bench.py --workload masked_fused --n 4000000
+    # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 4984.254 MB read
+    # + 73.270 MB written; scaled to the full corpus by rows scanned
+    ("k3_tensor", "masked_fused"): {"bytes_per_row": 1264.381, "src": "exact_inner_product_b200/csrc/k_tensor.cu",
+                                    "sha": "de8f36cb5cd9b834950b076a917f656f291e63dd7a3a7ad71247af58d6443feb"},
 }
 
 
