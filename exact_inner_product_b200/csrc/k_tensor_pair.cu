@@ -346,16 +346,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         const int col0 = (2 * pair + h) * 32;  // within this warp's 128 columns
-                        // Fast test: four independent or-chains.
+                        // Fast test. One threshold per thread: compare the
+                        // maximum of the 32 scores (four chains of
+                        // three-input max, half an instruction per score).
                         bool h0 = false, h1 = false, h2 = false, h3 = false;
+                        float gmax[4];
                         if (uniform_c) {
 #pragma unroll
-                            for (int i = 0; i < 32; i += 4) {
-                                h0 |= v[h].x[i + 0] >= t_fast;
-                                h1 |= v[h].x[i + 1] >= t_fast;
-                                h2 |= v[h].x[i + 2] >= t_fast;
-                                h3 |= v[h].x[i + 3] >= t_fast;
+                            for (int j = 0; j < 4; ++j) {  // chain j: scores 8j .. 8j+7
+                                const float* x = v[h].x + 8 * j;
+                                gmax[j] = fmaxf(max3f(max3f(max3f(x[0], x[1], x[2]), x[3], x[4]), x[5], x[6]), x[7]);
                             }
+                            h0 = fmaxf(max3f(gmax[0], gmax[1], gmax[2]), gmax[3]) >= t_fast;
                         } else {
                             // all-negative test: AND of the sign words
                             const float4* c4 = reinterpret_cast<const float4*>(cw + col0);
@@ -374,9 +376,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
                         if (h0 | h1 | h2 | h3) {
                             uint32_t m = 0;
                             if (uniform_c) {
+                                // only the groups of eight whose maximum passed
 #pragma unroll
-                                for (int i = 0; i < 32; ++i)
-                                    m |= (v[h].x[i] >= t_fast) ? (1u << i) : 0u;
+                                for (int j = 0; j < 4; ++j) {
+                                    if (gmax[j] >= t_fast) {
+#pragma unroll
+                                        for (int i = 8 * j; i < 8 * j + 8; ++i)
+                                            m |= (v[h].x[i] >= t_fast) ? (1u << i) : 0u;
+                                    }
+                                }
                             } else {
                                 const float4* c4 = reinterpret_cast<const float4*>(cw + col0);
 #pragma unroll

@@ -211,7 +211,15 @@ static int sm_count_current() {
 constexpr int STRIDE_RATIO = 64;
 constexpr int DEFAULT_CAP = 16384;
 constexpr int MAX_DEEPEST_ROWS = 4096;  // the deepest level keeps every key
+// Floors of the ranks. The survivors of a pass whose threshold is the r-th
+// best key of a 1/64 sample number about Gamma(r, 64); a pass that must keep
+// `need` keys falls short with probability P(Poisson(need / 64) >= r).
+// Level 1 sets the threshold of the full pass (need = k): r >= max(3k/64, 32)
+// puts that below 1e-8 per query. Deeper levels only feed a coarser pass
+// (need <= a few dozen, so need / 64 < 1) and 10 suffices there, with far
+// fewer keys kept per pass.
 constexpr int MIN_RANK = 32;
+constexpr int MIN_RANK_DEEP = 10;
 constexpr int MAX_LEVELS = 4;
 constexpr int MAX_RESCANS = 64;
 // Batches at least this large, on a corpus stored normalised, go to the
@@ -265,7 +273,8 @@ static tt_status make_plan(int64_t n, int32_t k, const tt_options* opt, Plan* p)
         p->rows[i] = n > 0 ? (n + st - 1) / st : 0;
         if (i >= 1) {
             int64_t r = (3 * (int64_t)need + STRIDE_RATIO - 1) / STRIDE_RATIO;
-            if (r < MIN_RANK) r = MIN_RANK;
+            const int floor_r = i == 1 ? MIN_RANK : MIN_RANK_DEEP;
+            if (r < floor_r) r = floor_r;
             r = r * scale / 100;
             if (r < 1) r = 1;
             p->rank[i] = (int)r;

@@ -134,12 +134,12 @@ def test_plan_levels():
             assert p["ranks"][i] * 64 <= p["cap"] // 2
     assert tt.tt_plan(400, 10)["levels"] == 1
     assert tt.tt_plan(10 ** 6, 100) == {"levels": 3, "rows": [10 ** 6, 15625, 245], "strides": [1, 64, 4096],
-                                        "ranks": [100, 32, 32], "cap": 16384}
-    assert tt.tt_plan(5 * 10 ** 7, 1000)["ranks"] == [1000, 47, 32, 32]
+                                        "ranks": [100, 32, 10], "cap": 16384}
+    assert tt.tt_plan(5 * 10 ** 7, 1000)["ranks"] == [1000, 47, 10, 10]
     assert tt.tt_plan(4096, 10)["levels"] == 1 and tt.tt_plan(4097, 10)["levels"] == 2
     assert tt.tt_plan(10 ** 6, 100, force_levels=1)["levels"] == 1
     assert tt.tt_plan(10 ** 6, 100, force_levels=3)["levels"] == 3
-    assert tt.tt_plan(10 ** 6, 100, rank_scale_pct=50)["ranks"] == [100, 16, 16]
+    assert tt.tt_plan(10 ** 6, 100, rank_scale_pct=50)["ranks"] == [100, 16, 5]
     with pytest.raises(tt.TTError):
         tt.tt_plan(10, 0)
     with pytest.raises(tt.TTError):
