@@ -8,10 +8,14 @@ select the exact top-k. Inputs are seeded synthetic data (``workloads.py``)
 resident in HBM before timing starts. The default workload is the streaming
 single-query case (N = 1,000,000, d = 128, B = 1, k = 100).
 
-Multi-GPU (torchrun, one process per GPU): every rank runs an independent
-replica of the workload on its own queries - the path has no exchange step,
-so there is no collective in the data path; the value is the total over ranks
-(weak scaling), timed as the max over ranks.
+Multi-GPU (torchrun, one process per GPU), two modes:
+  --mode replicas (default): every rank runs an independent replica of the
+    workload on its own queries - no collective in the data path; the value
+    is the total over ranks (weak scaling), timed as the max over ranks.
+  --mode shard: the ranks split one corpus by rows; every step each rank
+    normalises and scores its shard, the [b, k] lists are all-gathered over
+    NCCL and merged (tt_merge_topk) on every rank; the value is the one
+    workload's scores per second (strong scaling).
 
 Prints one JSON line (rank 0).
 """
@@ -19,6 +23,7 @@ from __future__ import annotations
 
 import argparse
 import csv
+import dataclasses
 import datetime as dt
 import json
 import math
@@ -264,14 +269,25 @@ def workload_from_args(args) -> W.Workload:
 
 def run_ours(args, world, rank, local):
     import exact_inner_product_b200 as tt
+    from exact_inner_product_b200 import shard
 
+    sharded = args.mode == "shard"
     w = workload_from_args(args)
-    if world > 1:  # each rank: its own queries (independent replica)
+    if world > 1 and not sharded:  # each rank: its own queries (independent replica)
         w = W.workload(w.name, n=w.n, b=w.b, k=w.k, seed=w.seed + 7919 * rank)
     dev = torch.device("cuda", local)
     raw_c = W.corpus(w, dev)
     raw_q = W.queries(w, dev)
     excl = W.exclusion_bits(w, dev)
+    w_all = w
+    if sharded:
+        # this rank's rows of the one corpus; queries are the same on every rank
+        bounds = shard.shard_bounds(w.n, world)
+        start, count = bounds[rank]
+        raw_c = raw_c[start:start + count].clone()
+        excl = shard.exclude_slice(excl, start, count)
+        torch.cuda.empty_cache()
+        w = dataclasses.replace(w, n=count)
     if w.store == "raw":
         prepared = torch.empty((w.n,), dtype=torch.float32, device=dev)
         mode = tt.TT_NORM_FUSED
@@ -299,8 +315,11 @@ def run_ours(args, world, rank, local):
             e1.record(stream)
             ev_k1.append((e0, e1))
         tt.tt_normalize_candidates(raw_q, qn, tt.TT_NORM_STORE, make_index=False)
-        tt.tt_score_topk(index, qn, w.k, tau=w.tau, exclude=excl, out_ids=out_ids, out_scores=out_scores,
-                         path=args.path)
+        if sharded:
+            shard.sharded_score_topk(index, qn, w.k, bounds, tau=w.tau, exclude_local=excl, path=args.path)
+        else:
+            tt.tt_score_topk(index, qn, w.k, tau=w.tau, exclude=excl, out_ids=out_ids, out_scores=out_scores,
+                             path=args.path)
         return index
 
     for _ in range(args.warmup):
@@ -332,8 +351,9 @@ def run_ours(args, world, rank, local):
     ms_total = max_over_ranks(ms_total, world)
     ms_step = ms_total / args.steps
 
-    value = world * w.b * w.n / (ms_step / 1e3)
-    qps = world * w.b / (ms_step / 1e3)
+    # replicas: every rank did a whole workload; shards: the ranks did one together
+    value = (1 if sharded else world) * w_all.b * w_all.n / (ms_step / 1e3)
+    qps = (1 if sharded else world) * w_all.b / (ms_step / 1e3)
 
     # ---- roofline of the dominant kernel ----
     peaks, peak_src = load_peaks()
@@ -374,7 +394,7 @@ def run_ours(args, world, rank, local):
 
     # ---- end to end through the public API, host buffers ----
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not sharded:
         host_c = raw_c.cpu().pin_memory()
         host_q = raw_q.cpu().pin_memory()
         host_x = excl.cpu().pin_memory() if excl is not None else None
@@ -400,14 +420,16 @@ def run_ours(args, world, rank, local):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.store != "f32" else "f32",
+        "scaling": "strong" if sharded else "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.store != "f32" else "f32",
         "data": "synthetic (seeded, workloads.py)",
-        "config": {"workload": w.name, "n": w.n, "d": w.d, "b": w.b, "k": w.k, "tau": w.tau,
+        "config": {"workload": w.name, "n": w_all.n, "d": w.d, "b": w.b, "k": w.k, "tau": w.tau,
                    "corpus_raw": w.raw_dtype, "corpus_store": w.store, "queries": w.query_dtype,
                    "mask_rate": w.mask_rate, "l2": "inputs larger than L2 (raw corpus "
                    f"{w.n * w.d * elem_bytes(w.raw_dtype) / 1e6:.0f} MB > 126 MB)",
                    "path": PATH_NAMES[stats["path"]], "levels": plan["rows"],
-                   "parallelism": f"replicas x{world}"},
+                   "parallelism": (f"corpus shards x{world} (all-gather of [b, k] lists + merge)" if sharded
+                                   else f"replicas x{world}")},
         "topk_queries_per_s": qps,
         "roofline": roof,
         "kernels": kernels,
@@ -463,6 +485,8 @@ def main():
     ap.add_argument("--k", type=int, default=0, help="override the workload's k")
     ap.add_argument("--path", type=int, default=0, choices=[0, 1, 2, 3],
                     help="scorer: 0 auto, 1 streaming, 2 tensor-core, 3 tensor-core on SM pairs")
+    ap.add_argument("--mode", default="replicas", choices=["replicas", "shard"],
+                    help="N > 1: independent replicas (default) or one corpus sharded by rows over the ranks")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -82,6 +82,7 @@ _sig("tt_plan", ctypes.c_int, [_i64, _i32, ctypes.POINTER(tt_options), ctypes.PO
                                ctypes.POINTER(_i32)])
 _sig("tt_score_topk_noalloc", ctypes.c_int, [_vp, ctypes.c_int, _i64, _i32, _vp, _vp, ctypes.c_int, _i32,
                                              _vp, ctypes.c_float, _i32, _vp, _vp, _vp])
+_sig("tt_merge_topk", ctypes.c_int, [_vp, _vp, _i32, _i32, _i32, ctypes.POINTER(_i64), _i32, _vp, _vp, _vp])
 _sig("tt_free", None, [_vp])
 _sig("tt_launch_count", _i64, [])
 _sig("tt_profile_begin", ctypes.c_int, [])
@@ -93,7 +94,7 @@ _sig("tt_last_error", ctypes.c_char_p, [])
 _sig("tt_version", ctypes.c_char_p, [])
 
 EXPORTED = ("tt_normalize_candidates", "tt_index_wrap", "tt_score_topk", "tt_score_topk_ex",
-            "tt_score_topk_noalloc",
+            "tt_score_topk_noalloc", "tt_merge_topk",
             "tt_last_stats", "tt_plan", "tt_free", "tt_launch_count", "tt_profile_begin",
             "tt_profile_end", "tt_profile_launches", "tt_status_string", "tt_last_error", "tt_version")
 
@@ -247,6 +248,32 @@ def tt_score_topk_noalloc(rows: torch.Tensor, queries: torch.Tensor, k: int, tau
                                     _dtype(queries), b, _ptr(exclude), float(tau), int(k), _ptr(out_ids),
                                     _ptr(out_scores), _stream(stream))
     _check(st, "tt_score_topk_noalloc")
+    return out_ids, out_scores
+
+
+def tt_merge_topk(ids: torch.Tensor, scores: torch.Tensor, id_offsets, k_out: int,
+                  out_ids: torch.Tensor | None = None, out_scores: torch.Tensor | None = None, stream=None):
+    """Top-k_out of the union of per-shard lists (``tt_merge_topk``).
+
+    ``ids`` int32 / ``scores`` float32, contiguous [parts, b, k_in] on the GPU
+    (each part: one shard's tt_score_topk output, local ids); ``id_offsets``:
+    the global id of each shard's row 0. Returns ``(ids int32 [b, k_out],
+    scores float32 [b, k_out])`` with global ids."""
+    if ids.dim() != 3 or ids.shape != scores.shape or not ids.is_contiguous() or not scores.is_contiguous():
+        raise ValueError("ids and scores must be contiguous [parts, b, k_in] tensors of one shape")
+    if ids.dtype != torch.int32 or scores.dtype != torch.float32:
+        raise TypeError("ids must be int32 and scores float32")
+    parts, b, k_in = ids.shape
+    offs = (_i64 * max(1, parts))(*[int(o) for o in id_offsets])
+    if len(id_offsets) != parts:
+        raise ValueError("one offset per part")
+    dev = ids.device
+    if out_ids is None:
+        out_ids = torch.empty((b, k_out), dtype=torch.int32, device=dev)
+    if out_scores is None:
+        out_scores = torch.empty((b, k_out), dtype=torch.float32, device=dev)
+    _check(_lib.tt_merge_topk(_ptr(ids), _ptr(scores), parts, b, k_in, offs, int(k_out), _ptr(out_ids),
+                              _ptr(out_scores), _stream(stream)), "tt_merge_topk")
     return out_ids, out_scores
 
 

@@ -56,7 +56,7 @@ __device__ const uint64_t* stage_keys(const uint64_t* __restrict__ g, int n, K4S
     return sm.keys;
 }
 
-// r-th largest (1-based) of n distinct keys; 1 <= r <= n. Block-wide.
+// r-th largest (1-based, counting repeats) of n keys; 1 <= r <= n. Block-wide.
 // Radix passes narrow the candidates to a digit prefix; once at most
 // K4_THREADS keys share the prefix they are gathered and ranked directly.
 __device__ uint64_t block_kth_largest(const uint64_t* keys, int n, int r, K4Smem& sm) {
@@ -131,15 +131,110 @@ __device__ uint64_t block_kth_largest(const uint64_t* keys, int n, int r, K4Smem
             __syncthreads();
             if (tid < (int)count) {
                 const uint64_t mine = sm.sorted[tid];
-                uint32_t above_me = 0;
-                for (uint32_t j = 0; j < count; ++j) above_me += sm.sorted[j] > mine;
-                if (above_me == remaining - 1) sm.result = mine;
+                uint32_t above_me = 0, equal = 0;
+                for (uint32_t j = 0; j < count; ++j) {
+                    above_me += sm.sorted[j] > mine;
+                    equal += sm.sorted[j] == mine;
+                }
+                if (above_me < remaining && remaining <= above_me + equal) sm.result = mine;
             }
             __syncthreads();
             return sm.result;
         }
     }
     return prefix;
+}
+
+// The min(n, k) largest of n distinct keys, sorted descending, written as
+// (id, score); slots past n get (-1, -inf). Block-wide; out_* point at one
+// query's row of k entries.
+__device__ void write_sorted_topk(const uint64_t* keys, int n, int k, K4Smem& sm, int32_t* out_ids,
+                                  float* out_scores) {
+    const int tid = threadIdx.x;
+    const int r = n < k ? n : k;
+    if (r > 0) {
+        const uint64_t kth = block_kth_largest(keys, n, r, sm);
+        if (tid == 0) sm.n_collected = 0;
+        __syncthreads();
+        // fewer than r keys are above the r-th largest; the rest of the r
+        // slots hold it (one copy when keys are distinct)
+        for (int i = tid; i < n; i += K4_THREADS) {
+            const uint64_t key = keys[i];
+            if (key > kth) {
+                const uint32_t slot = atomicAdd(&sm.n_collected, 1u);
+                if (slot < (uint32_t)r) sm.sorted[slot] = key;
+            }
+        }
+        __syncthreads();
+        const int above = (int)sm.n_collected < r ? (int)sm.n_collected : r;
+        for (int i = above + tid; i < r; i += K4_THREADS) sm.sorted[i] = kth;
+        __syncthreads();
+        int P = 1;
+        while (P < r) P <<= 1;
+        for (int i = r + tid; i < P; i += K4_THREADS) sm.sorted[i] = KEY_MIN;
+        __syncthreads();
+        // bitonic sort, descending
+        for (int size = 2; size <= P; size <<= 1) {
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                for (int i = tid; i < P; i += K4_THREADS) {
+                    const int j = i ^ stride;
+                    if (j > i) {
+                        const uint64_t x = sm.sorted[i], y = sm.sorted[j];
+                        const bool desc = (i & size) == 0;
+                        if (desc ? (x < y) : (x > y)) {
+                            sm.sorted[i] = y;
+                            sm.sorted[j] = x;
+                        }
+                    }
+                }
+                __syncthreads();
+            }
+        }
+    }
+    for (int i = tid; i < k; i += K4_THREADS) {
+        int32_t id = -1;
+        float sc = -INFINITY;
+        if (i < r) {
+            id = (int32_t)key_id(sm.sorted[i]);
+            sc = key_score(sm.sorted[i]);
+        }
+        out_ids[i] = id;
+        out_scores[i] = sc;
+    }
+}
+
+// Merge of per-shard results: part p holds, for every query, its shard's
+// top-k_in as (local id, score); local ids plus id_offset[p] are global ids;
+// -1 entries are padding. Each query's keys are built in shared memory (or
+// in scratch[q * parts * k_in ...] when they do not fit) and the k_out best
+// are written sorted. Exact: every member of the global top-k_out is in its
+// own shard's top-k_in when k_out <= k_in.
+struct MergeOffsets {
+    int64_t v[TT_MAX_PARTS];
+};
+
+__global__ void __launch_bounds__(K4_THREADS)
+    k4_merge(const int32_t* __restrict__ ids, const float* __restrict__ scores, int parts, int b, int k_in,
+             const MergeOffsets id_offset, int k_out, uint64_t* __restrict__ scratch,
+             int32_t* __restrict__ out_ids, float* __restrict__ out_scores) {
+    extern __shared__ __align__(16) uint8_t k4_smem_raw[];
+    K4Smem& sm = *reinterpret_cast<K4Smem*>(k4_smem_raw);
+    const int q = blockIdx.x;
+    const int tid = threadIdx.x;
+    const int m = parts * k_in;
+    uint64_t* keys = m <= K4_SMEM_KEYS ? sm.keys : scratch + (int64_t)q * m;
+    if (tid == 0) sm.n_collected = 0;
+    __syncthreads();
+    for (int i = tid; i < m; i += K4_THREADS) {
+        const int p = i / k_in, j = i - p * k_in;
+        const int64_t src = ((int64_t)p * b + q) * k_in + j;
+        const int32_t id = ids[src];
+        if (id >= 0) keys[atomicAdd(&sm.n_collected, 1u)] = make_key(scores[src], (uint32_t)(id + id_offset.v[p]));
+    }
+    __syncthreads();
+    const int n = (int)sm.n_collected;
+    __syncthreads();
+    write_sorted_topk(keys, n, k_out, sm, out_ids + (int64_t)q * k_out, out_scores + (int64_t)q * k_out);
 }
 
 __global__ void __launch_bounds__(K4_THREADS)
@@ -179,48 +274,7 @@ __global__ void __launch_bounds__(K4_THREADS)
     const uint64_t* qkeys = stage_keys(keys + (int64_t)q * cap, n, sm);
     const bool exact = (c <= (uint32_t)cap) && (c >= (uint32_t)k || th == KEY_MIN);
     if (exact) {
-        const int r = n < k ? n : k;
-        if (r > 0) {
-            const uint64_t kth = block_kth_largest(qkeys, n, r, sm);
-            if (tid == 0) sm.n_collected = 0;
-            __syncthreads();
-            for (int i = tid; i < n; i += K4_THREADS) {
-                const uint64_t key = qkeys[i];
-                if (key >= kth) sm.sorted[atomicAdd(&sm.n_collected, 1u)] = key;
-            }
-            __syncthreads();
-            int P = 1;
-            while (P < r) P <<= 1;
-            for (int i = r + tid; i < P; i += K4_THREADS) sm.sorted[i] = KEY_MIN;
-            __syncthreads();
-            // bitonic sort, descending
-            for (int size = 2; size <= P; size <<= 1) {
-                for (int stride = size >> 1; stride > 0; stride >>= 1) {
-                    for (int i = tid; i < P; i += K4_THREADS) {
-                        const int j = i ^ stride;
-                        if (j > i) {
-                            const uint64_t x = sm.sorted[i], y = sm.sorted[j];
-                            const bool desc = (i & size) == 0;
-                            if (desc ? (x < y) : (x > y)) {
-                                sm.sorted[i] = y;
-                                sm.sorted[j] = x;
-                            }
-                        }
-                    }
-                    __syncthreads();
-                }
-            }
-        }
-        for (int i = tid; i < k; i += K4_THREADS) {
-            int32_t id = -1;
-            float sc = -INFINITY;
-            if (i < r) {
-                id = (int32_t)key_id(sm.sorted[i]);
-                sc = key_score(sm.sorted[i]);
-            }
-            out_ids[(int64_t)q * k + i] = id;
-            out_scores[(int64_t)q * k + i] = sc;
-        }
+        write_sorted_topk(qkeys, n, k, sm, out_ids + (int64_t)q * k, out_scores + (int64_t)q * k);
         if (tid == 0) status[q] = 0;
     } else {
         uint64_t th_new = KEY_MIN;
@@ -311,6 +365,24 @@ cudaError_t launch_select_final(const uint64_t* keys, uint32_t* count, int cap, 
     note_launch_end(TT_KIND_SELECT, s);
     return cudaGetLastError();
 }
+
+cudaError_t launch_merge(const int32_t* ids, const float* scores, int parts, int b, int k_in,
+                         const int64_t* id_offset_host, int k_out, uint64_t* scratch, int32_t* out_ids,
+                         float* out_scores, cudaStream_t s) {
+    if (b == 0) return cudaSuccess;
+    if (parts < 1 || parts > TT_MAX_PARTS) return cudaErrorInvalidValue;
+    MergeOffsets id_offset;
+    for (int p = 0; p < TT_MAX_PARTS; ++p) id_offset.v[p] = p < parts ? id_offset_host[p] : 0;
+    const int smem = (int)sizeof(K4Smem);
+    cudaFuncSetAttribute(k4_merge, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    note_launch_begin(TT_KIND_SELECT, s);
+    k4_merge<<<b, K4_THREADS, smem, s>>>(ids, scores, parts, b, k_in, id_offset, k_out, scratch, out_ids,
+                                         out_scores);
+    note_launch_end(TT_KIND_SELECT, s);
+    return cudaGetLastError();
+}
+
+int merge_smem_keys() { return K4_SMEM_KEYS; }
 
 cudaError_t launch_prepare_repair(uint64_t* theta, float* thf, const int32_t* status, int b,
                                   int* flags, cudaStream_t s) {

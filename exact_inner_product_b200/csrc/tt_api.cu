@@ -789,6 +789,40 @@ tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtyp
     return TT_OK;
 }
 
+tt_status tt_merge_topk(const int32_t* ids, const float* scores, int32_t parts, int32_t b, int32_t k_in,
+                        const int64_t* id_offsets, int32_t k_out, int32_t* out_ids, float* out_scores,
+                        void* stream) {
+    if (b < 0 || parts < 1 || k_in < 1 || k_out < 1) return TT_ERR_INVALID_ARG;
+    if (parts > TT_MAX_PARTS || k_in > TT_MAX_K) return TT_ERR_UNSUPPORTED;
+    if (k_out > k_in) return TT_ERR_INVALID_ARG;
+    if (id_offsets == nullptr) return TT_ERR_INVALID_ARG;
+    for (int p = 0; p < parts; ++p)
+        if (id_offsets[p] < 0 || id_offsets[p] >= ((int64_t)1 << 31)) return TT_ERR_INVALID_ARG;
+    if (b > 0 && (ids == nullptr || scores == nullptr || out_ids == nullptr || out_scores == nullptr))
+        return TT_ERR_INVALID_ARG;
+    if (!aligned(ids, 4) || !aligned(scores, 4) || !aligned(out_ids, 4) || !aligned(out_scores, 4))
+        return TT_ERR_INVALID_ARG;
+    if (b == 0) return TT_OK;
+    tt_status st;
+    if ((st = check_device_ptr(ids, "ids")) != TT_OK) return st;
+    if ((st = check_device_ptr(scores, "scores")) != TT_OK) return st;
+    if ((st = check_device_ptr(out_ids, "out_ids")) != TT_OK) return st;
+    if ((st = check_device_ptr(out_scores, "out_scores")) != TT_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t m = (int64_t)parts * k_in;
+    uint64_t* scratch = nullptr;
+    if (m > merge_smem_keys()) {
+        // keys of the lists that do not fit in shared memory, stream-ordered
+        TT_CUDA(cudaMallocAsync(reinterpret_cast<void**>(&scratch), (size_t)b * m * sizeof(uint64_t), s),
+                "merge scratch");
+    }
+    cudaError_t e = launch_merge(ids, scores, parts, b, k_in, id_offsets, k_out, scratch, out_ids,
+                                 out_scores, s);
+    if (scratch) cudaFreeAsync(scratch, s);
+    if (e != cudaSuccess) return cuda_fail(e, "merge");
+    return TT_OK;
+}
+
 tt_status tt_score_topk(tt_index* index, const void* queries, tt_dtype q_dtype, int32_t b,
                         const uint32_t* exclude_bits, float tau, int32_t k, int32_t* out_ids,
                         float* out_scores, void* stream) {

@@ -69,6 +69,13 @@ cudaError_t launch_select_threshold(const uint64_t* keys, uint32_t* count, int c
 cudaError_t launch_select_final(const uint64_t* keys, uint32_t* count, int cap, int b, int k,
                                 uint64_t* theta, float* thf, int32_t* status, int* flags,
                                 int repair, int32_t* out_ids, float* out_scores, cudaStream_t s);
+// Merge per-shard top-k lists (see k4_merge); id_offset_host: host array of
+// `parts` global-id offsets; scratch: b * parts * k_in keys when parts * k_in
+// exceeds merge_smem_keys(), else unused (may be null).
+cudaError_t launch_merge(const int32_t* ids, const float* scores, int parts, int b, int k_in,
+                         const int64_t* id_offset_host, int k_out, uint64_t* scratch, int32_t* out_ids,
+                         float* out_scores, cudaStream_t s);
+int merge_smem_keys();
 // Before a repair round: theta[q] = KEY_MAX where status[q] == 0; flags[0] = 0.
 cudaError_t launch_prepare_repair(uint64_t* theta, float* thf, const int32_t* status, int b,
                                   int* flags, cudaStream_t s);

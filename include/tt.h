@@ -63,6 +63,7 @@ typedef enum tt_norm_mode {
 /* Limits. */
 #define TT_MAX_D 512        /* d must be a multiple of 16 and at most 512 (f32 corpus: 256) */
 #define TT_MAX_K 2048       /* k at most 2048 */
+#define TT_MAX_PARTS 64     /* shards merged by one tt_merge_topk call */
 #define TT_MAX_N 2147483647 /* candidate ids are int32: n < 2^31 */
 
 /* Opaque handle describing a prepared corpus. Owned by the library; release
@@ -190,6 +191,38 @@ TT_API tt_status tt_last_stats(const tt_index* index, tt_stats* out);
  */
 TT_API tt_status tt_plan(int64_t n, int32_t k, const tt_options* options, int32_t* levels, int64_t* rows,
                   int64_t* strides, int32_t* ranks, int32_t* cap);
+
+/*
+ * tt_merge_topk - the top-k of a corpus split into row shards, from the
+ * shards' own top-k lists (e.g. one shard per GPU: tt_score_topk on each,
+ * then an all-gather of the lists, then this call on every GPU or on one).
+ *
+ * (recsys_two_tower_model.py `forward` shards the corpus over devices on the
+ *  `expert` axis and combines the per-device scores before `top_k_by_key`;
+ *  here only each shard's top-k crosses devices, and this call combines them.)
+ *
+ * ids, scores  device [parts, b, k_in] int32 / f32: part p's list for each
+ *              query, in tt_score_topk's output form (local ids within the
+ *              shard, sorted or not; id -1 = padding, ignored)
+ * parts        1 <= parts <= TT_MAX_PARTS
+ * b            queries, b >= 0
+ * k_in         entries per list, 1 <= k_in <= TT_MAX_K
+ * id_offsets   HOST [parts]: global id of the shard's local id 0 (>= 0);
+ *              local id + offset must stay below 2^31; shards must be
+ *              disjoint (equal global ids are not merged into one)
+ * k_out        1 <= k_out <= k_in: entries per query in the result
+ * out_ids,     device [b, k_out]: the k_out best (score, global id) of the
+ * out_scores   union, sorted by score descending then id ascending; padded
+ *              with (-1, -INFINITY). Equal to the single-corpus result when
+ *              every shard's list is that shard's exact top-k_in.
+ * stream       cudaStream_t; the call is asynchronous (no synchronisation)
+ *
+ * Errors: TT_ERR_INVALID_ARG (bad sizes, pointers, offsets),
+ * TT_ERR_UNSUPPORTED (parts or k beyond the limits), TT_ERR_CUDA.
+ */
+TT_API tt_status tt_merge_topk(const int32_t* ids, const float* scores, int32_t parts, int32_t b,
+                               int32_t k_in, const int64_t* id_offsets, int32_t k_out,
+                               int32_t* out_ids, float* out_scores, void* stream);
 
 /* Release a handle. Its scratch memory returns to a per-device pool that
  * later handles reuse (it is not returned to CUDA before the process exits).

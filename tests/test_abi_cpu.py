@@ -116,6 +116,26 @@ def test_host_validation_rejects_before_any_device_call():
     lib.tt_free(ixw)
 
 
+def test_merge_validation_before_device_calls():
+    lib = tt._lib
+    fake = ctypes.c_void_p(0x10000)
+    offs = (ctypes.c_int64 * 3)(0, 100, 200)
+    call = lambda **kw: lib.tt_merge_topk(kw.get("ids", fake), kw.get("sc", fake), kw.get("parts", 3),
+                                          kw.get("b", 4), kw.get("k_in", 10), kw.get("offs", offs),
+                                          kw.get("k_out", 10), fake, fake, None)
+    assert call(parts=0) == tt.TT_ERR_INVALID_ARG
+    assert call(parts=65) == tt.TT_ERR_UNSUPPORTED
+    assert call(k_in=4096, k_out=10) == tt.TT_ERR_UNSUPPORTED
+    assert call(k_out=11) == tt.TT_ERR_INVALID_ARG  # k_out > k_in
+    assert call(k_out=0) == tt.TT_ERR_INVALID_ARG
+    assert call(b=-1) == tt.TT_ERR_INVALID_ARG
+    assert call(offs=None) == tt.TT_ERR_INVALID_ARG
+    assert call(offs=(ctypes.c_int64 * 3)(0, -5, 10)) == tt.TT_ERR_INVALID_ARG
+    assert call(offs=(ctypes.c_int64 * 3)(0, 1 << 31, 10)) == tt.TT_ERR_INVALID_ARG
+    assert call(ids=ctypes.c_void_p(0x10002)) == tt.TT_ERR_INVALID_ARG  # misaligned
+    assert call(b=0) == tt.TT_OK
+
+
 def test_plan_levels():
     # the deepest level holds at most `cap` rows; strides are powers of 64
     for n, k in ((400, 10), (10 ** 6, 100), (10 ** 7, 500), (5 * 10 ** 7, 1000), (2 * 10 ** 7, 256),
