@@ -8,8 +8,8 @@
 // HBM-bound: every row is read once with 16-byte loads and written once with
 // 16-byte (or 8-byte) stores. L lanes of a warp share one row (L = 32 for
 // rows of >= 512 bytes), each lane keeping up to 4 chunks in registers, and
-// each warp works on two to four row groups at a time to keep enough bytes
-// in flight. fp32 arithmetic with IEEE sqrt and division; the result is rounded
+// each warp works on two to four row groups at a time, with the loads of the
+// next groups already issued, to keep enough bytes in flight. fp32 arithmetic with IEEE sqrt and division; the result is rounded
 // to the output type to nearest-even.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -103,21 +103,41 @@ __global__ void __launch_bounds__(K1_THREADS)
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const int64_t step = nwarps * (U * ROWS_PER_GROUP);
 
-    for (int64_t base = warp * (U * ROWS_PER_GROUP); base < n; base += step) {
+    // The loads of the next row groups are issued before the current ones
+    // are reduced, so each warp keeps two groups of loads in flight.
+    auto load_group = [&](int64_t gbase, uint4 (&dst)[U][CPL]) {
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t r = gbase + u * ROWS_PER_GROUP + grp;
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                const int c = sub + i * L;
+                if (r < n && c < chunks)
+                    dst[u][i] = ld_stream(in + r * d + (int64_t)c * E);
+                else
+                    dst[u][i] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+    };
+    // (Rows of 512 bytes and more, where the doubled registers fit: up to 4
+    // chunks per lane and group.)
+    constexpr bool PREFETCH = L == 32 && U * CPL <= 4;
+    uint4 nxt[U][CPL];
+    int64_t base = warp * (U * ROWS_PER_GROUP);
+    if (PREFETCH && base < n) load_group(base, nxt);
+    for (; base < n; base += step) {
         int64_t row[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) row[u] = base + u * ROWS_PER_GROUP + grp;
         uint4 raw[U][CPL];
+        if (PREFETCH) {
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
+            for (int u = 0; u < U; ++u)
 #pragma unroll
-            for (int i = 0; i < CPL; ++i) {
-                const int c = sub + i * L;
-                if (row[u] < n && c < chunks)
-                    raw[u][i] = ld_stream(in + row[u] * d + (int64_t)c * E);
-                else
-                    raw[u][i] = make_uint4(0u, 0u, 0u, 0u);
-            }
+                for (int i = 0; i < CPL; ++i) raw[u][i] = nxt[u][i];
+            if (base + step < n) load_group(base + step, nxt);
+        } else {
+            load_group(base, raw);
         }
         float ss[U];
 #pragma unroll
