@@ -71,6 +71,12 @@ class OracleLib:
         lib.oracle_topk.restype = ctypes.c_int
         lib.oracle_scores.argtypes = [vp, i32, i64, vp, i32, i32, vp, ctypes.c_double, vp, i64, vp]
         lib.oracle_scores.restype = None
+        lib.oracle_quantize_rows.argtypes = [vp, i32, i64, i32, i32, vp, vp]
+        lib.oracle_quantize_rows.restype = None
+        lib.oracle_topk_q8.argtypes = [vp, vp, i64, vp, vp, i64, i32, vp, ctypes.c_double, i64, vp, vp]
+        lib.oracle_topk_q8.restype = ctypes.c_int
+        lib.oracle_scores_q8.argtypes = [vp, vp, i64, vp, vp, i32, ctypes.c_double, vp, i64, vp]
+        lib.oracle_scores_q8.restype = None
         lib.oracle_set_threads.argtypes = [i32]
         lib.oracle_set_threads.restype = None
         lib.oracle_max_threads.argtypes = []
@@ -145,6 +151,45 @@ class OracleLib:
                                _ptr(ids), ids.shape[0], _ptr(out))
         return out
 
+    def quantize(self, rows: np.ndarray, normalise: bool):
+        """Symmetric per-row int8 codes in fp32 arithmetic: ``(codes int8
+        [n,d], scales float32 [n])``; with ``normalise`` the row is first
+        L2-normalised (fp64 norm, value held in fp32)."""
+        rows = _c2(rows)
+        codes = np.empty(rows.shape, dtype=np.int8)
+        scales = np.empty(rows.shape[0], dtype=np.float32)
+        self.lib.oracle_quantize_rows(_ptr(rows), _dtype_code(rows), rows.shape[0], rows.shape[1],
+                                      1 if normalise else 0, _ptr(codes), _ptr(scales))
+        return codes, scales
+
+    def topk_q8(self, qcodes: np.ndarray, qscales: np.ndarray, vcodes: np.ndarray, vscales: np.ndarray,
+                k: int, tau: float = 1.0, exclude: np.ndarray | None = None):
+        """Exact top-k of (sum q8 v8) * qscale * vscale / tau (fp64, every score sorted)."""
+        qcodes, vcodes = _c2(qcodes), _c2(vcodes)
+        assert qcodes.dtype == np.int8 and vcodes.dtype == np.int8
+        b, d = qcodes.shape
+        n = vcodes.shape[0]
+        qscales = np.ascontiguousarray(qscales, dtype=np.float32)
+        vscales = np.ascontiguousarray(vscales, dtype=np.float32)
+        if exclude is not None:
+            exclude = np.ascontiguousarray(exclude).view(np.uint32)
+        ids = np.empty((b, k), dtype=np.int32)
+        scores = np.empty((b, k), dtype=np.float64)
+        rc = self.lib.oracle_topk_q8(_ptr(qcodes), _ptr(qscales), b, _ptr(vcodes), _ptr(vscales), n, d,
+                                     _ptr(exclude), float(tau), int(k), _ptr(ids), _ptr(scores))
+        if rc != 0:
+            raise MemoryError("oracle_topk_q8 could not allocate its work buffer")
+        return ids, scores
+
+    def scores_for_q8(self, qcodes, qscales, qrow, vcodes, vscales, ids, tau=1.0) -> np.ndarray:
+        qcodes, vcodes = _c2(qcodes), _c2(vcodes)
+        ids = np.ascontiguousarray(ids, dtype=np.int64)
+        out = np.empty(ids.shape[0], dtype=np.float64)
+        self.lib.oracle_scores_q8(_ptr(qcodes), _ptr(np.ascontiguousarray(qscales, dtype=np.float32)),
+                                  int(qrow), _ptr(vcodes), _ptr(np.ascontiguousarray(vscales, dtype=np.float32)),
+                                  qcodes.shape[1], float(tau), _ptr(ids), ids.shape[0], _ptr(out))
+        return out
+
     def set_threads(self, n: int) -> None:
         self.lib.oracle_set_threads(int(n))
 
@@ -181,6 +226,18 @@ def topk(queries, corpus, k, tau=1.0, norms=None, exclude=None):
 
 def scores_for(queries, qrow, corpus, ids, tau=1.0, norms=None):
     return default().scores_for(queries, qrow, corpus, ids, tau=tau, norms=norms)
+
+
+def quantize(rows, normalise):
+    return default().quantize(rows, normalise)
+
+
+def topk_q8(qcodes, qscales, vcodes, vscales, k, tau=1.0, exclude=None):
+    return default().topk_q8(qcodes, qscales, vcodes, vscales, k, tau=tau, exclude=exclude)
+
+
+def scores_for_q8(qcodes, qscales, qrow, vcodes, vscales, ids, tau=1.0):
+    return default().scores_for_q8(qcodes, qscales, qrow, vcodes, vscales, ids, tau=tau)
 
 
 def set_threads(n):

@@ -26,6 +26,17 @@
  *     section, `Towers::top_k` (score every item, stable sort descending, take
  *     k: a stable sort keeps the lower index first on equal scores).
  *
+ * int8 scoring (recsys_two_tower_model.py `forward`, inner
+ * `compute_top_k_int8`): each query row u is quantised symmetrically in fp32,
+ * us = max(max_i |u_i| / 127, 1e-12), u8_i = clip(round(u_i / us), -127, 127)
+ * (round half to even), and the candidate rows arrive as int8 codes with one
+ * fp32 scale each; the score is the int32 dot product of the codes times
+ * us times the candidate's scale. The pages do not show how the candidate
+ * codes are made; they are taken to be the same scheme applied to the
+ * L2-normalised candidate row (held in fp32). Here the score is the fp64
+ * value of the dequantised vectors, (sum_i u8_i v8_ij) * us * scale_j / tau,
+ * whose integer sum is exact.
+ *
  * Storage rounding: where the corpus or the queries are stored in bf16 or
  * fp32, the fp64 normalised value is rounded once, to nearest with ties to
  * even, to the storage type (recsys_two_tower_model.py keeps the candidate
@@ -43,7 +54,9 @@
 
 #define ORACLE_F32 0
 #define ORACLE_BF16 1
+#define ORACLE_I8 2
 #define ORACLE_EPS 1e-12
+#define ORACLE_Q8_FLOOR 1e-12f
 
 /* ---- element access ---------------------------------------------------- */
 
@@ -59,6 +72,8 @@ static double load_elem(const void *base, int dtype, int64_t idx)
 {
     if (dtype == ORACLE_F32)
         return (double)((const float *)base)[idx];
+    if (dtype == ORACLE_I8)
+        return (double)((const int8_t *)base)[idx];
     return bf16_bits_to_double(((const uint16_t *)base)[idx]);
 }
 
@@ -128,6 +143,53 @@ void oracle_normalize(const void *in, int in_dtype, int64_t n, int d, void *out,
     }
 }
 
+/* ---- int8 quantisation -------------------------------------------------- */
+
+/* Symmetric per-row int8 codes, in fp32 arithmetic as written on the page:
+ * row values w_i (fp32), us = max(max|w_i| / 127, 1e-12),
+ * code_i = clip(round_half_even(w_i / us), -127, 127).
+ * normalise != 0: w_i = fl32(v_i / norm) with the fp64 norm of
+ * oracle_normalize (the L2-normalised candidate row held in fp32);
+ * normalise == 0: w_i = v_i as given (a query row). */
+void oracle_quantize_rows(const void *in, int in_dtype, int64_t n, int d, int normalise,
+                          int8_t *codes, float *scales)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < n; ++j) {
+        double norm = 1.0;
+        if (normalise) {
+            double ss = 0.0;
+            for (int i = 0; i < d; ++i) {
+                double x = load_elem(in, in_dtype, j * (int64_t)d + i);
+                ss += x * x;
+            }
+            norm = sqrt(ss > ORACLE_EPS ? ss : ORACLE_EPS);
+        }
+        float maxabs = 0.0f;
+        for (int i = 0; i < d; ++i) {
+            double x = load_elem(in, in_dtype, j * (int64_t)d + i);
+            float w = normalise ? (float)(x / norm) : (float)x;
+            float a = fabsf(w);
+            if (a > maxabs)
+                maxabs = a;
+        }
+        float us = maxabs / 127.0f;
+        if (us < ORACLE_Q8_FLOOR)
+            us = ORACLE_Q8_FLOOR;
+        scales[j] = us;
+        for (int i = 0; i < d; ++i) {
+            double x = load_elem(in, in_dtype, j * (int64_t)d + i);
+            float w = normalise ? (float)(x / norm) : (float)x;
+            float r = rintf(w / us); /* nearest, ties to even */
+            if (r > 127.0f)
+                r = 127.0f;
+            if (r < -127.0f)
+                r = -127.0f;
+            codes[j * (int64_t)d + i] = (int8_t)r;
+        }
+    }
+}
+
 /* ---- scoring and top-k ------------------------------------------------- */
 
 static int is_excluded(const uint32_t *exclude, int64_t j)
@@ -137,9 +199,11 @@ static int is_excluded(const uint32_t *exclude, int64_t j)
     return (int)((exclude[j >> 5] >> (j & 31)) & 1u);
 }
 
-/* s = (q . v_j) [/ norm_j] / tau, summed in index order. */
+/* s = (q . v_j) [/ norm_j] [* qscale_q * vscale_j] / tau, summed in index
+ * order (for int8 codes every partial sum is an exact integer). */
 static double score_one(const void *q, int q_dtype, int64_t qrow, const void *v, int v_dtype,
-                        int64_t j, int d, const double *norms, double tau)
+                        int64_t j, int d, const double *norms, const float *qscales,
+                        const float *vscales, double tau)
 {
     double dot = 0.0;
     for (int i = 0; i < d; ++i)
@@ -147,6 +211,8 @@ static double score_one(const void *q, int q_dtype, int64_t qrow, const void *v,
                load_elem(v, v_dtype, j * (int64_t)d + i);
     if (norms)
         dot = dot / norms[j];
+    if (qscales)
+        dot = dot * (double)qscales[qrow] * (double)vscales[j];
     return dot / tau;
 }
 
@@ -174,9 +240,10 @@ static int cmp_pair(const void *pa, const void *pb)
 /* For each of the b queries: score every eligible candidate, sort all of
  * them, keep the first k. out_ids [b,k] (int32), out_scores [b,k] (fp64).
  * Returns 0, or -1 if a work buffer could not be allocated. */
-int oracle_topk(const void *q, int q_dtype, int64_t b, const void *v, int v_dtype, int64_t n,
-                int d, const double *norms, const uint32_t *exclude, double tau, int64_t k,
-                int32_t *out_ids, double *out_scores)
+static int topk_impl(const void *q, int q_dtype, int64_t b, const void *v, int v_dtype, int64_t n,
+                     int d, const double *norms, const float *qscales, const float *vscales,
+                     const uint32_t *exclude, double tau, int64_t k, int32_t *out_ids,
+                     double *out_scores)
 {
     int failed = 0;
 #pragma omp parallel for schedule(dynamic, 1)
@@ -191,7 +258,7 @@ int oracle_topk(const void *q, int q_dtype, int64_t b, const void *v, int v_dtyp
         for (int64_t j = 0; j < n; ++j) {
             if (is_excluded(exclude, j))
                 continue;
-            pairs[m].s = score_one(q, q_dtype, qi, v, v_dtype, j, d, norms, tau);
+            pairs[m].s = score_one(q, q_dtype, qi, v, v_dtype, j, d, norms, qscales, vscales, tau);
             pairs[m].id = j;
             ++m;
         }
@@ -210,13 +277,38 @@ int oracle_topk(const void *q, int q_dtype, int64_t b, const void *v, int v_dtyp
     return failed ? -1 : 0;
 }
 
+int oracle_topk(const void *q, int q_dtype, int64_t b, const void *v, int v_dtype, int64_t n,
+                int d, const double *norms, const uint32_t *exclude, double tau, int64_t k,
+                int32_t *out_ids, double *out_scores)
+{
+    return topk_impl(q, q_dtype, b, v, v_dtype, n, d, norms, NULL, NULL, exclude, tau, k, out_ids,
+                     out_scores);
+}
+
+/* Top-k over int8 codes: s = (sum_i q8_i v8_ji) * qscales[q] * vscales[j] / tau. */
+int oracle_topk_q8(const int8_t *q, const float *qscales, int64_t b, const int8_t *v,
+                   const float *vscales, int64_t n, int d, const uint32_t *exclude, double tau,
+                   int64_t k, int32_t *out_ids, double *out_scores)
+{
+    return topk_impl(q, ORACLE_I8, b, v, ORACLE_I8, n, d, NULL, qscales, vscales, exclude, tau, k,
+                     out_ids, out_scores);
+}
+
 /* Scores of listed candidates for one query: out[t] = s(qrow, ids[t]). */
 void oracle_scores(const void *q, int q_dtype, int64_t qrow, const void *v, int v_dtype, int d,
                    const double *norms, double tau, const int64_t *ids, int64_t count,
                    double *out)
 {
     for (int64_t t = 0; t < count; ++t)
-        out[t] = score_one(q, q_dtype, qrow, v, v_dtype, ids[t], d, norms, tau);
+        out[t] = score_one(q, q_dtype, qrow, v, v_dtype, ids[t], d, norms, NULL, NULL, tau);
+}
+
+void oracle_scores_q8(const int8_t *q, const float *qscales, int64_t qrow, const int8_t *v,
+                      const float *vscales, int d, double tau, const int64_t *ids, int64_t count,
+                      double *out)
+{
+    for (int64_t t = 0; t < count; ++t)
+        out[t] = score_one(q, ORACLE_I8, qrow, v, ORACLE_I8, ids[t], d, NULL, qscales, vscales, tau);
 }
 
 /* ---- threading ---------------------------------------------------------- */

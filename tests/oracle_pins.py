@@ -5,7 +5,8 @@ a mismatch. ``test_oracle_pins.py`` runs them against the oracle as built;
 ``test_oracle_mutants.py`` runs them against copies of ``oracle.c`` with one
 planted mistake each and expects every copy to fail at least one check.
 
-The pins are: hand-worked closed forms (``golden/hand_worked.json``), the
+The pins are: hand-worked closed forms (``golden/hand_worked.json``, H1-H3
+for the fp path, H5-H7 for int8 coding and scoring), the
 rank characterisation of top-k evaluated in exact rational arithmetic on tiny
 inputs, fp32 -> bf16 rounding by an independent library routine, and
 invariants that any correct implementation satisfies (unit norms, scaling by
@@ -304,7 +305,98 @@ def check_bf16_inputs(o):
     assert np.allclose(scores[0], [1.0, 0.8017837257372732, 0.5], rtol=1e-12)
 
 
+def _check_quantize_golden(o, g):
+    rows = np.array(g["rows"], dtype=np.float32)
+    codes, scales = o.quantize(rows, g["normalise"])
+    assert codes.tolist() == g["expected_codes"], (codes, g["expected_codes"])
+    for s, want in zip(scales.tolist(), g["expected_scales"]):
+        assert abs(s - want) <= g["scale_rel_tol"] * abs(want) + 1e-30, (s, want)
+
+
+def check_h5_quantize(o):
+    _check_quantize_golden(o, golden()["H5_quantize"])
+
+
+def check_h6_quantize_ties(o):
+    _check_quantize_golden(o, golden()["H6_quantize_ties"])
+
+
+def check_h7_int8_score(o):
+    g = golden()["H7_int8_score"]
+    vc, vs = o.quantize(np.array(g["corpus_raw"], dtype=np.float32), True)
+    qc, qs = o.quantize(np.array([g["query"]], dtype=np.float32), False)
+    ids, scores = o.topk_q8(qc, qs, vc, vs, g["k"], tau=g["tau"])
+    assert ids[0].tolist() == g["expected_ids"]
+    for s, want in zip(scores[0].tolist(), g["expected_scores"]):
+        assert abs(s - want) <= g["rel_tol"] * abs(want) + 1e-12, (s, want)
+    # the listed-candidate scorer agrees
+    s2 = o.scores_for_q8(qc, qs, 0, vc, vs, [2, 0], tau=g["tau"])
+    assert s2.tolist() == [scores[0, 2], scores[0, 0]]
+
+
+def check_quantize_invariants(o):
+    """Codes stay in [-127, 127]; a non-zero row reaches 127 in magnitude; each
+    dequantised value is within half a scale step of the fp32 row value it
+    codes; signs agree; the scale is max|w| / 127 to fp32 rounding; a power of
+    two times a row (not normalised) keeps the codes and scales the scale."""
+    rng = np.random.default_rng(17)
+    for d in (16, 64, 128, 256):
+        x = (rng.standard_normal((80, d)) * rng.lognormal(0, 1, (80, 1))).astype(np.float32)
+        for normalise in (False, True):
+            codes, scales = o.quantize(x, normalise)
+            assert codes.dtype == np.int8 and np.abs(codes.astype(np.int32)).max() <= 127
+            assert (np.abs(codes.astype(np.int32)).max(axis=1) == 127).all()
+            w = x.astype(np.float64)
+            if normalise:
+                w = w / np.sqrt(np.maximum((w * w).sum(axis=1, keepdims=True), 1e-12))
+            w32 = w.astype(np.float32).astype(np.float64)
+            maxabs = np.abs(w32).max(axis=1)
+            assert np.allclose(scales, maxabs / 127, rtol=2.4e-7, atol=0)
+            deq = codes.astype(np.float64) * scales.astype(np.float64)[:, None]
+            assert (np.abs(deq - w32) <= 0.5 * scales.astype(np.float64)[:, None] * (1 + 2e-5)).all()
+            nz = codes != 0
+            assert (np.sign(codes[nz]) == np.sign(w32[nz])).all()
+        c1, s1 = o.quantize(x, False)
+        c2, s2 = o.quantize((x * 8).astype(np.float32), False)
+        assert (c1 == c2).all() and np.allclose(s2, s1 * 8, rtol=0, atol=0)
+        # normalising first makes the codes independent of the row's length
+        c3, _ = o.quantize((x * 8).astype(np.float32), True)
+        c4, _ = o.quantize(x, True)
+        assert (c3 == c4).all()
+
+
+def check_int8_topk_invariants(o):
+    """The int8 top-k is the top-k of the dequantised vectors' dot products:
+    compared with the fp64 top-k of (codes * scale) rows, and 1/tau only scales."""
+    rng = np.random.default_rng(23)
+    n, d, b, k = 400, 32, 5, 25
+    V = rng.standard_normal((n, d)).astype(np.float32)
+    Q = rng.standard_normal((b, d)).astype(np.float32)
+    vc, vs = o.quantize(V, True)
+    qc, qs = o.quantize(Q, False)
+    ids, scores = o.topk_q8(qc, qs, vc, vs, k)
+    deq_v = (vc.astype(np.float64) * vs.astype(np.float64)[:, None])
+    deq_q = (qc.astype(np.float64) * qs.astype(np.float64)[:, None])
+    full = deq_q @ deq_v.T
+    for q in range(b):
+        order = sorted(range(n), key=lambda j: (-full[q, j], j))[:k]
+        assert ids[q].tolist() == order
+        assert np.allclose(scores[q], full[q, order], rtol=1e-12, atol=1e-15)
+    ids2, scores2 = o.topk_q8(qc, qs, vc, vs, k, tau=0.25)
+    assert (ids2 == ids).all() and np.allclose(scores2, scores * 4, rtol=1e-15)
+    # exclusion removes exactly the excluded ids
+    ex = np.zeros(n, dtype=bool)
+    ex[ids[:, 0]] = True
+    ids3, _ = o.topk_q8(qc, qs, vc, vs, k, exclude=pack_bits(ex))
+    assert not np.isin(ids3, np.nonzero(ex)[0]).any()
+
+
 ALL_CHECKS = [
+    check_h5_quantize,
+    check_h6_quantize_ties,
+    check_h7_int8_score,
+    check_quantize_invariants,
+    check_int8_topk_invariants,
     check_bf16_rounding,
     check_bf16_inputs,
     check_h1_normalize,

@@ -1,6 +1,6 @@
 """Planted mistakes: each copy of oracle.c below carries one plausible bug
 (a dropped term, a wrong sign, index or operand, a misplaced floor, a broken
-tie rule or rounding). Every copy must fail at least one pin; a copy that
+tie rule or rounding, in the fp path and in int8 coding and scoring). Every copy must fail at least one pin; a copy that
 passes them all would show a gap in the pins. CPU only; the copies are built
 in a temporary directory and never touch the real oracle."""
 import os
@@ -32,6 +32,15 @@ MUTANTS = {
     "bf16_one_bit_short": ("ldexp(1.0, lead - 7)", "ldexp(1.0, lead - 6)"),
     "bf16_load_shift": ("(uint32_t)h << 16", "(uint32_t)h << 15"),
     "pad_score_zero": ("out_scores[qi * k + r] = -INFINITY;", "out_scores[qi * k + r] = 0.0;"),
+    # int8 coding and scoring
+    "q8_scale_over_128": ("maxabs / 127.0f", "maxabs / 128.0f"),
+    "q8_round_half_away": ("rintf(w / us)", "roundf(w / us)"),
+    "q8_truncate": ("rintf(w / us)", "truncf(w / us)"),
+    "q8_scale_floor_missing": ("if (us < ORACLE_Q8_FLOOR)\n            us = ORACLE_Q8_FLOOR;", ""),
+    "q8_not_normalised": ("float w = normalise ? (float)(x / norm) : (float)x;", "float w = (float)x;"),
+    "q8_row_scale_dropped": ("dot = dot * (double)qscales[qrow] * (double)vscales[j];",
+                             "dot = dot * (double)qscales[qrow];"),
+    "q8_code_sign_lost": ("codes[j * (int64_t)d + i] = (int8_t)r;", "codes[j * (int64_t)d + i] = (int8_t)fabsf(r);"),
 }
 
 
