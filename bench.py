@@ -107,9 +107,12 @@ def elem_bytes(name):
     return {"f32": 4, "bf16": 2}[name]
 
 
-def work_model(w: W.Workload, plan: dict):
+def work_model(w: W.Workload, plan: dict, int8: bool = False):
     s_in = elem_bytes(w.raw_dtype)
-    if w.store == "raw":
+    if int8:  # normalise + code: read the raw rows, write codes and one scale per row
+        k1_bytes = w.n * w.d * s_in + w.n * w.d + w.n * 4
+        s_corpus = 1
+    elif w.store == "raw":
         k1_bytes = w.n * w.d * s_in + w.n * 4
         s_corpus = s_in
     else:
@@ -117,7 +120,7 @@ def work_model(w: W.Workload, plan: dict):
         k1_bytes = w.n * w.d * (s_in + s_out)
         s_corpus = s_out
     rows_scanned = sum(plan["rows"])
-    per_row = w.d * s_corpus + (4 if w.store == "raw" else 0)
+    per_row = w.d * s_corpus + (4 if (w.store == "raw" or int8) else 0)
     score_bytes = rows_scanned * per_row + (w.n // 8 if w.masked else 0)
     score_flops = 2.0 * w.b * w.d * rows_scanned
     return {"k1_bytes": k1_bytes, "score_bytes": score_bytes, "score_flops": score_flops,
@@ -288,7 +291,12 @@ def run_ours(args, world, rank, local):
         excl = shard.exclude_slice(excl, start, count)
         torch.cuda.empty_cache()
         w = dataclasses.replace(w, n=count)
-    if w.store == "raw":
+    int8 = args.quant == "int8"
+    if int8:
+        prepared = torch.empty((w.n, w.d), dtype=torch.int8, device=dev)
+        scales = torch.empty((w.n,), dtype=torch.float32, device=dev)
+        mode = None
+    elif w.store == "raw":
         prepared = torch.empty((w.n,), dtype=torch.float32, device=dev)
         mode = tt.TT_NORM_FUSED
     else:
@@ -304,13 +312,19 @@ def run_ours(args, world, rank, local):
 
     # The index handle refers to `prepared`; every step rewrites `prepared`
     # from the raw corpus, so one handle (and its scratch) serves all steps.
-    index = tt.tt_normalize_candidates(raw_c, prepared, mode)
+    if int8:
+        index = tt.tt_quantize_candidates(raw_c, prepared, scales)
+    else:
+        index = tt.tt_normalize_candidates(raw_c, prepared, mode)
 
     def step(record_k1=False):
         if record_k1:
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-        tt.tt_normalize_candidates(raw_c, prepared, mode, make_index=False)
+        if int8:
+            tt.tt_quantize_candidates(raw_c, prepared, scales, make_index=False)
+        else:
+            tt.tt_normalize_candidates(raw_c, prepared, mode, make_index=False)
         if record_k1:
             e1.record(stream)
             ev_k1.append((e0, e1))
@@ -357,16 +371,20 @@ def run_ours(args, world, rank, local):
 
     # ---- roofline of the dominant kernel ----
     peaks, peak_src = load_peaks()
-    work = work_model(w, plan)
+    work = work_model(w, plan, int8)
+    # int8 contraction: the bf16 measured peak times the nominal int8 / bf16 ratio (4.5 / 2.25)
+    tensor_peak = peaks["bf16_tflops_sustained"] * (2.0 if int8 else 1.0)
+    peak_note = " (sustained bf16 x 2, the nominal int8 ratio)" if int8 else " (sustained bf16)"
     k1_ms = sum(a.elapsed_time(b) for a, b in ev_k1) / max(1, len(ev_k1))
     score_kind = "tensor" if stats["path"] >= 2 else "stream"
     score_kernel = {1: "k2_stream", 2: "k3_tensor", 3: "k3_pair"}[stats["path"]]
     score_ms = prof[score_kind]["ms"] / args.steps
     if k1_ms >= score_ms:
-        dom = {"kernel": "k1_normalize (corpus)", "bound": "hbm", "ms": k1_ms, "bytes": work["k1_bytes"],
+        dom = {"kernel": "k1_normalize (corpus" + (", int8 codes)" if int8 else ")"), "bound": "hbm", "ms": k1_ms,
+               "bytes": work["k1_bytes"],
                "launches_per_step": 1}
     else:
-        t_flops = work["score_flops"] / (peaks["bf16_tflops_sustained"] * 1e12)
+        t_flops = work["score_flops"] / (tensor_peak * 1e12)
         t_bytes = work["score_bytes"] / (peaks["hbm_gbs"] * 1e9)
         bound = "tensor" if (stats["path"] >= 2 and t_flops > t_bytes) else "hbm"
         dom = {"kernel": f"{score_kernel} (all levels)", "bound": bound,
@@ -378,14 +396,16 @@ def run_ours(args, world, rank, local):
                 "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None}
     else:
         achieved = dom["flops"] / (dom["ms"] / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peaks["bf16_tflops_sustained"],
-                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops_sustained"], 4), "traffic": None}
-    if dom["kernel"].startswith("k1"):
+        roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": tensor_peak,
+                "unit": "TOP/s" if int8 else "TFLOP/s", "frac": round(achieved / tensor_peak, 4), "traffic": None}
+    if int8:
+        roof["traffic"] = None  # no capture recorded for the int8 kernels
+    elif dom["kernel"].startswith("k1"):
         roof["traffic"] = recorded_traffic("k1_normalize", w.name, w.n)
     else:
         roof["traffic"] = recorded_traffic(score_kernel, w.name, work["rows_scanned"])
     roof["kernel"] = dom["kernel"]
-    roof["peak_source"] = peak_src + (" (sustained bf16)" if roof["bound"] == "tensor" else " (copy)")
+    roof["peak_source"] = peak_src + (peak_note if roof["bound"] == "tensor" else " (copy)")
     roof["kernel_ms"] = round(dom["ms"], 5)
 
     kernels = {k: {"ms_per_step": round(v["ms"] / args.steps, 5), "launches_per_step": v["launches"] / args.steps}
@@ -421,10 +441,11 @@ def run_ours(args, world, rank, local):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
         "scaling": "strong" if sharded else "weak", "vs_baseline": None,
-        "dtype": "bf16" if w.store != "f32" else "f32",
+        "dtype": "i8" if int8 else ("bf16" if w.store != "f32" else "f32"),
         "data": "synthetic (seeded, workloads.py)",
         "config": {"workload": w.name, "n": w_all.n, "d": w.d, "b": w.b, "k": w.k, "tau": w.tau,
-                   "corpus_raw": w.raw_dtype, "corpus_store": w.store, "queries": w.query_dtype,
+                   "corpus_raw": w.raw_dtype, "corpus_store": "i8 codes + f32 scales" if int8 else w.store,
+                   "queries": w.query_dtype,
                    "mask_rate": w.mask_rate, "l2": "inputs larger than L2 (raw corpus "
                    f"{w.n * w.d * elem_bytes(w.raw_dtype) / 1e6:.0f} MB > 126 MB)",
                    "path": PATH_NAMES[stats["path"]], "levels": plan["rows"],
@@ -485,6 +506,8 @@ def main():
     ap.add_argument("--k", type=int, default=0, help="override the workload's k")
     ap.add_argument("--path", type=int, default=0, choices=[0, 1, 2, 3],
                     help="scorer: 0 auto, 1 streaming, 2 tensor-core, 3 tensor-core on SM pairs")
+    ap.add_argument("--quant", default="none", choices=["none", "int8"],
+                    help="int8: code the normalised corpus in int8 and score int8 codes (tensor cores kind::i8)")
     ap.add_argument("--mode", default="replicas", choices=["replicas", "shard"],
                     help="N > 1: independent replicas (default) or one corpus sharded by rows over the ranks")
     ap.add_argument("--no-e2e", action="store_true")

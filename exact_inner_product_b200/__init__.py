@@ -32,6 +32,7 @@ TT_ERR_INTERNAL = 6
 
 TT_F32 = 0
 TT_BF16 = 1
+TT_I8 = 2
 TT_NORM_STORE = 0
 TT_NORM_FUSED = 1
 TT_MAX_D = 512
@@ -72,6 +73,7 @@ def _sig(name, res, args):
 _sig("tt_normalize_candidates", ctypes.c_int, [_vp, ctypes.c_int, _i64, _i32, _vp, ctypes.c_int, _i32, _vp,
                                                ctypes.POINTER(_vp)])
 _sig("tt_index_wrap", ctypes.c_int, [_vp, ctypes.c_int, _i64, _i32, _vp, ctypes.POINTER(_vp)])
+_sig("tt_quantize_candidates", ctypes.c_int, [_vp, ctypes.c_int, _i64, _i32, _vp, _vp, _vp, ctypes.POINTER(_vp)])
 _sig("tt_score_topk", ctypes.c_int, [_vp, _vp, ctypes.c_int, _i32, _vp, ctypes.c_float, _i32, _vp, _vp,
                                      _vp])
 _sig("tt_score_topk_ex", ctypes.c_int, [_vp, _vp, ctypes.c_int, _i32, _vp, ctypes.c_float, _i32, _vp,
@@ -93,7 +95,7 @@ _sig("tt_status_string", ctypes.c_char_p, [ctypes.c_int])
 _sig("tt_last_error", ctypes.c_char_p, [])
 _sig("tt_version", ctypes.c_char_p, [])
 
-EXPORTED = ("tt_normalize_candidates", "tt_index_wrap", "tt_score_topk", "tt_score_topk_ex",
+EXPORTED = ("tt_normalize_candidates", "tt_quantize_candidates", "tt_index_wrap", "tt_score_topk", "tt_score_topk_ex",
             "tt_score_topk_noalloc", "tt_merge_topk",
             "tt_last_stats", "tt_plan", "tt_free", "tt_launch_count", "tt_profile_begin",
             "tt_profile_end", "tt_profile_launches", "tt_status_string", "tt_last_error", "tt_version")
@@ -117,7 +119,9 @@ def _dtype(t: torch.Tensor) -> int:
         return TT_F32
     if t.dtype == torch.bfloat16:
         return TT_BF16
-    raise TypeError(f"tensors must be float32 or bfloat16, got {t.dtype}")
+    if t.dtype == torch.int8:
+        return TT_I8
+    raise TypeError(f"tensors must be float32, bfloat16 or int8 (codes), got {t.dtype}")
 
 
 def _ptr(t):
@@ -179,6 +183,25 @@ def tt_normalize_candidates(x: torch.Tensor, out: torch.Tensor, mode: int = TT_N
     if mode == TT_NORM_STORE:
         return Index(handle.value, out, None, n, d)
     return Index(handle.value, x, out, n, d)
+
+
+def tt_quantize_candidates(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, stream=None,
+                           make_index: bool = True) -> Index | None:
+    """L2-normalise each row and code it in int8 with one scale per row
+    (``tt_quantize_candidates``). ``x``: [n, d] float32/bfloat16 on the GPU;
+    ``codes``: [n, d] int8; ``scales``: [n] float32. Returns an int8 ``Index``
+    (or None when ``make_index`` is False)."""
+    if x.dim() != 2 or not x.is_contiguous() or not codes.is_contiguous() or not scales.is_contiguous():
+        raise ValueError("x, codes and scales must be contiguous")
+    if codes.dtype != torch.int8 or scales.dtype != torch.float32:
+        raise TypeError("codes must be int8 and scales float32")
+    n, d = x.shape
+    handle = ctypes.c_void_p()
+    _check(_lib.tt_quantize_candidates(_ptr(x), _dtype(x), n, d, _ptr(codes), _ptr(scales), _stream(stream),
+                                       ctypes.byref(handle) if make_index else None), "tt_quantize_candidates")
+    if not make_index:
+        return None
+    return Index(handle.value, codes, scales, n, d)
 
 
 def tt_index_wrap(rows: torch.Tensor, inv_norm: torch.Tensor | None = None) -> Index:
@@ -336,8 +359,10 @@ def search(corpus: torch.Tensor, queries: torch.Tensor, k: int, tau: float = 1.0
 
     ``corpus`` [n, d] and ``queries`` [b, d] are CPU tensors (pinned memory
     makes the copies asynchronous). ``fused`` keeps the corpus raw and folds
-    the norms into the scores. ``query_dtype`` defaults to float32 for small
-    batches (b <= 8) and bfloat16 otherwise."""
+    the norms into the scores; ``store_dtype=torch.int8`` codes the
+    normalised corpus in int8 (``tt_quantize_candidates``) and scores with
+    int8 codes. ``query_dtype`` defaults to float32 for small batches
+    (b <= 8) and bfloat16 otherwise."""
     n, d = corpus.shape
     b = queries.shape[0]
     dc = corpus.to(device, non_blocking=True)
@@ -346,6 +371,10 @@ def search(corpus: torch.Tensor, queries: torch.Tensor, k: int, tau: float = 1.0
     if fused:
         inv = torch.empty((n,), dtype=torch.float32, device=device)
         index = tt_normalize_candidates(dc, inv, TT_NORM_FUSED)
+    elif store_dtype == torch.int8:
+        codes = torch.empty((n, d), dtype=torch.int8, device=device)
+        scales = torch.empty((n,), dtype=torch.float32, device=device)
+        index = tt_quantize_candidates(dc, codes, scales)
     else:
         rows = torch.empty((n, d), dtype=store_dtype, device=device)
         index = tt_normalize_candidates(dc, rows, TT_NORM_STORE)

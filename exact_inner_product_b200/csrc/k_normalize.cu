@@ -86,7 +86,28 @@ __device__ __forceinline__ void store_chunk<__nv_bfloat16, 8>(__nv_bfloat16* row
                    pack_bf16x2(y[6], y[7]));
 }
 
+// Store E int8 codes at element offset e0 of the row.
+template <int E>
+__device__ __forceinline__ void store_codes(int8_t* row_out, int e0, const int* q);
+template <>
+__device__ __forceinline__ void store_codes<4>(int8_t* row_out, int e0, const int* q) {
+    const uint32_t w = (uint32_t)(q[0] & 0xFF) | ((uint32_t)(q[1] & 0xFF) << 8) |
+                       ((uint32_t)(q[2] & 0xFF) << 16) | ((uint32_t)(q[3] & 0xFF) << 24);
+    *reinterpret_cast<uint32_t*>(row_out + e0) = w;
+}
+template <>
+__device__ __forceinline__ void store_codes<8>(int8_t* row_out, int e0, const int* q) {
+    uint32_t w[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+        w[h] = (uint32_t)(q[4 * h] & 0xFF) | ((uint32_t)(q[4 * h + 1] & 0xFF) << 8) |
+               ((uint32_t)(q[4 * h + 2] & 0xFF) << 16) | ((uint32_t)(q[4 * h + 3] & 0xFF) << 24);
+    *reinterpret_cast<uint2*>(row_out + e0) = make_uint2(w[0], w[1]);
+}
+
 // MODE 0: out rows = v / norm (Tout). MODE 1: inv_norm[j] = 1 / norm.
+// MODE 2: w = v / norm, then int8 codes of w to out (Tout = int8_t) and the
+// row's scale to inv_norm. MODE 3: the same coding of v as given (queries).
 // L lanes per row, CPL 16-byte chunks per lane (d * elem <= 2048 bytes),
 // U row groups per warp in flight at once.
 template <typename Tin, typename Tout, int MODE, int L, int CPL, int U>
@@ -156,22 +177,71 @@ __global__ void __launch_bounds__(K1_THREADS)
 #pragma unroll
             for (int u = 0; u < U; ++u) ss[u] += __shfl_xor_sync(0xFFFFFFFFu, ss[u], off);
         }
+        if constexpr (MODE >= 2) {
+            // int8 coding (recsys_two_tower_model.py `compute_top_k_int8`):
+            // scale = max(max|w| / 127, 1e-12), code = clip(round(w / scale)),
+            // round half to even, in fp32 as written there.
+            // The row values w are computed once (one IEEE division each when
+            // normalising) and kept in registers for the coding pass.
+            float mx[U];
+            float wv[U][CPL][E];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            if (row[u] >= n) continue;
-            const float norm = __fsqrt_rn(fmaxf(ss[u], 1e-12f));
-            if (MODE == 1) {
-                if (sub == 0) inv_norm[row[u]] = __fdiv_rn(1.0f, norm);
-            } else {
+            for (int u = 0; u < U; ++u) {
+                const float norm = MODE == 2 ? __fsqrt_rn(fmaxf(ss[u], 1e-12f)) : 1.0f;
+                mx[u] = 0.f;
+#pragma unroll
+                for (int i = 0; i < CPL; ++i) {
+                    float x[E];
+                    Elem<Tin>::unpack(raw[u][i], x);
+#pragma unroll
+                    for (int e = 0; e < E; ++e) {
+                        wv[u][i][e] = MODE == 2 ? __fdiv_rn(x[e], norm) : x[e];
+                        mx[u] = fmaxf(mx[u], fabsf(wv[u][i][e]));
+                    }
+                }
+            }
+#pragma unroll
+            for (int off = L / 2; off > 0; off >>= 1) {
+#pragma unroll
+                for (int u = 0; u < U; ++u) mx[u] = fmaxf(mx[u], __shfl_xor_sync(0xFFFFFFFFu, mx[u], off));
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (row[u] >= n) continue;
+                const float scale = fmaxf(__fdiv_rn(mx[u], 127.0f), 1e-12f);
+                if (sub == 0) inv_norm[row[u]] = scale;
 #pragma unroll
                 for (int i = 0; i < CPL; ++i) {
                     const int c = sub + i * L;
                     if (c < chunks) {
-                        float x[E], y[E];
-                        Elem<Tin>::unpack(raw[u][i], x);
+                        int q[E];
 #pragma unroll
-                        for (int e = 0; e < E; ++e) y[e] = __fdiv_rn(x[e], norm);
-                        store_chunk<Tout, E>(out + row[u] * d, c * E, y);
+                        for (int e = 0; e < E; ++e) {
+                            const float r = fminf(fmaxf(rintf(__fdiv_rn(wv[u][i][e], scale)), -127.f), 127.f);
+                            q[e] = (int)r;
+                        }
+                        store_codes<E>(reinterpret_cast<int8_t*>(out) + row[u] * d, c * E, q);
+                    }
+                }
+            }
+        } else {
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (row[u] >= n) continue;
+                const float norm = __fsqrt_rn(fmaxf(ss[u], 1e-12f));
+                if constexpr (MODE == 1) {
+                    if (sub == 0) inv_norm[row[u]] = __fdiv_rn(1.0f, norm);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < CPL; ++i) {
+                        const int c = sub + i * L;
+                        if (c < chunks) {
+                            float x[E], y[E];
+                            Elem<Tin>::unpack(raw[u][i], x);
+#pragma unroll
+                            for (int e = 0; e < E; ++e) y[e] = __fdiv_rn(x[e], norm);
+                            store_chunk<Tout, E>(out + row[u] * d, c * E, y);
+                        }
                     }
                 }
             }
@@ -188,7 +258,7 @@ __global__ void k0_cast_bf16(const float4* __restrict__ in, int64_t count4, uint
 }
 
 template <typename Tin, typename Tout, int MODE>
-cudaError_t dispatch_lanes(const void* in, int64_t n, int d, void* out, cudaStream_t s) {
+cudaError_t dispatch_lanes(const void* in, int64_t n, int d, void* out, cudaStream_t s, void* aux = nullptr) {
     constexpr int E = Elem<Tin>::per_chunk;
     const int chunks = d / E;
     int L = 32;
@@ -204,8 +274,8 @@ cudaError_t dispatch_lanes(const void* in, int64_t n, int d, void* out, cudaStre
     if (blocks > max_blocks) blocks = max_blocks;
     if (blocks < 1) blocks = 1;
     const Tin* pin = static_cast<const Tin*>(in);
-    Tout* pout = MODE == 0 ? static_cast<Tout*>(out) : nullptr;
-    float* pinv = MODE == 1 ? static_cast<float*>(out) : nullptr;
+    Tout* pout = (MODE == 0 || MODE >= 2) ? static_cast<Tout*>(out) : nullptr;
+    float* pinv = MODE == 1 ? static_cast<float*>(out) : static_cast<float*>(aux);
     note_launch_begin(TT_KIND_NORMALIZE, s);
     const dim3 g((unsigned)blocks), t(K1_THREADS);
     if (L == 32 && cpl == 1) k1_normalize<Tin, Tout, MODE, 32, 1, 4><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
@@ -232,6 +302,16 @@ cudaError_t launch_normalize(const void* in, int in_dtype, int64_t n, int d, voi
     if (mode == TT_NORM_FUSED) return dispatch_lanes<__nv_bfloat16, float, 1>(in, n, d, out, s);
     if (out_dtype == TT_F32) return dispatch_lanes<__nv_bfloat16, float, 0>(in, n, d, out, s);
     return dispatch_lanes<__nv_bfloat16, __nv_bfloat16, 0>(in, n, d, out, s);
+}
+
+cudaError_t launch_quantize(const void* in, int in_dtype, int64_t n, int d, int8_t* codes, float* scales,
+                            bool normalise, cudaStream_t s) {
+    if (n == 0) return cudaSuccess;
+    if (in_dtype == TT_F32)
+        return normalise ? dispatch_lanes<float, int8_t, 2>(in, n, d, codes, s, scales)
+                         : dispatch_lanes<float, int8_t, 3>(in, n, d, codes, s, scales);
+    return normalise ? dispatch_lanes<__nv_bfloat16, int8_t, 2>(in, n, d, codes, s, scales)
+                     : dispatch_lanes<__nv_bfloat16, int8_t, 3>(in, n, d, codes, s, scales);
 }
 
 cudaError_t launch_cast_bf16(const float* in, int64_t count, __nv_bfloat16* out, cudaStream_t s) {

@@ -13,7 +13,11 @@
 // Score and filter, per (query b, row j):
 //   s = fl(dot * c_j), c_j = fl(inv_norm_j * inv_tau) (inv_norm_j = 1 when
 //   the corpus is stored normalised); candidate kept iff it is not excluded
-//   and key(s, j) > theta[b]. Kept keys are appended to the query's buffer;
+//   and key(s, j) > theta[b].
+// int8 rows (k2_stream_i8; recsys_two_tower_model.py `compute_top_k_int8`):
+//   the queries are int8 codes with scales us_b, staged as packed words; dot
+//   is the exact int32 sum of code products (dp4a), s = fl(fl(fl(dot) * us_b)
+//   * c_j) with c_j = fl(scale_j * inv_tau). Kept keys are appended to the query's buffer;
 //   the append is warp-aggregated (one atomicAdd per query per warp).
 // (recsys_two_tower_model.py `forward`: scores = user . post_embeddings^T,
 // masked candidates dropped; the top-k is taken from the kept keys by the
@@ -158,6 +162,98 @@ __global__ void __launch_bounds__(K2_THREADS)
     }
 }
 
+// Kept keys of one warp appended to query q's buffer (warp-aggregated).
+__device__ __forceinline__ void append_warp(const PassArgs& a, int q, bool keep, uint64_t key, int lane) {
+    const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, keep);
+    if (ballot) {
+        const int leader = __ffs(ballot) - 1;
+        uint32_t slot0 = 0;
+        if (lane == leader) slot0 = atomicAdd(a.count + q, (uint32_t)__popc(ballot));
+        slot0 = __shfl_sync(0xFFFFFFFFu, slot0, leader);
+        if (keep) {
+            const uint32_t slot = slot0 + __popc(ballot & lanemask_lt());
+            if (slot < (uint32_t)a.cap) a.keys[(int64_t)q * a.cap + slot] = key;
+        }
+    }
+}
+
+// int8 rows: one thread per row, 32 codes per 32-byte piece, dp4a against
+// the staged query code words. d % 32 == 0; four pieces (128 codes) in
+// flight per thread.
+constexpr int K2_BATCH_I8 = 4;
+
+template <int QB, bool V8>
+__global__ void __launch_bounds__(K2_THREADS)
+    k2_stream_i8(const PassArgs a) {
+    extern __shared__ __align__(16) int qw[];  // [QB][d / 4] packed codes
+    const int lane = threadIdx.x & 31;
+    const int q0 = blockIdx.y * QB;
+    const int d = a.d;
+    const int dw = d / 4;
+    const int pieces = d / 32;
+    for (int i = threadIdx.x; i < QB * dw; i += blockDim.x) {
+        const int qb = i / dw, w = i % dw;
+        const int q = q0 + qb;
+        qw[i] = q < a.b ? reinterpret_cast<const int*>(a.queries)[(int64_t)q * dw + w] : 0;
+    }
+    uint64_t th[QB];
+    float us[QB];
+#pragma unroll
+    for (int qb = 0; qb < QB; ++qb) {
+        th[qb] = (q0 + qb < a.b) ? a.theta[q0 + qb] : KEY_MAX;
+        us[qb] = (q0 + qb < a.b) ? a.qscale[q0 + qb] : 1.0f;
+    }
+    __syncthreads();
+
+    const int64_t pitch = (int64_t)a.stride * d;
+    const uint8_t* base = static_cast<const uint8_t*>(a.rows);
+    const int64_t n_threads = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r - lane < a.n_rows; r += n_threads) {
+        const bool valid = r < a.n_rows;
+        const uint8_t* row = base + (valid ? r : 0) * pitch;
+        int acc[QB];
+#pragma unroll
+        for (int qb = 0; qb < QB; ++qb) acc[qb] = 0;
+        for (int p0 = 0; p0 < pieces; p0 += K2_BATCH_I8) {
+            Raw32 raw[K2_BATCH_I8];
+#pragma unroll
+            for (int j = 0; j < K2_BATCH_I8; ++j)
+                if (p0 + j < pieces && valid) raw[j] = ld32<V8>(row + (int64_t)(p0 + j) * 32);
+#pragma unroll
+            for (int j = 0; j < K2_BATCH_I8; ++j) {
+                if (p0 + j >= pieces) break;
+                const int w0 = (p0 + j) * 8;
+#pragma unroll
+                for (int qb = 0; qb < QB; ++qb) {
+                    const int4* qv = reinterpret_cast<const int4*>(qw + qb * dw + w0);
+                    const int4 qa = qv[0], qc = qv[1];
+                    acc[qb] = __dp4a((int)raw[j].w[0], qa.x, acc[qb]);
+                    acc[qb] = __dp4a((int)raw[j].w[1], qa.y, acc[qb]);
+                    acc[qb] = __dp4a((int)raw[j].w[2], qa.z, acc[qb]);
+                    acc[qb] = __dp4a((int)raw[j].w[3], qa.w, acc[qb]);
+                    acc[qb] = __dp4a((int)raw[j].w[4], qc.x, acc[qb]);
+                    acc[qb] = __dp4a((int)raw[j].w[5], qc.y, acc[qb]);
+                    acc[qb] = __dp4a((int)raw[j].w[6], qc.z, acc[qb]);
+                    acc[qb] = __dp4a((int)raw[j].w[7], qc.w, acc[qb]);
+                }
+            }
+        }
+        const int64_t id = r * a.stride;
+        bool row_ok = valid;
+        float c = a.inv_tau;
+        if (valid) {
+            if (a.exclude) row_ok = !((a.exclude[id >> 5] >> (id & 31)) & 1u);
+            c = a.inv_norm[id] * a.inv_tau;
+        }
+#pragma unroll
+        for (int qb = 0; qb < QB; ++qb) {
+            // |acc| < 2^24 (127 * 127 * 512), so fl(acc) is exact
+            const uint64_t key = make_key((float)acc[qb] * us[qb] * c, (uint32_t)id);
+            append_warp(a, q0 + qb, row_ok && key > th[qb], key, lane);
+        }
+    }
+}
+
 template <typename T, int QB>
 cudaError_t launch_qb(const PassArgs& a, dim3 grid, size_t smem, bool v8, cudaStream_t s) {
     if (v8)
@@ -165,6 +261,24 @@ cudaError_t launch_qb(const PassArgs& a, dim3 grid, size_t smem, bool v8, cudaSt
     else
         k2_stream<T, QB, false><<<grid, K2_THREADS, smem, s>>>(a);
     return cudaGetLastError();
+}
+
+template <int QB>
+cudaError_t launch_i8_qb(const PassArgs& a, dim3 grid, size_t smem, bool v8, cudaStream_t s) {
+    if (v8)
+        k2_stream_i8<QB, true><<<grid, K2_THREADS, smem, s>>>(a);
+    else
+        k2_stream_i8<QB, false><<<grid, K2_THREADS, smem, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_i8(const PassArgs& a, int qb, dim3 grid, size_t smem, bool v8, cudaStream_t s) {
+    switch (qb) {
+        case 1: return launch_i8_qb<1>(a, grid, smem, v8, s);
+        case 2: return launch_i8_qb<2>(a, grid, smem, v8, s);
+        case 4: return launch_i8_qb<4>(a, grid, smem, v8, s);
+        default: return launch_i8_qb<8>(a, grid, smem, v8, s);
+    }
 }
 
 template <typename T>
@@ -192,8 +306,9 @@ cudaError_t launch_stream_pass(const PassArgs& a, cudaStream_t s, int sm_count) 
     if (gx < 1) gx = 1;
     const dim3 grid((unsigned)gx, (unsigned)gy);
     note_launch_begin(TT_KIND_STREAM, s);
-    cudaError_t e = a.dtype == TT_F32 ? launch_t<float>(a, qb, grid, smem, v8, s)
-                                      : launch_t<__nv_bfloat16>(a, qb, grid, smem, v8, s);
+    cudaError_t e = a.dtype == TT_F32    ? launch_t<float>(a, qb, grid, smem, v8, s)
+                    : a.dtype == TT_I8 ? launch_i8(a, qb, grid, smem, v8, s)
+                                       : launch_t<__nv_bfloat16>(a, qb, grid, smem, v8, s);
     note_launch_end(TT_KIND_STREAM, s);
     return e;
 }

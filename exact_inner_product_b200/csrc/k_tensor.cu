@@ -40,7 +40,7 @@ namespace tt {
 namespace {
 
 constexpr int K3_M = 128;                  // corpus rows per tile
-constexpr int K3_KC = 64;                  // bf16 elements per 128-byte swizzle row
+constexpr int K3_ROW_BYTES = 128;          // one 128-byte swizzle row of K per operand row
 constexpr int K3_STAGE_BYTES = K3_M * 128; // one K chunk of a corpus tile
 constexpr int K3_MAX_STAGES = 12;
 constexpr int K3_EPI_WARPS = 8;
@@ -61,9 +61,10 @@ struct K3Ctl {
     uint32_t tmem_base;
     int abort;
     // per epilogue warp: fast-path thresholds and exact threshold keys of its
-    // columns for the current unit
+    // columns for the current unit (int8 rows: and the query scales)
     alignas(16) float th_fast[K3_EPI_WARPS][K3_WARP_COLS];  // read as float4
     uint64_t th_key[K3_EPI_WARPS][K3_WARP_COLS];
+    float q_us[K3_EPI_WARPS][K3_WARP_COLS];
 };
 static_assert(offsetof(K3Ctl, th_fast) % 16 == 0, "float4 reads of th_fast need 16-byte alignment");
 
@@ -71,7 +72,7 @@ struct K3Params {
     PassArgs a;
     int nq;          // queries per tile (multiple of 32, <= 256)
     int q_tiles;     // ceil(b / nq)
-    int kchunks;     // ceil(d / 64)
+    int kchunks;     // 128-byte chunks of K: ceil(d * element size / 128)
     int stages;
     int64_t tiles;   // corpus tiles of 128 rows in this level
     int chunks;      // corpus chunks (units = q_tiles * chunks)
@@ -86,9 +87,13 @@ __device__ __forceinline__ void unit_range(const K3Params& p, int u, int* qt, in
     *t1 = p.tiles * (ch + 1) / p.chunks;
 }
 
+// I8: int8 codes (kind::i8, int32 accumulators; recsys_two_tower_model.py
+// `compute_top_k_int8`), else bf16 (kind::f16, fp32 accumulators).
+template <bool I8>
 __global__ void __launch_bounds__(K3_THREADS, 1)
     k3_tensor(const __grid_constant__ CUtensorMap tm_rows, const __grid_constant__ CUtensorMap tm_q,
               const K3Params p) {
+    constexpr int KC = I8 ? 128 : 64;  // elements per 128-byte row of a chunk
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -142,7 +147,7 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
                 q_issued = uc;
                 mbar_arrive_expect_tx(&ctl->qfull, (uint32_t)(p.kchunks * q_chunk_bytes));
                 for (int kc = 0; kc < p.kchunks; ++kc)
-                    tma_load_2d(qsm + (size_t)kc * q_chunk_bytes, &tm_q, &ctl->qfull, kc * K3_KC,
+                    tma_load_2d(qsm + (size_t)kc * q_chunk_bytes, &tm_q, &ctl->qfull, kc * KC,
                                 qt * p.nq);
                 for (int64_t t = t0; ok && t < t1; ++t) {
                     for (int kc = 0; kc < p.kchunks; ++kc, ++it) {
@@ -153,7 +158,7 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
                         }
                         mbar_arrive_expect_tx(&ctl->full[s], K3_STAGE_BYTES);
                         tma_load_2d(ring + (size_t)s * K3_STAGE_BYTES, &tm_rows, &ctl->full[s],
-                                    kc * K3_KC, (int32_t)(t * K3_M));
+                                    kc * KC, (int32_t)(t * K3_M));
                     }
                 }
             }
@@ -193,10 +198,15 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
                         const uint32_t a_addr = rbase + (uint32_t)(s * K3_STAGE_BYTES);
                         const uint32_t b_addr = qbase + (uint32_t)(kc * q_chunk_bytes);
 #pragma unroll
-                        for (int kk = 0; kk < K3_KC / 16; ++kk) {
-                            umma_bf16(d_tmem, umma_desc_kmajor_sw128(a_addr + kk * 32),
-                                      umma_desc_kmajor_sw128(b_addr + kk * 32), p.idesc,
-                                      (kc | kk) != 0 ? 1u : 0u);
+                        for (int kk = 0; kk < K3_ROW_BYTES / 32; ++kk) {  // 32 bytes of K per MMA
+                            if constexpr (I8)
+                                umma_i8(d_tmem, umma_desc_kmajor_sw128(a_addr + kk * 32),
+                                        umma_desc_kmajor_sw128(b_addr + kk * 32), p.idesc,
+                                        (kc | kk) != 0 ? 1u : 0u);
+                            else
+                                umma_bf16(d_tmem, umma_desc_kmajor_sw128(a_addr + kk * 32),
+                                          umma_desc_kmajor_sw128(b_addr + kk * 32), p.idesc,
+                                          (kc | kk) != 0 ? 1u : 0u);
                         }
                         umma_commit(&ctl->empty[s]);  // stage free once these MMAs finish
                     }
@@ -229,6 +239,7 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
         const bool uniform_c = a.inv_norm == nullptr;
         float* th_fast = ctl->th_fast[ew];
         uint64_t* th_key = ctl->th_key[ew];
+        float* q_us = ctl->q_us[ew];
         uint32_t tc = 0;
         bool ok = true;
         for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
@@ -242,14 +253,25 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
                 const int ch = half + 2 * (j >> 5);
                 float t = INFINITY;
                 th_key[j] = ch < nchunk32 ? __ldg(th_unit + ch * 32 + (j & 31)) : KEY_MAX;
+                float us = 1.0f;
                 if (ch < nchunk32) {
                     t = __ldg(thf_unit + ch * 32 + (j & 31));
-                    if (uniform_c && t != INFINITY && t != -INFINITY) {
+                    if (I8) {
+                        // score = fl(fl(acc * us) * c): the fast test compares
+                        // fl(acc * c) with th / us, lowered like th / c below
+                        const int q = qt * p.nq + ch * 32 + (j & 31);
+                        us = q < a.b ? __ldg(a.qscale + q) : 1.0f;
+                        if (t != INFINITY && t != -INFINITY) {
+                            const float r = t / us;
+                            t = r - fabsf(r) * 0x1p-20f - 1e-30f;
+                        }
+                    } else if (uniform_c && t != INFINITY && t != -INFINITY) {
                         const float r = t / a.inv_tau;
                         t = r - fabsf(r) * 0x1p-20f - 1e-30f;
                     }
                 }
                 th_fast[j] = t;
+                q_us[j] = us;
             }
             __syncwarp();
             for (int64_t t = t0; t < t1; ++t, ++tc) {
@@ -287,6 +309,12 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
                     tmem_ld_32cols(tbase + (uint32_t)((half + 2 * cja) * 32), v[0].x);
                     if (has_b) tmem_ld_32cols(tbase + (uint32_t)((half + 2 * cjb) * 32), v[1].x);
                     tmem_ld_wait();
+                    if constexpr (I8) {  // int32 accumulators: exact in fp32 (|acc| < 2^24)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) v[h].x[i] = (float)__float_as_int(v[h].x[i]);
+                    }
                     const bool last = pair == 1 || half + 2 * (cjb + 1) >= nchunk32;
                     if (last) {
                         tc_fence_before();
@@ -327,7 +355,8 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
                             while (m) {
                                 const int i = __ffs(m) - 1;
                                 m &= m - 1;
-                                const uint64_t key = make_key(select32(v[h], i) * c, (uint32_t)id);
+                                const float acc = I8 ? select32(v[h], i) * q_us[cj * 32 + i] : select32(v[h], i);
+                                const uint64_t key = make_key(acc * c, (uint32_t)id);
                                 if (key > th_key[cj * 32 + i]) {
                                     const int q = qt * p.nq + col0 + i;
                                     const uint32_t slot = atomicAdd(a.count + q, 1u);
@@ -355,8 +384,8 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
 
 }  // namespace
 
-int tensor_pass_smem_bytes(int d, int nq) {
-    const int kchunks = (d + K3_KC - 1) / K3_KC;
+int tensor_pass_smem_bytes(int d, int nq, int esize) {
+    const int kchunks = (d * esize + K3_ROW_BYTES - 1) / K3_ROW_BYTES;
     const int q_bytes = kchunks * nq * 128;
     const int fixed = 1024 + q_bytes + (int)sizeof(K3Ctl);
     int stages = (K3_SMEM_BUDGET - fixed) / K3_STAGE_BYTES;
@@ -365,10 +394,10 @@ int tensor_pass_smem_bytes(int d, int nq) {
     return fixed + stages * K3_STAGE_BYTES;
 }
 
-int tensor_pass_max_nq(int d) {
+int tensor_pass_max_nq(int d, int esize) {
     for (int nq = K3_MAX_NQ; nq >= 32; nq -= 32)
-        if (tensor_pass_smem_bytes(d, nq) > 0 && tensor_pass_smem_bytes(d, nq) <= K3_SMEM_BUDGET &&
-            ((d + K3_KC - 1) / K3_KC) * nq * 128 <= 128 * 1024)
+        if (tensor_pass_smem_bytes(d, nq, esize) > 0 && tensor_pass_smem_bytes(d, nq, esize) <= K3_SMEM_BUDGET &&
+            ((d * esize + K3_ROW_BYTES - 1) / K3_ROW_BYTES) * nq * 128 <= 128 * 1024)
             return nq;
     return 0;
 }
@@ -381,8 +410,10 @@ cudaError_t launch_tensor_pass(const PassArgs& a, const CUtensorMap& tm_rows,
     p.a = a;
     p.nq = nq;
     p.q_tiles = (a.b + nq - 1) / nq;
-    p.kchunks = (a.d + K3_KC - 1) / K3_KC;
-    const int smem = tensor_pass_smem_bytes(a.d, nq);
+    const bool i8 = a.dtype == TT_I8;
+    const int esize = i8 ? 1 : 2;
+    p.kchunks = (a.d * esize + K3_ROW_BYTES - 1) / K3_ROW_BYTES;
+    const int smem = tensor_pass_smem_bytes(a.d, nq, esize);
     if (smem <= 0) return cudaErrorInvalidValue;
     const int fixed = 1024 + p.kchunks * nq * 128 + (int)sizeof(K3Ctl);
     p.stages = (smem - fixed) / K3_STAGE_BYTES;
@@ -397,13 +428,17 @@ cudaError_t launch_tensor_pass(const PassArgs& a, const CUtensorMap& tm_rows,
     if (chunks < 1) chunks = 1;
     if (chunks > p.tiles) chunks = (int)p.tiles;
     p.chunks = chunks;
-    p.idesc = umma_idesc_bf16(K3_M, nq);
+    p.idesc = i8 ? umma_idesc_s8(K3_M, nq) : umma_idesc_bf16(K3_M, nq);
     const int n_units = p.q_tiles * p.chunks;
     const int grid = n_units < sm_count ? n_units : sm_count;
-    cudaError_t e = cudaFuncSetAttribute(k3_tensor, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = i8 ? cudaFuncSetAttribute(k3_tensor<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+                       : cudaFuncSetAttribute(k3_tensor<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     note_launch_begin(TT_KIND_TENSOR, s);
-    k3_tensor<<<grid, K3_THREADS, smem, s>>>(tm_rows, tm_queries, p);
+    if (i8)
+        k3_tensor<true><<<grid, K3_THREADS, smem, s>>>(tm_rows, tm_queries, p);
+    else
+        k3_tensor<false><<<grid, K3_THREADS, smem, s>>>(tm_rows, tm_queries, p);
     note_launch_end(TT_KIND_TENSOR, s);
     return cudaGetLastError();
 }

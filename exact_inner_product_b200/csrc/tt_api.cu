@@ -161,12 +161,26 @@ bool bf16_tile_tensor_map(const void* base, int64_t rows, int d, int64_t row_pit
                      CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// int8 rows: boxes of 128 codes (one 128-byte swizzle row) x box_rows rows.
+static bool i8_tile_tensor_map(const void* base, int64_t rows, int d, int64_t row_pitch_elems,
+                               int box_rows, CUtensorMap* tm) {
+    return encode_2d(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, (uint64_t)d, (uint64_t)rows,
+                     (uint64_t)row_pitch_elems, 128, (uint32_t)box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+static bool tile_tensor_map(int dtype, const void* base, int64_t rows, int d, int64_t row_pitch_elems,
+                            int box_rows, CUtensorMap* tm) {
+    return dtype == TT_I8 ? i8_tile_tensor_map(base, rows, d, row_pitch_elems, box_rows, tm)
+                          : bf16_tile_tensor_map(base, rows, d, row_pitch_elems, box_rows, tm);
+}
+
 // ---------------------------------------------------------------------------
 // validation helpers
 // ---------------------------------------------------------------------------
 static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 static bool valid_dtype(int dt) { return dt == TT_F32 || dt == TT_BF16; }
+static bool valid_index_dtype(int dt) { return valid_dtype(dt) || dt == TT_I8; }
 
 static tt_status check_d(int32_t d) {
     if (d <= 0) return TT_ERR_INVALID_ARG;
@@ -296,6 +310,8 @@ struct Scratch {
     int32_t* status;
     int* flags;
     __nv_bfloat16* qcast;
+    int8_t* qcodes;   // int8 index: the queries' codes [b, d]
+    float* qscale;    // and their scales [b]
 };
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -359,7 +375,7 @@ static void pinned_give(int* p) {
 }
 
 static tt_status get_scratch(tt_index* ix, int b, int b_pad, int cap, int d, bool need_qcast,
-                             Scratch* out) {
+                             bool need_q8, Scratch* out) {
     size_t off = 0;
     const size_t o_keys = off;
     off = align_up(off + (size_t)b * cap * 8, 256);
@@ -375,6 +391,10 @@ static tt_status get_scratch(tt_index* ix, int b, int b_pad, int cap, int d, boo
     off = align_up(off + 64, 256);
     const size_t o_q = off;
     off = align_up(off + (need_qcast ? (size_t)b * d * 2 : 0), 256);
+    const size_t o_q8 = off;
+    off = align_up(off + (need_q8 ? (size_t)b * d : 0), 256);
+    const size_t o_qs = off;
+    off = align_up(off + (need_q8 ? (size_t)b_pad * 4 : 0), 256);
     if (off > ix->scratch_bytes) {
         if (ix->scratch) {
             // the old block may still be read by work queued on the stream
@@ -403,6 +423,8 @@ static tt_status get_scratch(tt_index* ix, int b, int b_pad, int cap, int d, boo
     out->status = reinterpret_cast<int32_t*>(base + o_status);
     out->flags = reinterpret_cast<int*>(base + o_flags);
     out->qcast = need_qcast ? reinterpret_cast<__nv_bfloat16*>(base + o_q) : nullptr;
+    out->qcodes = need_q8 ? reinterpret_cast<int8_t*>(base + o_q8) : nullptr;
+    out->qscale = need_q8 ? reinterpret_cast<float*>(base + o_qs) : nullptr;
     if (!ix->h_flags) {
         ix->h_flags = pinned_take();
         if (!ix->h_flags) {
@@ -421,6 +443,7 @@ struct PathCfg {
     int nq;             // tensor path: queries per tile
     const void* queries;
     int q_dtype;
+    const float* qscale;  // int8 index: query scales
     CUtensorMap tm_q;
 };
 
@@ -438,6 +461,7 @@ static tt_status run_pass(const tt_index* ix, const PathCfg& pc, const Plan& pla
     a.inv_tau = inv_tau;
     a.queries = pc.queries;
     a.q_dtype = pc.q_dtype;
+    a.qscale = pc.qscale;
     a.b = b;
     a.theta = sc.theta;
     a.thf = sc.thf;
@@ -448,7 +472,7 @@ static tt_status run_pass(const tt_index* ix, const PathCfg& pc, const Plan& pla
     cudaError_t e;
     if (pc.path == 2) {
         CUtensorMap tm_rows;
-        if (!bf16_tile_tensor_map(ix->rows, a.n_rows, ix->d, a.stride * ix->d, 128, &tm_rows))
+        if (!tile_tensor_map(ix->dtype, ix->rows, a.n_rows, ix->d, a.stride * ix->d, 128, &tm_rows))
             return TT_ERR_CUDA;
         e = launch_tensor_pass(a, tm_rows, pc.tm_q, pc.nq, s, sms);
     } else if (pc.path == 3) {
@@ -611,6 +635,28 @@ tt_status tt_normalize_candidates(const void* in, tt_dtype in_dtype, int64_t n, 
     return TT_OK;
 }
 
+tt_status tt_quantize_candidates(const void* in, tt_dtype in_dtype, int64_t n, int32_t d, int8_t* out_codes,
+                                 float* out_scales, void* stream, tt_index** index_out) {
+    if (index_out) *index_out = nullptr;
+    if (n < 0) return TT_ERR_INVALID_ARG;
+    if (n > TT_MAX_N) return TT_ERR_UNSUPPORTED;
+    tt_status st = check_d(d);
+    if (st != TT_OK) return st;
+    if (!valid_dtype(in_dtype)) return TT_ERR_INVALID_ARG;
+    if (n > 0 && (in == nullptr || out_codes == nullptr || out_scales == nullptr)) return TT_ERR_INVALID_ARG;
+    if (!aligned(in, 16) || !aligned(out_codes, 16) || !aligned(out_scales, 4)) return TT_ERR_INVALID_ARG;
+    if (n > 0) {
+        if ((st = check_device_ptr(in, "in")) != TT_OK) return st;
+        if ((st = check_device_ptr(out_codes, "out_codes")) != TT_OK) return st;
+        if ((st = check_device_ptr(out_scales, "out_scales")) != TT_OK) return st;
+        cudaError_t e = launch_quantize(in, in_dtype, n, d, out_codes, out_scales, true,
+                                        static_cast<cudaStream_t>(stream));
+        if (e != cudaSuccess) return cuda_fail(e, "quantize");
+    }
+    if (index_out) return new_index(out_codes, TT_I8, n, d, out_scales, index_out);
+    return TT_OK;
+}
+
 tt_status tt_index_wrap(const void* rows, tt_dtype dtype, int64_t n, int32_t d,
                         const float* inv_norm, tt_index** index_out) {
     if (!index_out) return TT_ERR_INVALID_ARG;
@@ -619,8 +665,9 @@ tt_status tt_index_wrap(const void* rows, tt_dtype dtype, int64_t n, int32_t d,
     if (n > TT_MAX_N) return TT_ERR_UNSUPPORTED;
     tt_status st = check_d(d);
     if (st != TT_OK) return st;
-    if (!valid_dtype(dtype)) return TT_ERR_INVALID_ARG;
+    if (!valid_index_dtype(dtype)) return TT_ERR_INVALID_ARG;
     if (n > 0 && rows == nullptr) return TT_ERR_INVALID_ARG;
+    if (dtype == TT_I8 && n > 0 && inv_norm == nullptr) return TT_ERR_INVALID_ARG;  // scales required
     if (!aligned(rows, 16) || !aligned(inv_norm, 4)) return TT_ERR_INVALID_ARG;
     if (n > 0) {
         if ((st = check_device_ptr(rows, "rows")) != TT_OK) return st;
@@ -663,7 +710,12 @@ tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtyp
     tt_status st = make_plan(index->n, k, options, &plan);
     if (st != TT_OK) return st;
     if (index->dtype == TT_F32 && index->d > 256) return TT_ERR_UNSUPPORTED;
-    const bool tc_possible = index->dtype == TT_BF16 && index->d >= 64 && tensor_pass_max_nq(index->d) > 0;
+    const bool i8 = index->dtype == TT_I8;
+    // int8 rows are read in 32-byte pieces by the streaming scorer
+    if (i8 && index->d % 32 != 0) return TT_ERR_UNSUPPORTED;
+    const int esize = i8 ? 1 : 2;
+    const bool tc_possible = (index->dtype == TT_BF16 || i8) && index->d >= 64 &&
+                             tensor_pass_max_nq(index->d, esize) > 0;
     const bool pair_possible = index->dtype == TT_BF16 && index->d >= 64 && tensor_pair_smem_bytes(index->d) > 0;
     int path = path_req;
     if (path == 0) {
@@ -711,7 +763,7 @@ tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtyp
     // threshold arrays are padded to whole query tiles plus one 32-column chunk).
     int nq = 0, q_tiles = 1;
     if (path == 2) {
-        const int max_nq = tensor_pass_max_nq(index->d);
+        const int max_nq = tensor_pass_max_nq(index->d, esize);
         q_tiles = (b + max_nq - 1) / max_nq;
         nq = (b + q_tiles - 1) / q_tiles;
         nq = (nq + 31) / 32 * 32;  // whole 32-column chunks: no chunk reads past the tile
@@ -719,9 +771,9 @@ tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtyp
     }
     if (path == 3) q_tiles = (b + 255) / 256;
     const int b_pad = (path == 2 ? q_tiles * nq : path == 3 ? q_tiles * 256 : b) + 64;
-    const bool need_qcast = path >= 2 && q_dtype == TT_F32;
+    const bool need_qcast = !i8 && path >= 2 && q_dtype == TT_F32;
     Scratch sc;
-    if ((st = get_scratch(index, b, b_pad, plan.cap, index->d, need_qcast, &sc)) != TT_OK) return st;
+    if ((st = get_scratch(index, b, b_pad, plan.cap, index->d, need_qcast, i8, &sc)) != TT_OK) return st;
     const int sms = sm_count_current();
     const float inv_tau = 1.0f / tau;
 
@@ -730,6 +782,14 @@ tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtyp
     pc.path = path;
     pc.queries = queries;
     pc.q_dtype = q_dtype;
+    if (i8) {
+        // code the queries as given (recsys_two_tower_model.py `compute_top_k_int8`)
+        cudaError_t e = launch_quantize(queries, q_dtype, b, index->d, sc.qcodes, sc.qscale, false, s);
+        if (e != cudaSuccess) return cuda_fail(e, "query coding");
+        pc.queries = sc.qcodes;
+        pc.q_dtype = TT_I8;
+        pc.qscale = sc.qscale;
+    }
     if (path >= 2) {
         if (need_qcast) {
             cudaError_t e = launch_cast_bf16(static_cast<const float*>(queries), (int64_t)b * index->d,
@@ -740,7 +800,7 @@ tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtyp
         }
         pc.nq = path == 2 ? nq : 256;
         // single-CTA kernel: boxes of nq queries; pairs: each CTA loads 128
-        if (!bf16_tile_tensor_map(pc.queries, b, index->d, index->d, path == 2 ? nq : 128, &pc.tm_q))
+        if (!tile_tensor_map(pc.q_dtype, pc.queries, b, index->d, index->d, path == 2 ? nq : 128, &pc.tm_q))
             return TT_ERR_CUDA;
     }
 

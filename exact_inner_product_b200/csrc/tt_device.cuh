@@ -197,6 +197,18 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint6
         : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T, signed int8 inputs, exact int32
+// accumulation (K = 32 per instruction).
+__device__ __forceinline__ void umma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive on `bar` once every tcgen05 operation issued so far by this thread
 // has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -249,6 +261,16 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int m, int n) {
     return (1u << 4)                          // accumulator format: f32
            | (1u << 7)                        // A format: bf16
            | (1u << 10)                       // B format: bf16
+           | ((uint32_t)(n >> 3) << 17)       // N / 8
+           | ((uint32_t)(m >> 4) << 24);      // M / 16
+}
+
+// Instruction descriptor: kind::i8 with signed int8 A and B (both K-major),
+// int32 accumulator, shape M x N.
+__host__ __device__ constexpr uint32_t umma_idesc_s8(int m, int n) {
+    return (2u << 4)                          // accumulator format: s32
+           | (1u << 7)                        // A format: signed 8-bit
+           | (1u << 10)                       // B format: signed 8-bit
            | ((uint32_t)(n >> 3) << 17)       // N / 8
            | ((uint32_t)(m >> 4) << 24);      // M / 16
 }

@@ -21,10 +21,10 @@ struct PassArgs {
     int64_t n_rows;            // rows in this level
     int64_t stride;            // corpus rows between consecutive level rows
     int d;
-    const float* inv_norm;     // [n] or null
+    const float* inv_norm;     // [n] or null (int8 rows: the per-row scales)
     const uint32_t* exclude;   // [ceil(n/32)] or null
     float inv_tau;
-    const void* queries;       // [b, d]
+    const void* queries;       // [b, d] (int8 rows: the query codes)
     int q_dtype;
     int b;
     const uint64_t* theta;     // [b_pad] threshold keys (KEY_MAX past b)
@@ -33,6 +33,7 @@ struct PassArgs {
     uint64_t* keys;            // [b * cap]
     int cap;
     int* err;                  // device error word
+    const float* qscale;       // [b] query scales of int8 rows, else null
 };
 
 // Set the text tt_last_error() returns on the calling thread.
@@ -46,6 +47,10 @@ void note_launch_end(int kind, cudaStream_t s);
 cudaError_t launch_normalize(const void* in, int in_dtype, int64_t n, int d, void* out,
                              int out_dtype, int mode, cudaStream_t s);
 cudaError_t launch_cast_bf16(const float* in, int64_t count, __nv_bfloat16* out, cudaStream_t s);
+// int8 coding of rows (normalised first when `normalise`): codes [n, d],
+// scales [n] (see tt_quantize_candidates).
+cudaError_t launch_quantize(const void* in, int in_dtype, int64_t n, int d, int8_t* codes, float* scales,
+                            bool normalise, cudaStream_t s);
 cudaError_t launch_stream_pass(const PassArgs& a, cudaStream_t s, int sm_count);
 cudaError_t launch_tensor_pass(const PassArgs& a, const CUtensorMap& tm_rows,
                                const CUtensorMap& tm_queries, int nq_tile, cudaStream_t s,
@@ -87,8 +92,9 @@ bool bf16_tile_tensor_map(const void* base, int64_t rows, int d, int64_t row_pit
 cudaError_t launch_pad(int32_t* out_ids, float* out_scores, int64_t count, cudaStream_t s);
 
 // Shared-memory bytes the tensor-core pass needs for a given d and query tile.
-int tensor_pass_smem_bytes(int d, int nq_tile);
-int tensor_pass_max_nq(int d);
+// esize: bytes per element of the rows (2 bf16, 1 int8).
+int tensor_pass_smem_bytes(int d, int nq_tile, int esize);
+int tensor_pass_max_nq(int d, int esize);
 int tensor_pair_smem_bytes(int d);  // -1 when d does not fit
 
 }  // namespace tt

@@ -114,11 +114,11 @@ tt_status tt_score_topk_noalloc(const void* rows, tt_dtype dtype, int64_t n, int
     int64_t lrows[4] = {0}, lstride[4] = {0};
     tt_status st = tt_plan(n, k, nullptr, &levels, lrows, lstride, ranks, &cap);
     if (st != TT_OK) return st;
-    const bool tc_possible = dtype == TT_BF16 && d >= 64 && tensor_pass_max_nq(d) > 0;
+    const bool tc_possible = dtype == TT_BF16 && d >= 64 && tensor_pass_max_nq(d, 2) > 0;
     const int path = (tc_possible && b > 8) ? 2 : 1;
     int nq = 0, q_tiles = 1;
     if (path == 2) {
-        const int max_nq = tensor_pass_max_nq(d);
+        const int max_nq = tensor_pass_max_nq(d, 2);
         q_tiles = (b + max_nq - 1) / max_nq;
         nq = ((b + q_tiles - 1) / q_tiles + 31) / 32 * 32;  // whole 32-column chunks
         if (nq > max_nq) nq = max_nq;
@@ -198,6 +198,7 @@ tt_status tt_score_topk_noalloc(const void* rows, tt_dtype dtype, int64_t n, int
         a.inv_tau = inv_tau;
         a.queries = q_use;
         a.q_dtype = q_dt_use;
+        a.qscale = nullptr;
         a.b = b;
         a.theta = theta;
         a.thf = thf;

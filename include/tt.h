@@ -51,7 +51,11 @@ typedef enum tt_status {
     TT_ERR_INTERNAL = 6     /* the exactness check could not be satisfied (not expected) */
 } tt_status;
 
-typedef enum tt_dtype { TT_F32 = 0, TT_BF16 = 1 } tt_dtype;
+typedef enum tt_dtype {
+    TT_F32 = 0,
+    TT_BF16 = 1,
+    TT_I8 = 2 /* int8 codes with one f32 scale per row (tt_quantize_candidates) */
+} tt_dtype;
 
 /* How tt_normalize_candidates prepares the corpus. */
 typedef enum tt_norm_mode {
@@ -102,10 +106,39 @@ TT_API tt_status tt_normalize_candidates(const void* in, tt_dtype in_dtype, int6
                                   tt_index** index_out);
 
 /*
+ * tt_quantize_candidates - L2-normalise each row and code it in int8 with
+ * one scale per row, for int8 scoring.
+ *
+ *   w_ji = fl(v_ji / norm_j)   (norm_j as in tt_normalize_candidates, fp32)
+ *   scale_j = max(fl(max_i |w_ji| / 127), 1e-12)
+ *   code_ji = clip(round_half_even(fl(w_ji / scale_j)), -127, 127)
+ *
+ * (recsys_two_tower_model.py `forward`, `compute_top_k_int8`: the user rows
+ *  are coded this way and the candidate index arrives as int8 codes with one
+ *  scale per candidate; the pages do not show how those are made, and this
+ *  call applies the same scheme to the normalised candidate rows.)
+ *
+ * in          device [n, d] rows, in_dtype (TT_F32 or TT_BF16)
+ * n, d        as in tt_normalize_candidates
+ * out_codes   device [n, d] int8 (caller-owned)
+ * out_scales  device [n] f32 (caller-owned)
+ * stream      cudaStream_t
+ * index_out   optional: receives a handle over (out_codes, out_scales),
+ *             dtype TT_I8, released with tt_free
+ *
+ * Errors as tt_normalize_candidates; out_codes and out_scales must be
+ * 16-byte and 4-byte aligned device pointers.
+ */
+TT_API tt_status tt_quantize_candidates(const void* in, tt_dtype in_dtype, int64_t n, int32_t d,
+                                        int8_t* out_codes, float* out_scales, void* stream,
+                                        tt_index** index_out);
+
+/*
  * tt_index_wrap - a handle over a corpus that is already prepared (rows
- * normalised and stored, or raw rows plus their f32 inv_norm), e.g. loaded
- * from a checkpoint. No device work. rows: device [n, d] dtype; inv_norm:
- * device [n] f32 or NULL. Limits as for tt_normalize_candidates.
+ * normalised and stored, or raw rows plus their f32 inv_norm, or int8 codes
+ * plus their f32 scales), e.g. loaded from a checkpoint. No device work.
+ * rows: device [n, d] dtype; inv_norm: device [n] f32 or NULL (for TT_I8
+ * rows: the per-row scales, required). Limits as for tt_normalize_candidates.
  */
 TT_API tt_status tt_index_wrap(const void* rows, tt_dtype dtype, int64_t n, int32_t d,
                         const float* inv_norm, tt_index** index_out);
@@ -116,6 +149,11 @@ TT_API tt_status tt_index_wrap(const void* rows, tt_dtype dtype, int64_t n, int3
  *   s_bj = fl(dot_bj * c_j),  c_j = fl(inv_norm_j * fl(1/tau))  (inv_norm_j = 1
  *          unless the handle was prepared with TT_NORM_FUSED)
  *   dot_bj = sum_i q_bi * v_ji with fp32 accumulation
+ *   int8 handle (TT_I8): each query row is coded as in tt_quantize_candidates
+ *   but without normalisation (codes u8_b, scale us_b), and
+ *   s_bj = fl(fl(fl(acc_bj) * us_b) * c_j), c_j = fl(scale_j * fl(1/tau)),
+ *   acc_bj = sum_i u8_bi * v8_ji exactly in int32
+ *   (recsys_two_tower_model.py `compute_top_k_int8`)
  *   For each query: the k eligible candidates with the largest s_bj, sorted by
  *   s descending; equal scores are ordered by ascending id. Candidates whose
  *   exclusion bit is set never appear. When fewer than k candidates are

@@ -86,6 +86,69 @@ class OracleSide:
         return ((words[ids >> 5] >> (ids & 31).astype(np.uint32)) & 1).astype(bool)
 
 
+class OracleSideQ8(OracleSide):
+    """The oracle's view of an int8 index: its own codes of its own
+    normalised corpus rows, and of its own stored queries coded as given."""
+
+    def __init__(self, w: W.Workload, raw_corpus_np: np.ndarray, raw_queries_np: np.ndarray,
+                 exclude_np: np.ndarray | None, qids: np.ndarray):
+        self.w = w
+        self.qids = qids
+        self.exclude = exclude_np
+        self.vcodes, self.vscales = oracle.quantize(raw_corpus_np, True)
+        stored_q = oracle.normalize(np.ascontiguousarray(raw_queries_np[qids]), w.query_dtype)
+        self.qcodes, self.qscales = oracle.quantize(stored_q, False)
+
+    def topk(self, k: int):
+        return oracle.topk_q8(self.qcodes, self.qscales, self.vcodes, self.vscales, k, tau=self.tau,
+                              exclude=self.exclude)
+
+    def scores_for(self, row: int, ids) -> np.ndarray:
+        return oracle.scores_for_q8(self.qcodes, self.qscales, row, self.vcodes, self.vscales, ids, tau=self.tau)
+
+
+def gpu_prepare_q8(w: W.Workload, raw_corpus: torch.Tensor, raw_queries: torch.Tensor):
+    """int8 index of the corpus (normalise + code on the GPU) and the stored
+    (normalised) queries; tt_score_topk codes the queries itself."""
+    import exact_inner_product_b200 as tt
+    codes = torch.empty((w.n, w.d), dtype=torch.int8, device=raw_corpus.device)
+    scales = torch.empty((w.n,), dtype=torch.float32, device=raw_corpus.device)
+    index = tt.tt_quantize_candidates(raw_corpus, codes, scales)
+    qdt = torch.float32 if w.query_dtype == "f32" else torch.bfloat16
+    qn = torch.empty((w.b, w.d), dtype=qdt, device=raw_queries.device)
+    tt.tt_normalize_candidates(raw_queries, qn, tt.TT_NORM_STORE, make_index=False)
+    return index, qn
+
+
+def q8_tolerance(w: W.Workload) -> float:
+    """Score tolerance of the int8 path: 2e-3 / tau. A code that rounds the
+    other way on the two sides (their normalised rows can differ in the last
+    fp32 bit) moves a score by us * scale * |code| / tau <= max|u| max|v| / 127
+    / tau, about 7e-4 / tau for unit rows at d = 128; such flips are rare (a
+    value must sit within ~1e-5 of a half step)."""
+    return 2e-3 / float(np.float32(w.tau))
+
+
+def run_case_q8(w: W.Workload, device="cuda", **options):
+    """int8 index: generate, run both sides, compare."""
+    import exact_inner_product_b200 as tt
+    raw_c = W.corpus(w, device)
+    raw_q = W.queries(w, device)
+    excl = W.exclusion_bits(w, device)
+    index, qn = gpu_prepare_q8(w, raw_c, raw_q)
+    ids, scores = tt.tt_score_topk(index, qn, w.k, tau=w.tau, exclude=excl, **options)
+    torch.cuda.synchronize()
+    qids = W.oracle_query_ids(w)
+    gi = ids.cpu().numpy()[qids]
+    gs = scores.cpu().numpy()[qids]
+    st = tt.tt_last_stats(index)
+    side = OracleSideQ8(w, W.to_numpy_rows(raw_c), raw_q.cpu().numpy(),
+                        None if excl is None else excl.cpu().numpy().view(np.uint32), qids)
+    del raw_c
+    res = compare(gi, gs, side, w.k, q8_tolerance(w))
+    return res, st
+
+
 def compare(gpu_ids: np.ndarray, gpu_scores: np.ndarray, side: OracleSide, k: int, tol: float,
             o_ids: np.ndarray | None = None, o_scores: np.ndarray | None = None) -> dict:
     """Apply the comparison rule to the sampled rows. gpu_* are [len(qids), k]."""

@@ -1,0 +1,113 @@
+"""The int8 path (recsys_two_tower_model.py `compute_top_k_int8`) against
+the oracle: corpus coding on the GPU against the oracle's codes, and exact
+top-k over int8 codes on the streaming (dp4a) and tensor-core (kind::i8)
+scorers, with masks, tau, ties and edge cases. (GPU)"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import parity
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+tt = pytest.importorskip("exact_inner_product_b200")
+
+
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+@pytest.mark.parametrize("name,n", [("stream_b1", 50_003), ("masked_fused", 20_011), ("tiny_f32", 400)])
+def test_coding_matches_oracle(name, n):
+    """Codes equal the oracle's except where the two sides' normalised values
+    (fp32 norm here, fp64 there) straddle a rounding half step: then they
+    differ by one. Scales agree to fp32 rounding."""
+    _cuda()
+    w = W.workload(name, n=n)
+    raw = W.corpus(w, "cuda")
+    codes = torch.empty((n, w.d), dtype=torch.int8, device="cuda")
+    scales = torch.empty((n,), dtype=torch.float32, device="cuda")
+    tt.tt_quantize_candidates(raw, codes, scales, make_index=False)
+    oc, os_ = oracle.quantize(W.to_numpy_rows(raw), True)
+    diff = np.abs(codes.cpu().numpy().astype(np.int32) - oc.astype(np.int32))
+    assert diff.max() <= 1
+    assert (diff == 0).mean() > 0.9995
+    assert np.allclose(scales.cpu().numpy(), os_, rtol=5e-7, atol=0)
+    assert np.abs(codes.cpu().numpy().astype(np.int32)).max() <= 127
+
+
+CASES = [
+    # name, overrides, expected path
+    ("stream_b1", {"n": 200_037}, 1),
+    ("stream_b1", {"n": 150_001, "b": 5, "k": 64}, 1),
+    ("small_batch", {"n": 300_077, "tau": 1.0}, 2),
+    ("small_batch", {"n": 100_003, "b": 9, "k": 17}, 2),
+    ("large_batch", {"n": 400_005, "b": 300, "k": 1000, "oracle_queries": 12}, 2),
+    ("masked_fused", {"n": 200_099, "b": 260, "oracle_queries": 12}, 2),
+    ("masked_fused", {"n": 120_031, "b": 3, "k": 256}, 1),
+]
+
+
+@pytest.mark.parametrize("name,over,path", CASES, ids=[f"{c[0]}-{i}" for i, c in enumerate(CASES)])
+def test_int8_parity(name, over, path):
+    _cuda()
+    w = W.workload(name, **over)
+    res, st = parity.run_case_q8(w)
+    assert st["path"] == path, st
+    assert res["max_abs_err"] <= parity.q8_tolerance(w)
+    assert res.get("sure_checked", 0) > 0
+
+
+def test_int8_both_scorers_agree():
+    """The dp4a streaming scorer and the kind::i8 tensor-core scorer compute
+    the same exact integer sums, so their results are identical."""
+    _cuda()
+    w = W.workload("small_batch", n=70_001, b=40, k=100, tau=1.0)
+    raw_c, raw_q = W.corpus(w, "cuda"), W.queries(w, "cuda")
+    index, qn = parity.gpu_prepare_q8(w, raw_c, raw_q)
+    a = tt.tt_score_topk(index, qn, w.k, path=1)
+    assert tt.tt_last_stats(index)["path"] == 1
+    b = tt.tt_score_topk(index, qn, w.k, path=2)
+    assert tt.tt_last_stats(index)["path"] == 2
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    res, _ = parity.run_case_q8(w, path=1)
+    assert res["max_abs_err"] <= parity.q8_tolerance(w)
+
+
+def test_int8_ties_and_edges():
+    _cuda()
+    d = 64
+    # identical rows: every score ties; ids must come out 0..k-1 on both scorers
+    row = torch.nn.functional.normalize(torch.randn(1, d), dim=1)
+    raw = row.repeat(5000, 1).cuda().contiguous()
+    codes = torch.empty((5000, d), dtype=torch.int8, device="cuda")
+    scales = torch.empty((5000,), dtype=torch.float32, device="cuda")
+    index = tt.tt_quantize_candidates(raw, codes, scales)
+    for path, b in ((1, 2), (2, 40)):
+        q = torch.randn(b, d, device="cuda")
+        ids, sc = tt.tt_score_topk(index, q, 300, path=path)
+        assert (ids.cpu() == torch.arange(300, dtype=torch.int32)[None, :]).all()
+        assert (sc == sc[:, :1]).all()
+    # k > n pads; everything excluded pads
+    small = tt.tt_index_wrap(codes[:40].contiguous(), scales[:40].contiguous())
+    q = torch.randn(12, d, device="cuda")
+    ids, sc = tt.tt_score_topk(small, q, 50)
+    assert (ids[:, 40:] == -1).all() and torch.isinf(sc[:, 40:]).all()
+    excl = torch.full((2,), -1, dtype=torch.int32, device="cuda")
+    ids, _ = tt.tt_score_topk(small, q, 5, exclude=excl)
+    assert (ids == -1).all()
+    # int8 rows need the scales, d % 32 == 0, and no SM-pair kernel
+    with pytest.raises(tt.TTError) as e:
+        tt.tt_index_wrap(codes)
+    assert e.value.status == tt.TT_ERR_INVALID_ARG
+    odd = torch.empty((10, 48), dtype=torch.int8, device="cuda")
+    ix48 = tt.tt_index_wrap(odd, torch.ones(10, device="cuda"))
+    with pytest.raises(tt.TTError) as e:
+        tt.tt_score_topk(ix48, torch.randn(2, 48, device="cuda"), 3)
+    assert e.value.status == tt.TT_ERR_UNSUPPORTED
+    with pytest.raises(tt.TTError) as e:
+        tt.tt_score_topk(index, torch.randn(300, d, device="cuda"), 3, path=3)
+    assert e.value.status == tt.TT_ERR_UNSUPPORTED
