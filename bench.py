@@ -56,9 +56,9 @@ PATH_NAMES = {1: "streaming", 2: "tensor-core", 3: "tensor-core (SM pairs)"}
 # applied to every level of a step, like `achieved`).
 TRAFFIC = {
     # ncu --set full -k regex:k1_normalize -s 5 -c 1 on `python bench.py --steps 50 --warmup 3
-    # --no-e2e --no-cpu-baseline`: 512.016 MB read + 201.165 MB written for 1,000,000 rows
-    ("k1_normalize", "stream_b1"): {"bytes_per_row": 713.181, "src": "exact_inner_product_b200/csrc/k_normalize.cu",
-                                    "sha": "6d3e520d16da8b6d042167b6dd9594cc512d14f3cc131115f5cdfec93e963db7"},
+    # --no-e2e --no-cpu-baseline`: 512.019 MB read + 200.806 MB written for 1,000,000 rows
+    ("k1_normalize", "stream_b1"): {"bytes_per_row": 712.825, "src": "exact_inner_product_b200/csrc/k_normalize.cu",
+                                    "sha": "4273a9f8869b74ec01b8762c20eb598dc6f0b1597fcd3e5f8ad9afde664127f4"},
     # ncu --set full -k regex:k3_pair -s 5 -c 1 on `python bench.py --workload large_batch --n 4000000
     # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 1587.723 MB read
     # + 27.798 MB written; scaled to the full corpus by rows scanned
