@@ -60,15 +60,15 @@ TRAFFIC = {
     ("k1_normalize", "stream_b1"): {"bytes_per_row": 712.825, "src": "exact_inner_product_b200/csrc/k_normalize.cu",
                                     "sha": "4273a9f8869b74ec01b8762c20eb598dc6f0b1597fcd3e5f8ad9afde664127f4"},
     # ncu --set full -k regex:k3_pair -s 5 -c 1 on `python bench.py --workload large_batch --n 4000000
-    # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 1587.723 MB read
-    # + 27.798 MB written; scaled to the full corpus by rows scanned
-    ("k3_pair", "large_batch"): {"bytes_per_row": 403.880, "src": "exact_inner_product_b200/csrc/k_tensor_pair.cu",
-                                 "sha": "43e2c4b1ce6837870992c30a53efa9ec8d8dfb0ced721048ba161508dce63734"},
+    # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 1738.856 MB read
+    # + 26.853 MB written; scaled to the full corpus by rows scanned
+    ("k3_pair", "large_batch"): {"bytes_per_row": 441.427, "src": "exact_inner_product_b200/csrc/k_tensor_pair.cu",
+                                 "sha": "10e96adf483df1eed057e58de3cca01783ba80d0d841dc4d9b22c65146f76f0d"},
     # ncu --set full -k regex:k3_tensor -s 5 -c 1 on `python bench.py --workload masked_fused --n 4000000
-    # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 4984.254 MB read
-    # + 73.270 MB written; scaled to the full corpus by rows scanned
-    ("k3_tensor", "masked_fused"): {"bytes_per_row": 1264.381, "src": "exact_inner_product_b200/csrc/k_tensor.cu",
-                                    "sha": "de8f36cb5cd9b834950b076a917f656f291e63dd7a3a7ad71247af58d6443feb"},
+    # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 4557.230 MB read
+    # + 69.327 MB written; scaled to the full corpus by rows scanned
+    ("k3_tensor", "masked_fused"): {"bytes_per_row": 1156.639, "src": "exact_inner_product_b200/csrc/k_tensor.cu",
+                                    "sha": "e272fbce88a48a18de133cbebd3c8729fab9cc163a4c3bb86fa6fb30575524b8"},
 }
 
 

@@ -85,6 +85,10 @@ _sig("tt_plan", ctypes.c_int, [_i64, _i32, ctypes.POINTER(tt_options), ctypes.PO
 _sig("tt_score_topk_noalloc", ctypes.c_int, [_vp, ctypes.c_int, _i64, _i32, _vp, _vp, ctypes.c_int, _i32,
                                              _vp, ctypes.c_float, _i32, _vp, _vp, _vp])
 _sig("tt_merge_topk", ctypes.c_int, [_vp, _vp, _i32, _i32, _i32, ctypes.POINTER(_i64), _i32, _vp, _vp, _vp])
+_sig("tt_score_topk_ranges", ctypes.c_int, [_vp, _vp, ctypes.c_int, _i32, _vp, ctypes.c_float, _i32, _i32,
+                                            ctypes.POINTER(_i64), _vp, _vp, _vp])
+_sig("tt_score_topk_types", ctypes.c_int, [_vp, _vp, ctypes.c_int, _i32, _vp, ctypes.c_float, _i32, _vp, _i32,
+                                           ctypes.POINTER(_i32), _vp, _vp, _vp])
 _sig("tt_free", None, [_vp])
 _sig("tt_launch_count", _i64, [])
 _sig("tt_profile_begin", ctypes.c_int, [])
@@ -96,7 +100,7 @@ _sig("tt_last_error", ctypes.c_char_p, [])
 _sig("tt_version", ctypes.c_char_p, [])
 
 EXPORTED = ("tt_normalize_candidates", "tt_quantize_candidates", "tt_index_wrap", "tt_score_topk", "tt_score_topk_ex",
-            "tt_score_topk_noalloc", "tt_merge_topk",
+            "tt_score_topk_noalloc", "tt_merge_topk", "tt_score_topk_ranges", "tt_score_topk_types",
             "tt_last_stats", "tt_plan", "tt_free", "tt_launch_count", "tt_profile_begin",
             "tt_profile_end", "tt_profile_launches", "tt_status_string", "tt_last_error", "tt_version")
 
@@ -297,6 +301,50 @@ def tt_merge_topk(ids: torch.Tensor, scores: torch.Tensor, id_offsets, k_out: in
         out_scores = torch.empty((b, k_out), dtype=torch.float32, device=dev)
     _check(_lib.tt_merge_topk(_ptr(ids), _ptr(scores), parts, b, k_in, offs, int(k_out), _ptr(out_ids),
                               _ptr(out_scores), _stream(stream)), "tt_merge_topk")
+    return out_ids, out_scores
+
+
+def _check_queries(index: Index, queries: torch.Tensor, exclude):
+    if queries.dim() != 2 or not queries.is_contiguous():
+        raise ValueError("queries must be a contiguous [b, d] tensor")
+    if queries.shape[1] != index.d:
+        raise ValueError(f"queries have d={queries.shape[1]}, index has d={index.d}")
+    if exclude is not None and (exclude.dtype != torch.int32 or not exclude.is_contiguous()):
+        raise TypeError("exclude must be a contiguous int32 tensor of packed bits")
+
+
+def tt_score_topk_ranges(index: Index, queries: torch.Tensor, k: int, ranges, tau: float = 1.0,
+                         exclude: torch.Tensor | None = None, stream=None):
+    """One top-k per candidate range [start, end) (``tt_score_topk_ranges``).
+    Returns ``(ids int32 [R, b, k], scores float32 [R, b, k])`` with corpus ids."""
+    _check_queries(index, queries, exclude)
+    b = queries.shape[0]
+    R = len(ranges)
+    flat = (_i64 * (2 * max(1, R)))(*[int(v) for rng in ranges for v in rng])
+    out_ids = torch.empty((R, b, k), dtype=torch.int32, device=queries.device)
+    out_scores = torch.empty((R, b, k), dtype=torch.float32, device=queries.device)
+    _check(_lib.tt_score_topk_ranges(index.handle, _ptr(queries), _dtype(queries), b, _ptr(exclude), float(tau),
+                                     int(k), R, flat, _ptr(out_ids), _ptr(out_scores), _stream(stream)),
+           "tt_score_topk_ranges")
+    return out_ids, out_scores
+
+
+def tt_score_topk_types(index: Index, queries: torch.Tensor, k: int, types: torch.Tensor, set_types,
+                        tau: float = 1.0, exclude: torch.Tensor | None = None, stream=None):
+    """One top-k per candidate type (``tt_score_topk_types``): ``types`` is a
+    uint8 [n] tensor on the GPU, ``set_types`` the types to report. Returns
+    ``(ids int32 [T, b, k], scores float32 [T, b, k])``."""
+    _check_queries(index, queries, exclude)
+    if types.dtype != torch.uint8 or not types.is_contiguous():
+        raise TypeError("types must be a contiguous uint8 tensor")
+    b = queries.shape[0]
+    T = len(set_types)
+    st_arr = (_i32 * max(1, T))(*[int(t) for t in set_types])
+    out_ids = torch.empty((T, b, k), dtype=torch.int32, device=queries.device)
+    out_scores = torch.empty((T, b, k), dtype=torch.float32, device=queries.device)
+    _check(_lib.tt_score_topk_types(index.handle, _ptr(queries), _dtype(queries), b, _ptr(exclude), float(tau),
+                                    int(k), _ptr(types), T, st_arr, _ptr(out_ids), _ptr(out_scores),
+                                    _stream(stream)), "tt_score_topk_types")
     return out_ids, out_scores
 
 

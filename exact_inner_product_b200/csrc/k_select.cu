@@ -325,6 +325,37 @@ __global__ void k4_pad(int32_t* out_ids, float* out_scores, int64_t count) {
     }
 }
 
+// Exclusion words of rows [start, start + count): bit i of out word w is bit
+// (start + 32w + i) of the input mask (0 past the end, or when there is no
+// input mask). With `types`, a row whose type differs from `want` is
+// excluded as well.
+__global__ void k4_mask_slice(const uint32_t* __restrict__ in, int64_t start, int64_t count,
+                              const uint8_t* __restrict__ types, int want, uint32_t* __restrict__ out) {
+    const int64_t words = (count + 31) / 32;
+    for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < words;
+         w += (int64_t)gridDim.x * blockDim.x) {
+        uint32_t v = 0;
+        for (int i = 0; i < 32; ++i) {
+            const int64_t r = 32 * w + i;
+            if (r >= count) break;
+            const int64_t j = start + r;
+            bool ex = in != nullptr && ((in[j >> 5] >> (j & 31)) & 1u);
+            if (types != nullptr && types[j] != (uint8_t)want) ex = true;
+            v |= (ex ? 1u : 0u) << i;
+        }
+        out[w] = v;
+    }
+}
+
+// ids += offset where ids >= 0 (padding stays -1).
+__global__ void k4_offset_ids(int32_t* ids, int64_t count, int64_t offset) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int32_t v = ids[i];
+        if (v >= 0) ids[i] = (int32_t)(v + offset);
+    }
+}
+
 unsigned small_grid(int64_t n) {
     int64_t g = (n + 255) / 256;
     if (g < 1) g = 1;
@@ -388,6 +419,23 @@ cudaError_t launch_prepare_repair(uint64_t* theta, float* thf, const int32_t* st
                                   int* flags, cudaStream_t s) {
     note_launch_begin(TT_KIND_AUX, s);
     k4_prepare_repair<<<small_grid(b), 256, 0, s>>>(theta, thf, status, b, flags);
+    note_launch_end(TT_KIND_AUX, s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_mask_slice(const uint32_t* in, int64_t start, int64_t count, const uint8_t* types, int want,
+                              uint32_t* out, cudaStream_t s) {
+    if (count == 0) return cudaSuccess;
+    note_launch_begin(TT_KIND_AUX, s);
+    k4_mask_slice<<<small_grid((count + 31) / 32), 256, 0, s>>>(in, start, count, types, want, out);
+    note_launch_end(TT_KIND_AUX, s);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_offset_ids(int32_t* ids, int64_t count, int64_t offset, cudaStream_t s) {
+    if (count == 0 || offset == 0) return cudaSuccess;
+    note_launch_begin(TT_KIND_AUX, s);
+    k4_offset_ids<<<small_grid(count), 256, 0, s>>>(ids, count, offset);
     note_launch_end(TT_KIND_AUX, s);
     return cudaGetLastError();
 }

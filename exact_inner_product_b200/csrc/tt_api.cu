@@ -883,6 +883,107 @@ tt_status tt_merge_topk(const int32_t* ids, const float* scores, int32_t parts, 
     return TT_OK;
 }
 
+// One result set: rows [start, start + count) of the index, a mask already
+// sliced to those rows (or null), ids reported as corpus ids.
+static tt_status score_rows(tt_index* index, int64_t start, int64_t count, const void* queries, tt_dtype q_dtype,
+                            int32_t b, const uint32_t* mask, float tau, int32_t k, int32_t* out_ids,
+                            float* out_scores, cudaStream_t s) {
+    const int esize = index->dtype == TT_F32 ? 4 : index->dtype == TT_BF16 ? 2 : 1;
+    tt_index* sub = nullptr;
+    tt_status st = new_index(static_cast<const uint8_t*>(index->rows) + start * index->d * esize, index->dtype,
+                             count, index->d, index->inv_norm ? index->inv_norm + start : nullptr, &sub);
+    if (st != TT_OK) return st;
+    st = tt_score_topk_ex(sub, queries, q_dtype, b, mask, tau, k, out_ids, out_scores, s, nullptr);
+    index->last = sub->last;
+    tt_free(sub);  // the call above synchronised its stream: the scratch is idle
+    if (st != TT_OK) return st;
+    cudaError_t e = launch_offset_ids(out_ids, (int64_t)b * k, start, s);
+    if (e != cudaSuccess) return cuda_fail(e, "id offset");
+    return TT_OK;
+}
+
+// Common host checks of the multi-set calls (no device calls).
+static tt_status check_sets(const tt_index* index, int32_t b, int32_t k, int32_t n_sets, const void* queries,
+                            const int32_t* out_ids, const float* out_scores) {
+    if (!index || b < 0 || k <= 0) return TT_ERR_INVALID_ARG;
+    if (k > TT_MAX_K) return TT_ERR_UNSUPPORTED;
+    if (n_sets < 1) return TT_ERR_INVALID_ARG;
+    if (n_sets > TT_MAX_PARTS) return TT_ERR_UNSUPPORTED;
+    if (b > 0 && (queries == nullptr || out_ids == nullptr || out_scores == nullptr)) return TT_ERR_INVALID_ARG;
+    if (!aligned(out_ids, 4) || !aligned(out_scores, 4)) return TT_ERR_INVALID_ARG;
+    return TT_OK;
+}
+
+tt_status tt_score_topk_ranges(tt_index* index, const void* queries, tt_dtype q_dtype, int32_t b,
+                               const uint32_t* exclude_bits, float tau, int32_t k, int32_t n_ranges,
+                               const int64_t* ranges, int32_t* out_ids, float* out_scores, void* stream) {
+    tt_status st = check_sets(index, b, k, n_ranges, queries, out_ids, out_scores);
+    if (st != TT_OK) return st;
+    if (!ranges) return TT_ERR_INVALID_ARG;
+    for (int r = 0; r < n_ranges; ++r)
+        if (ranges[2 * r] < 0 || ranges[2 * r] > ranges[2 * r + 1] || ranges[2 * r + 1] > index->n)
+            return TT_ERR_INVALID_ARG;
+    if (!aligned(exclude_bits, 4)) return TT_ERR_INVALID_ARG;
+    if (b == 0) return TT_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t per_set = (int64_t)b * k;
+    for (int r = 0; r < n_ranges; ++r) {
+        const int64_t start = ranges[2 * r], count = ranges[2 * r + 1] - start;
+        uint32_t* mask = nullptr;
+        if (exclude_bits && count > 0) {
+            if ((st = check_device_ptr(exclude_bits, "exclude_bits")) != TT_OK) return st;
+            TT_CUDA(cudaMallocAsync(reinterpret_cast<void**>(&mask), (size_t)((count + 31) / 32) * 4, s),
+                    "range mask");
+            cudaError_t e = launch_mask_slice(exclude_bits, start, count, nullptr, 0, mask, s);
+            if (e != cudaSuccess) {
+                cudaFreeAsync(mask, s);
+                return cuda_fail(e, "range mask");
+            }
+        }
+        st = score_rows(index, start, count, queries, q_dtype, b, mask, tau, k, out_ids + r * per_set,
+                        out_scores + r * per_set, s);
+        if (mask) cudaFreeAsync(mask, s);
+        if (st != TT_OK) return st;
+    }
+    return TT_OK;
+}
+
+tt_status tt_score_topk_types(tt_index* index, const void* queries, tt_dtype q_dtype, int32_t b,
+                              const uint32_t* exclude_bits, float tau, int32_t k, const uint8_t* types,
+                              int32_t n_sets, const int32_t* set_types, int32_t* out_ids, float* out_scores,
+                              void* stream) {
+    tt_status st = check_sets(index, b, k, n_sets, queries, out_ids, out_scores);
+    if (st != TT_OK) return st;
+    if (!set_types || (index->n > 0 && !types)) return TT_ERR_INVALID_ARG;
+    for (int t = 0; t < n_sets; ++t)
+        if (set_types[t] < 0 || set_types[t] > 255) return TT_ERR_INVALID_ARG;
+    if (!aligned(exclude_bits, 4)) return TT_ERR_INVALID_ARG;
+    if (b == 0) return TT_OK;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (index->n > 0) {
+        if ((st = check_device_ptr(types, "types")) != TT_OK) return st;
+        if ((st = check_device_ptr(exclude_bits, "exclude_bits")) != TT_OK) return st;
+    }
+    const int64_t per_set = (int64_t)b * k;
+    const int64_t words = (index->n + 31) / 32;
+    uint32_t* mask = nullptr;
+    if (words > 0) TT_CUDA(cudaMallocAsync(reinterpret_cast<void**>(&mask), (size_t)words * 4, s), "type mask");
+    for (int t = 0; t < n_sets; ++t) {
+        if (mask) {
+            cudaError_t e = launch_mask_slice(exclude_bits, 0, index->n, types, set_types[t], mask, s);
+            if (e != cudaSuccess) {
+                cudaFreeAsync(mask, s);
+                return cuda_fail(e, "type mask");
+            }
+        }
+        st = score_rows(index, 0, index->n, queries, q_dtype, b, mask, tau, k, out_ids + t * per_set,
+                        out_scores + t * per_set, s);
+        if (st != TT_OK) break;
+    }
+    if (mask) cudaFreeAsync(mask, s);
+    return st;
+}
+
 tt_status tt_score_topk(tt_index* index, const void* queries, tt_dtype q_dtype, int32_t b,
                         const uint32_t* exclude_bits, float tau, int32_t k, int32_t* out_ids,
                         float* out_scores, void* stream) {

@@ -90,6 +90,12 @@ cudaError_t launch_prepare_repair(uint64_t* theta, float* thf, const int32_t* st
 bool bf16_tile_tensor_map(const void* base, int64_t rows, int d, int64_t row_pitch_elems,
                           int box_rows, CUtensorMap* tm);
 cudaError_t launch_pad(int32_t* out_ids, float* out_scores, int64_t count, cudaStream_t s);
+// Exclusion words for rows [start, start + count) of a mask (null: none),
+// optionally also excluding rows whose types[j] != want (types null: none).
+cudaError_t launch_mask_slice(const uint32_t* in, int64_t start, int64_t count, const uint8_t* types, int want,
+                              uint32_t* out, cudaStream_t s);
+// ids[i] += offset where ids[i] >= 0.
+cudaError_t launch_offset_ids(int32_t* ids, int64_t count, int64_t offset, cudaStream_t s);
 
 // Shared-memory bytes the tensor-core pass needs for a given d and query tile.
 // esize: bytes per element of the rows (2 bf16, 1 int8).

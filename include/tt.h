@@ -262,6 +262,52 @@ TT_API tt_status tt_merge_topk(const int32_t* ids, const float* scores, int32_t 
                                int32_t k_in, const int64_t* id_offsets, int32_t k_out,
                                int32_t* out_ids, float* out_scores, void* stream);
 
+/*
+ * tt_score_topk_ranges - one top-k list per candidate range, from one call.
+ *
+ * (recsys_two_tower_model.py `forward`, the `dataset_ranges` path: for each
+ *  (start, end) the candidate slice [start, end) gets its own top-k, with
+ *  indices offset by start.)
+ *
+ * For range r = [ranges[2r], ranges[2r+1]) the result is exactly
+ * tt_score_topk over the rows of that range (same scores, same order and
+ * padding), with ids reported as corpus ids. Ranges may be empty or
+ * overlap. Each range is scanned once, so disjoint ranges together read
+ * each row at most once.
+ *
+ * ranges    HOST int64 [n_ranges * 2]: 0 <= start <= end <= n
+ * n_ranges  1 <= n_ranges <= TT_MAX_PARTS
+ * out_ids, out_scores  device [n_ranges, b, k]
+ * other arguments, the exactness and the errors as tt_score_topk; the call
+ * returns once the results are complete on `stream`.
+ */
+TT_API tt_status tt_score_topk_ranges(tt_index* index, const void* queries, tt_dtype q_dtype, int32_t b,
+                                      const uint32_t* exclude_bits, float tau, int32_t k, int32_t n_ranges,
+                                      const int64_t* ranges, int32_t* out_ids, float* out_scores,
+                                      void* stream);
+
+/*
+ * tt_score_topk_types - one top-k list per candidate type, from one call.
+ *
+ * (recsys_two_tower_model.py `forward`, the `target_dataset_types` path: for
+ *  each target type, `mask_and_top_k` over the candidates whose dataset type
+ *  matches.)
+ *
+ * Set s keeps only candidates j with types[j] == set_types[s] (and not
+ * excluded by exclude_bits); the result is exactly tt_score_topk with that
+ * combined mask. Each set is a separate pass over the corpus.
+ *
+ * types      device uint8 [n]: the type of every candidate
+ * set_types  HOST int32 [n_sets], each 0..255
+ * n_sets     1 <= n_sets <= TT_MAX_PARTS
+ * out_ids, out_scores  device [n_sets, b, k]
+ * other arguments, the exactness and the errors as tt_score_topk.
+ */
+TT_API tt_status tt_score_topk_types(tt_index* index, const void* queries, tt_dtype q_dtype, int32_t b,
+                                     const uint32_t* exclude_bits, float tau, int32_t k, const uint8_t* types,
+                                     int32_t n_sets, const int32_t* set_types, int32_t* out_ids,
+                                     float* out_scores, void* stream);
+
 /* Release a handle. Its scratch memory returns to a per-device pool that
  * later handles reuse (it is not returned to CUDA before the process exits).
  * NULL is a no-op. Must not be called while work using the handle is still

@@ -136,6 +136,31 @@ def test_merge_validation_before_device_calls():
     assert call(b=0) == tt.TT_OK
 
 
+def test_set_calls_validate_before_device_calls():
+    lib = tt._lib
+    fake = ctypes.c_void_p(0x10000)
+    ix = _empty_index()
+    rng = (ctypes.c_int64 * 2)(0, 0)
+    call = lambda **kw: lib.tt_score_topk_ranges(kw.get("ix", ix), fake, 1, kw.get("b", 0), None, 1.0,
+                                                 kw.get("k", 5), kw.get("nr", 1), kw.get("rng", rng), fake,
+                                                 fake, None)
+    assert call() == tt.TT_OK  # b = 0: nothing to do
+    assert call(ix=None) == tt.TT_ERR_INVALID_ARG
+    assert call(nr=0) == tt.TT_ERR_INVALID_ARG
+    assert call(nr=65) == tt.TT_ERR_UNSUPPORTED
+    assert call(k=0) == tt.TT_ERR_INVALID_ARG
+    assert call(k=4096) == tt.TT_ERR_UNSUPPORTED
+    assert call(rng=None) == tt.TT_ERR_INVALID_ARG
+    assert call(rng=(ctypes.c_int64 * 2)(0, 1)) == tt.TT_ERR_INVALID_ARG  # end past n = 0
+    types_call = lambda st, n=1: lib.tt_score_topk_types(ix, fake, 1, 0, None, 1.0, 5, None, n, st, fake, fake,
+                                                         None)
+    assert types_call((ctypes.c_int32 * 1)(3)) == tt.TT_OK
+    assert types_call(None) == tt.TT_ERR_INVALID_ARG
+    assert types_call((ctypes.c_int32 * 1)(256)) == tt.TT_ERR_INVALID_ARG
+    assert types_call((ctypes.c_int32 * 1)(3), n=0) == tt.TT_ERR_INVALID_ARG
+    lib.tt_free(ix)
+
+
 def test_plan_levels():
     # the deepest level holds at most `cap` rows; strides are powers of 64
     for n, k in ((400, 10), (10 ** 6, 100), (10 ** 7, 500), (5 * 10 ** 7, 1000), (2 * 10 ** 7, 256),
