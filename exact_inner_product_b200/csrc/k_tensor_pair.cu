@@ -283,13 +283,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
             uint64_t* qkeys = a.keys + (int64_t)q * a.cap;
             // Per-row data of this warp's 128 columns of a tile, fetched one
             // tile ahead: lane l holds rows l, l+32, l+64, l+96 - the inverse
-            // norm (rows with norms; 0 past the last row) and the mask word
-            // holding the row's exclusion bit. That bit sits at position l
-            // when level rows are corpus rows, and at 0 on coarser levels
-            // (their strides are multiples of 64).
+            // norm (rows with norms; 0 past the last row), the mask word
+            // holding the row's exclusion bit and that bit's position.
             float cl[4];
-            uint32_t xl[4];
-            const uint32_t xshift = a.stride == 1 ? (uint32_t)lane : 0u;
+            uint32_t xl[4], xs[4];
             auto fetch_rows = [&](int64_t tile) {
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -297,7 +294,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
                     const bool valid = r < a.n_rows;
                     // raw values: nothing waits for these loads until the next tile
                     if (!uniform_c) cl[j] = valid ? __ldg(a.inv_norm + r * a.stride) : 0.0f;
-                    if (a.exclude) xl[j] = valid ? __ldg(a.exclude + ((r * a.stride) >> 5)) : 0u;
+                    if (a.exclude) {
+                        xl[j] = valid ? __ldg(a.exclude + ((r * a.stride) >> 5)) : 0u;
+                        xs[j] = (uint32_t)((r * a.stride) & 31);
+                    }
                 }
             };
             if (!uniform_c || a.exclude) fetch_rows(t0);
@@ -309,7 +309,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     bool bad = row0 + lane + 32 * j >= a.n_rows;
-                    if (a.exclude) bad |= ((xl[j] >> xshift) & 1u) != 0u;
+                    if (a.exclude) bad |= ((xl[j] >> xs[j]) & 1u) != 0u;
                     skip[j] = __ballot_sync(0xFFFFFFFFu, bad);
                 }
                 if (!uniform_c) {

@@ -5,8 +5,8 @@
 // each scoring pass keeps, per query, only candidates whose key (score, id)
 // beats a threshold key theta, and the final selection checks that the pass
 // kept everything it had to. Thresholds are estimated on coarser levels of
-// the corpus (every 64th row, every 4096th row, ...): the r-th best key of a
-// level, taken with r about 3k/64, predicts a filter that keeps about 3k
+// the corpus (every 61st row, every 3721st row, ...): the r-th best key of a
+// level, taken with r about 3k/61, predicts a filter that keeps about 3k
 // candidates of the next finer level. The deepest level is small enough to
 // keep every key (no threshold). A query's final pass is exact when it kept
 // at least k keys (so every member of the true top-k beat the threshold) and
@@ -222,15 +222,18 @@ static int sm_count_current() {
 // ---------------------------------------------------------------------------
 // scan plan
 // ---------------------------------------------------------------------------
-constexpr int STRIDE_RATIO = 64;
+// Level i samples every 61^i-th row. A prime stride keeps the samples spread
+// over masks that repeat with a period of 2, 4, 8, ... rows (with a stride
+// of 64, every sample of `type = id % 4` would have the same type).
+constexpr int STRIDE_RATIO = 61;
 constexpr int DEFAULT_CAP = 16384;
 constexpr int MAX_DEEPEST_ROWS = 4096;  // the deepest level keeps every key
 // Floors of the ranks. The survivors of a pass whose threshold is the r-th
-// best key of a 1/64 sample number about Gamma(r, 64); a pass that must keep
-// `need` keys falls short with probability P(Poisson(need / 64) >= r).
-// Level 1 sets the threshold of the full pass (need = k): r >= max(3k/64, 32)
+// best key of a 1/61 sample number about Gamma(r, 61); a pass that must keep
+// `need` keys falls short with probability P(Poisson(need / 61) >= r).
+// Level 1 sets the threshold of the full pass (need = k): r >= max(3k/61, 32)
 // puts that below 1e-8 per query. Deeper levels only feed a coarser pass
-// (need <= a few dozen, so need / 64 < 1) and 10 suffices there, with far
+// (need <= a few dozen, so need / 61 < 1) and 10 suffices there, with far
 // fewer keys kept per pass.
 constexpr int MIN_RANK = 32;
 constexpr int MIN_RANK_DEEP = 10;

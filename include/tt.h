@@ -222,7 +222,7 @@ TT_API tt_status tt_last_stats(const tt_index* index, tt_stats* out);
 /*
  * tt_plan - the scan plan tt_score_topk would use for a corpus of n rows and
  * a given k (host only, no device work). Level 0 is the whole corpus; level i
- * scans every (64^i)-th row. The deepest level keeps every key; the r-th best
+ * scans every (61^i)-th row. The deepest level keeps every key; the r-th best
  * key of level i (ranks[i], i >= 1) sets the filter threshold of level i-1.
  * Arrays receive up to 4 entries. Any output pointer may be NULL.
  * Errors as tt_score_topk for n, k and options.

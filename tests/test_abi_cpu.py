@@ -162,25 +162,25 @@ def test_set_calls_validate_before_device_calls():
 
 
 def test_plan_levels():
-    # the deepest level holds at most `cap` rows; strides are powers of 64
+    # the deepest level holds at most `cap` rows; strides are powers of 61
     for n, k in ((400, 10), (10 ** 6, 100), (10 ** 7, 500), (5 * 10 ** 7, 1000), (2 * 10 ** 7, 256),
                  (2 ** 31 - 1, 2048), (1, 1), (0, 7)):
         p = tt.tt_plan(n, k)
         assert p["rows"][-1] <= 4096 or p["levels"] == 4
         assert p["rows"][0] == n
         for i, (r, s) in enumerate(zip(p["rows"], p["strides"])):
-            assert s == 64 ** i
+            assert s == 61 ** i
             assert r == (n + s - 1) // s
-        # expected survivors at each finer level ~ rank * 64, comfortably above
+        # expected survivors at each finer level ~ rank * 61, comfortably above
         # the rank needed there and within the buffer
         for i in range(1, p["levels"]):
             need = p["ranks"][i - 1]
-            assert p["ranks"][i] * 64 >= 3 * need
-            assert p["ranks"][i] * 64 <= p["cap"] // 2
+            assert p["ranks"][i] * 61 >= 3 * need
+            assert p["ranks"][i] * 61 <= p["cap"] // 2
     assert tt.tt_plan(400, 10)["levels"] == 1
-    assert tt.tt_plan(10 ** 6, 100) == {"levels": 3, "rows": [10 ** 6, 15625, 245], "strides": [1, 64, 4096],
+    assert tt.tt_plan(10 ** 6, 100) == {"levels": 3, "rows": [10 ** 6, 16394, 269], "strides": [1, 61, 3721],
                                         "ranks": [100, 32, 10], "cap": 16384}
-    assert tt.tt_plan(5 * 10 ** 7, 1000)["ranks"] == [1000, 47, 10, 10]
+    assert tt.tt_plan(5 * 10 ** 7, 1000)["ranks"] == [1000, 50, 10, 10]
     assert tt.tt_plan(4096, 10)["levels"] == 1 and tt.tt_plan(4097, 10)["levels"] == 2
     assert tt.tt_plan(10 ** 6, 100, force_levels=1)["levels"] == 1
     assert tt.tt_plan(10 ** 6, 100, force_levels=3)["levels"] == 3
