@@ -60,10 +60,10 @@ TRAFFIC = {
     ("k1_normalize", "stream_b1"): {"bytes_per_row": 712.825, "src": "exact_inner_product_b200/csrc/k_normalize.cu",
                                     "sha": "4273a9f8869b74ec01b8762c20eb598dc6f0b1597fcd3e5f8ad9afde664127f4"},
     # ncu --set full -k regex:k3_pair -s 5 -c 1 on `python bench.py --workload large_batch --n 4000000
-    # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 1738.856 MB read
-    # + 26.853 MB written; scaled to the full corpus by rows scanned
-    ("k3_pair", "large_batch"): {"bytes_per_row": 441.427, "src": "exact_inner_product_b200/csrc/k_tensor_pair.cu",
-                                 "sha": "10e96adf483df1eed057e58de3cca01783ba80d0d841dc4d9b22c65146f76f0d"},
+    # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 1773.760 MB read
+    # + 27.450 MB written; scaled to the full corpus by rows scanned
+    ("k3_pair", "large_batch"): {"bytes_per_row": 450.303, "src": "exact_inner_product_b200/csrc/k_tensor_pair.cu",
+                                 "sha": "26cccee2055038f9327e3160f5bd52beaace8eafa31f85c3b78cdb0b3eaa44db"},
     # ncu --set full -k regex:k3_tensor -s 5 -c 1 on `python bench.py --workload masked_fused --n 4000000
     # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 4557.230 MB read
     # + 69.327 MB written; scaled to the full corpus by rows scanned

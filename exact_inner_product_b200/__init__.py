@@ -49,7 +49,7 @@ if not os.path.exists(LIB_PATH):
 
 class tt_options(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int32), ("rank_scale_pct", ctypes.c_int32),
-                ("force_levels", ctypes.c_int32), ("cap", ctypes.c_int32)]
+                ("force_levels", ctypes.c_int32), ("cap", ctypes.c_int32), ("withhold_copy", ctypes.c_int32)]
 
 
 class tt_stats(ctypes.Structure):
@@ -138,8 +138,8 @@ def _stream(stream):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _options(path=0, rank_scale_pct=0, force_levels=0, cap=0):
-    return tt_options(int(path), int(rank_scale_pct), int(force_levels), int(cap))
+def _options(path=0, rank_scale_pct=0, force_levels=0, cap=0, withhold_copy=0):
+    return tt_options(int(path), int(rank_scale_pct), int(force_levels), int(cap), int(withhold_copy))
 
 
 class Index:

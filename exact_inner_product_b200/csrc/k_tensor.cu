@@ -156,6 +156,7 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
                             ok = false;
                             break;
                         }
+                        if (p.a.withhold_copy && it == 0) continue;  // test hook: never lands
                         mbar_arrive_expect_tx(&ctl->full[s], K3_STAGE_BYTES);
                         tma_load_2d(ring + (size_t)s * K3_STAGE_BYTES, &tm_rows, &ctl->full[s],
                                     kc * KC, (int32_t)(t * K3_M));

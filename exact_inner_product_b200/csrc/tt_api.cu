@@ -447,6 +447,7 @@ struct PathCfg {
     const void* queries;
     int q_dtype;
     const float* qscale;  // int8 index: query scales
+    int withhold_copy;    // test hook, see tt_options
     CUtensorMap tm_q;
 };
 
@@ -465,6 +466,7 @@ static tt_status run_pass(const tt_index* ix, const PathCfg& pc, const Plan& pla
     a.queries = pc.queries;
     a.q_dtype = pc.q_dtype;
     a.qscale = pc.qscale;
+    a.withhold_copy = pc.withhold_copy;
     a.b = b;
     a.theta = sc.theta;
     a.thf = sc.thf;
@@ -785,6 +787,7 @@ tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtyp
     pc.path = path;
     pc.queries = queries;
     pc.q_dtype = q_dtype;
+    pc.withhold_copy = options ? options->withhold_copy : 0;
     if (i8) {
         // code the queries as given (recsys_two_tower_model.py `compute_top_k_int8`)
         cudaError_t e = launch_quantize(queries, q_dtype, b, index->d, sc.qcodes, sc.qscale, false, s);

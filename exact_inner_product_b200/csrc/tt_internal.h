@@ -34,6 +34,7 @@ struct PassArgs {
     int cap;
     int* err;                  // device error word
     const float* qscale;       // [b] query scales of int8 rows, else null
+    int withhold_copy;         // test hook (tensor-core pass): skip the first corpus copy
 };
 
 // Set the text tt_last_error() returns on the calling thread.

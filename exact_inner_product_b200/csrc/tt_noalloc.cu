@@ -199,6 +199,7 @@ tt_status tt_score_topk_noalloc(const void* rows, tt_dtype dtype, int64_t n, int
         a.queries = q_use;
         a.q_dtype = q_dt_use;
         a.qscale = nullptr;
+        a.withhold_copy = 0;
         a.b = b;
         a.theta = theta;
         a.thf = thf;

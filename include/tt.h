@@ -199,6 +199,11 @@ typedef struct tt_options {
     int32_t force_levels;   /* 0 auto; > 0 = number of levels (1 = single pass) */
     int32_t cap;            /* 0 auto (16384); candidate buffer per query, power of 2,
                                256..16384 (test hook: small values provoke overflow) */
+    int32_t withhold_copy;  /* test hook, 0 = off. 1: the single-SM tensor-core pass
+                               (path 2) never issues its first corpus copy, so the wait
+                               for it gives up after its time limit (about 2 s) and the
+                               call returns TT_ERR_TIMEOUT; the device and the handle
+                               stay usable. Exercises the bounded-wait failure path. */
 } tt_options;
 
 TT_API tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtype, int32_t b,

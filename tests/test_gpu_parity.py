@@ -221,6 +221,26 @@ def test_repeat_runs_are_bitwise_identical():
     assert torch.equal(single[0], first[0]) and torch.equal(single[1], first[1])
 
 
+def test_bounded_wait_expiry_is_reported():
+    """The tensor-core pass is told (test hook) to withhold its first corpus
+    copy: the wait for it gives up after its time limit, every role of the
+    kernel drains and exits, and the call reports TT_ERR_TIMEOUT. The device
+    and the handle stay usable: the next call gives the earlier answer."""
+    import time
+    _cuda()
+    w = W.workload("small_batch", n=100_003, b=40, k=50)
+    raw_c, raw_q = W.corpus(w, "cuda"), W.queries(w, "cuda")
+    index, qn = parity.gpu_prepare(w, raw_c, raw_q)
+    good = tt.tt_score_topk(index, qn, w.k, path=2)
+    t0 = time.time()
+    with pytest.raises(tt.TTError) as e:
+        tt.tt_score_topk(index, qn, w.k, path=2, force_levels=1, withhold_copy=1)
+    assert e.value.status == tt.TT_ERR_TIMEOUT
+    assert time.time() - t0 < 60
+    again = tt.tt_score_topk(index, qn, w.k, path=2)
+    assert torch.equal(good[0], again[0]) and torch.equal(good[1], again[1])
+
+
 def test_rejects_host_pointers_and_bad_args():
     _cuda()
     rows = torch.randn(100, 64, device="cuda").to(torch.bfloat16)
