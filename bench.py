@@ -65,10 +65,10 @@ TRAFFIC = {
     ("k3_pair", "large_batch"): {"bytes_per_row": 450.303, "src": "exact_inner_product_b200/csrc/k_tensor_pair.cu",
                                  "sha": "26cccee2055038f9327e3160f5bd52beaace8eafa31f85c3b78cdb0b3eaa44db"},
     # ncu --set full -k regex:k3_tensor -s 5 -c 1 on `python bench.py --workload masked_fused --n 4000000
-    # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 4557.230 MB read
-    # + 69.327 MB written; scaled to the full corpus by rows scanned
-    ("k3_tensor", "masked_fused"): {"bytes_per_row": 1156.639, "src": "exact_inner_product_b200/csrc/k_tensor.cu",
-                                    "sha": "e272fbce88a48a18de133cbebd3c8729fab9cc163a4c3bb86fa6fb30575524b8"},
+    # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 4599.171 MB read
+    # + 66.280 MB written; scaled to the full corpus by rows scanned
+    ("k3_tensor", "masked_fused"): {"bytes_per_row": 1166.363, "src": "exact_inner_product_b200/csrc/k_tensor.cu",
+                                    "sha": "1074ee60d7ac4f9dd8a45c54fb73ec1c8ab54218cc60b75d7307328d39225625"},
 }
 
 

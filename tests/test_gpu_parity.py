@@ -45,6 +45,18 @@ def test_parity_scaled(name, over, path):
     assert res["max_abs_err"] <= w.tolerance
 
 
+@pytest.mark.parametrize("path,b", [(1, 3), (2, 40), (3, 260)])
+def test_limits_widest_rows_and_largest_k(path, b):
+    """d = 512 (the widest rows) with k = 2048 (the largest k) on every
+    scorer: the query tile and ring shrink to fit shared memory, and the
+    final selection sorts 2048 keys."""
+    _cuda()
+    w = W.workload("large_batch", n=30_011, d=512, b=b, k=2048, n_clusters=64, oracle_queries=6)
+    res, st = parity.run_case(w, path=path)
+    assert st["path"] == path
+    assert res["max_abs_err"] <= w.tolerance
+
+
 @pytest.mark.parametrize("path", [1, 2, 3])
 def test_every_scorer_agrees_with_oracle(path):
     _cuda()
