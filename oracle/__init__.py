@@ -77,6 +77,9 @@ class OracleLib:
         lib.oracle_topk_q8.restype = ctypes.c_int
         lib.oracle_scores_q8.argtypes = [vp, vp, i64, vp, vp, i32, ctypes.c_double, vp, i64, vp]
         lib.oracle_scores_q8.restype = None
+        lib.oracle_inbatch_softmax.argtypes = [vp, i32, i64, vp, i32, i64, i32, vp, vp, vp, ctypes.c_double,
+                                               vp, vp, vp]
+        lib.oracle_inbatch_softmax.restype = ctypes.c_int
         lib.oracle_set_threads.argtypes = [i32]
         lib.oracle_set_threads.restype = None
         lib.oracle_max_threads.argtypes = []
@@ -190,6 +193,41 @@ class OracleLib:
                                   qcodes.shape[1], float(tau), _ptr(ids), ids.shape[0], _ptr(out))
         return out
 
+    def inbatch_softmax(self, users: np.ndarray, items: np.ndarray, tau: float = 1.0,
+                        logq: np.ndarray | None = None, item_ids: np.ndarray | None = None,
+                        valid: np.ndarray | None = None):
+        """In-batch sampled softmax in fp64: row i's positive is candidate i,
+        every other valid column not holding row i's item is a negative.
+
+        ``users`` [b,d] and ``items`` [nc,d] (nc >= b) as float32 or bf16 bits;
+        ``logq`` [nc] is subtracted from every logit of its column; ``item_ids``
+        [nc] int64 marks accidental hits; ``valid`` [nc] bool drops columns and
+        (for i < b) rows. Returns ``(lse [b], loss [b], mean)`` as float64.
+        """
+        users, items = _c2(users), _c2(items)
+        b, d = users.shape
+        nc = items.shape[0]
+        if items.shape[1] != d or nc < b:
+            raise ValueError("need items [nc, d] with nc >= b")
+        if logq is not None:
+            logq = np.ascontiguousarray(logq, dtype=np.float64)
+            assert logq.shape == (nc,)
+        if item_ids is not None:
+            item_ids = np.ascontiguousarray(item_ids, dtype=np.int64)
+            assert item_ids.shape == (nc,)
+        if valid is not None:
+            valid = np.ascontiguousarray(valid, dtype=bool).view(np.uint8)
+            assert valid.shape == (nc,)
+        lse = np.empty(b, dtype=np.float64)
+        loss = np.empty(b, dtype=np.float64)
+        mean = np.empty(1, dtype=np.float64)
+        rc = self.lib.oracle_inbatch_softmax(_ptr(users), _dtype_code(users), b, _ptr(items),
+                                             _dtype_code(items), nc, d, _ptr(logq), _ptr(item_ids),
+                                             _ptr(valid), float(tau), _ptr(lse), _ptr(loss), _ptr(mean))
+        if rc != 0:
+            raise MemoryError("oracle_inbatch_softmax could not allocate its work buffer")
+        return lse, loss, float(mean[0])
+
     def set_threads(self, n: int) -> None:
         self.lib.oracle_set_threads(int(n))
 
@@ -238,6 +276,10 @@ def topk_q8(qcodes, qscales, vcodes, vscales, k, tau=1.0, exclude=None):
 
 def scores_for_q8(qcodes, qscales, qrow, vcodes, vscales, ids, tau=1.0):
     return default().scores_for_q8(qcodes, qscales, qrow, vcodes, vscales, ids, tau=tau)
+
+
+def inbatch_softmax(users, items, tau=1.0, logq=None, item_ids=None, valid=None):
+    return default().inbatch_softmax(users, items, tau=tau, logq=logq, item_ids=item_ids, valid=valid)
 
 
 def set_threads(n):

@@ -37,6 +37,25 @@
  * value of the dequantised vectors, (sum_i u8_i v8_ij) * us * scale_j / tau,
  * whose integer sum is exact.
  *
+ * In-batch sampled softmax (training loss): users u_i (i < b) against the
+ * candidate rows v_j (j < nc, nc >= b); row i's positive is candidate i and
+ * the rest of the columns are its negatives ("Two-Tower Retrieval at
+ * Industrial Scale", section 3, In-batch sampled softmax, `in_batch_loss`;
+ * columns j >= b are negatives shared by every row, like the global
+ * negatives of x-algorithm recsys_two_tower_model.py
+ * `compute_retrieval_loss`). The corrected logit is
+ * l_ij = (u_i . v_j) / tau - logq_j, with the correction on every column,
+ * the positive included (same article, section 4, The LogQ Correction,
+ * `corrected_in_batch_loss`). Column j enters row i's denominator when it is
+ * valid and is not an accidental hit: a column j != i whose item id equals
+ * item i's (`corrected_in_batch_loss`, masked with -inf; mhtirogla.ai
+ * "Two-tower retrieval", Code section, `step`). Then
+ * lse_i = log sum_j exp(l_ij) over that set, loss_i = lse_i - l_ii for a
+ * valid row (0 for an invalid one), and the loss is the mean of loss_i over
+ * the valid rows, 0 when there are none (`compute_retrieval_loss`:
+ * neg_log_probs = log_denominator - numerator_logits, averaged over valid
+ * positives, then over users with one).
+ *
  * Storage rounding: where the corpus or the queries are stored in bf16 or
  * fp32, the fp64 normalised value is rounded once, to nearest with ties to
  * even, to the storage type (recsys_two_tower_model.py keeps the candidate
@@ -309,6 +328,67 @@ void oracle_scores_q8(const int8_t *q, const float *qscales, int64_t qrow, const
 {
     for (int64_t t = 0; t < count; ++t)
         out[t] = score_one(q, ORACLE_I8, qrow, v, ORACLE_I8, ids[t], d, NULL, qscales, vscales, tau);
+}
+
+/* ---- in-batch sampled softmax ------------------------------------------- */
+
+static int inbatch_in_denominator(const int64_t *item_ids, const uint8_t *valid, int64_t i,
+                                  int64_t j)
+{
+    if (valid && !valid[j])
+        return 0;
+    if (item_ids && j != i && item_ids[j] == item_ids[i])
+        return 0; /* accidental hit: the same item as row i's positive */
+    return 1;
+}
+
+/* lse [b], loss [b], *mean: see the header comment. u [b,d] and v [nc,d] in
+ * their storage types; logq [nc] (NULL: no correction); item_ids [nc] (NULL:
+ * no accidental-hit mask); valid [nc] bytes (NULL: every row and column is
+ * valid). Returns 0, or -1 if a work buffer could not be allocated. */
+int oracle_inbatch_softmax(const void *u, int u_dtype, int64_t b, const void *v, int v_dtype,
+                           int64_t nc, int d, const double *logq, const int64_t *item_ids,
+                           const uint8_t *valid, double tau, double *lse, double *loss,
+                           double *mean)
+{
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < b; ++i) {
+        double *l = (double *)malloc((size_t)(nc > 0 ? nc : 1) * sizeof(double));
+        if (!l) {
+#pragma omp atomic write
+            failed = 1;
+            continue;
+        }
+        double m = -INFINITY;
+        for (int64_t j = 0; j < nc; ++j) {
+            l[j] = score_one(u, u_dtype, i, v, v_dtype, j, d, NULL, NULL, NULL, tau);
+            if (logq)
+                l[j] -= logq[j];
+            if (inbatch_in_denominator(item_ids, valid, i, j) && l[j] > m)
+                m = l[j];
+        }
+        /* log sum exp, with the largest term factored out so that nothing
+         * overflows: log sum_j exp(l_j) = m + log sum_j exp(l_j - m) */
+        double sum = 0.0;
+        for (int64_t j = 0; j < nc; ++j)
+            if (inbatch_in_denominator(item_ids, valid, i, j))
+                sum += exp(l[j] - m);
+        lse[i] = sum > 0.0 ? m + log(sum) : -INFINITY;
+        loss[i] = (!valid || valid[i]) ? lse[i] - l[i] : 0.0;
+        free(l);
+    }
+    if (failed)
+        return -1;
+    double total = 0.0;
+    int64_t rows = 0;
+    for (int64_t i = 0; i < b; ++i)
+        if (!valid || valid[i]) {
+            total += loss[i];
+            ++rows;
+        }
+    *mean = rows > 0 ? total / (double)rows : 0.0;
+    return 0;
 }
 
 /* ---- threading ---------------------------------------------------------- */

@@ -11,7 +11,11 @@ rank characterisation of top-k evaluated in exact rational arithmetic on tiny
 inputs, fp32 -> bf16 rounding by an independent library routine, and
 invariants that any correct implementation satisfies (unit norms, scaling by
 powers of two, permutation of the corpus, prefix property of top-k, 1/tau
-scaling, masks that exclude nothing, duplicate queries).
+scaling, masks that exclude nothing, duplicate queries). For the in-batch
+sampled softmax: the logQ article's printed three-item example (H8), torch's
+fp64 cross-entropy on the dense masked logits, the two-column logistic form,
+equal-logit counts, and invariants (a constant shift of log q, permutation of
+the batch, accidental hits as dropped columns, power-of-two scaling).
 """
 from __future__ import annotations
 
@@ -391,7 +395,173 @@ def check_int8_topk_invariants(o):
     assert not np.isin(ids3, np.nonzero(ex)[0]).any()
 
 
+# ---- in-batch sampled softmax ----------------------------------------------
+
+
+def _unit_rows(idx, d):
+    """Rows of the identity: row t is e_{idx[t]} (exact in every storage type)."""
+    out = np.zeros((len(idx), d), dtype=np.float32)
+    out[np.arange(len(idx)), idx] = 1.0
+    return out
+
+
+def check_h8_logq_worked(o):
+    """The logQ article's three-item example: a batch that holds each item in
+    proportion to q recovers the full-softmax denominator (times the batch
+    size) once log q is subtracted, and reproduces the printed pressure
+    ratios without it."""
+    g = golden()["H8_logq_worked"]
+    mult = g["multiplicities"]
+    col_item = np.repeat(np.arange(3), mult)
+    ncol = len(col_item)
+    d = 16
+    V = _unit_rows(col_item, d)
+    U = np.zeros((ncol, d), dtype=np.float32)
+    U[0, :3] = [2.0, 1.0, 0.0]  # user 0's logits against A, B, C (its positive is a copy of A)
+    q = np.array(g["q"], dtype=np.float64)[col_item]
+    press = g["printed_corrected_pressures"]
+    tol = 0.5 * 10.0 ** -g["printed_digits"]
+    lse, _, _ = o.inbatch_softmax(U, V, 1.0, logq=np.log(q))
+    assert abs(math.exp(lse[0]) - ncol * sum(press)) <= ncol * 3 * tol, (math.exp(lse[0]), ncol * sum(press))
+    lse_u, _, _ = o.inbatch_softmax(U, V, 1.0)
+    z_unc = math.exp(lse_u[0])
+    assert abs(z_unc - sum(m * p for m, p in zip(mult, press))) <= 20 * tol, z_unc
+    share_full = [p / sum(press) for p in press]
+    ratio_a = mult[0] * press[0] / z_unc / share_full[0]
+    ratio_c = mult[2] * press[2] / z_unc / share_full[2]
+    assert round(ratio_a, 2) == g["printed_ratio_uncorrected_to_correct"]["A"], ratio_a
+    assert round(ratio_c, 2) == g["printed_ratio_uncorrected_to_correct"]["C"], ratio_c
+
+
+def _random_batch(seed, b, nc, d, dup=True, invalid=True):
+    rng = np.random.default_rng(seed)
+    U = (rng.standard_normal((b, d)) / math.sqrt(d)).astype(np.float32)
+    V = (rng.standard_normal((nc, d)) / math.sqrt(d)).astype(np.float32)
+    logq = np.log(rng.uniform(1e-4, 1.0, nc))
+    ids = rng.integers(0, nc * 4, nc).astype(np.int64)
+    if dup:  # a few accidental hits: rows sharing an item, and a shared negative equal to a positive
+        ids[3] = ids[7]
+        ids[b - 1] = ids[5] = ids[0]
+        if nc > b:
+            ids[nc - 1] = ids[2]
+    valid = np.ones(nc, dtype=bool)
+    if invalid:
+        valid[[1, b - 2]] = False
+    return U, V, logq, ids, valid
+
+
+def _dense_reference(U, V, tau, logq, ids, valid):
+    """Row-wise cross-entropy of the masked logit matrix by torch's own
+    fp64 routine (the form `in_batch_loss` / `corrected_in_batch_loss` call)."""
+    b, nc = U.shape[0], V.shape[0]
+    logits = torch.from_numpy(U.astype(np.float64)) @ torch.from_numpy(V.astype(np.float64)).T / tau
+    if logq is not None:
+        logits = logits - torch.from_numpy(logq)[None, :]
+    keep = torch.ones((b, nc), dtype=torch.bool)
+    if valid is not None:
+        keep &= torch.from_numpy(valid)[None, :]
+    if ids is not None:
+        t = torch.from_numpy(ids)
+        hit = t[:b, None] == t[None, :]
+        hit[torch.arange(b), torch.arange(b)] = False
+        keep &= ~hit
+    logits = logits.masked_fill(~keep, -math.inf)
+    ce = torch.nn.functional.cross_entropy(logits, torch.arange(b), reduction="none")
+    lse = torch.logsumexp(logits, dim=1)
+    return lse.numpy(), ce.numpy()
+
+
+def check_inbatch_library(o):
+    """Against torch's fp64 cross-entropy and logsumexp on the dense masked
+    logits, with and without each of logq, item ids, validity and shared
+    negatives."""
+    for seed, b, nc, d in ((1, 12, 12, 16), (2, 16, 23, 32), (3, 9, 9, 64)):
+        U, V, logq, ids, valid = _random_batch(seed, b, nc, d)
+        for use_q in (False, True):
+            for use_ids in (False, True):
+                for use_valid in (False, True):
+                    tau = 0.07 if use_q else 1.0
+                    args = dict(logq=logq if use_q else None, item_ids=ids if use_ids else None,
+                                valid=valid if use_valid else None)
+                    lse, loss, mean = o.inbatch_softmax(U, V, tau, **args)
+                    want_lse, want_ce = _dense_reference(U, V, tau, args["logq"], args["item_ids"], args["valid"])
+                    assert np.allclose(lse, want_lse, rtol=1e-12, atol=1e-12), (seed, use_q, use_ids, use_valid)
+                    rows = valid[:b] if use_valid else np.ones(b, dtype=bool)
+                    assert np.allclose(loss[rows], want_ce[rows], rtol=1e-12, atol=1e-12)
+                    assert (loss[~rows] == 0).all()
+                    assert abs(mean - want_ce[rows].mean()) <= 1e-12 * max(1.0, abs(mean))
+
+
+def check_inbatch_closed_forms(o):
+    """Two columns: the softmax cross-entropy is the logistic loss
+    log(1 + exp(-margin)). Equal logits: the loss is log of the number of
+    columns in the row's denominator, counted from the masks."""
+    d = 16
+    U = np.zeros((2, d), dtype=np.float32)
+    V = np.zeros((2, d), dtype=np.float32)
+    U[0, 0], U[1, 1] = 1.0, 2.0
+    V[0, 0], V[1, 1], V[1, 0] = 2.0, 1.0, 0.5
+    logq = np.array([math.log(0.25), math.log(0.5)])
+    _, loss, _ = o.inbatch_softmax(U, V, 0.5, logq=logq)
+    # row 0: logits 2/0.5 - log 0.25 and 0.5/0.5 - log 0.5; row 1: 0 - log 0.25 and 2/0.5 - log 0.5
+    m0 = (4.0 - math.log(0.25)) - (1.0 - math.log(0.5))
+    m1 = (4.0 - math.log(0.5)) - (0.0 - math.log(0.25))
+    assert abs(loss[0] - math.log1p(math.exp(-m0))) <= 1e-14, loss
+    assert abs(loss[1] - math.log1p(math.exp(-m1))) <= 1e-14, loss
+    # equal logits (zero users): loss_i = log |D_i|
+    b, nc = 10, 14
+    _, _, _, ids, valid = _random_batch(5, b, nc, d)
+    Uz = np.zeros((b, d), dtype=np.float32)
+    Vr = np.ones((nc, d), dtype=np.float32)
+    lse, loss, mean = o.inbatch_softmax(Uz, Vr, 1.0, item_ids=ids, valid=valid)
+    for i in range(b):
+        count = sum(1 for j in range(nc) if valid[j] and (j == i or ids[j] != ids[i]))
+        assert abs(lse[i] - math.log(count)) <= 1e-14, (i, lse[i], count)
+        assert loss[i] == (lse[i] if valid[i] else 0.0)
+    # no valid row: the mean is 0
+    _, loss, mean = o.inbatch_softmax(Uz, Vr, 1.0, valid=np.zeros(nc, dtype=bool))
+    assert mean == 0.0 and (loss == 0).all()
+
+
+def check_inbatch_invariants(o):
+    """A constant added to every log q moves lse by minus that constant and
+    leaves the loss alone (the correction applies to every column, the
+    positive included); permuting the batch permutes the outputs; masking an
+    accidental hit equals dropping that column for the row; users scaled by 2
+    with tau scaled by 2 change nothing."""
+    b, nc, d = 14, 20, 32
+    U, V, logq, ids, valid = _random_batch(9, b, nc, d)
+    lse, loss, mean = o.inbatch_softmax(U, V, 0.1, logq=logq, item_ids=ids, valid=valid)
+    lse2, loss2, mean2 = o.inbatch_softmax(U, V, 0.1, logq=logq + 3.0, item_ids=ids, valid=valid)
+    assert np.allclose(lse2, lse - 3.0, rtol=0, atol=1e-12)
+    assert np.allclose(loss2, loss, rtol=0, atol=1e-12) and abs(mean2 - mean) <= 1e-12
+    # permutation of rows (with their columns) and of the shared negatives
+    rng = np.random.default_rng(4)
+    pr = rng.permutation(b)
+    pg = b + rng.permutation(nc - b)
+    cols = np.concatenate([pr, pg])
+    lse3, loss3, mean3 = o.inbatch_softmax(U[pr], V[cols], 0.1, logq=logq[cols], item_ids=ids[cols],
+                                           valid=valid[cols])
+    assert np.allclose(lse3, lse[pr], rtol=1e-13, atol=1e-13)
+    assert np.allclose(loss3, loss[pr], rtol=1e-13, atol=1e-13) and abs(mean3 - mean) <= 1e-12
+    # row 3 shares its item with row 7: its loss equals the loss with column 7 dropped and no id mask
+    assert ids[3] == ids[7] and valid[3] and valid[7]
+    drop7 = valid.copy()
+    drop7[7] = False
+    lse4, loss4, _ = o.inbatch_softmax(U, V, 0.1, logq=logq, valid=drop7)
+    assert abs(loss4[3] - loss[3]) <= 1e-12 and abs(lse4[3] - lse[3]) <= 1e-12
+    # the shared item does not mask the positive itself: row 0's item is also held by rows 5 and b-1
+    assert np.isfinite(loss[0]) and loss[0] > 0
+    # power-of-two scaling of users and tau
+    lse5, loss5, _ = o.inbatch_softmax((U * 2).astype(np.float32), V, 0.2, logq=logq, item_ids=ids, valid=valid)
+    assert np.array_equal(lse5, lse) and np.array_equal(loss5, loss)
+
+
 ALL_CHECKS = [
+    check_h8_logq_worked,
+    check_inbatch_library,
+    check_inbatch_closed_forms,
+    check_inbatch_invariants,
     check_h5_quantize,
     check_h6_quantize_ties,
     check_h7_int8_score,

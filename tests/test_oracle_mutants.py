@@ -1,6 +1,7 @@
 """Planted mistakes: each copy of oracle.c below carries one plausible bug
 (a dropped term, a wrong sign, index or operand, a misplaced floor, a broken
-tie rule or rounding, in the fp path and in int8 coding and scoring). Every copy must fail at least one pin; a copy that
+tie rule or rounding, in the fp path, in int8 coding and scoring and
+in the in-batch softmax). Every copy must fail at least one pin; a copy that
 passes them all would show a gap in the pins. CPU only; the copies are built
 in a temporary directory and never touch the real oracle."""
 import os
@@ -41,6 +42,18 @@ MUTANTS = {
     "q8_row_scale_dropped": ("dot = dot * (double)qscales[qrow] * (double)vscales[j];",
                              "dot = dot * (double)qscales[qrow];"),
     "q8_code_sign_lost": ("codes[j * (int64_t)d + i] = (int8_t)r;", "codes[j * (int64_t)d + i] = (int8_t)fabsf(r);"),
+    # in-batch sampled softmax
+    "logq_added": ("l[j] -= logq[j];", "l[j] += logq[j];"),
+    "logq_skips_positive": ("            if (logq)\n                l[j] -= logq[j];",
+                            "            if (logq && j != i)\n                l[j] -= logq[j];"),
+    "hit_masks_positive": ("if (item_ids && j != i && item_ids[j] == item_ids[i])",
+                           "if (item_ids && item_ids[j] == item_ids[i])"),
+    "hit_compares_index": ("item_ids[j] == item_ids[i])", "item_ids[j] == (int64_t)i)"),
+    "invalid_column_kept": ("    if (valid && !valid[j])\n        return 0;\n", ""),
+    "invalid_row_counted": ("loss[i] = (!valid || valid[i]) ? lse[i] - l[i] : 0.0;", "loss[i] = lse[i] - l[i];"),
+    "mean_over_all_rows": ("total / (double)rows", "total / (double)b"),
+    "max_not_factored_back": ("m + log(sum)", "log(sum)"),
+    "numerator_first_column": ("lse[i] - l[i]", "lse[i] - l[0]"),
 }
 
 
