@@ -38,7 +38,7 @@ TT_NORM_FUSED = 1
 TT_MAX_D = 512
 TT_MAX_K = 2048
 
-KIND_NAMES = ("normalize", "cast", "stream", "tensor", "select", "aux")
+KIND_NAMES = ("normalize", "cast", "stream", "tensor", "select", "aux", "softmax")
 TT_NUM_KINDS = len(KIND_NAMES)
 
 if not os.path.exists(LIB_PATH):
@@ -89,6 +89,10 @@ _sig("tt_score_topk_ranges", ctypes.c_int, [_vp, _vp, ctypes.c_int, _i32, _vp, c
                                             ctypes.POINTER(_i64), _vp, _vp, _vp])
 _sig("tt_score_topk_types", ctypes.c_int, [_vp, _vp, ctypes.c_int, _i32, _vp, ctypes.c_float, _i32, _vp, _i32,
                                            ctypes.POINTER(_i32), _vp, _vp, _vp])
+_sig("tt_inbatch_softmax_workspace", ctypes.c_int, [_i32, _i32, _i32, _i32, ctypes.POINTER(ctypes.c_size_t)])
+_sig("tt_inbatch_softmax", ctypes.c_int, [_vp, _vp, ctypes.c_int, _i32, _i32, _i32, ctypes.c_float, _vp, _vp, _vp,
+                                          _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp])
+_sig("tt_inbatch_softmax_check", ctypes.c_int, [_vp, _vp])
 _sig("tt_free", None, [_vp])
 _sig("tt_launch_count", _i64, [])
 _sig("tt_profile_begin", ctypes.c_int, [])
@@ -101,6 +105,7 @@ _sig("tt_version", ctypes.c_char_p, [])
 
 EXPORTED = ("tt_normalize_candidates", "tt_quantize_candidates", "tt_index_wrap", "tt_score_topk", "tt_score_topk_ex",
             "tt_score_topk_noalloc", "tt_merge_topk", "tt_score_topk_ranges", "tt_score_topk_types",
+            "tt_inbatch_softmax_workspace", "tt_inbatch_softmax", "tt_inbatch_softmax_check",
             "tt_last_stats", "tt_plan", "tt_free", "tt_launch_count", "tt_profile_begin",
             "tt_profile_end", "tt_profile_launches", "tt_status_string", "tt_last_error", "tt_version")
 
@@ -302,6 +307,57 @@ def tt_merge_topk(ids: torch.Tensor, scores: torch.Tensor, id_offsets, k_out: in
     _check(_lib.tt_merge_topk(_ptr(ids), _ptr(scores), parts, b, k_in, offs, int(k_out), _ptr(out_ids),
                               _ptr(out_scores), _stream(stream)), "tt_merge_topk")
     return out_ids, out_scores
+
+
+def tt_inbatch_softmax_workspace(b: int, nc: int, d: int, with_item_ids: bool) -> int:
+    """Bytes of device workspace ``tt_inbatch_softmax`` needs for these sizes."""
+    out = ctypes.c_size_t(0)
+    _check(_lib.tt_inbatch_softmax_workspace(int(b), int(nc), int(d), 1 if with_item_ids else 0,
+                                             ctypes.byref(out)), "tt_inbatch_softmax_workspace")
+    return int(out.value)
+
+
+def tt_inbatch_softmax(users: torch.Tensor, items: torch.Tensor, tau: float = 1.0,
+                       logq: torch.Tensor | None = None, item_ids: torch.Tensor | None = None,
+                       valid: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                       out: tuple | None = None, stream=None, check: bool = True):
+    """In-batch sampled softmax loss (``tt_inbatch_softmax``): row i of
+    ``users`` [b, d] has candidate row i of ``items`` [nc, d] (bf16, nc >= b)
+    as its positive. ``logq`` float32 [nc] is subtracted from every logit of
+    its column, ``item_ids`` int64 [nc] masks accidental hits, ``valid`` bool
+    or uint8 [nc] drops padding. Returns ``(lse [b], loss [b], mean [])`` as
+    float32 tensors on the device. ``workspace`` (uint8, at least
+    ``tt_inbatch_softmax_workspace`` bytes) and ``out`` (lse, loss, mean) may
+    be passed to avoid allocations; ``check`` waits for the result and raises
+    on a device-side timeout."""
+    if users.dim() != 2 or items.dim() != 2 or not users.is_contiguous() or not items.is_contiguous():
+        raise ValueError("users and items must be contiguous [b, d] and [nc, d] tensors")
+    if users.shape[1] != items.shape[1]:
+        raise ValueError("users and items disagree on d")
+    b, d = users.shape
+    nc = items.shape[0]
+    for name, t, dt in (("logq", logq, torch.float32), ("item_ids", item_ids, torch.int64)):
+        if t is not None and (t.dtype != dt or not t.is_contiguous() or t.numel() != nc):
+            raise TypeError(f"{name} must be a contiguous {dt} tensor of nc elements")
+    if valid is not None:
+        if valid.dtype == torch.bool:
+            valid = valid.view(torch.uint8)
+        if valid.dtype != torch.uint8 or not valid.is_contiguous() or valid.numel() != nc:
+            raise TypeError("valid must be a contiguous bool or uint8 tensor of nc elements")
+    need = tt_inbatch_softmax_workspace(b, nc, d, item_ids is not None)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=users.device)
+    if out is None:
+        out = (torch.empty(b, dtype=torch.float32, device=users.device),
+               torch.empty(b, dtype=torch.float32, device=users.device),
+               torch.empty((), dtype=torch.float32, device=users.device))
+    lse, loss, mean = out
+    _check(_lib.tt_inbatch_softmax(_ptr(users), _ptr(items), _dtype(users), b, nc, d, float(tau), _ptr(logq), _ptr(item_ids),
+                                   _ptr(valid), _ptr(lse), _ptr(loss), _ptr(mean), _ptr(workspace),
+                                   workspace.numel(), _stream(stream)), "tt_inbatch_softmax")
+    if check:
+        _check(_lib.tt_inbatch_softmax_check(_ptr(workspace), _stream(stream)), "tt_inbatch_softmax")
+    return lse, loss, mean
 
 
 def _check_queries(index: Index, queries: torch.Tensor, exclude):

@@ -889,6 +889,84 @@ tt_status tt_merge_topk(const int32_t* ids, const float* scores, int32_t parts, 
     return TT_OK;
 }
 
+// ---------------------------------------------------------------------------
+// in-batch sampled softmax
+// ---------------------------------------------------------------------------
+static tt_status softmax_sizes(int32_t b, int32_t nc, int32_t d, bool with_ids) {
+    if (b < 0 || nc < b) return TT_ERR_INVALID_ARG;
+    if (d <= 0) return TT_ERR_INVALID_ARG;
+    if (d % 16 != 0 || d > TT_MAX_D || !softmax_supported(d)) return TT_ERR_UNSUPPORTED;
+    if (with_ids && nc > (1 << 28)) return TT_ERR_UNSUPPORTED;
+    return TT_OK;
+}
+
+tt_status tt_inbatch_softmax_workspace(int32_t b, int32_t nc, int32_t d, int32_t with_item_ids, size_t* bytes) {
+    if (bytes == nullptr) return TT_ERR_INVALID_ARG;
+    tt_status st = softmax_sizes(b, nc, d, with_item_ids != 0);
+    if (st != TT_OK) return st;
+    *bytes = softmax_plan(b, nc, d, with_item_ids != 0, sm_count_current()).bytes;
+    return TT_OK;
+}
+
+tt_status tt_inbatch_softmax(const void* users, const void* items, tt_dtype dtype, int32_t b, int32_t nc,
+                             int32_t d, float tau, const float* logq, const int64_t* item_ids,
+                             const uint8_t* valid, float* lse, float* loss, float* mean, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+    // ---------------- host-side validation (no device calls) ----------------
+    if (dtype != TT_BF16) return valid_index_dtype(dtype) ? TT_ERR_UNSUPPORTED : TT_ERR_INVALID_ARG;
+    tt_status st = softmax_sizes(b, nc, d, item_ids != nullptr);
+    if (st != TT_OK) return st;
+    if (!(tau > 0.0f) || !isfinite(tau)) return TT_ERR_INVALID_ARG;
+    if (mean == nullptr || workspace == nullptr) return TT_ERR_INVALID_ARG;
+    if (b > 0 && (users == nullptr || items == nullptr || lse == nullptr || loss == nullptr))
+        return TT_ERR_INVALID_ARG;
+    if (!aligned(users, 16) || !aligned(items, 16) || !aligned(logq, 4) || !aligned(item_ids, 8) ||
+        !aligned(lse, 4) || !aligned(loss, 4) || !aligned(mean, 4) || !aligned(workspace, 256))
+        return TT_ERR_INVALID_ARG;
+    const int sms = sm_count_current();
+    const SoftmaxPlan pl = softmax_plan(b, nc, d, item_ids != nullptr, sms);
+    if (workspace_bytes < pl.bytes) {
+        snprintf(g_last_error, sizeof g_last_error, "workspace of %zu bytes, need %zu", workspace_bytes, pl.bytes);
+        return TT_ERR_INVALID_ARG;
+    }
+    // ---------------- device checks ----------------
+    if ((st = check_device_ptr(users, "users")) != TT_OK) return st;
+    if ((st = check_device_ptr(items, "items")) != TT_OK) return st;
+    if ((st = check_device_ptr(logq, "logq")) != TT_OK) return st;
+    if ((st = check_device_ptr(item_ids, "item_ids")) != TT_OK) return st;
+    if ((st = check_device_ptr(valid, "valid")) != TT_OK) return st;
+    if ((st = check_device_ptr(lse, "lse")) != TT_OK) return st;
+    if ((st = check_device_ptr(loss, "loss")) != TT_OK) return st;
+    if ((st = check_device_ptr(mean, "mean")) != TT_OK) return st;
+    if ((st = check_device_ptr(workspace, "workspace")) != TT_OK) return st;
+    CUtensorMap tm_users, tm_items;
+    memset(&tm_users, 0, sizeof tm_users);
+    memset(&tm_items, 0, sizeof tm_items);
+    if (b > 0) {
+        if (!bf16_tile_tensor_map(users, b, d, d, 128, &tm_users)) return TT_ERR_CUDA;
+        if (!bf16_tile_tensor_map(items, nc, d, d, 256, &tm_items)) return TT_ERR_CUDA;
+    }
+    cudaError_t e = launch_softmax(pl, tm_users, tm_items, b, nc, d, tau, logq, item_ids, valid, lse, loss, mean,
+                                   workspace, static_cast<cudaStream_t>(stream), sms);
+    if (e != cudaSuccess) return cuda_fail(e, "in-batch softmax");
+    return TT_OK;
+}
+
+tt_status tt_inbatch_softmax_check(const void* workspace, void* stream) {
+    if (workspace == nullptr || !aligned(workspace, 256)) return TT_ERR_INVALID_ARG;
+    tt_status st;
+    if ((st = check_device_ptr(workspace, "workspace")) != TT_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int err = 0;
+    TT_CUDA(cudaMemcpyAsync(&err, workspace, sizeof err, cudaMemcpyDeviceToHost, s), "error word readback");
+    TT_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+    if (err != 0) {
+        snprintf(g_last_error, sizeof g_last_error, "device wait expired (code %d)", err);
+        return TT_ERR_TIMEOUT;
+    }
+    return TT_OK;
+}
+
 // One result set: rows [start, start + count) of the index, a mask already
 // sliced to those rows (or null), ids reported as corpus ids.
 static tt_status score_rows(tt_index* index, int64_t start, int64_t count, const void* queries, tt_dtype q_dtype,

@@ -313,6 +313,56 @@ TT_API tt_status tt_score_topk_types(tt_index* index, const void* queries, tt_dt
                                      int32_t n_sets, const int32_t* set_types, int32_t* out_ids,
                                      float* out_scores, void* stream);
 
+/*
+ * tt_inbatch_softmax - the in-batch sampled-softmax training loss, fused:
+ * logits, masks, log-sum-exp and cross-entropy in one tensor-core pass that
+ * never writes the b x nc logit matrix.
+ *
+ * ("Two-Tower Retrieval at Industrial Scale", section 3, In-batch sampled
+ *  softmax, `in_batch_loss`; section 4, The LogQ Correction,
+ *  `corrected_in_batch_loss`; x-algorithm recsys_two_tower_model.py
+ *  `compute_retrieval_loss`, in-batch and global negatives.)
+ *
+ * Row i (i < b) is a user u_i whose positive is candidate row i; candidates
+ * b..nc-1 are negatives shared by every row. For every pair
+ *     l_ij = (u_i . v_j) / tau - logq_j
+ * (the correction on every column, the positive included). Column j enters
+ * row i's denominator when valid[j] and it is not an accidental hit: j == i,
+ * or item_ids[j] != item_ids[i]. Then
+ *     lse_i  = log sum_j exp(l_ij)          (-inf if no column enters)
+ *     loss_i = lse_i - l_ii for valid rows (valid[i]), 0 otherwise
+ *     mean   = sum of loss_i over valid rows / their number (0 if none)
+ * The dot products are exact products of the bf16 inputs accumulated in
+ * fp32 on the tensor cores; the exponentials are single-precision.
+ *
+ * users     device bf16 [b, d]
+ * items     device bf16 [nc, d], b <= nc
+ * dtype     TT_BF16 (other types: TT_ERR_UNSUPPORTED; cast first)
+ * d         multiple of 16, 64 <= d <= TT_MAX_D (zero-pad narrower rows)
+ * tau       > 0, finite
+ * logq      device f32 [nc] (finite), or NULL for no correction
+ * item_ids  device int64 [nc], or NULL for no accidental-hit mask
+ *           (with ids, nc is at most 2^28)
+ * valid     device uint8 [nc] (0 = padding), or NULL when every row is valid
+ * lse, loss device f32 [b]; mean device f32 [1]
+ * workspace device memory of at least tt_inbatch_softmax_workspace bytes,
+ *           256-byte aligned, owned by the caller, not shared with another
+ *           call in flight
+ *
+ * Asynchronous: the work is enqueued on `stream` and the call returns. If a
+ * bounded device-side wait expires (which a correct run never does), every
+ * output is NaN and tt_inbatch_softmax_check then returns TT_ERR_TIMEOUT.
+ */
+TT_API tt_status tt_inbatch_softmax_workspace(int32_t b, int32_t nc, int32_t d, int32_t with_item_ids,
+                                              size_t* bytes);
+TT_API tt_status tt_inbatch_softmax(const void* users, const void* items, tt_dtype dtype, int32_t b, int32_t nc,
+                                    int32_t d, float tau, const float* logq, const int64_t* item_ids,
+                                    const uint8_t* valid, float* lse, float* loss, float* mean, void* workspace,
+                                    size_t workspace_bytes, void* stream);
+/* Wait for the last tt_inbatch_softmax that used `workspace` (on `stream`)
+ * and report TT_OK or TT_ERR_TIMEOUT. */
+TT_API tt_status tt_inbatch_softmax_check(const void* workspace, void* stream);
+
 /* Release a handle. Its scratch memory returns to a per-device pool that
  * later handles reuse (it is not returned to CUDA before the process exits).
  * NULL is a no-op. Must not be called while work using the handle is still
@@ -364,7 +414,8 @@ TT_API tt_status tt_score_topk_noalloc(const void* rows, tt_dtype dtype, int64_t
 #define TT_KIND_TENSOR 3
 #define TT_KIND_SELECT 4
 #define TT_KIND_AUX 5
-#define TT_NUM_KINDS 6
+#define TT_KIND_SOFTMAX 6 /* tt_inbatch_softmax */
+#define TT_NUM_KINDS 7
 
 /* Total kernels this library has launched in the process. */
 TT_API int64_t tt_launch_count(void);

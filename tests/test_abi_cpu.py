@@ -161,6 +161,39 @@ def test_set_calls_validate_before_device_calls():
     lib.tt_free(ix)
 
 
+def test_softmax_validation_before_device_calls():
+    lib = tt._lib
+    fake = ctypes.c_void_p(0x10000)
+    size = ctypes.c_size_t(0)
+    assert lib.tt_inbatch_softmax_workspace(100, 300, 64, 1, ctypes.byref(size)) == tt.TT_OK
+    need = size.value
+    assert need > 300 * 8  # at least the per-column data
+    assert lib.tt_inbatch_softmax_workspace(100, 300, 64, 0, ctypes.byref(size)) == tt.TT_OK
+    assert size.value < need  # no hash table without item ids
+    assert lib.tt_inbatch_softmax_workspace(300, 100, 64, 0, ctypes.byref(size)) == tt.TT_ERR_INVALID_ARG
+    assert lib.tt_inbatch_softmax_workspace(10, 10, 24, 0, ctypes.byref(size)) == tt.TT_ERR_UNSUPPORTED
+    assert lib.tt_inbatch_softmax_workspace(10, 10, 64, 0, None) == tt.TT_ERR_INVALID_ARG
+
+    def call(**kw):
+        return lib.tt_inbatch_softmax(fake, fake, kw.get("dt", tt.TT_BF16), kw.get("b", 100), kw.get("nc", 300),
+                                      kw.get("d", 64), kw.get("tau", 0.05), None, kw.get("ids", fake), None, fake,
+                                      fake, kw.get("mean", fake), kw.get("ws", fake), kw.get("wsb", 1), None)
+    assert call(dt=tt.TT_F32) == tt.TT_ERR_UNSUPPORTED
+    assert call(dt=9) == tt.TT_ERR_INVALID_ARG
+    assert call(b=400) == tt.TT_ERR_INVALID_ARG  # nc < b
+    assert call(b=-1) == tt.TT_ERR_INVALID_ARG
+    assert call(d=40) == tt.TT_ERR_UNSUPPORTED
+    assert call(d=48) == tt.TT_ERR_UNSUPPORTED  # narrower than one 64-element box
+    assert call(d=1024) == tt.TT_ERR_UNSUPPORTED
+    assert call(tau=0.0) == tt.TT_ERR_INVALID_ARG
+    assert call(tau=float("inf")) == tt.TT_ERR_INVALID_ARG
+    assert call(mean=None) == tt.TT_ERR_INVALID_ARG
+    assert call(ws=ctypes.c_void_p(0x10010)) == tt.TT_ERR_INVALID_ARG  # workspace not 256-byte aligned
+    assert call(wsb=need - 1) == tt.TT_ERR_INVALID_ARG  # workspace too small
+    assert call(ids=ctypes.c_void_p(0x10004)) == tt.TT_ERR_INVALID_ARG  # misaligned ids
+    assert lib.tt_inbatch_softmax_check(None, None) == tt.TT_ERR_INVALID_ARG
+
+
 def test_plan_levels():
     # the deepest level holds at most `cap` rows; strides are powers of 61
     for n, k in ((400, 10), (10 ** 6, 100), (10 ** 7, 500), (5 * 10 ** 7, 1000), (2 * 10 ** 7, 256),

@@ -20,6 +20,16 @@ candidate-tower corpus and a batch of user-tower outputs):
 * exclusion mask: independent Bernoulli(rate) per candidate, packed 32 per
   uint32 word, bit (j & 31) of word (j >> 5) set = candidate j excluded.
 
+In-batch training batches (``Batch``, for the sampled-softmax loss): user and
+item vectors ~ N(0, I / d) (length close to 1, as unit-norm tower outputs are;
+"Two-Tower Retrieval at Industrial Scale", section 3, (B, 64) unit-norm user
+and item towers), stored in bf16. Each column's item id is drawn from a
+catalogue with Zipf popularity p(c) proportional to (c + 1)^-s, so popular
+items repeat inside a batch (the accidental hits); a repeated id carries the
+vector of its first occurrence; log q_j is the log of the drawing probability
+of column j's item. A column is padding with probability pad_rate. Columns
+b..nc-1 are drawn the same way and act as shared negatives.
+
 Every tensor is drawn with ``torch.Generator`` seeded from the workload seed,
 in fixed-size chunks, so the same call gives the same numbers on the same
 device type.
@@ -206,3 +216,71 @@ def to_numpy_rows(t: torch.Tensor) -> np.ndarray:
     if t.dtype == torch.bfloat16:
         return bf16_bits(t)
     return t.detach().contiguous().cpu().numpy()
+
+
+# ---------------------------------------------------------------------------
+# in-batch training batches
+# ---------------------------------------------------------------------------
+@dataclasses.dataclass(frozen=True)
+class Batch:
+    name: str
+    b: int               # users (rows); row i's positive is column i
+    nc: int              # candidate columns, nc >= b (columns >= b: shared negatives)
+    d: int
+    tau: float
+    catalogue: int       # items the ids are drawn from
+    zipf_s: float        # popularity exponent
+    pad_rate: float      # probability that a column (and its row) is padding
+    oracle_rows: int = 0  # 0: check every row; else a seeded sample of this many
+    seed: int = BASE_SEED + 11
+
+    def describe(self) -> dict:
+        return dataclasses.asdict(self)
+
+
+BATCHES = {
+    # the article's batch of 8192 rows with 64-wide towers
+    "inbatch_b8192_d64": Batch("inbatch_b8192_d64", b=8192, nc=8192, d=64, tau=0.05, catalogue=1_000_000,
+                               zipf_s=1.0, pad_rate=0.01, oracle_rows=64, seed=BASE_SEED + 11),
+    # a large global batch: 2^32 logits
+    "inbatch_b65536_d64": Batch("inbatch_b65536_d64", b=65536, nc=65536, d=64, tau=0.05, catalogue=1_000_000,
+                                zipf_s=1.0, pad_rate=0.01, oracle_rows=32, seed=BASE_SEED + 12),
+    # wider towers and as many shared negatives as in-batch ones
+    "inbatch_b16384_g16384_d128": Batch("inbatch_b16384_g16384_d128", b=16384, nc=32768, d=128, tau=0.05,
+                                        catalogue=1_000_000, zipf_s=1.0, pad_rate=0.01, oracle_rows=32,
+                                        seed=BASE_SEED + 13),
+}
+
+
+def batch(name: str, **overrides) -> Batch:
+    """A named training batch, optionally resized (``b=``, ``nc=``, ``d=`` ...)."""
+    return dataclasses.replace(BATCHES[name], **overrides)
+
+
+def batch_inputs(w: Batch, device="cpu") -> dict:
+    """users bf16 [b, d], items bf16 [nc, d], logq f32 [nc], item_ids int64 [nc],
+    valid bool [nc]; drawn on the CPU (the same numbers for every device) and
+    then moved to ``device``."""
+    g = _gen(w.seed, "cpu")
+    users = (torch.randn((w.b, w.d), generator=g) / math.sqrt(w.d)).to(torch.bfloat16)
+    weights = torch.arange(1, w.catalogue + 1, dtype=torch.float64) ** (-w.zipf_s)
+    prob = weights / weights.sum()
+    ids = torch.multinomial(prob, w.nc, replacement=True, generator=g)
+    vecs = (torch.randn((w.nc, w.d), generator=g) / math.sqrt(w.d)).to(torch.bfloat16)
+    # a repeated item carries the vector of its first occurrence
+    _, inverse = torch.unique(ids, return_inverse=True)
+    first = torch.full((int(inverse.max()) + 1 if w.nc else 0,), w.nc, dtype=torch.int64)
+    first = first.scatter_reduce(0, inverse, torch.arange(w.nc), reduce="amin")
+    items = vecs[first[inverse]]
+    logq = torch.log(prob[ids]).to(torch.float32)
+    valid = torch.rand(w.nc, generator=g) >= w.pad_rate
+    return {"users": users.to(device), "items": items.contiguous().to(device), "logq": logq.to(device),
+            "item_ids": ids.to(device), "valid": valid.to(device)}
+
+
+def oracle_row_ids(w: Batch) -> np.ndarray:
+    """The rows the oracle checks for a full-size batch (sorted, seeded)."""
+    if w.oracle_rows == 0 or w.oracle_rows >= w.b:
+        return np.arange(w.b, dtype=np.int64)
+    rng = np.random.Generator(np.random.Philox(w.seed + 5_000_011))
+    return np.sort(rng.choice(w.b, size=w.oracle_rows, replace=False)).astype(np.int64)
