@@ -17,6 +17,12 @@ Multi-GPU (torchrun, one process per GPU), two modes:
     NCCL and merged (tt_merge_topk) on every rank; the value is the one
     workload's scores per second (strong scaling).
 
+With --op inbatch_softmax the step is instead the in-batch sampled-softmax
+training loss (tt_inbatch_softmax: logits, logQ correction, accidental-hit and
+padding masks, log-sum-exp, cross-entropy and the mean) over one seeded
+training batch (--batch, default 65,536 users x 65,536 candidates, d = 64);
+the value is logits per second.
+
 Prints one JSON line (rank 0).
 """
 from __future__ import annotations
@@ -463,6 +469,201 @@ def run_ours(args, world, rank, local):
     return line
 
 
+# ---------------------------------------------------------------------------
+# in-batch sampled softmax
+# ---------------------------------------------------------------------------
+SOFTMAX_METRIC = "in-batch sampled-softmax logits/sec (fused loss)"
+SOFTMAX_UNIT = "logits/s"
+# ex2 results per clock per SM (the multi-function unit; CUDA C++ Programming
+# Guide, arithmetic instruction throughput, compute capability 10.0)
+MUFU_PER_CLK_SM = 16
+SM_COUNT = 148
+SM_MAX_MHZ = 1965.0
+
+
+def softmax_oracle_run(inp, rows, tau):
+    """fp64 oracle on the listed rows, each against every column."""
+    import oracle
+    nc = inp["items"].shape[0]
+    rest = np.setdiff1d(np.arange(nc), rows)
+    cols = np.concatenate([rows, rest])
+    users = W.bf16_bits(inp["users"][torch.from_numpy(rows)])
+    items = W.bf16_bits(inp["items"][torch.from_numpy(cols)])
+    logq = inp["logq"].numpy().astype(np.float64)[cols]
+    ids = inp["item_ids"].numpy()[cols]
+    valid = inp["valid"].numpy()[cols]
+    t0 = time.perf_counter()
+    oracle.inbatch_softmax(users, items, tau, logq=logq, item_ids=ids, valid=valid)
+    return time.perf_counter() - t0
+
+
+def softmax_oracle_sample(w, inp, seconds):
+    import oracle
+    threads = oracle.max_threads()
+    r = min(w.b, max(1, threads))
+    t = softmax_oracle_run(inp, np.arange(r), w.tau)
+    while r < w.b and t < seconds / 4:
+        r = min(w.b, r * 4)
+        t = softmax_oracle_run(inp, np.arange(r), w.tau)
+    if t > 0 and r < w.b:
+        r = int(min(w.b, max(1, r * seconds / t)))
+    return r, threads
+
+
+def softmax_cpu_baseline(w, inp, seconds):
+    r, threads = softmax_oracle_sample(w, inp, seconds)
+    t = softmax_oracle_run(inp, np.arange(r), w.tau)
+    return {"value": r * w.nc / t, "unit": SOFTMAX_UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"first {r} rows of {w.name} against all {w.nc} columns (fp64 logits, masks, "
+                      f"log-sum-exp, loss), one run of {t:.2f} s"}
+
+
+def run_softmax(args, world, rank, local):
+    import exact_inner_product_b200 as tt
+
+    w = W.batch(args.batch)
+    if world > 1:  # each rank: its own batch (data parallel; the losses stay per rank)
+        w = dataclasses.replace(w, seed=w.seed + 7919 * rank)
+    dev = torch.device("cuda", local)
+    host = W.batch_inputs(w, "cpu")
+    inp = {k: v.to(dev) for k, v in host.items()}
+    ws = torch.empty(tt.tt_inbatch_softmax_workspace(w.b, w.nc, w.d, True), dtype=torch.uint8, device=dev)
+    out = (torch.empty(w.b, device=dev), torch.empty(w.b, device=dev), torch.empty((), device=dev))
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)  # larger than the 126 MB L2
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        tt.tt_inbatch_softmax(inp["users"], inp["items"], w.tau, logq=inp["logq"], item_ids=inp["item_ids"],
+                              valid=inp["valid"], workspace=ws, out=out, check=False)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    if tt._lib.tt_inbatch_softmax_check(tt._ptr(ws), None) != tt.TT_OK:
+        raise RuntimeError("tt_inbatch_softmax: device-side timeout in warm-up")
+    torch.cuda.synchronize(dev)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    launches0 = tt.tt_launch_count()
+    tt.tt_profile_begin()
+    t_wall0 = time.time()
+    evs = []
+    for _ in range(args.steps):
+        flush.zero_()  # L2 flush, outside the step's events
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b_.record(stream)
+        evs.append((a, b_))
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    barrier(world)
+    recs = tt.tt_profile_launches()
+    tt.tt_profile_end()
+    launches = tt.tt_launch_count() - launches0
+    clk = clocks.stop(t_wall0, t_wall1)
+    if tt._lib.tt_inbatch_softmax_check(tt._ptr(ws), None) != tt.TT_OK:
+        raise RuntimeError("tt_inbatch_softmax: device-side timeout in the timed steps")
+    ms_total = max_over_ranks(sum(a.elapsed_time(b_) for a, b_ in evs), world)
+    ms_step = ms_total / args.steps
+    logits = w.b * w.nc
+    value = world * logits / (ms_step / 1e3)
+
+    # roofline: one ex2 per logit on the multi-function unit (the fused kernel
+    # is the third of the four launches of a step with item ids)
+    per_step = len(recs) // args.steps
+    main_ms = [recs[s * per_step + 2][1] for s in range(args.steps)]
+    k5_ms = float(np.mean(main_ms))
+    achieved = logits / (k5_ms / 1e3) / 1e12
+    peak = MUFU_PER_CLK_SM * SM_COUNT * SM_MAX_MHZ * 1e6 / 1e12
+    roof = {"bound": "alu", "achieved": round(achieved, 4), "peak": round(peak, 4), "unit": "Tex2/s",
+            "frac": round(achieved / peak, 4), "traffic": recorded_traffic("k5_softmax", w.name, logits),
+            "kernel": "k5_softmax", "kernel_ms": round(k5_ms, 5),
+            "peak_source": f"derived: {MUFU_PER_CLK_SM} ex2 per clock per SM x {SM_COUNT} SMs x {SM_MAX_MHZ:.0f} MHz "
+                           "(clocks.max.sm)"}
+    if clk.get("sm_mhz"):
+        roof["frac_at_sampled_clock"] = round(achieved / (peak * clk["sm_mhz"] / SM_MAX_MHZ), 4)
+    kernels = {}
+    names = ["k5_table_clear", "k5_columns", "k5_softmax", "k5_merge"]
+    for j in range(per_step):
+        kernels[names[j] if per_step == 4 else f"launch{j}"] = {
+            "ms_per_step": round(float(np.mean([recs[s * per_step + j][1] for s in range(args.steps)])), 5),
+            "launches_per_step": 1}
+
+    # end to end: pinned host batch -> device, the call, the mean back to the host
+    e2e = None
+    if not args.no_e2e:
+        pinned = {k: v.pin_memory() for k, v in host.items()}
+        mean_host = torch.empty((), dtype=torch.float32).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+
+        def e2e_step():
+            d = {k: v.to(dev, non_blocking=True) for k, v in pinned.items()}
+            _, _, mean = tt.tt_inbatch_softmax(d["users"], d["items"], w.tau, logq=d["logq"],
+                                               item_ids=d["item_ids"], valid=d["valid"], workspace=ws,
+                                               check=False)
+            mean_host.copy_(mean, non_blocking=True)
+
+        e2e_step()
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        e2e_steps = max(3, min(args.steps, args.e2e_steps))
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(a.elapsed_time(b_) / e2e_steps, world)
+        e2e = {"value": world * logits / (e2e_ms / 1e3), "unit": SOFTMAX_UNIT, "ms_per_step": round(e2e_ms, 4),
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": 4, "steps": e2e_steps}
+
+    line = {
+        "metric": SOFTMAX_METRIC, "value": value, "unit": SOFTMAX_UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded, workloads.py)",
+        "config": {"workload": w.name, "b": w.b, "nc": w.nc, "d": w.d, "tau": w.tau, "catalogue": w.catalogue,
+                   "zipf_s": w.zipf_s, "pad_rate": w.pad_rate, "logq": True, "item_ids": True,
+                   "l2": "flushed before every step (256 MB write outside the step's events)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": roof,
+        "kernels": kernels,
+        "clocks": clk,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = softmax_cpu_baseline(w, host, seconds=args.cpu_seconds)
+    return line
+
+
+def run_softmax_reference(args, world, rank):
+    """The fp64 oracle as the reference arm of --op inbatch_softmax."""
+    if rank != 0:
+        return None
+    w = W.batch(args.batch)
+    host = W.batch_inputs(w, "cpu")
+    budget = args.ref_seconds or max(0.05, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    r, threads = softmax_oracle_sample(w, host, budget)
+    for _ in range(args.warmup):
+        softmax_oracle_run(host, np.arange(r), w.tau)
+    t = sum(softmax_oracle_run(host, np.arange(r), w.tau) for _ in range(args.steps))
+    ms = t / args.steps * 1e3
+    value = r * w.nc / (ms / 1e3)
+    sample = f"each step: first {r} rows of {w.name} against all {w.nc} columns (fp64)"
+    return {"impl": "reference", "metric": SOFTMAX_METRIC, "value": value, "unit": SOFTMAX_UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, workloads.py)",
+            "config": {"workload": w.name, "b": w.b, "nc": w.nc, "d": w.d, "tau": w.tau},
+            "cpu_baseline": {"value": value, "unit": SOFTMAX_UNIT, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": SOFTMAX_UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
 def run_reference(args, world, rank):
     """The fp64 oracle as the reference arm, on this host's cores."""
     if rank != 0:
@@ -475,7 +676,7 @@ def run_reference(args, world, rank):
     raw_c_np = W.to_numpy_rows(raw_c)
     raw_q_np = raw_q.numpy()
     excl_np = None if excl is None else excl.numpy().view(np.uint32)
-    budget = max(0.05, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
+    budget = args.ref_seconds or max(0.05, min(10.0, 150.0 / max(1, args.steps + args.warmup)))
     n_s, b_s, threads = oracle_sample_size(w, raw_c_np, raw_q_np, excl_np, budget)
     for _ in range(args.warmup):
         oracle_sample_run(w, raw_c_np, raw_q_np, excl_np, n_s, b_s)
@@ -510,19 +711,26 @@ def main():
                     help="int8: code the normalised corpus in int8 and score int8 codes (tensor cores kind::i8)")
     ap.add_argument("--mode", default="replicas", choices=["replicas", "shard"],
                     help="N > 1: independent replicas (default) or one corpus sharded by rows over the ranks")
+    ap.add_argument("--op", default="topk", choices=["topk", "inbatch_softmax"],
+                    help="topk: the retrieval step (default); inbatch_softmax: the fused training loss")
+    ap.add_argument("--batch", default="inbatch_b65536_d64", choices=sorted(W.BATCHES),
+                    help="training batch of --op inbatch_softmax")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-seconds", type=float, default=0.0,
+                    help="reference arm: oracle seconds per step (default: sized so the run ends in minutes)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = dist_setup(args)
     try:
+        softmax = args.op == "inbatch_softmax"
         if args.impl == "reference":
-            line = run_reference(args, world, rank)
+            line = run_softmax_reference(args, world, rank) if softmax else run_reference(args, world, rank)
         else:
-            line = run_ours(args, world, rank, local)
+            line = run_softmax(args, world, rank, local) if softmax else run_ours(args, world, rank, local)
         if rank == 0 and line is not None:
             print(json.dumps(line), flush=True)
     finally:

@@ -48,18 +48,22 @@ namespace tt {
 namespace {
 
 constexpr int K5_M = 128;                    // users per tile (TMEM lanes)
-constexpr int K5_N = 256;                    // candidates per tile (TMEM columns)
+constexpr int K5_N = 192;                    // candidates per tile (TMEM columns, <= K5_ACC_COLS)
 constexpr int K5_USER_CHUNK = K5_M * 128;    // one 128-byte K chunk of the user tile
 constexpr int K5_STAGE_BYTES = K5_N * 128;   // one 128-byte K chunk of a candidate tile
 constexpr int K5_MAX_STAGES = 8;
-constexpr int K5_EPI_WARPS = 8;
+constexpr int K5_EPI_WARPS = 12;              // 4 TMEM lane quarters x K5_COL_GROUPS
+constexpr int K5_COL_GROUPS = K5_EPI_WARPS / 4;
+constexpr int K5_WARP_COLS = K5_N / K5_COL_GROUPS;  // columns of one epilogue warp
+constexpr int K5_WARP_CHUNKS = K5_WARP_COLS / 32;   // 32-column TMEM loads per warp and tile
+static_assert(K5_EPI_WARPS % 4 == 0 && K5_WARP_CHUNKS % 2 == 0 && K5_WARP_COLS * K5_COL_GROUPS == K5_N,
+              "epilogue split");
 constexpr int K5_THREADS = 32 * (2 + K5_EPI_WARPS);
 constexpr int K5_TMEM_COLS = 512;
 constexpr int K5_ACC_COLS = 256;
 constexpr int K5_SMEM_BUDGET = 227 * 1024;
-constexpr int K5_HALF = K5_N / 2;            // columns of one epilogue warp
 constexpr float K5_MAX_FLOOR = -1e30f;       // running max before any column (base-2 units)
-constexpr float K5_LAG = 8.0f;               // the running max may trail the true one by 8
+constexpr float K5_SUM_LIMIT = 0x1p64f;      // largest chunk sum taken without raising the max
 constexpr float K5_LOG2E = 1.4426950408889634f;
 constexpr float K5_LN2 = 0.6931471805599453f;
 constexpr unsigned long long K5_EMPTY = 0x8000000000000000ull;  // free table slot
@@ -78,9 +82,9 @@ struct K5Ctl {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
-    // per epilogue warp: biases and groups of its 128 columns of the current tile
-    alignas(16) float nb[K5_EPI_WARPS][K5_HALF];
-    alignas(16) int grp[K5_EPI_WARPS][K5_HALF];
+    // per epilogue warp: biases and groups of its columns of the current tile
+    alignas(16) float nb[K5_EPI_WARPS][K5_WARP_COLS];
+    alignas(16) int grp[K5_EPI_WARPS][K5_WARP_COLS];
 };
 static_assert(offsetof(K5Ctl, nb) % 16 == 0 && offsetof(K5Ctl, grp) % 16 == 0,
               "float4 / int4 reads of the column data need 16-byte alignment");
@@ -88,7 +92,7 @@ static_assert(offsetof(K5Ctl, nb) % 16 == 0 && offsetof(K5Ctl, grp) % 16 == 0,
 struct K5Params {
     const ColInfo* col;  // [nc]
     float* numer;        // [b] diagonal logit, base-2 units
-    float2* part;        // [chunks * 2][b] (running max, sum)
+    float2* part;        // [chunks * K5_COL_GROUPS][b] (running max, sum)
     int* err;
     int b, nc;
     float a2;            // log2(e) / tau
@@ -99,6 +103,39 @@ struct K5Params {
     int stages;
     uint32_t idesc;
 };
+
+// Packed fp32 pairs (sm_100 f32x2): two lanes of work per instruction.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// Keep the compiler from moving uses of TMEM-loaded registers above the
+// tcgen05.wait::ld that makes them valid.
+__device__ __forceinline__ void fence_regs(Cols32& c) {
+    asm volatile(""
+                 : "+f"(c.x[0]), "+f"(c.x[1]), "+f"(c.x[2]), "+f"(c.x[3]), "+f"(c.x[4]), "+f"(c.x[5]),
+                   "+f"(c.x[6]), "+f"(c.x[7]), "+f"(c.x[8]), "+f"(c.x[9]), "+f"(c.x[10]), "+f"(c.x[11]),
+                   "+f"(c.x[12]), "+f"(c.x[13]), "+f"(c.x[14]), "+f"(c.x[15]), "+f"(c.x[16]), "+f"(c.x[17]),
+                   "+f"(c.x[18]), "+f"(c.x[19]), "+f"(c.x[20]), "+f"(c.x[21]), "+f"(c.x[22]), "+f"(c.x[23]),
+                   "+f"(c.x[24]), "+f"(c.x[25]), "+f"(c.x[26]), "+f"(c.x[27]), "+f"(c.x[28]), "+f"(c.x[29]),
+                   "+f"(c.x[30]), "+f"(c.x[31]));
+}
 
 __device__ __forceinline__ float ex2_approx(float x) {
     float y;
@@ -297,14 +334,27 @@ __global__ void __launch_bounds__(K5_THREADS, 1)
         }
     } else {
         // ------------------------------ epilogue ------------------------------
-        // Warp w reads TMEM lanes 32*(w%4).. (its 32 users) and one half of
-        // the tile's 256 columns; each thread keeps (max, sum) for its user.
+        // Warp w reads TMEM lanes 32*(w%4).. (its 32 users) and one group of
+        // K5_WARP_COLS of the tile's 256 columns; each thread keeps (max, sum)
+        // for its user.
         const int ew = warp - 2;
         const int quarter = warp & 3;
-        const int half = ew >> 2;
+        const int cgrp = ew >> 2;
         float* nb_s = ctl->nb[ew];
         int* g_s = ctl->grp[ew];
-        uint32_t tc = 0;
+        const float2 a2v = make_float2(p.a2, p.a2);
+        // TMEM address of chunk c (32 columns) of this warp's slice of accumulator tile tcx
+        auto tmem_chunk = [&](uint32_t tcx, int c) -> uint32_t {
+            return tmem_base + ((uint32_t)(quarter * 32) << 16) +
+                   (uint32_t)((tcx & 1) * K5_ACC_COLS + cgrp * K5_WARP_COLS + c * 32);
+        };
+        // this warp is done reading accumulator tile tcx
+        auto release = [&](uint32_t tcx) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->tempty[tcx & 1]);
+        };
+        uint32_t tc = 0;  // accumulator tiles this CTA has consumed
         bool ok = true;
         for (int u = blockIdx.x; ok && u < n_units; u += gridDim.x) {
             int ut, ch, t0, t1;
@@ -312,98 +362,160 @@ __global__ void __launch_bounds__(K5_THREADS, 1)
             const int i = ut * K5_M + quarter * 32 + lane;  // this thread's user
             const bool row_ok = i < p.b;
             const int my_g = (HITS && row_ok) ? p.col[i].g : -1;
+            // Running max m (base-2 units) and sum of 2^(x - m). m is raised
+            // only when a chunk's sum leaves [0, 2^64] (terms up to 2^64 are
+            // exact enough and far from overflow), so the common path needs
+            // no maximum at all.
             float m = K5_MAX_FLOOR;
-            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
-            for (int t = t0; t < t1; ++t, ++tc) {
-                const int buf = tc & 1;
-                const int jbase = t * K5_N + half * K5_HALF;
-                // this warp's column data, fetched before waiting for the accumulator
-                int2 ci0, ci1, ci2, ci3;  // (bias bits, group) of columns jbase + 32 e + lane
-                ci0 = load_col(p, jbase + lane);
-                ci1 = load_col(p, jbase + 32 + lane);
-                ci2 = load_col(p, jbase + 64 + lane);
-                ci3 = load_col(p, jbase + 96 + lane);
-                __syncwarp();  // the previous tile's reads of nb_s / g_s are done
-                nb_s[lane] = __int_as_float(ci0.x);
-                nb_s[32 + lane] = __int_as_float(ci1.x);
-                nb_s[64 + lane] = __int_as_float(ci2.x);
-                nb_s[96 + lane] = __int_as_float(ci3.x);
-                g_s[lane] = ci0.y;
-                g_s[32 + lane] = ci1.y;
-                g_s[64 + lane] = ci2.y;
-                g_s[96 + lane] = ci3.y;
-                __syncwarp();
-                if (!mbar_wait(&ctl->tfull[buf], (tc >> 1) & 1, abort)) {
-                    ok = false;
-                    break;
+            float sum = 0.f;
+
+            // One chunk (32 columns) of logits: x = acc * log2(e)/tau + nb_j,
+            // then the sum of 2^(x - m) without hits (this row's group).
+            auto process = [&](float* x, int jbase, int c) {
+                const float4* nb4 = reinterpret_cast<const float4*>(nb_s + c * 32);
+#pragma unroll
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    const float4 b4 = nb4[e4];
+                    const float2 lo = fma2(make_float2(x[4 * e4], x[4 * e4 + 1]), a2v, make_float2(b4.x, b4.y));
+                    const float2 hi = fma2(make_float2(x[4 * e4 + 2], x[4 * e4 + 3]), a2v, make_float2(b4.z, b4.w));
+                    x[4 * e4] = lo.x;
+                    x[4 * e4 + 1] = lo.y;
+                    x[4 * e4 + 2] = hi.x;
+                    x[4 * e4 + 3] = hi.y;
                 }
-                tc_fence_after();
-                const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) +
-                                       (uint32_t)(buf * K5_ACC_COLS + half * K5_HALF);
+                // the positive's logit, taken before the group test masks it
+                const int col0 = jbase + c * 32;
+                if (row_ok && (unsigned)(i - col0) < 32u) {
+                    Cols32 tmp;
 #pragma unroll
-                for (int pair = 0; pair < 2; ++pair) {
-                    Cols32 v[2];
-                    tmem_ld_32cols(tbase + (uint32_t)(2 * pair * 32), v[0].x);
-                    tmem_ld_32cols(tbase + (uint32_t)((2 * pair + 1) * 32), v[1].x);
-                    tmem_ld_wait();
-                    if (pair == 1) {
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&ctl->tempty[buf]);  // values are in registers now
+                    for (int e = 0; e < 32; ++e) tmp.x[e] = x[e];
+                    p.numer[i] = select32(tmp, i - col0);
+                }
+                const float2 nm = make_float2(-m, -m);
+                float2 c0 = make_float2(0.f, 0.f), c1 = c0;
+                const int4* g4 = reinterpret_cast<const int4*>(g_s + c * 32);
+#pragma unroll
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    float2 lo = add2(make_float2(x[4 * e4], x[4 * e4 + 1]), nm);
+                    float2 hi = add2(make_float2(x[4 * e4 + 2], x[4 * e4 + 3]), nm);
+                    lo.x = ex2_approx(lo.x);
+                    lo.y = ex2_approx(lo.y);
+                    hi.x = ex2_approx(hi.x);
+                    hi.y = ex2_approx(hi.y);
+                    if constexpr (HITS) {
+                        const int4 gg = g4[e4];
+                        lo.x = gg.x == my_g ? 0.f : lo.x;
+                        lo.y = gg.y == my_g ? 0.f : lo.y;
+                        hi.x = gg.z == my_g ? 0.f : hi.x;
+                        hi.y = gg.w == my_g ? 0.f : hi.y;
                     }
+                    c0 = add2(c0, lo);
+                    c1 = add2(c1, hi);
+                }
+                const float2 cc = add2(c0, c1);
+                const float csum = cc.x + cc.y;
+                if (csum <= K5_SUM_LIMIT) {
+                    sum += csum;
+                    return;
+                }
+                // rare: the running max is too low for this chunk (always on a
+                // unit's first chunk). Mask, take the exact chunk max, rescale.
+                if constexpr (HITS) {
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int c = 2 * pair + h;
-                        const float4* nb4 = reinterpret_cast<const float4*>(nb_s + c * 32);
+                    for (int e = 0; e < 32; ++e)
+                        if (g_s[c * 32 + e] == my_g) x[e] = -INFINITY;
+                }
+                float ca = x[0], cb = x[1];
 #pragma unroll
-                        for (int e4 = 0; e4 < 8; ++e4) {
-                            const float4 b4 = nb4[e4];
-                            v[h].x[4 * e4 + 0] = fmaf(v[h].x[4 * e4 + 0], p.a2, b4.x);
-                            v[h].x[4 * e4 + 1] = fmaf(v[h].x[4 * e4 + 1], p.a2, b4.y);
-                            v[h].x[4 * e4 + 2] = fmaf(v[h].x[4 * e4 + 2], p.a2, b4.z);
-                            v[h].x[4 * e4 + 3] = fmaf(v[h].x[4 * e4 + 3], p.a2, b4.w);
-                        }
-                        // the positive's logit, taken before the group test masks it
-                        const int col0 = jbase + c * 32;
-                        if (row_ok && (unsigned)(i - col0) < 32u) p.numer[i] = select32(v[h], i - col0);
-                        if constexpr (HITS) {
-                            const int4* g4 = reinterpret_cast<const int4*>(g_s + c * 32);
+                for (int e = 2; e < 32; e += 4) {
+                    ca = max3f(ca, x[e], x[e + 1]);
+                    cb = max3f(cb, x[e + 2], x[e + 3]);
+                }
+                const float cmax = fmaxf(ca, cb);
+                if (cmax > m) {
+                    sum *= ex2_approx(m - cmax);
+                    m = cmax;
+                }
+                float r0 = 0.f, r1 = 0.f;
 #pragma unroll
-                            for (int e4 = 0; e4 < 8; ++e4) {
-                                const int4 gg = g4[e4];
-                                if (gg.x == my_g) v[h].x[4 * e4 + 0] = -INFINITY;
-                                if (gg.y == my_g) v[h].x[4 * e4 + 1] = -INFINITY;
-                                if (gg.z == my_g) v[h].x[4 * e4 + 2] = -INFINITY;
-                                if (gg.w == my_g) v[h].x[4 * e4 + 3] = -INFINITY;
-                            }
-                        }
-                        float ca = v[h].x[0], cb = v[h].x[1];
+                for (int e = 0; e < 32; e += 2) {
+                    r0 += ex2_approx(x[e] - m);
+                    r1 += ex2_approx(x[e + 1] - m);
+                }
+                sum += r0 + r1;
+            };
+
+            // column data: tile t0 into shared memory, t0 + 1 into registers
+            int2 ci[K5_WARP_CHUNKS];
 #pragma unroll
-                        for (int e = 2; e < 32; e += 4) {
-                            ca = max3f(ca, v[h].x[e], v[h].x[e + 1]);
-                            cb = max3f(cb, v[h].x[e + 2], v[h].x[e + 3]);
-                        }
-                        const float cmax = fmaxf(ca, cb);
-                        if (cmax > m + K5_LAG) {  // raise the running max, rescale the sums
-                            const float r = ex2_approx(m - cmax);
-                            s0 *= r;
-                            s1 *= r;
-                            s2 *= r;
-                            s3 *= r;
-                            m = cmax;
-                        }
+            for (int e = 0; e < K5_WARP_CHUNKS; ++e) ci[e] = load_col(p, t0 * K5_N + cgrp * K5_WARP_COLS + 32 * e + lane);
+            __syncwarp();  // the previous unit's reads of nb_s / g_s are done
 #pragma unroll
-                        for (int e4 = 0; e4 < 8; ++e4) {
-                            s0 += ex2_approx(v[h].x[4 * e4 + 0] - m);
-                            s1 += ex2_approx(v[h].x[4 * e4 + 1] - m);
-                            s2 += ex2_approx(v[h].x[4 * e4 + 2] - m);
-                            s3 += ex2_approx(v[h].x[4 * e4 + 3] - m);
+            for (int e = 0; e < K5_WARP_CHUNKS; ++e) {
+                nb_s[32 * e + lane] = __int_as_float(ci[e].x);
+                g_s[32 * e + lane] = ci[e].y;
+            }
+            __syncwarp();
+            if (t0 + 1 < t1) {
+#pragma unroll
+                for (int e = 0; e < K5_WARP_CHUNKS; ++e)
+                    ci[e] = load_col(p, (t0 + 1) * K5_N + cgrp * K5_WARP_COLS + 32 * e + lane);
+            }
+            // Chunks are loaded from TMEM one ahead of the one being processed,
+            // alternating between two register sets (K5_WARP_CHUNKS is even,
+            // so chunk c of every tile uses set c & 1).
+            Cols32 v[2];
+            if (!mbar_wait(&ctl->tfull[tc & 1], (tc >> 1) & 1, abort)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            tmem_ld_32cols(tmem_chunk(tc, 0), v[0].x);
+            tmem_ld_wait();
+            fence_regs(v[0]);
+            for (int t = t0; t < t1; ++t, ++tc) {
+                const int jbase = t * K5_N + cgrp * K5_WARP_COLS;
+#pragma unroll
+                for (int c = 0; c < K5_WARP_CHUNKS; ++c) {
+                    bool more = true;
+                    if (c + 1 < K5_WARP_CHUNKS) {
+                        tmem_ld_32cols(tmem_chunk(tc, c + 1), v[(c + 1) & 1].x);
+                    } else if (t + 1 < t1) {
+                        if (!mbar_wait(&ctl->tfull[(tc + 1) & 1], ((tc + 1) >> 1) & 1, abort)) {
+                            ok = false;
+                            break;
                         }
+                        tc_fence_after();
+                        tmem_ld_32cols(tmem_chunk(tc + 1, 0), v[0].x);
+                    } else {
+                        more = false;
+                    }
+                    process(v[c & 1].x, jbase, c);
+                    if (more) {
+                        tmem_ld_wait();
+                        fence_regs(v[(c + 1) & 1]);
+                        if (c + 1 == K5_WARP_CHUNKS - 1) release(tc);  // tile tc fully loaded
+                    }
+                }
+                if (!ok) break;
+                // column data of tile t + 1 (every read of tile t's is done)
+                if (t + 1 < t1) {
+                    __syncwarp();
+#pragma unroll
+                    for (int e = 0; e < K5_WARP_CHUNKS; ++e) {
+                        nb_s[32 * e + lane] = __int_as_float(ci[e].x);
+                        g_s[32 * e + lane] = ci[e].y;
+                    }
+                    __syncwarp();
+                    if (t + 2 < t1) {
+#pragma unroll
+                        for (int e = 0; e < K5_WARP_CHUNKS; ++e)
+                            ci[e] = load_col(p, jbase + 2 * K5_N + 32 * e + lane);
                     }
                 }
             }
             if (!ok) break;
-            if (row_ok) p.part[(int64_t)(ch * 2 + half) * p.b + i] = make_float2(m, (s0 + s1) + (s2 + s3));
+            if (row_ok) p.part[(int64_t)(ch * K5_COL_GROUPS + cgrp) * p.b + i] = make_float2(m, sum);
         }
         if (!ok) {
             atomicExch(p.err, ERR_TIMEOUT_EPI);
@@ -511,6 +623,7 @@ int log2_ceil(int64_t x) {
 SoftmaxPlan softmax_plan(int b, int nc, int d, bool item_ids, int sm_count) {
     SoftmaxPlan pl;
     pl.u_tiles = (b + K5_M - 1) / K5_M;
+    pl.tile_cols = K5_N;
     pl.c_tiles = (nc + K5_N - 1) / K5_N;
     pl.stages = softmax_stages(d);
     // column ranges: make u_tiles * chunks a multiple of the SM count when
@@ -537,7 +650,7 @@ SoftmaxPlan softmax_plan(int b, int nc, int d, bool item_ids, int sm_count) {
     pl.off_ticket = take(sizeof(unsigned));
     pl.off_col = take((size_t)nc * sizeof(ColInfo));
     pl.off_numer = take((size_t)b * sizeof(float));
-    pl.off_part = take((size_t)chunks * 2 * b * sizeof(float2));
+    pl.off_part = take((size_t)chunks * K5_COL_GROUPS * b * sizeof(float2));
     pl.off_keys = take(item_ids ? ((size_t)1 << pl.log2_slots) * sizeof(unsigned long long) : 0);
     pl.off_block_sum = take((size_t)(pl.merge_blocks > 0 ? pl.merge_blocks : 1) * sizeof(double));
     pl.off_block_rows = take((size_t)(pl.merge_blocks > 0 ? pl.merge_blocks : 1) * sizeof(int));
@@ -607,7 +720,7 @@ cudaError_t launch_softmax(const SoftmaxPlan& pl, const CUtensorMap& tm_users, c
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     note_launch_begin(TT_KIND_SOFTMAX, s);
-    k5_merge<<<pl.merge_blocks, K5_MERGE_THREADS, 0, s>>>(part, pl.chunks * 2, numer, valid, b, hits ? 1 : 0,
+    k5_merge<<<pl.merge_blocks, K5_MERGE_THREADS, 0, s>>>(part, pl.chunks * K5_COL_GROUPS, numer, valid, b, hits ? 1 : 0,
                                                            err, lse, loss, mean, block_sum, block_rows, ticket);
     note_launch_end(TT_KIND_SOFTMAX, s);
     return cudaGetLastError();

@@ -944,7 +944,7 @@ tt_status tt_inbatch_softmax(const void* users, const void* items, tt_dtype dtyp
     memset(&tm_items, 0, sizeof tm_items);
     if (b > 0) {
         if (!bf16_tile_tensor_map(users, b, d, d, 128, &tm_users)) return TT_ERR_CUDA;
-        if (!bf16_tile_tensor_map(items, nc, d, d, 256, &tm_items)) return TT_ERR_CUDA;
+        if (!bf16_tile_tensor_map(items, nc, d, d, pl.tile_cols, &tm_items)) return TT_ERR_CUDA;
     }
     cudaError_t e = launch_softmax(pl, tm_users, tm_items, b, nc, d, tau, logq, item_ids, valid, lse, loss, mean,
                                    workspace, static_cast<cudaStream_t>(stream), sms);

@@ -99,6 +99,7 @@ cudaError_t launch_mask_slice(const uint32_t* in, int64_t start, int64_t count, 
 // In-batch sampled softmax (k_softmax.cu): work split and workspace layout
 // (byte offsets of each region; the error word is at offset 0).
 struct SoftmaxPlan {
+    int tile_cols;  // candidates per tile (rows of one items box)
     int u_tiles, c_tiles, chunks, stages, log2_slots, merge_blocks;
     size_t off_err, off_ticket, off_col, off_numer, off_part, off_keys, off_block_sum, off_block_rows;
     size_t bytes;
@@ -106,7 +107,7 @@ struct SoftmaxPlan {
 SoftmaxPlan softmax_plan(int b, int nc, int d, bool item_ids, int sm_count);
 bool softmax_supported(int d);
 // users [b, d] and items [nc, d] bf16 through tm_users (boxes of 64 x 128)
-// and tm_items (boxes of 64 x 256).
+// and tm_items (boxes of 64 x tile_cols).
 cudaError_t launch_softmax(const SoftmaxPlan& pl, const CUtensorMap& tm_users, const CUtensorMap& tm_items,
                            int b, int nc, int d, float tau, const float* logq, const int64_t* item_ids,
                            const uint8_t* valid, float* lse, float* loss, float* mean, void* workspace,

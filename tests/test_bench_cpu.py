@@ -40,6 +40,19 @@ def test_reference_arm_prints_one_line():
     assert line["e2e"]["h2d_bytes_per_step"] == 0
 
 
+def test_softmax_reference_arm_prints_one_line():
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--op", "inbatch_softmax", "--batch",
+                        "inbatch_b8192_d64", "--steps", "3", "--warmup", "3", "--ref-seconds", "0.2"], cwd=ROOT,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr
+    lines = _json_lines(r.stdout)
+    assert len(lines) == 1
+    line = lines[0]
+    assert line["impl"] == "reference" and line["unit"] == "logits/s" and line["value"] > 0
+    assert line["config"]["workload"] == "inbatch_b8192_d64"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["d2h_bytes_per_step"] == 0
+
+
 def test_reference_arm_under_two_ranks():
     port = _free_port()
     r = subprocess.run([sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
