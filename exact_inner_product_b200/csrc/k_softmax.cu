@@ -370,7 +370,7 @@ __global__ void __launch_bounds__(K5_THREADS, 1)
             float sum = 0.f;
 
             // One chunk (32 columns) of logits: x = acc * log2(e)/tau + nb_j,
-            // then the sum of 2^(x - m) without hits (this row's group).
+            // hits (this row's group) set to -inf, then the sum of 2^(x - m).
             auto process = [&](float* x, int jbase, int c) {
                 const float4* nb4 = reinterpret_cast<const float4*>(nb_s + c * 32);
 #pragma unroll
@@ -391,9 +391,19 @@ __global__ void __launch_bounds__(K5_THREADS, 1)
                     for (int e = 0; e < 32; ++e) tmp.x[e] = x[e];
                     p.numer[i] = select32(tmp, i - col0);
                 }
+                if constexpr (HITS) {  // hits (this row's group) leave the sum: x = -inf
+                    const int4* g4 = reinterpret_cast<const int4*>(g_s + c * 32);
+#pragma unroll
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        const int4 gg = g4[e4];
+                        x[4 * e4] = gg.x == my_g ? -INFINITY : x[4 * e4];
+                        x[4 * e4 + 1] = gg.y == my_g ? -INFINITY : x[4 * e4 + 1];
+                        x[4 * e4 + 2] = gg.z == my_g ? -INFINITY : x[4 * e4 + 2];
+                        x[4 * e4 + 3] = gg.w == my_g ? -INFINITY : x[4 * e4 + 3];
+                    }
+                }
                 const float2 nm = make_float2(-m, -m);
                 float2 c0 = make_float2(0.f, 0.f), c1 = c0;
-                const int4* g4 = reinterpret_cast<const int4*>(g_s + c * 32);
 #pragma unroll
                 for (int e4 = 0; e4 < 8; ++e4) {
                     float2 lo = add2(make_float2(x[4 * e4], x[4 * e4 + 1]), nm);
@@ -402,13 +412,6 @@ __global__ void __launch_bounds__(K5_THREADS, 1)
                     lo.y = ex2_approx(lo.y);
                     hi.x = ex2_approx(hi.x);
                     hi.y = ex2_approx(hi.y);
-                    if constexpr (HITS) {
-                        const int4 gg = g4[e4];
-                        lo.x = gg.x == my_g ? 0.f : lo.x;
-                        lo.y = gg.y == my_g ? 0.f : lo.y;
-                        hi.x = gg.z == my_g ? 0.f : hi.x;
-                        hi.y = gg.w == my_g ? 0.f : hi.y;
-                    }
                     c0 = add2(c0, lo);
                     c1 = add2(c1, hi);
                 }
@@ -419,12 +422,7 @@ __global__ void __launch_bounds__(K5_THREADS, 1)
                     return;
                 }
                 // rare: the running max is too low for this chunk (always on a
-                // unit's first chunk). Mask, take the exact chunk max, rescale.
-                if constexpr (HITS) {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (g_s[c * 32 + e] == my_g) x[e] = -INFINITY;
-                }
+                // unit's first chunk). Take the exact chunk max, rescale.
                 float ca = x[0], cb = x[1];
 #pragma unroll
                 for (int e = 2; e < 32; e += 4) {
