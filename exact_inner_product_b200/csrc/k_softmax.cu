@@ -82,9 +82,9 @@ struct K5Ctl {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
-    // per epilogue warp: biases and groups of its columns of the current tile
-    alignas(16) float nb[K5_EPI_WARPS][K5_WARP_COLS];
-    alignas(16) int grp[K5_EPI_WARPS][K5_WARP_COLS];
+    // per epilogue warp: biases and groups of its columns, for two tiles in flight
+    alignas(16) float nb[K5_EPI_WARPS][2][K5_WARP_COLS];
+    alignas(16) int grp[K5_EPI_WARPS][2][K5_WARP_COLS];
 };
 static_assert(offsetof(K5Ctl, nb) % 16 == 0 && offsetof(K5Ctl, grp) % 16 == 0,
               "float4 / int4 reads of the column data need 16-byte alignment");
@@ -340,8 +340,7 @@ __global__ void __launch_bounds__(K5_THREADS, 1)
         const int ew = warp - 2;
         const int quarter = warp & 3;
         const int cgrp = ew >> 2;
-        float* nb_s = ctl->nb[ew];
-        int* g_s = ctl->grp[ew];
+
         const float2 a2v = make_float2(p.a2, p.a2);
         // TMEM address of chunk c (32 columns) of this warp's slice of accumulator tile tcx
         auto tmem_chunk = [&](uint32_t tcx, int c) -> uint32_t {
@@ -369,9 +368,13 @@ __global__ void __launch_bounds__(K5_THREADS, 1)
             float m = K5_MAX_FLOOR;
             float sum = 0.f;
 
-            // One chunk (32 columns) of logits: x = acc * log2(e)/tau + nb_j,
-            // hits (this row's group) set to -inf, then the sum of 2^(x - m).
-            auto process = [&](float* x, int jbase, int c) {
+            // One chunk (32 columns) in three parts, so that the next chunk's
+            // logits can be formed while this chunk's sum is reduced and tested.
+            // Part 1: x = acc * log2(e)/tau + nb_j; the positive's logit; hits
+            // (this row's group) set to -inf. Needs no running max.
+            auto logits = [&](float* x, int t, int c) {
+                const float* nb_s = ctl->nb[ew][t & 1];
+                const int* g_s = ctl->grp[ew][t & 1];
                 const float4* nb4 = reinterpret_cast<const float4*>(nb_s + c * 32);
 #pragma unroll
                 for (int e4 = 0; e4 < 8; ++e4) {
@@ -383,15 +386,14 @@ __global__ void __launch_bounds__(K5_THREADS, 1)
                     x[4 * e4 + 2] = hi.x;
                     x[4 * e4 + 3] = hi.y;
                 }
-                // the positive's logit, taken before the group test masks it
-                const int col0 = jbase + c * 32;
+                const int col0 = t * K5_N + cgrp * K5_WARP_COLS + c * 32;
                 if (row_ok && (unsigned)(i - col0) < 32u) {
                     Cols32 tmp;
 #pragma unroll
                     for (int e = 0; e < 32; ++e) tmp.x[e] = x[e];
                     p.numer[i] = select32(tmp, i - col0);
                 }
-                if constexpr (HITS) {  // hits (this row's group) leave the sum: x = -inf
+                if constexpr (HITS) {
                     const int4* g4 = reinterpret_cast<const int4*>(g_s + c * 32);
 #pragma unroll
                     for (int e4 = 0; e4 < 8; ++e4) {
@@ -402,6 +404,9 @@ __global__ void __launch_bounds__(K5_THREADS, 1)
                         x[4 * e4 + 3] = gg.w == my_g ? -INFINITY : x[4 * e4 + 3];
                     }
                 }
+            };
+            // Part 2: the chunk's sum of 2^(x - m).
+            auto chunk_sum = [&](const float* x) -> float {
                 const float2 nm = make_float2(-m, -m);
                 float2 c0 = make_float2(0.f, 0.f), c1 = c0;
 #pragma unroll
@@ -416,13 +421,16 @@ __global__ void __launch_bounds__(K5_THREADS, 1)
                     c1 = add2(c1, hi);
                 }
                 const float2 cc = add2(c0, c1);
-                const float csum = cc.x + cc.y;
+                return cc.x + cc.y;
+            };
+            // Part 3: take the sum, or (rare: the running max is too low for this
+            // chunk, always on a unit's first chunk) raise the max to the exact
+            // chunk max, rescale and sum again.
+            auto accumulate = [&](const float* x, float csum) {
                 if (csum <= K5_SUM_LIMIT) {
                     sum += csum;
                     return;
                 }
-                // rare: the running max is too low for this chunk (always on a
-                // unit's first chunk). Take the exact chunk max, rescale.
                 float ca = x[0], cb = x[1];
 #pragma unroll
                 for (int e = 2; e < 32; e += 4) {
@@ -442,24 +450,28 @@ __global__ void __launch_bounds__(K5_THREADS, 1)
                 }
                 sum += r0 + r1;
             };
+            // column data of tile t into shared-memory buffer t & 1
+            auto stage_cols = [&](int t, const int2* cv) {
+                __syncwarp();  // earlier reads of that buffer are done
+#pragma unroll
+                for (int e = 0; e < K5_WARP_CHUNKS; ++e) {
+                    ctl->nb[ew][t & 1][32 * e + lane] = __int_as_float(cv[e].x);
+                    ctl->grp[ew][t & 1][32 * e + lane] = cv[e].y;
+                }
+                __syncwarp();
+            };
 
             // column data: tile t0 into shared memory, t0 + 1 into registers
             int2 ci[K5_WARP_CHUNKS];
 #pragma unroll
             for (int e = 0; e < K5_WARP_CHUNKS; ++e) ci[e] = load_col(p, t0 * K5_N + cgrp * K5_WARP_COLS + 32 * e + lane);
-            __syncwarp();  // the previous unit's reads of nb_s / g_s are done
-#pragma unroll
-            for (int e = 0; e < K5_WARP_CHUNKS; ++e) {
-                nb_s[32 * e + lane] = __int_as_float(ci[e].x);
-                g_s[32 * e + lane] = ci[e].y;
-            }
-            __syncwarp();
+            stage_cols(t0, ci);
             if (t0 + 1 < t1) {
 #pragma unroll
                 for (int e = 0; e < K5_WARP_CHUNKS; ++e)
                     ci[e] = load_col(p, (t0 + 1) * K5_N + cgrp * K5_WARP_COLS + 32 * e + lane);
             }
-            // Chunks are loaded from TMEM one ahead of the one being processed,
+            // Chunks are loaded from TMEM one ahead of the one being summed,
             // alternating between two register sets (K5_WARP_CHUNKS is even,
             // so chunk c of every tile uses set c & 1).
             Cols32 v[2];
@@ -471,8 +483,18 @@ __global__ void __launch_bounds__(K5_THREADS, 1)
             tmem_ld_32cols(tmem_chunk(tc, 0), v[0].x);
             tmem_ld_wait();
             fence_regs(v[0]);
+            logits(v[0].x, t0, 0);
             for (int t = t0; t < t1; ++t, ++tc) {
-                const int jbase = t * K5_N + cgrp * K5_WARP_COLS;
+                // column data of tile t + 1 (its first chunk's logits are formed
+                // during this tile's last chunk)
+                if (t + 1 < t1) {
+                    stage_cols(t + 1, ci);
+                    if (t + 2 < t1) {
+#pragma unroll
+                        for (int e = 0; e < K5_WARP_CHUNKS; ++e)
+                            ci[e] = load_col(p, (t + 2) * K5_N + cgrp * K5_WARP_COLS + 32 * e + lane);
+                    }
+                }
 #pragma unroll
                 for (int c = 0; c < K5_WARP_CHUNKS; ++c) {
                     bool more = true;
@@ -488,29 +510,19 @@ __global__ void __launch_bounds__(K5_THREADS, 1)
                     } else {
                         more = false;
                     }
-                    process(v[c & 1].x, jbase, c);
+                    const float csum = chunk_sum(v[c & 1].x);
                     if (more) {
                         tmem_ld_wait();
                         fence_regs(v[(c + 1) & 1]);
                         if (c + 1 == K5_WARP_CHUNKS - 1) release(tc);  // tile tc fully loaded
+                        if (c + 1 < K5_WARP_CHUNKS)
+                            logits(v[(c + 1) & 1].x, t, c + 1);
+                        else
+                            logits(v[0].x, t + 1, 0);
                     }
+                    accumulate(v[c & 1].x, csum);
                 }
                 if (!ok) break;
-                // column data of tile t + 1 (every read of tile t's is done)
-                if (t + 1 < t1) {
-                    __syncwarp();
-#pragma unroll
-                    for (int e = 0; e < K5_WARP_CHUNKS; ++e) {
-                        nb_s[32 * e + lane] = __int_as_float(ci[e].x);
-                        g_s[32 * e + lane] = ci[e].y;
-                    }
-                    __syncwarp();
-                    if (t + 2 < t1) {
-#pragma unroll
-                        for (int e = 0; e < K5_WARP_CHUNKS; ++e)
-                            ci[e] = load_col(p, jbase + 2 * K5_N + 32 * e + lane);
-                    }
-                }
             }
             if (!ok) break;
             if (row_ok) p.part[(int64_t)(ch * K5_COL_GROUPS + cgrp) * p.b + i] = make_float2(m, sum);
