@@ -448,4 +448,32 @@ cudaError_t launch_pad(int32_t* out_ids, float* out_scores, int64_t count, cudaS
     return cudaGetLastError();
 }
 
+// Per query: the loosest of its sets' thresholds, which every kernel's first
+// test uses before the exact per-set test.
+__global__ void k4_sets_min(const uint64_t* __restrict__ theta_v, const float* __restrict__ thf_v, int n_sets,
+                            int b, int b_pad, uint64_t* __restrict__ theta_min, float* __restrict__ thf_min) {
+    const int q = blockIdx.x * blockDim.x + threadIdx.x;
+    if (q >= b_pad) return;
+    uint64_t t = KEY_MAX;
+    float f = key_floor(KEY_MAX);
+    if (q < b) {
+        for (int s = 0; s < n_sets; ++s) {
+            const uint64_t ts = theta_v[(int64_t)s * b + q];
+            if (ts < t) t = ts;
+            f = fminf(f, thf_v[(int64_t)s * b + q]);
+        }
+    }
+    theta_min[q] = t;
+    thf_min[q] = f;
+}
+
+cudaError_t launch_sets_min(const uint64_t* theta_v, const float* thf_v, int n_sets, int b, int b_pad,
+                            uint64_t* theta_min, float* thf_min, cudaStream_t s) {
+    if (b_pad <= 0) return cudaSuccess;
+    note_launch_begin(TT_KIND_AUX, s);
+    k4_sets_min<<<(b_pad + 255) / 256, 256, 0, s>>>(theta_v, thf_v, n_sets, b, b_pad, theta_min, thf_min);
+    note_launch_end(TT_KIND_AUX, s);
+    return cudaGetLastError();
+}
+
 }  // namespace tt

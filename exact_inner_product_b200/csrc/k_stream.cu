@@ -19,6 +19,9 @@
 //   is the exact int32 sum of code products (dp4a), s = fl(fl(fl(dot) * us_b)
 //   * c_j) with c_j = fl(scale_j * inv_tau). Kept keys are appended to the query's buffer;
 //   the append is warp-aggregated (one atomicAdd per query per warp).
+// Several result sets by candidate type: the first test uses the query's
+//   loosest set threshold; a key that passes goes to its row's set if it
+//   beats that set's threshold.
 // (recsys_two_tower_model.py `forward`: scores = user . post_embeddings^T,
 // masked candidates dropped; the top-k is taken from the kept keys by the
 // select kernel.)
@@ -69,6 +72,17 @@ __device__ __forceinline__ void unpack32(const Raw32& r, float* x, __nv_bfloat16
     for (int i = 0; i < 8; ++i) {
         x[2 * i] = __uint_as_float(r.w[i] << 16);
         x[2 * i + 1] = __uint_as_float(r.w[i] & 0xFFFF0000u);
+    }
+}
+
+// Several result sets: a key that beat the query's loosest set threshold is
+// kept if it beats the threshold of its row's set, in that set's buffer.
+__device__ __forceinline__ void append_set(const PassArgs& a, int q, int rset, bool keep, uint64_t key) {
+    if (!keep) return;
+    const int64_t v = (int64_t)rset * a.b + q;
+    if (key > a.theta_v[v]) {
+        const uint32_t slot = atomicAdd(a.count + v, 1u);
+        if (slot < (uint32_t)a.cap) a.keys[v * a.cap + slot] = key;
     }
 }
 
@@ -138,14 +152,23 @@ __global__ void __launch_bounds__(K2_THREADS)
         const int64_t id = r * a.stride;
         bool row_ok = valid;
         float c = a.inv_tau;
+        int rset = 0;
         if (valid) {
             if (a.exclude) row_ok = !((a.exclude[id >> 5] >> (id & 31)) & 1u);
             if (a.inv_norm) c = a.inv_norm[id] * a.inv_tau;
+            if (a.types) {
+                rset = a.set_of[a.types[id]];
+                if (rset < 0) row_ok = false;
+            }
         }
 #pragma unroll
         for (int qb = 0; qb < QB; ++qb) {
             const uint64_t key = make_key(acc[qb] * c, (uint32_t)id);
             const bool keep = row_ok && key > th[qb];
+            if (a.types) {  // this row's set: its own threshold and buffer
+                append_set(a, q0 + qb, rset, keep, key);
+                continue;
+            }
             const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, keep);
             if (ballot) {
                 const int q = q0 + qb;
@@ -241,15 +264,23 @@ __global__ void __launch_bounds__(K2_THREADS)
         const int64_t id = r * a.stride;
         bool row_ok = valid;
         float c = a.inv_tau;
+        int rset = 0;
         if (valid) {
             if (a.exclude) row_ok = !((a.exclude[id >> 5] >> (id & 31)) & 1u);
             c = a.inv_norm[id] * a.inv_tau;
+            if (a.types) {
+                rset = a.set_of[a.types[id]];
+                if (rset < 0) row_ok = false;
+            }
         }
 #pragma unroll
         for (int qb = 0; qb < QB; ++qb) {
             // |acc| < 2^24 (127 * 127 * 512), so fl(acc) is exact
             const uint64_t key = make_key((float)acc[qb] * us[qb] * c, (uint32_t)id);
-            append_warp(a, q0 + qb, row_ok && key > th[qb], key, lane);
+            if (a.types)
+                append_set(a, q0 + qb, rset, row_ok && key > th[qb], key);
+            else
+                append_warp(a, q0 + qb, row_ok && key > th[qb], key, lane);
         }
     }
 }

@@ -283,9 +283,14 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
                 const int64_t id = j * a.stride;
                 bool row_ok = valid;
                 float c = a.inv_tau;
+                int rset = 0;  // several result sets: this row's set
                 if (valid) {
                     if (a.exclude) row_ok = !((a.exclude[id >> 5] >> (id & 31)) & 1u);
                     if (a.inv_norm) c = a.inv_norm[id] * a.inv_tau;
+                    if (a.types) {
+                        rset = a.set_of[a.types[id]];
+                        if (rset < 0) row_ok = false;
+                    }
                 }
                 if (!mbar_wait(&ctl->tfull[buf], (tc >> 1) & 1, abort)) {
                     ok = false;
@@ -358,8 +363,16 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
                                 m &= m - 1;
                                 const float acc = I8 ? select32(v[h], i) * q_us[cj * 32 + i] : select32(v[h], i);
                                 const uint64_t key = make_key(acc * c, (uint32_t)id);
-                                if (key > th_key[cj * 32 + i]) {
-                                    const int q = qt * p.nq + col0 + i;
+                                const int q = qt * p.nq + col0 + i;
+                                if (a.types) {  // the row's set: its threshold and buffer
+                                    if (q < a.b) {
+                                        const int64_t v = (int64_t)rset * a.b + q;
+                                        if (key > a.theta_v[v]) {
+                                            const uint32_t slot = atomicAdd(a.count + v, 1u);
+                                            if (slot < (uint32_t)a.cap) a.keys[v * a.cap + slot] = key;
+                                        }
+                                    }
+                                } else if (key > th_key[cj * 32 + i]) {
                                     const uint32_t slot = atomicAdd(a.count + q, 1u);
                                     if (slot < (uint32_t)a.cap) a.keys[(int64_t)q * a.cap + slot] = key;
                                 }

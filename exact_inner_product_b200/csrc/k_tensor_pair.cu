@@ -403,7 +403,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
                                 const int64_t id = (row0 + col0 + i) * a.stride;
                                 const float c = uniform_c ? a.inv_tau : cw[col0 + i];
                                 const uint64_t key = make_key(select32(v[h], i) * c, (uint32_t)id);
-                                if (key > th_key) {
+                                if (a.types) {  // several result sets: the row's set
+                                    const int rset = a.set_of[a.types[id]];
+                                    if (rset >= 0 && q < a.b) {
+                                        const int64_t vq = (int64_t)rset * a.b + q;
+                                        if (key > a.theta_v[vq]) {
+                                            const uint32_t slot = atomicAdd(a.count + vq, 1u);
+                                            if (slot < (uint32_t)a.cap) a.keys[vq * a.cap + slot] = key;
+                                        }
+                                    }
+                                } else if (key > th_key) {
                                     const uint32_t slot = atomicAdd(cnt, 1u);
                                     if (slot < (uint32_t)a.cap) qkeys[slot] = key;
                                 }

@@ -315,6 +315,11 @@ struct Scratch {
     __nv_bfloat16* qcast;
     int8_t* qcodes;   // int8 index: the queries' codes [b, d]
     float* qscale;    // and their scales [b]
+    // several result sets by type: per-query minima of the virtual
+    // thresholds [b_pad] and the type -> set map [256]
+    uint64_t* theta_min;
+    float* thf_min;
+    int8_t* set_of;
 };
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -377,19 +382,28 @@ static void pinned_give(int* p) {
     g_pinned_pool.push_back(p);
 }
 
-static tt_status get_scratch(tt_index* ix, int b, int b_pad, int cap, int d, bool need_qcast,
-                             bool need_q8, Scratch* out) {
+// b, b_pad: queries (with the padding of the query tiles); vq, vpad: the
+// lists kept (vq = b, or sets * b for several result sets, padded to vpad);
+// n_min: entries of the per-query minima (0 without result sets).
+static tt_status get_scratch(tt_index* ix, int b, int b_pad, int vq, int vpad, int n_min, int cap, int d,
+                             bool need_qcast, bool need_q8, Scratch* out) {
     size_t off = 0;
     const size_t o_keys = off;
-    off = align_up(off + (size_t)b * cap * 8, 256);
+    off = align_up(off + (size_t)vq * cap * 8, 256);
     const size_t o_count = off;
-    off = align_up(off + (size_t)b_pad * 4, 256);
+    off = align_up(off + (size_t)vpad * 4, 256);
     const size_t o_theta = off;
-    off = align_up(off + (size_t)b_pad * 8, 256);
+    off = align_up(off + (size_t)vpad * 8, 256);
     const size_t o_thf = off;
-    off = align_up(off + (size_t)b_pad * 4, 256);
+    off = align_up(off + (size_t)vpad * 4, 256);
     const size_t o_status = off;
-    off = align_up(off + (size_t)b_pad * 4, 256);
+    off = align_up(off + (size_t)vpad * 4, 256);
+    const size_t o_tmin = off;
+    off = align_up(off + (size_t)n_min * 8, 256);
+    const size_t o_fmin = off;
+    off = align_up(off + (size_t)n_min * 4, 256);
+    const size_t o_setof = off;
+    off = align_up(off + (n_min > 0 ? 256 : 0), 256);
     const size_t o_flags = off;
     off = align_up(off + 64, 256);
     const size_t o_q = off;
@@ -428,6 +442,9 @@ static tt_status get_scratch(tt_index* ix, int b, int b_pad, int cap, int d, boo
     out->qcast = need_qcast ? reinterpret_cast<__nv_bfloat16*>(base + o_q) : nullptr;
     out->qcodes = need_q8 ? reinterpret_cast<int8_t*>(base + o_q8) : nullptr;
     out->qscale = need_q8 ? reinterpret_cast<float*>(base + o_qs) : nullptr;
+    out->theta_min = n_min > 0 ? reinterpret_cast<uint64_t*>(base + o_tmin) : nullptr;
+    out->thf_min = n_min > 0 ? reinterpret_cast<float*>(base + o_fmin) : nullptr;
+    out->set_of = n_min > 0 ? reinterpret_cast<int8_t*>(base + o_setof) : nullptr;
     if (!ix->h_flags) {
         ix->h_flags = pinned_take();
         if (!ix->h_flags) {
@@ -448,6 +465,7 @@ struct PathCfg {
     int q_dtype;
     const float* qscale;  // int8 index: query scales
     int withhold_copy;    // test hook, see tt_options
+    const uint8_t* types; // several result sets by type: the candidates' types, else null
     CUtensorMap tm_q;
 };
 
@@ -474,6 +492,13 @@ static tt_status run_pass(const tt_index* ix, const PathCfg& pc, const Plan& pla
     a.keys = sc.keys;
     a.cap = plan.cap;
     a.err = sc.flags + 1;
+    a.types = pc.types;
+    a.set_of = pc.types ? sc.set_of : nullptr;
+    a.theta_v = pc.types ? sc.theta : nullptr;
+    if (pc.types) {  // first tests against each query's loosest set threshold
+        a.theta = sc.theta_min;
+        a.thf = sc.thf_min;
+    }
     cudaError_t e;
     if (pc.path == 2) {
         CUtensorMap tm_rows;
@@ -694,9 +719,13 @@ tt_status tt_last_stats(const tt_index* index, tt_stats* out) {
     return TT_OK;
 }
 
-tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtype, int32_t b,
-                           const uint32_t* exclude_bits, float tau, int32_t k, int32_t* out_ids,
-                           float* out_scores, void* stream, const tt_options* options) {
+// The whole search. With `types`, one pass serves n_sets result sets: set t
+// takes the candidates whose type maps to t (set_of_host, 256 entries, -1 for
+// none), and its lists are out_ids[t * b * k ...] (virtual queries t * b + q).
+static tt_status score_core(tt_index* index, const void* queries, tt_dtype q_dtype, int32_t b,
+                            const uint32_t* exclude_bits, float tau, int32_t k, int32_t* out_ids,
+                            float* out_scores, void* stream, const tt_options* options, const uint8_t* types,
+                            int n_sets, const int8_t* set_of_host) {
     // ---------------- host-side validation (no device calls) ----------------
     if (!index) return TT_ERR_INVALID_ARG;
     if (b < 0) return TT_ERR_INVALID_ARG;
@@ -731,6 +760,7 @@ tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtyp
     if (path == 2 && !tc_possible) return TT_ERR_UNSUPPORTED;
     if (path == 3 && !pair_possible) return TT_ERR_UNSUPPORTED;
     if (b == 0) return TT_OK;
+    const int V = types ? n_sets * b : b;  // lists kept: one per (set, query)
 
     // ---------------- device checks ----------------
     if ((st = check_device_ptr(queries, "queries")) != TT_OK) return st;
@@ -757,7 +787,7 @@ tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtyp
     }
 
     if (index->n == 0) {
-        cudaError_t e = launch_pad(out_ids, out_scores, (int64_t)b * k, s);
+        cudaError_t e = launch_pad(out_ids, out_scores, (int64_t)V * k, s);
         if (e != cudaSuccess) return cuda_fail(e, "pad");
         stats.launches = (int)(g_launches.load() - launches0);
         index->last = stats;
@@ -778,7 +808,10 @@ tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtyp
     const int b_pad = (path == 2 ? q_tiles * nq : path == 3 ? q_tiles * 256 : b) + 64;
     const bool need_qcast = !i8 && path >= 2 && q_dtype == TT_F32;
     Scratch sc;
-    if ((st = get_scratch(index, b, b_pad, plan.cap, index->d, need_qcast, i8, &sc)) != TT_OK) return st;
+    const int v_pad = types ? V + 64 : b_pad;
+    if ((st = get_scratch(index, b, b_pad, V, v_pad, types ? b_pad : 0, plan.cap, index->d, need_qcast, i8, &sc)) !=
+        TT_OK)
+        return st;
     const int sms = sm_count_current();
     const float inv_tau = 1.0f / tau;
 
@@ -788,6 +821,13 @@ tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtyp
     pc.queries = queries;
     pc.q_dtype = q_dtype;
     pc.withhold_copy = options ? options->withhold_copy : 0;
+    pc.types = types;
+    if (types) TT_CUDA(cudaMemcpyAsync(sc.set_of, set_of_host, 256, cudaMemcpyHostToDevice, s), "set map");
+    // several result sets: every kernel's first test uses each query's loosest set threshold
+    auto sets_min = [&]() -> cudaError_t {
+        return types ? launch_sets_min(sc.theta, sc.thf, n_sets, b, b_pad, sc.theta_min, sc.thf_min, s)
+                     : cudaSuccess;
+    };
     if (i8) {
         // code the queries as given (recsys_two_tower_model.py `compute_top_k_int8`)
         cudaError_t e = launch_quantize(queries, q_dtype, b, index->d, sc.qcodes, sc.qscale, false, s);
@@ -810,16 +850,19 @@ tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtyp
             return TT_ERR_CUDA;
     }
 
-    cudaError_t e = launch_init(sc.count, sc.theta, sc.thf, KEY_MIN, b, b_pad, sc.flags, s);
+    cudaError_t e = launch_init(sc.count, sc.theta, sc.thf, KEY_MIN, V, v_pad, sc.flags, s);
+    if (e == cudaSuccess) e = sets_min();
     if (e != cudaSuccess) return cuda_fail(e, "init");
     for (int lv = plan.levels - 1; lv >= 0; --lv) {
         if ((st = run_pass(index, pc, plan, lv, sc, exclude_bits, inv_tau, b, s, sms)) != TT_OK) return st;
-        if (lv > 0)
-            e = launch_select_threshold(sc.keys, sc.count, plan.cap, b, plan.rank[lv], sc.theta,
+        if (lv > 0) {
+            e = launch_select_threshold(sc.keys, sc.count, plan.cap, V, plan.rank[lv], sc.theta,
                                         sc.thf, s);
-        else
-            e = launch_select_final(sc.keys, sc.count, plan.cap, b, k, sc.theta, sc.thf, sc.status,
+            if (e == cudaSuccess) e = sets_min();
+        } else {
+            e = launch_select_final(sc.keys, sc.count, plan.cap, V, k, sc.theta, sc.thf, sc.status,
                                     sc.flags, 0, out_ids, out_scores, s);
+        }
         if (e != cudaSuccess) return cuda_fail(e, "select");
     }
     int rescans = 0;
@@ -841,10 +884,11 @@ tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtyp
                      rescans);
             return TT_ERR_INTERNAL;
         }
-        e = launch_prepare_repair(sc.theta, sc.thf, sc.status, b, sc.flags, s);
+        e = launch_prepare_repair(sc.theta, sc.thf, sc.status, V, sc.flags, s);
+        if (e == cudaSuccess) e = sets_min();
         if (e != cudaSuccess) return cuda_fail(e, "prepare rescan");
         if ((st = run_pass(index, pc, plan, 0, sc, exclude_bits, inv_tau, b, s, sms)) != TT_OK) return st;
-        e = launch_select_final(sc.keys, sc.count, plan.cap, b, k, sc.theta, sc.thf, sc.status,
+        e = launch_select_final(sc.keys, sc.count, plan.cap, V, k, sc.theta, sc.thf, sc.status,
                                 sc.flags, 1, out_ids, out_scores, s);
         if (e != cudaSuccess) return cuda_fail(e, "select");
         ++rescans;
@@ -853,6 +897,13 @@ tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtyp
     stats.launches = (int)(g_launches.load() - launches0);
     index->last = stats;
     return TT_OK;
+}
+
+tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype q_dtype, int32_t b,
+                           const uint32_t* exclude_bits, float tau, int32_t k, int32_t* out_ids,
+                           float* out_scores, void* stream, const tt_options* options) {
+    return score_core(index, queries, q_dtype, b, exclude_bits, tau, k, out_ids, out_scores, stream, options,
+                      nullptr, 0, nullptr);
 }
 
 tt_status tt_merge_topk(const int32_t* ids, const float* scores, int32_t parts, int32_t b, int32_t k_in,
@@ -1043,29 +1094,32 @@ tt_status tt_score_topk_types(tt_index* index, const void* queries, tt_dtype q_d
         if (set_types[t] < 0 || set_types[t] > 255) return TT_ERR_INVALID_ARG;
     if (!aligned(exclude_bits, 4)) return TT_ERR_INVALID_ARG;
     if (b == 0) return TT_OK;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (index->n > 0) {
-        if ((st = check_device_ptr(types, "types")) != TT_OK) return st;
-        if ((st = check_device_ptr(exclude_bits, "exclude_bits")) != TT_OK) return st;
-    }
-    const int64_t per_set = (int64_t)b * k;
-    const int64_t words = (index->n + 31) / 32;
-    uint32_t* mask = nullptr;
-    if (words > 0) TT_CUDA(cudaMallocAsync(reinterpret_cast<void**>(&mask), (size_t)words * 4, s), "type mask");
+    if (index->n > 0 && (st = check_device_ptr(types, "types")) != TT_OK) return st;
+    // type -> set; a type asked for twice is scored once and its lists copied
+    int8_t set_of[256];
+    memset(set_of, -1, sizeof set_of);
+    int distinct = 0;
+    int first_of[TT_MAX_PARTS];
     for (int t = 0; t < n_sets; ++t) {
-        if (mask) {
-            cudaError_t e = launch_mask_slice(exclude_bits, 0, index->n, types, set_types[t], mask, s);
-            if (e != cudaSuccess) {
-                cudaFreeAsync(mask, s);
-                return cuda_fail(e, "type mask");
-            }
-        }
-        st = score_rows(index, 0, index->n, queries, q_dtype, b, mask, tau, k, out_ids + t * per_set,
-                        out_scores + t * per_set, s);
-        if (st != TT_OK) break;
+        if (set_of[set_types[t]] < 0) set_of[set_types[t]] = (int8_t)distinct++;
+        first_of[t] = set_of[set_types[t]];
     }
-    if (mask) cudaFreeAsync(mask, s);
-    return st;
+    // the distinct sets' lists go to the front of the output, in first-seen order
+    st = score_core(index, queries, q_dtype, b, exclude_bits, tau, k, out_ids, out_scores, stream, nullptr,
+                    types, distinct, set_of);
+    if (st != TT_OK) return st;
+    // move each requested set to its place (from the back, so that no list is
+    // overwritten before it is read: set t's source is at index first_of[t] <= t)
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t per_set = (size_t)b * k;
+    for (int t = n_sets - 1; t >= 0; --t) {
+        if (first_of[t] == t) continue;
+        TT_CUDA(cudaMemcpyAsync(out_ids + t * per_set, out_ids + first_of[t] * per_set, per_set * 4,
+                                cudaMemcpyDeviceToDevice, s), "set copy");
+        TT_CUDA(cudaMemcpyAsync(out_scores + t * per_set, out_scores + first_of[t] * per_set, per_set * 4,
+                                cudaMemcpyDeviceToDevice, s), "set copy");
+    }
+    return TT_OK;
 }
 
 tt_status tt_score_topk(tt_index* index, const void* queries, tt_dtype q_dtype, int32_t b,

@@ -35,6 +35,14 @@ struct PassArgs {
     int* err;                  // device error word
     const float* qscale;       // [b] query scales of int8 rows, else null
     int withhold_copy;         // test hook (tensor-core pass): skip the first corpus copy
+    // Several result sets by candidate type, from one pass (null types: one
+    // set). Row j belongs to set s = set_of[types[j]] (-1: to none); its
+    // keys go to the virtual query v = s * b + q and must beat theta_v[v];
+    // count and keys are indexed by v. theta and thf then hold, per query,
+    // the minimum over the sets, for the kernels' first (fast) tests.
+    const uint8_t* types;      // [n] or null
+    const int8_t* set_of;      // [256]
+    const uint64_t* theta_v;   // [n_sets * b]
 };
 
 // Set the text tt_last_error() returns on the calling thread.
@@ -112,6 +120,10 @@ cudaError_t launch_softmax(const SoftmaxPlan& pl, const CUtensorMap& tm_users, c
                            int b, int nc, int d, float tau, const float* logq, const int64_t* item_ids,
                            const uint8_t* valid, float* lse, float* loss, float* mean, void* workspace,
                            cudaStream_t s, int sm_count);
+// Per query, the minimum over n_sets of the virtual thresholds (v = s * b + q):
+// theta_min[q], thf_min[q] for q < b; KEY_MAX / +inf for b <= q < b_pad.
+cudaError_t launch_sets_min(const uint64_t* theta_v, const float* thf_v, int n_sets, int b, int b_pad,
+                            uint64_t* theta_min, float* thf_min, cudaStream_t s);
 cudaError_t launch_offset_ids(int32_t* ids, int64_t count, int64_t offset, cudaStream_t s);
 
 // Shared-memory bytes the tensor-core pass needs for a given d and query tile.

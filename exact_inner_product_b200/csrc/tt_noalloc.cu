@@ -200,6 +200,9 @@ tt_status tt_score_topk_noalloc(const void* rows, tt_dtype dtype, int64_t n, int
         a.q_dtype = q_dt_use;
         a.qscale = nullptr;
         a.withhold_copy = 0;
+        a.types = nullptr;
+        a.set_of = nullptr;
+        a.theta_v = nullptr;
         a.b = b;
         a.theta = theta;
         a.thf = thf;

@@ -300,7 +300,11 @@ TT_API tt_status tt_score_topk_ranges(tt_index* index, const void* queries, tt_d
  *
  * Set s keeps only candidates j with types[j] == set_types[s] (and not
  * excluded by exclude_bits); the result is exactly tt_score_topk with that
- * combined mask. Each set is a separate pass over the corpus.
+ * combined mask. All sets come from the same passes over the corpus: every
+ * score is computed once, and a candidate that beats its query's loosest
+ * set threshold is kept in the list of its own type's set. A type asked for
+ * twice is scored once and its lists copied. The work buffers hold n_sets * b
+ * lists.
  *
  * types      device uint8 [n]: the type of every candidate
  * set_types  HOST int32 [n_sets], each 0..255

@@ -79,20 +79,25 @@ def test_ranges_against_oracle():
         assert set(sure.tolist()) <= set(got_i[q].tolist())
 
 
-def test_types_equal_masked_calls_and_oracle():
+@pytest.mark.parametrize("b,path", [(3, 1), (40, 2), (260, 3)])
+def test_types_equal_masked_calls_and_oracle(b, path):
+    """One fused pass for all the requested types (a type asked twice gets the
+    same lists twice), on each scorer."""
     _cuda()
-    w = W.workload("large_batch", n=90_001, b=260, k=80, mask_rate=0.1)
+    w = W.workload("large_batch", n=90_001, b=b, k=80, mask_rate=0.1)
     raw_c, raw_q = W.corpus(w, "cuda"), W.queries(w, "cuda")
     excl = W.exclusion_bits(w, "cuda")
     index, qn = parity.gpu_prepare(w, raw_c, raw_q)
     g = torch.Generator(device="cpu").manual_seed(31)
     types_np = torch.randint(0, 4, (w.n,), generator=g, dtype=torch.uint8).numpy()
     types = torch.from_numpy(types_np).cuda()
-    sets = [2, 0, 7]  # type 7 has no candidates: all padding
+    sets = [2, 0, 7, 2]  # type 7 has no candidates: all padding
     ids, scores = tt.tt_score_topk_types(index, qn, w.k, types, sets, exclude=excl)
+    assert tt.tt_last_stats(index)["path"] == path
     ex_all = _bits(excl, w.n)
     corpus = oracle.normalize(W.to_numpy_rows(raw_c), w.store)
     queries = oracle.normalize(raw_q.cpu().numpy()[:8], w.query_dtype)
+    nq_check = min(8, w.b)
     for t_i, t in enumerate(sets):
         combined = ex_all | (types_np != t)
         wi, ws = tt.tt_score_topk(index, qn, w.k, exclude=_mask_from_bool(combined))
@@ -101,9 +106,9 @@ def test_types_equal_masked_calls_and_oracle():
             assert (ids[t_i] == -1).all()
             continue
         oi, os_ = oracle.topk(queries, corpus, w.k, exclude=oracle_pins.pack_bits(combined))
-        got = ids[t_i, :8].cpu().numpy()
+        got = ids[t_i, :nq_check].cpu().numpy()
         assert (types_np[got[got >= 0]] == t).all()
-        for q in range(8):
+        for q in range(nq_check):
             sure = oi[q][os_[q] > os_[q][-1] + w.tolerance]
             assert set(sure.tolist()) <= set(got[q].tolist())
 
