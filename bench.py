@@ -66,15 +66,15 @@ TRAFFIC = {
     ("k1_normalize", "stream_b1"): {"bytes_per_row": 712.825, "src": "exact_inner_product_b200/csrc/k_normalize.cu",
                                     "sha": "4273a9f8869b74ec01b8762c20eb598dc6f0b1597fcd3e5f8ad9afde664127f4"},
     # ncu --set full -k regex:k3_pair -s 5 -c 1 on `python bench.py --workload large_batch --n 4000000
-    # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 1773.760 MB read
-    # + 27.450 MB written; scaled to the full corpus by rows scanned
-    ("k3_pair", "large_batch"): {"bytes_per_row": 450.303, "src": "exact_inner_product_b200/csrc/k_tensor_pair.cu",
-                                 "sha": "26cccee2055038f9327e3160f5bd52beaace8eafa31f85c3b78cdb0b3eaa44db"},
+    # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 1592.981 MB read
+    # + 28.070 MB written; scaled to the full corpus by rows scanned
+    ("k3_pair", "large_batch"): {"bytes_per_row": 405.263, "src": "exact_inner_product_b200/csrc/k_tensor_pair.cu",
+                                 "sha": "6f303eca084c883abd77d28ff639f8375a1558b5412efecc66fc5478f0e084eb"},
     # ncu --set full -k regex:k3_tensor -s 5 -c 1 on `python bench.py --workload masked_fused --n 4000000
-    # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 4599.171 MB read
-    # + 66.280 MB written; scaled to the full corpus by rows scanned
-    ("k3_tensor", "masked_fused"): {"bytes_per_row": 1166.363, "src": "exact_inner_product_b200/csrc/k_tensor.cu",
-                                    "sha": "1074ee60d7ac4f9dd8a45c54fb73ec1c8ab54218cc60b75d7307328d39225625"},
+    # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 4385.550 MB read
+    # + 66.286 MB written; scaled to the full corpus by rows scanned
+    ("k3_tensor", "masked_fused"): {"bytes_per_row": 1112.959, "src": "exact_inner_product_b200/csrc/k_tensor.cu",
+                                    "sha": "dcfd00e71e06c525df0eb6aac897f7ad09d53050bd7abde0b4238ef405fb3486"},
 }
 
 
