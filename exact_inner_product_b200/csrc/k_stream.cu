@@ -161,14 +161,18 @@ __global__ void __launch_bounds__(K2_THREADS)
                 if (rset < 0) row_ok = false;
             }
         }
+        if (a.types) {  // this row's set: its own threshold and buffer
+#pragma unroll
+            for (int qb = 0; qb < QB; ++qb) {
+                const uint64_t key = make_key(acc[qb] * c, (uint32_t)id);
+                append_set(a, q0 + qb, rset, row_ok && key > th[qb], key);
+            }
+            continue;
+        }
 #pragma unroll
         for (int qb = 0; qb < QB; ++qb) {
             const uint64_t key = make_key(acc[qb] * c, (uint32_t)id);
             const bool keep = row_ok && key > th[qb];
-            if (a.types) {  // this row's set: its own threshold and buffer
-                append_set(a, q0 + qb, rset, keep, key);
-                continue;
-            }
             const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, keep);
             if (ballot) {
                 const int q = q0 + qb;
