@@ -1093,6 +1093,8 @@ tt_status tt_score_topk_types(tt_index* index, const void* queries, tt_dtype q_d
     for (int t = 0; t < n_sets; ++t)
         if (set_types[t] < 0 || set_types[t] > 255) return TT_ERR_INVALID_ARG;
     if (!aligned(exclude_bits, 4)) return TT_ERR_INVALID_ARG;
+    // one list per (set, query): their number must stay a modest int
+    if ((int64_t)n_sets * b > TT_MAX_SET_LISTS) return TT_ERR_UNSUPPORTED;
     if (b == 0) return TT_OK;
     if (index->n > 0 && (st = check_device_ptr(types, "types")) != TT_OK) return st;
     // type -> set; a type asked for twice is scored once and its lists copied

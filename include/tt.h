@@ -67,7 +67,8 @@ typedef enum tt_norm_mode {
 /* Limits. */
 #define TT_MAX_D 512        /* d must be a multiple of 16 and at most 512 (f32 corpus: 256) */
 #define TT_MAX_K 2048       /* k at most 2048 */
-#define TT_MAX_PARTS 64     /* shards merged by one tt_merge_topk call */
+#define TT_MAX_PARTS 64     /* shards merged by one tt_merge_topk call; result sets of one call */
+#define TT_MAX_SET_LISTS (1 << 24) /* tt_score_topk_types: n_sets * b at most this */
 #define TT_MAX_N 2147483647 /* candidate ids are int32: n < 2^31 */
 
 /* Opaque handle describing a prepared corpus. Owned by the library; release
@@ -308,7 +309,7 @@ TT_API tt_status tt_score_topk_ranges(tt_index* index, const void* queries, tt_d
  *
  * types      device uint8 [n]: the type of every candidate
  * set_types  HOST int32 [n_sets], each 0..255
- * n_sets     1 <= n_sets <= TT_MAX_PARTS
+ * n_sets     1 <= n_sets <= TT_MAX_PARTS, and n_sets * b <= TT_MAX_SET_LISTS
  * out_ids, out_scores  device [n_sets, b, k]
  * other arguments, the exactness and the errors as tt_score_topk.
  */

@@ -158,6 +158,10 @@ def test_set_calls_validate_before_device_calls():
     assert types_call(None) == tt.TT_ERR_INVALID_ARG
     assert types_call((ctypes.c_int32 * 1)(256)) == tt.TT_ERR_INVALID_ARG
     assert types_call((ctypes.c_int32 * 1)(3), n=0) == tt.TT_ERR_INVALID_ARG
+    # too many (set, query) lists: refused before any device call
+    many = lib.tt_score_topk_types(ix, fake, 1, 1 << 20, None, 1.0, 5, None, 32, (ctypes.c_int32 * 32)(*range(32)),
+                                   fake, fake, None)
+    assert many == tt.TT_ERR_UNSUPPORTED
     lib.tt_free(ix)
 
 
