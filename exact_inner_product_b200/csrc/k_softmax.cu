@@ -20,7 +20,7 @@
 //   k5_columns      per column: bias nb_j = -log q_j * log2(e) (-inf for an
 //                   invalid column) and item group g_j (the table slot of its
 //                   id, so equal ids <=> equal groups); zero the error word
-//   k5_softmax      tcgen05 MMAs of 128 users x 256 candidates into TMEM;
+//   k5_softmax      tcgen05 MMAs of 128 users x 192 candidates into TMEM;
 //                   the epilogue turns each accumulator row into running
 //                   (max, sum of 2^(x - max)) pairs, x = acc * log2(e)/tau + nb_j,
 //                   so the exponentials never leave registers
@@ -97,7 +97,7 @@ struct K5Params {
     int b, nc;
     float a2;            // log2(e) / tau
     int u_tiles;         // ceil(b / 128)
-    int c_tiles;         // ceil(nc / 256)
+    int c_tiles;         // ceil(nc / K5_N)
     int chunks;          // column ranges (units = u_tiles * chunks)
     int kchunks;         // ceil(d / 64)
     int stages;
@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(K5_THREADS, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* usm = smem;                                              // [kchunks][128 x 128 B]
-    uint8_t* ring = smem + (size_t)p.kchunks * K5_USER_CHUNK;         // [stages][256 x 128 B]
+    uint8_t* ring = smem + (size_t)p.kchunks * K5_USER_CHUNK;         // [stages][K5_N x 128 B]
     K5Ctl* ctl = reinterpret_cast<K5Ctl*>(ring + (size_t)p.stages * K5_STAGE_BYTES);
 
     const int warp = threadIdx.x >> 5;
@@ -335,7 +335,7 @@ __global__ void __launch_bounds__(K5_THREADS, 1)
     } else {
         // ------------------------------ epilogue ------------------------------
         // Warp w reads TMEM lanes 32*(w%4).. (its 32 users) and one group of
-        // K5_WARP_COLS of the tile's 256 columns; each thread keeps (max, sum)
+        // K5_WARP_COLS of the tile's K5_N columns; each thread keeps (max, sum)
         // for its user.
         const int ew = warp - 2;
         const int quarter = warp & 3;
