@@ -79,6 +79,9 @@ _sig("tt_score_topk", ctypes.c_int, [_vp, _vp, ctypes.c_int, _i32, _vp, ctypes.c
 _sig("tt_score_topk_ex", ctypes.c_int, [_vp, _vp, ctypes.c_int, _i32, _vp, ctypes.c_float, _i32, _vp,
                                         _vp, _vp, ctypes.POINTER(tt_options)])
 _sig("tt_last_stats", ctypes.c_int, [_vp, ctypes.POINTER(tt_stats)])
+_sig("tt_index_check", ctypes.c_int, [_vp, _vp])
+_sig("tt_score_topk_host", ctypes.c_int, [_vp, _vp, ctypes.c_int, _i32, _i32, ctypes.c_int, _vp, ctypes.c_float,
+                                          _i32, _vp, _vp, _vp])
 _sig("tt_plan", ctypes.c_int, [_i64, _i32, ctypes.POINTER(tt_options), ctypes.POINTER(_i32),
                                ctypes.POINTER(_i64), ctypes.POINTER(_i64), ctypes.POINTER(_i32),
                                ctypes.POINTER(_i32)])
@@ -104,6 +107,7 @@ _sig("tt_last_error", ctypes.c_char_p, [])
 _sig("tt_version", ctypes.c_char_p, [])
 
 EXPORTED = ("tt_normalize_candidates", "tt_quantize_candidates", "tt_index_wrap", "tt_score_topk", "tt_score_topk_ex",
+            "tt_index_check", "tt_score_topk_host",
             "tt_score_topk_noalloc", "tt_merge_topk", "tt_score_topk_ranges", "tt_score_topk_types",
             "tt_inbatch_softmax_workspace", "tt_inbatch_softmax", "tt_inbatch_softmax_check",
             "tt_last_stats", "tt_plan", "tt_free", "tt_launch_count", "tt_profile_begin",
@@ -231,9 +235,10 @@ def tt_score_topk(index: Index, queries: torch.Tensor, k: int, tau: float = 1.0,
 
     ``queries``: [b, d] float32/bfloat16 on the GPU. ``exclude``: packed
     exclusion bits, int32 tensor of ceil(n/32) words (bit j&31 of word j>>5).
-    Returns ``(ids int32 [b,k], scores float32 [b,k])``. Keyword options
-    (``path``, ``rank_scale_pct``, ``force_levels``, ``cap``) go to
-    ``tt_score_topk_ex``."""
+    Returns ``(ids int32 [b,k], scores float32 [b,k])``, complete once the
+    stream reaches the call's work (the call itself does not wait; see
+    ``tt_index_check``). Keyword options (``path``, ``rank_scale_pct``,
+    ``force_levels``, ``cap``, ``withhold_copy``) go to ``tt_score_topk_ex``."""
     if queries.dim() != 2 or not queries.is_contiguous():
         raise ValueError("queries must be a contiguous [b, d] tensor")
     b, d = queries.shape
@@ -272,14 +277,63 @@ def tt_score_topk_noalloc(rows: torch.Tensor, queries: torch.Tensor, k: int, tau
         raise ValueError("rows and queries must be contiguous 2-D tensors")
     n, d = rows.shape
     b = queries.shape[0]
+    if queries.shape[1] != d:
+        raise ValueError(f"queries have d={queries.shape[1]}, rows have d={d}")
+    dev = queries.device
     if out_ids is None:
-        out_ids = torch.empty((b, k), dtype=torch.int32, device=queries.device)
+        out_ids = torch.empty((b, k), dtype=torch.int32, device=dev)
     if out_scores is None:
-        out_scores = torch.empty((b, k), dtype=torch.float32, device=queries.device)
+        out_scores = torch.empty((b, k), dtype=torch.float32, device=dev)
+    for name, t, dt in (("out_ids", out_ids, torch.int32), ("out_scores", out_scores, torch.float32)):
+        if t.dtype != dt or tuple(t.shape) != (b, k) or not t.is_contiguous() or t.device != dev:
+            raise ValueError(f"{name} must be a contiguous {dt} tensor of shape ({b}, {k}) on {dev}")
+    if exclude is not None and (exclude.dtype != torch.int32 or not exclude.is_contiguous()
+                                or exclude.numel() < (n + 31) // 32):
+        raise TypeError("exclude must be a contiguous int32 tensor of ceil(n/32) packed words")
+    if inv_norm is not None and (inv_norm.dtype != torch.float32 or not inv_norm.is_contiguous()
+                                 or inv_norm.numel() != n):
+        raise TypeError("inv_norm must be a contiguous float32 tensor of n elements")
     st = _lib.tt_score_topk_noalloc(_ptr(rows), _dtype(rows), n, d, _ptr(inv_norm), _ptr(queries),
                                     _dtype(queries), b, _ptr(exclude), float(tau), int(k), _ptr(out_ids),
                                     _ptr(out_scores), _stream(stream))
     _check(st, "tt_score_topk_noalloc")
+    return out_ids, out_scores
+
+
+def tt_index_check(index: Index, stream=None) -> None:
+    """Wait for the work enqueued on ``stream`` and raise ``TTError``
+    (TT_ERR_TIMEOUT) if a device-side wait of a search on this handle
+    expired (``tt_index_check``)."""
+    _check(_lib.tt_index_check(index.handle, _stream(stream)), "tt_index_check")
+
+
+def tt_score_topk_host(index: Index, queries: torch.Tensor, k: int, tau: float = 1.0,
+                       exclude: torch.Tensor | None = None, normalize: bool = True,
+                       norm_dtype=torch.bfloat16, out_ids: torch.Tensor | None = None,
+                       out_scores: torch.Tensor | None = None, stream=None):
+    """The search from host to host (``tt_score_topk_host``): ``queries`` is
+    a CPU [b, d] tensor (pinned memory copies faster), copied to the device,
+    L2-normalised there into ``norm_dtype`` when ``normalize``, scored against
+    the resident index; returns CPU ``(ids int32 [b, k], scores float32 [b, k])``
+    once they are there. ``exclude`` stays a device tensor."""
+    if queries.dim() != 2 or not queries.is_contiguous() or queries.is_cuda:
+        raise ValueError("queries must be a contiguous [b, d] CPU tensor")
+    b, d = queries.shape
+    if d != index.d:
+        raise ValueError(f"queries have d={d}, index has d={index.d}")
+    if out_ids is None:
+        out_ids = torch.empty((b, k), dtype=torch.int32, pin_memory=torch.cuda.is_available())
+    if out_scores is None:
+        out_scores = torch.empty((b, k), dtype=torch.float32, pin_memory=torch.cuda.is_available())
+    for name, t, dt in (("out_ids", out_ids, torch.int32), ("out_scores", out_scores, torch.float32)):
+        if t.dtype != dt or tuple(t.shape) != (b, k) or not t.is_contiguous() or t.is_cuda:
+            raise ValueError(f"{name} must be a contiguous CPU {dt} tensor of shape ({b}, {k})")
+    if exclude is not None and (exclude.dtype != torch.int32 or not exclude.is_contiguous() or not exclude.is_cuda):
+        raise TypeError("exclude must be a contiguous int32 CUDA tensor of packed bits")
+    norm_dt = TT_F32 if norm_dtype == torch.float32 else TT_BF16
+    _check(_lib.tt_score_topk_host(index.handle, _ptr(queries), _dtype(queries), b, 1 if normalize else 0,
+                                   norm_dt, _ptr(exclude), float(tau), int(k), _ptr(out_ids), _ptr(out_scores),
+                                   _stream(stream)), "tt_score_topk_host")
     return out_ids, out_scores
 
 
@@ -409,6 +463,8 @@ def tt_free(index: Index) -> None:
 
 
 def tt_last_stats(index: Index) -> dict:
+    """What the last search on the handle did; ``rescans`` (lists the exact
+    fallback recomputed) is -1 until that search's work has completed."""
     s = tt_stats()
     _check(_lib.tt_last_stats(index.handle, ctypes.byref(s)), "tt_last_stats")
     return {"path": s.path, "levels": s.levels, "rescans": s.rescans, "launches": s.launches,

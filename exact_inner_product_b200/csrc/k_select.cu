@@ -17,7 +17,8 @@
 // positions past the number of eligible candidates get (-1, -inf). The
 // result is exact when the pass kept every key above its threshold
 // (count <= cap) and either found at least k of them or had no threshold;
-// otherwise the query is flagged for a rescan with a corrected threshold.
+// otherwise the list is handed to the exact fallback scan (k_exact.cu),
+// which runs in the same stream right after, with no host involvement.
 // (Order: score descending, ties by ascending id - mhtirogla.ai Two-tower
 // retrieval, Code, Towers::top_k; padding replaces the bf16.min fill of
 // recsys_two_tower_model.py `mask_and_top_k`.)
@@ -26,182 +27,10 @@
 
 #include "tt_device.cuh"
 #include "tt_internal.h"
+#include "tt_select.cuh"
 
 namespace tt {
 namespace {
-
-constexpr int K4_THREADS = 256;
-constexpr int K4_SORT_MAX = 2048;  // >= TT_MAX_K
-constexpr int K4_BINS = 2048;
-constexpr int K4_SMEM_KEYS = 4096;  // kept keys copied to shared memory when they fit
-
-struct K4Smem {
-    uint32_t hist[K4_BINS];
-    uint32_t part[K4_THREADS];
-    uint32_t above[K4_THREADS];
-    uint64_t sorted[K4_SORT_MAX];
-    uint64_t found_prefix;
-    uint32_t found_remaining;
-    uint32_t found_count;
-    uint32_t n_collected;
-    uint64_t result;
-    uint64_t keys[K4_SMEM_KEYS];
-};
-
-// The query's kept keys: copied to shared memory when they fit, else read in place.
-__device__ const uint64_t* stage_keys(const uint64_t* __restrict__ g, int n, K4Smem& sm) {
-    if (n > K4_SMEM_KEYS) return g;
-    for (int i = threadIdx.x; i < n; i += K4_THREADS) sm.keys[i] = g[i];
-    __syncthreads();
-    return sm.keys;
-}
-
-// r-th largest (1-based, counting repeats) of n keys; 1 <= r <= n. Block-wide.
-// Radix passes narrow the candidates to a digit prefix; once at most
-// K4_THREADS keys share the prefix they are gathered and ranked directly.
-__device__ uint64_t block_kth_largest(const uint64_t* keys, int n, int r, K4Smem& sm) {
-    const int tid = threadIdx.x;
-    // digits, most significant first: widths 11, 11, 10, 11, 11, 10
-    uint64_t prefix = 0, mask = 0;
-    uint32_t remaining = (uint32_t)r;
-    int shift = 64;
-#pragma unroll 1
-    for (int pass = 0; pass < 6; ++pass) {
-        const int w = (pass == 2 || pass == 5) ? 10 : 11;
-        shift -= w;
-        const int nb = 1 << w;
-        for (int i = tid; i < nb; i += K4_THREADS) sm.hist[i] = 0;
-        __syncthreads();
-        for (int i = tid; i < n; i += K4_THREADS) {
-            const uint64_t key = keys[i];
-            if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & (uint64_t)(nb - 1)], 1u);
-        }
-        __syncthreads();
-        // Thread t owns bins [t*per, (t+1)*per); above[t] = count in higher bins.
-        const int per = nb / K4_THREADS;
-        uint32_t local = 0;
-        for (int i = 0; i < per; ++i) local += sm.hist[tid * per + i];
-        sm.part[tid] = local;
-        __syncthreads();
-        if (tid < 32) {
-            uint32_t s = 0;
-            for (int i = 0; i < 8; ++i) s += sm.part[tid * 8 + i];
-            // suffix sum over lanes: sum of lanes > tid
-            uint32_t incl = s;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const uint32_t v = __shfl_down_sync(0xFFFFFFFFu, incl, off);
-                if (tid + off < 32) incl += v;
-            }
-            uint32_t run = incl - s;  // lanes above this one
-            for (int i = 7; i >= 0; --i) {
-                sm.above[tid * 8 + i] = run;
-                run += sm.part[tid * 8 + i];
-            }
-        }
-        __syncthreads();
-        const uint32_t above = sm.above[tid];
-        if (above < remaining && remaining <= above + local) {
-            uint32_t run = above;
-            for (int i = per - 1; i >= 0; --i) {
-                const uint32_t c = sm.hist[tid * per + i];
-                if (remaining <= run + c) {
-                    sm.found_prefix = (uint64_t)(tid * per + i);
-                    sm.found_remaining = remaining - run;
-                    sm.found_count = c;
-                    break;
-                }
-                run += c;
-            }
-        }
-        __syncthreads();
-        prefix |= sm.found_prefix << shift;
-        mask |= (uint64_t)(nb - 1) << shift;
-        remaining = sm.found_remaining;
-        const uint32_t count = sm.found_count;
-        __syncthreads();
-        if (count <= (uint32_t)K4_THREADS) {
-            // gather the keys with this prefix and rank them by counting
-            if (tid == 0) sm.n_collected = 0;
-            __syncthreads();
-            for (int i = tid; i < n; i += K4_THREADS) {
-                const uint64_t key = keys[i];
-                if ((key & mask) == prefix) sm.sorted[atomicAdd(&sm.n_collected, 1u)] = key;
-            }
-            __syncthreads();
-            if (tid < (int)count) {
-                const uint64_t mine = sm.sorted[tid];
-                uint32_t above_me = 0, equal = 0;
-                for (uint32_t j = 0; j < count; ++j) {
-                    above_me += sm.sorted[j] > mine;
-                    equal += sm.sorted[j] == mine;
-                }
-                if (above_me < remaining && remaining <= above_me + equal) sm.result = mine;
-            }
-            __syncthreads();
-            return sm.result;
-        }
-    }
-    return prefix;
-}
-
-// The min(n, k) largest of n distinct keys, sorted descending, written as
-// (id, score); slots past n get (-1, -inf). Block-wide; out_* point at one
-// query's row of k entries.
-__device__ void write_sorted_topk(const uint64_t* keys, int n, int k, K4Smem& sm, int32_t* out_ids,
-                                  float* out_scores) {
-    const int tid = threadIdx.x;
-    const int r = n < k ? n : k;
-    if (r > 0) {
-        const uint64_t kth = block_kth_largest(keys, n, r, sm);
-        if (tid == 0) sm.n_collected = 0;
-        __syncthreads();
-        // fewer than r keys are above the r-th largest; the rest of the r
-        // slots hold it (one copy when keys are distinct)
-        for (int i = tid; i < n; i += K4_THREADS) {
-            const uint64_t key = keys[i];
-            if (key > kth) {
-                const uint32_t slot = atomicAdd(&sm.n_collected, 1u);
-                if (slot < (uint32_t)r) sm.sorted[slot] = key;
-            }
-        }
-        __syncthreads();
-        const int above = (int)sm.n_collected < r ? (int)sm.n_collected : r;
-        for (int i = above + tid; i < r; i += K4_THREADS) sm.sorted[i] = kth;
-        __syncthreads();
-        int P = 1;
-        while (P < r) P <<= 1;
-        for (int i = r + tid; i < P; i += K4_THREADS) sm.sorted[i] = KEY_MIN;
-        __syncthreads();
-        // bitonic sort, descending
-        for (int size = 2; size <= P; size <<= 1) {
-            for (int stride = size >> 1; stride > 0; stride >>= 1) {
-                for (int i = tid; i < P; i += K4_THREADS) {
-                    const int j = i ^ stride;
-                    if (j > i) {
-                        const uint64_t x = sm.sorted[i], y = sm.sorted[j];
-                        const bool desc = (i & size) == 0;
-                        if (desc ? (x < y) : (x > y)) {
-                            sm.sorted[i] = y;
-                            sm.sorted[j] = x;
-                        }
-                    }
-                }
-                __syncthreads();
-            }
-        }
-    }
-    for (int i = tid; i < k; i += K4_THREADS) {
-        int32_t id = -1;
-        float sc = -INFINITY;
-        if (i < r) {
-            id = (int32_t)key_id(sm.sorted[i]);
-            sc = key_score(sm.sorted[i]);
-        }
-        out_ids[i] = id;
-        out_scores[i] = sc;
-    }
-}
 
 // Merge of per-shard results: part p holds, for every query, its shard's
 // top-k_in as (local id, score); local ids plus id_offset[p] are global ids;
@@ -234,7 +63,7 @@ __global__ void __launch_bounds__(K4_THREADS)
     __syncthreads();
     const int n = (int)sm.n_collected;
     __syncthreads();
-    write_sorted_topk(keys, n, k_out, sm, out_ids + (int64_t)q * k_out, out_scores + (int64_t)q * k_out);
+    write_sorted_topk(keys, n, n, k_out, sm, out_ids + (int64_t)q * k_out, out_scores + (int64_t)q * k_out);
 }
 
 __global__ void __launch_bounds__(K4_THREADS)
@@ -258,32 +87,36 @@ __global__ void __launch_bounds__(K4_THREADS)
     }
 }
 
+// Final mode. A list whose pass kept everything above its threshold is
+// exact: its sorted top-k is written. Otherwise it is handed to the exact
+// fallback scan (k_exact.cu): its index goes to flagged[atomicAdd(flags[0])]
+// and theta[q] receives a valid lower bound on its true k-th best key (the
+// k-th best kept key minus one after an overflow, else KEY_MIN).
 __global__ void __launch_bounds__(K4_THREADS)
     k4_select_final(const uint64_t* __restrict__ keys, uint32_t* __restrict__ count, int cap, int k,
-                    uint64_t* __restrict__ theta, float* __restrict__ thf, int32_t* __restrict__ status,
-                    int* __restrict__ flags, int repair, int32_t* __restrict__ out_ids,
-                    float* __restrict__ out_scores) {
+                    uint64_t* __restrict__ theta, float* __restrict__ thf, int32_t* __restrict__ flagged,
+                    int* __restrict__ flags, int32_t* __restrict__ out_ids, float* __restrict__ out_scores) {
     extern __shared__ __align__(16) uint8_t k4_smem_raw[];
     K4Smem& sm = *reinterpret_cast<K4Smem*>(k4_smem_raw);
     const int q = blockIdx.x;
     const int tid = threadIdx.x;
-    if (repair && status[q] == 0) return;  // block-uniform
+    if (flags[1] != 0) return;  // a device wait expired earlier in this call: nothing is valid
     const uint32_t c = count[q];
     const int n = c < (uint32_t)cap ? (int)c : cap;
     const uint64_t th = theta[q];
     const uint64_t* qkeys = stage_keys(keys + (int64_t)q * cap, n, sm);
     const bool exact = (c <= (uint32_t)cap) && (c >= (uint32_t)k || th == KEY_MIN);
     if (exact) {
-        write_sorted_topk(qkeys, n, k, sm, out_ids + (int64_t)q * k, out_scores + (int64_t)q * k);
-        if (tid == 0) status[q] = 0;
+        write_sorted_topk(qkeys, n, n, k, sm, out_ids + (int64_t)q * k, out_scores + (int64_t)q * k);
     } else {
+        // After an overflow every key above th survived, and n >= k of them
+        // were kept: the k-th best kept key is at most the true k-th best.
         uint64_t th_new = KEY_MIN;
         if (c > (uint32_t)cap && n >= k) th_new = block_kth_largest(qkeys, n, k, sm) - 1;
         if (tid == 0) {
             theta[q] = th_new;
             thf[q] = key_floor(th_new);
-            status[q] = 1;
-            atomicOr(flags, 1);
+            flagged[atomicAdd(flags, 1)] = q;
         }
     }
     __syncthreads();
@@ -304,17 +137,6 @@ __global__ void k4_init(uint32_t* count, uint64_t* theta, float* thf, uint64_t t
         }
     }
     if (blockIdx.x == 0 && threadIdx.x < 2) flags[threadIdx.x] = 0;
-}
-
-__global__ void k4_prepare_repair(uint64_t* theta, float* thf, const int32_t* status, int b, int* flags) {
-    const float fmax = key_floor(KEY_MAX);
-    for (int q = blockIdx.x * blockDim.x + threadIdx.x; q < b; q += gridDim.x * blockDim.x) {
-        if (status[q] == 0) {
-            theta[q] = KEY_MAX;
-            thf[q] = fmax;
-        }
-    }
-    if (blockIdx.x == 0 && threadIdx.x == 0) flags[0] = 0;
 }
 
 __global__ void k4_pad(int32_t* out_ids, float* out_scores, int64_t count) {
@@ -385,14 +207,14 @@ cudaError_t launch_select_threshold(const uint64_t* keys, uint32_t* count, int c
 }
 
 cudaError_t launch_select_final(const uint64_t* keys, uint32_t* count, int cap, int b, int k,
-                                uint64_t* theta, float* thf, int32_t* status, int* flags,
-                                int repair, int32_t* out_ids, float* out_scores, cudaStream_t s) {
+                                uint64_t* theta, float* thf, int32_t* flagged, int* flags,
+                                int32_t* out_ids, float* out_scores, cudaStream_t s) {
     if (b == 0) return cudaSuccess;
     const int smem = (int)sizeof(K4Smem);
     cudaFuncSetAttribute(k4_select_final, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     note_launch_begin(TT_KIND_SELECT, s);
-    k4_select_final<<<b, K4_THREADS, smem, s>>>(keys, count, cap, k, theta, thf, status, flags, repair,
-                                                out_ids, out_scores);
+    k4_select_final<<<b, K4_THREADS, smem, s>>>(keys, count, cap, k, theta, thf, flagged, flags, out_ids,
+                                                out_scores);
     note_launch_end(TT_KIND_SELECT, s);
     return cudaGetLastError();
 }
@@ -414,14 +236,6 @@ cudaError_t launch_merge(const int32_t* ids, const float* scores, int parts, int
 }
 
 int merge_smem_keys() { return K4_SMEM_KEYS; }
-
-cudaError_t launch_prepare_repair(uint64_t* theta, float* thf, const int32_t* status, int b,
-                                  int* flags, cudaStream_t s) {
-    note_launch_begin(TT_KIND_AUX, s);
-    k4_prepare_repair<<<small_grid(b), 256, 0, s>>>(theta, thf, status, b, flags);
-    note_launch_end(TT_KIND_AUX, s);
-    return cudaGetLastError();
-}
 
 cudaError_t launch_mask_slice(const uint32_t* in, int64_t start, int64_t count, const uint8_t* types, int want,
                               uint32_t* out, cudaStream_t s) {

@@ -60,6 +60,7 @@ struct K3Ctl {
     uint64_t drain;
     uint32_t tmem_base;
     int abort;
+    int skip;
     // per epilogue warp: fast-path thresholds and exact threshold keys of its
     // columns for the current unit (int8 rows: and the query scales)
     alignas(16) float th_fast[K3_EPI_WARPS][K3_WARP_COLS];  // read as float4
@@ -105,6 +106,13 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int n_units = p.q_tiles * p.chunks;
+
+    // A bounded wait of an earlier pass of this search expired: nothing that
+    // follows is valid, so skip the work (decided once for the whole CTA,
+    // before any barrier or tensor memory is set up).
+    if (threadIdx.x == 0) ctl->skip = *reinterpret_cast<volatile int*>(p.a.err);
+    __syncthreads();
+    if (ctl->skip) return;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {

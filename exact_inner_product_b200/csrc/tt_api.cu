@@ -11,8 +11,10 @@
 // keep every key (no threshold). A query's final pass is exact when it kept
 // at least k keys (so every member of the true top-k beat the threshold) and
 // its buffer did not overflow; if either fails - which the estimate makes
-// rare but never impossible - the query is rescanned with a threshold that
-// is correct by construction (the k-th best kept key, or none).
+// rare but never impossible - the query's list is recomputed by the exact
+// fallback scan (k_exact.cu), launched at the end of every search, which has
+// no capacity limit. The whole search is enqueued on the caller's stream and
+// the call returns without waiting: the host never reads a result.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -22,13 +24,14 @@
 
 #include <atomic>
 #include <mutex>
+#include <new>
 #include <vector>
 
 #include "../../include/tt.h"
 #include "tt_device.cuh"
 #include "tt_internal.h"
 
-#define TT_VERSION_STRING "tt 0.1.0 (sm_100a)"
+#define TT_VERSION_STRING "tt 0.2.0 (sm_100a)"
 
 struct tt_index {
     const void* rows;
@@ -37,10 +40,18 @@ struct tt_index {
     int32_t d;
     const float* inv_norm;
     int device;
-    // scratch (device), grown on demand
+    // work memory (device), grown on demand, and the stream it was last used on
     void* scratch;
     size_t scratch_bytes;
-    int* h_flags;  // pinned, 2 ints: [0] rescan needed, [1] device error code
+    void* io;  // staging of tt_score_topk_host: queries in, results out
+    size_t io_bytes;
+    cudaStream_t last_stream;
+    bool used;
+    // status block in host-mapped memory, written by the last kernel of a search
+    tt::HostStatus* hstat;
+    tt::HostStatus* dstat;  // the same block, as the device addresses it
+    int64_t seq;            // calls issued on the handle
+    int64_t last_pending;   // seq of the last search whose status block reports it (0: none)
     tt_stats last;
 };
 
@@ -238,7 +249,6 @@ constexpr int MAX_DEEPEST_ROWS = 4096;  // the deepest level keeps every key
 constexpr int MIN_RANK = 32;
 constexpr int MIN_RANK_DEEP = 10;
 constexpr int MAX_LEVELS = 4;
-constexpr int MAX_RESCANS = 64;
 // Batches at least this large, on a corpus stored normalised, go to the
 // tensor-core kernel on SM pairs (queries in tiles of 256 on TMEM lanes);
 // the rest to the single-SM kernel (queries in tiles of up to 256 on TMEM
@@ -310,8 +320,8 @@ struct Scratch {
     uint32_t* count;
     uint64_t* theta;
     float* thf;
-    int32_t* status;
-    int* flags;
+    int32_t* flagged;  // lists handed to the exact fallback
+    int* flags;        // [0] flagged lists, [1] error word of expired device waits
     __nv_bfloat16* qcast;
     int8_t* qcodes;   // int8 index: the queries' codes [b, d]
     float* qscale;    // and their scales [b]
@@ -324,69 +334,150 @@ struct Scratch {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Scratch blocks released by tt_free are kept here (per device) and handed
-// to later handles, so that short-lived handles do not cudaMalloc/cudaFree on
-// every call (cudaFree waits for the whole device). Blocks stay with the
-// process until it exits.
+// Work blocks released by a handle (tt_free, or growth) are kept here, per
+// device, and handed to later handles, so that short-lived handles do not
+// cudaMalloc/cudaFree on every call (cudaFree waits for the whole device).
+// Work still queued on the stream that last used a block may read it, so a
+// block carries an event recorded on that stream, and a later user's stream
+// waits for it before any of its own work touches the block. Blocks stay with
+// the process until it exits.
 struct PooledBlock {
     int device;
     void* ptr;
     size_t bytes;
+    cudaEvent_t ready;  // null: nothing queued used it
 };
 static std::mutex g_pool_mu;
 static std::vector<PooledBlock> g_pool;
 
-static void* pool_take(int device, size_t need, size_t* got) {
-    std::lock_guard<std::mutex> lock(g_pool_mu);
-    int best = -1;
-    for (int i = 0; i < (int)g_pool.size(); ++i)
-        if (g_pool[i].device == device && g_pool[i].bytes >= need &&
-            (best < 0 || g_pool[i].bytes < g_pool[best].bytes))
-            best = i;
-    if (best < 0) return nullptr;
-    void* p = g_pool[best].ptr;
-    *got = g_pool[best].bytes;
-    g_pool.erase(g_pool.begin() + best);
-    return p;
-}
-
-static void pool_give(int device, void* ptr, size_t bytes) {
-    if (!ptr) return;
-    std::lock_guard<std::mutex> lock(g_pool_mu);
-    g_pool.push_back({device, ptr, bytes});
-}
-
-// Pinned host words for reading back the exactness flags, reused the same way.
-static std::vector<int*> g_pinned_pool;
-
-static int* pinned_take() {
+static void* pool_take(int device, size_t need, size_t* got, cudaStream_t s) {
+    PooledBlock blk{};
     {
         std::lock_guard<std::mutex> lock(g_pool_mu);
-        if (!g_pinned_pool.empty()) {
-            int* p = g_pinned_pool.back();
-            g_pinned_pool.pop_back();
-            return p;
+        int best = -1;
+        for (int i = 0; i < (int)g_pool.size(); ++i)
+            if (g_pool[i].device == device && g_pool[i].bytes >= need &&
+                (best < 0 || g_pool[i].bytes < g_pool[best].bytes))
+                best = i;
+        if (best < 0) return nullptr;
+        blk = g_pool[best];
+        g_pool.erase(g_pool.begin() + best);
+    }
+    if (blk.ready) {
+        cudaStreamWaitEvent(s, blk.ready, 0);
+        cudaEventDestroy(blk.ready);
+    }
+    *got = blk.bytes;
+    return blk.ptr;
+}
+
+static void pool_give(int device, void* ptr, size_t bytes, cudaStream_t last, bool used) {
+    if (!ptr) return;
+    cudaEvent_t ev = nullptr;
+    if (used && cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) == cudaSuccess) {
+        if (cudaEventRecord(ev, last) != cudaSuccess) {
+            cudaGetLastError();
+            cudaEventDestroy(ev);
+            ev = nullptr;
+            cudaStreamSynchronize(last);  // no event: make sure nothing queued still reads the block
+            cudaGetLastError();
         }
     }
-    int* p = nullptr;
-    if (cudaMallocHost(&p, 2 * sizeof(int)) != cudaSuccess) {
+    std::lock_guard<std::mutex> lock(g_pool_mu);
+    g_pool.push_back({device, ptr, bytes, ev});
+}
+
+// A block of at least `need` bytes for *slot (a handle's scratch or io),
+// replacing the current one when it is too small.
+static tt_status grow_block(tt_index* ix, void** slot, size_t* slot_bytes, size_t need, cudaStream_t s,
+                            const char* what) {
+    if (need <= *slot_bytes) return TT_OK;
+    if (*slot) {
+        pool_give(ix->device, *slot, *slot_bytes, ix->last_stream, ix->used);
+        *slot = nullptr;
+        *slot_bytes = 0;
+    }
+    size_t got = 0;
+    void* p = pool_take(ix->device, need, &got, s);
+    if (!p) {
+        got = need + need / 4;
+        cudaError_t e = cudaMalloc(&p, got);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return cuda_fail(e, what);
+        }
+    }
+    *slot = p;
+    *slot_bytes = got;
+    return TT_OK;
+}
+
+// Status blocks (host-mapped, one per handle), reused the same way; a block
+// is handed out again only once the work that may still write it is done.
+struct PooledStatus {
+    HostStatus* p;
+    cudaEvent_t done;  // null: nothing queued writes it
+};
+static std::vector<PooledStatus> g_status_pool;
+
+static HostStatus* status_take() {
+    {
+        std::lock_guard<std::mutex> lock(g_pool_mu);
+        for (size_t i = 0; i < g_status_pool.size(); ++i) {
+            PooledStatus ps = g_status_pool[i];
+            if (ps.done) {
+                if (cudaEventQuery(ps.done) != cudaSuccess) {
+                    cudaGetLastError();
+                    continue;
+                }
+                cudaEventDestroy(ps.done);
+            }
+            g_status_pool.erase(g_status_pool.begin() + (long)i);
+            return ps.p;
+        }
+    }
+    void* p = nullptr;
+    if (cudaHostAlloc(&p, 64, cudaHostAllocMapped) != cudaSuccess) {
         cudaGetLastError();
         return nullptr;
     }
-    return p;
+    return static_cast<HostStatus*>(p);
 }
 
-static void pinned_give(int* p) {
+static void status_give(HostStatus* p, cudaStream_t last = nullptr, bool used = false) {
     if (!p) return;
+    cudaEvent_t ev = nullptr;
+    if (used && cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) == cudaSuccess &&
+        cudaEventRecord(ev, last) != cudaSuccess) {
+        cudaGetLastError();
+        cudaEventDestroy(ev);
+        ev = nullptr;
+        cudaStreamSynchronize(last);
+        cudaGetLastError();
+    }
     std::lock_guard<std::mutex> lock(g_pool_mu);
-    g_pinned_pool.push_back(p);
+    g_status_pool.push_back({p, ev});
+}
+
+// A device wait of an earlier search on this handle expired (its outputs were
+// set to id -1, score NaN): report it once, as TT_ERR_TIMEOUT.
+static tt_status report_pending(tt_index* ix) {
+    if (ix->hstat && ix->hstat->err != 0) {
+        const int code = ix->hstat->err;
+        ix->hstat->err = 0;
+        snprintf(g_last_error, sizeof g_last_error,
+                 "a device-side wait expired in a search on this handle (code %d); that search's outputs "
+                 "hold id -1 and score NaN", code);
+        return TT_ERR_TIMEOUT;
+    }
+    return TT_OK;
 }
 
 // b, b_pad: queries (with the padding of the query tiles); vq, vpad: the
 // lists kept (vq = b, or sets * b for several result sets, padded to vpad);
 // n_min: entries of the per-query minima (0 without result sets).
 static tt_status get_scratch(tt_index* ix, int b, int b_pad, int vq, int vpad, int n_min, int cap, int d,
-                             bool need_qcast, bool need_q8, Scratch* out) {
+                             bool need_qcast, bool need_q8, cudaStream_t s, Scratch* out) {
     size_t off = 0;
     const size_t o_keys = off;
     off = align_up(off + (size_t)vq * cap * 8, 256);
@@ -396,7 +487,7 @@ static tt_status get_scratch(tt_index* ix, int b, int b_pad, int vq, int vpad, i
     off = align_up(off + (size_t)vpad * 8, 256);
     const size_t o_thf = off;
     off = align_up(off + (size_t)vpad * 4, 256);
-    const size_t o_status = off;
+    const size_t o_flagged = off;
     off = align_up(off + (size_t)vpad * 4, 256);
     const size_t o_tmin = off;
     off = align_up(off + (size_t)n_min * 8, 256);
@@ -412,32 +503,14 @@ static tt_status get_scratch(tt_index* ix, int b, int b_pad, int vq, int vpad, i
     off = align_up(off + (need_q8 ? (size_t)b * d : 0), 256);
     const size_t o_qs = off;
     off = align_up(off + (need_q8 ? (size_t)b_pad * 4 : 0), 256);
-    if (off > ix->scratch_bytes) {
-        if (ix->scratch) {
-            // the old block may still be read by work queued on the stream
-            pool_give(ix->device, ix->scratch, ix->scratch_bytes);
-            ix->scratch = nullptr;
-            ix->scratch_bytes = 0;
-        }
-        size_t got = 0;
-        void* p = pool_take(ix->device, off, &got);
-        if (!p) {
-            got = off + off / 4;
-            cudaError_t e = cudaMalloc(&p, got);
-            if (e != cudaSuccess) {
-                cudaGetLastError();
-                return cuda_fail(e, "scratch allocation");
-            }
-        }
-        ix->scratch = p;
-        ix->scratch_bytes = got;
-    }
+    tt_status st = grow_block(ix, &ix->scratch, &ix->scratch_bytes, off, s, "scratch allocation");
+    if (st != TT_OK) return st;
     uint8_t* base = static_cast<uint8_t*>(ix->scratch);
     out->keys = reinterpret_cast<uint64_t*>(base + o_keys);
     out->count = reinterpret_cast<uint32_t*>(base + o_count);
     out->theta = reinterpret_cast<uint64_t*>(base + o_theta);
     out->thf = reinterpret_cast<float*>(base + o_thf);
-    out->status = reinterpret_cast<int32_t*>(base + o_status);
+    out->flagged = reinterpret_cast<int32_t*>(base + o_flagged);
     out->flags = reinterpret_cast<int*>(base + o_flags);
     out->qcast = need_qcast ? reinterpret_cast<__nv_bfloat16*>(base + o_q) : nullptr;
     out->qcodes = need_q8 ? reinterpret_cast<int8_t*>(base + o_q8) : nullptr;
@@ -445,12 +518,20 @@ static tt_status get_scratch(tt_index* ix, int b, int b_pad, int vq, int vpad, i
     out->theta_min = n_min > 0 ? reinterpret_cast<uint64_t*>(base + o_tmin) : nullptr;
     out->thf_min = n_min > 0 ? reinterpret_cast<float*>(base + o_fmin) : nullptr;
     out->set_of = n_min > 0 ? reinterpret_cast<int8_t*>(base + o_setof) : nullptr;
-    if (!ix->h_flags) {
-        ix->h_flags = pinned_take();
-        if (!ix->h_flags) {
-            snprintf(g_last_error, sizeof g_last_error, "pinned flag allocation failed");
+    if (!ix->hstat) {
+        ix->hstat = status_take();
+        void* dp = nullptr;
+        if (!ix->hstat || cudaHostGetDevicePointer(&dp, (void*)ix->hstat, 0) != cudaSuccess) {
+            cudaGetLastError();
+            status_give(ix->hstat);
+            ix->hstat = nullptr;
+            snprintf(g_last_error, sizeof g_last_error, "mapped status block allocation failed");
             return TT_ERR_NO_MEMORY;
         }
+        ix->dstat = static_cast<HostStatus*>(dp);
+        ix->hstat->err = 0;
+        ix->hstat->repaired = 0;
+        ix->hstat->seq = 0;
     }
     return TT_OK;
 }
@@ -708,15 +789,25 @@ tt_status tt_index_wrap(const void* rows, tt_dtype dtype, int64_t n, int32_t d,
 
 void tt_free(tt_index* index) {
     if (!index) return;
-    pool_give(index->device, index->scratch, index->scratch_bytes);
-    pinned_give(index->h_flags);
+    pool_give(index->device, index->scratch, index->scratch_bytes, index->last_stream, index->used);
+    pool_give(index->device, index->io, index->io_bytes, index->last_stream, index->used);
+    status_give(index->hstat, index->last_stream, index->used);
     delete index;
 }
 
 tt_status tt_last_stats(const tt_index* index, tt_stats* out) {
     if (!index || !out) return TT_ERR_INVALID_ARG;
     *out = index->last;
+    if (index->last_pending != 0)  // known once the call's last kernel has run
+        out->rescans = (index->hstat && index->hstat->seq == index->last_pending) ? index->hstat->repaired : -1;
     return TT_OK;
+}
+
+tt_status tt_index_check(tt_index* index, void* stream) {
+    if (!index) return TT_ERR_INVALID_ARG;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+    return report_pending(index);
 }
 
 // The whole search. With `types`, one pass serves n_sets result sets: set t
@@ -774,6 +865,7 @@ static tt_status score_core(tt_index* index, const void* queries, tt_dtype q_dty
                  index->device, dev);
         return TT_ERR_INVALID_ARG;
     }
+    if ((st = report_pending(index)) != TT_OK) return st;  // an earlier search's expired wait
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int64_t launches0 = g_launches.load();
     tt_stats stats;
@@ -791,6 +883,7 @@ static tt_status score_core(tt_index* index, const void* queries, tt_dtype q_dty
         if (e != cudaSuccess) return cuda_fail(e, "pad");
         stats.launches = (int)(g_launches.load() - launches0);
         index->last = stats;
+        index->last_pending = 0;
         return TT_OK;
     }
 
@@ -809,9 +902,12 @@ static tt_status score_core(tt_index* index, const void* queries, tt_dtype q_dty
     const bool need_qcast = !i8 && path >= 2 && q_dtype == TT_F32;
     Scratch sc;
     const int v_pad = types ? V + 64 : b_pad;
-    if ((st = get_scratch(index, b, b_pad, V, v_pad, types ? b_pad : 0, plan.cap, index->d, need_qcast, i8, &sc)) !=
-        TT_OK)
+    if ((st = get_scratch(index, b, b_pad, V, v_pad, types ? b_pad : 0, plan.cap, index->d, need_qcast, i8, s,
+                          &sc)) != TT_OK)
         return st;
+    index->last_stream = s;
+    index->used = true;
+    const int64_t seq = ++index->seq;
     const int sms = sm_count_current();
     const float inv_tau = 1.0f / tau;
 
@@ -860,42 +956,47 @@ static tt_status score_core(tt_index* index, const void* queries, tt_dtype q_dty
                                         sc.thf, s);
             if (e == cudaSuccess) e = sets_min();
         } else {
-            e = launch_select_final(sc.keys, sc.count, plan.cap, V, k, sc.theta, sc.thf, sc.status,
-                                    sc.flags, 0, out_ids, out_scores, s);
+            e = launch_select_final(sc.keys, sc.count, plan.cap, V, k, sc.theta, sc.thf, sc.flagged,
+                                    sc.flags, out_ids, out_scores, s);
         }
         if (e != cudaSuccess) return cuda_fail(e, "select");
     }
-    int rescans = 0;
-    while (true) {
-        TT_CUDA(cudaMemcpyAsync(index->h_flags, sc.flags, 2 * sizeof(int), cudaMemcpyDeviceToHost, s),
-                "flag readback");
-        TT_CUDA(cudaStreamSynchronize(s), "stream synchronize");
-        if (index->h_flags[1] != 0) {
-            snprintf(g_last_error, sizeof g_last_error, "device wait expired (code %d)",
-                     index->h_flags[1]);
-            stats.rescans = rescans;
-            stats.launches = (int)(g_launches.load() - launches0);
-            index->last = stats;
-            return TT_ERR_TIMEOUT;
-        }
-        if (index->h_flags[0] == 0) break;
-        if (rescans >= MAX_RESCANS) {
-            snprintf(g_last_error, sizeof g_last_error, "exactness check not met after %d rescans",
-                     rescans);
-            return TT_ERR_INTERNAL;
-        }
-        e = launch_prepare_repair(sc.theta, sc.thf, sc.status, V, sc.flags, s);
-        if (e == cudaSuccess) e = sets_min();
-        if (e != cudaSuccess) return cuda_fail(e, "prepare rescan");
-        if ((st = run_pass(index, pc, plan, 0, sc, exclude_bits, inv_tau, b, s, sms)) != TT_OK) return st;
-        e = launch_select_final(sc.keys, sc.count, plan.cap, V, k, sc.theta, sc.thf, sc.status,
-                                sc.flags, 1, out_ids, out_scores, s);
-        if (e != cudaSuccess) return cuda_fail(e, "select");
-        ++rescans;
-    }
-    stats.rescans = rescans;
+    // Lists the final select could not prove exact are recomputed on the
+    // device, in the same stream; with none, every block returns at once.
+    ExactArgs ea;
+    memset(&ea, 0, sizeof ea);
+    ea.rows = index->rows;
+    ea.dtype = index->dtype;
+    ea.n = index->n;
+    ea.d = index->d;
+    ea.inv_norm = index->inv_norm;
+    ea.exclude = exclude_bits;
+    ea.inv_tau = inv_tau;
+    ea.queries = pc.queries;
+    ea.q_dtype = pc.q_dtype;
+    ea.qscale = pc.qscale;
+    ea.b = b;
+    ea.V = V;
+    ea.types = types;
+    ea.set_of = types ? sc.set_of : nullptr;
+    ea.keys = sc.keys;
+    ea.cap = plan.cap;
+    ea.k = k;
+    ea.theta = sc.theta;
+    ea.done = sc.count;
+    ea.flagged = sc.flagged;
+    ea.flags = sc.flags;
+    ea.out_ids = out_ids;
+    ea.out_scores = out_scores;
+    ea.status = index->dstat;
+    ea.seq = seq;
+    ea.chunks = exact_chunks(index->n, k, plan.cap);
+    e = launch_exact(ea, s, sms);
+    if (e != cudaSuccess) return cuda_fail(e, "exact fallback");
+    stats.rescans = -1;  // known once the work has run (tt_last_stats)
     stats.launches = (int)(g_launches.load() - launches0);
     index->last = stats;
+    index->last_pending = seq;
     return TT_OK;
 }
 
@@ -1024,13 +1125,17 @@ static tt_status score_rows(tt_index* index, int64_t start, int64_t count, const
                             int32_t b, const uint32_t* mask, float tau, int32_t k, int32_t* out_ids,
                             float* out_scores, cudaStream_t s) {
     const int esize = index->dtype == TT_F32 ? 4 : index->dtype == TT_BF16 ? 2 : 1;
-    tt_index* sub = nullptr;
-    tt_status st = new_index(static_cast<const uint8_t*>(index->rows) + start * index->d * esize, index->dtype,
-                             count, index->d, index->inv_norm ? index->inv_norm + start : nullptr, &sub);
-    if (st != TT_OK) return st;
-    st = tt_score_topk_ex(sub, queries, q_dtype, b, mask, tau, k, out_ids, out_scores, s, nullptr);
-    index->last = sub->last;
-    tt_free(sub);  // the call above synchronised its stream: the scratch is idle
+    // a view of the rows that borrows the handle's work memory and status block
+    tt_index sub = *index;
+    sub.rows = static_cast<const uint8_t*>(index->rows) + start * index->d * esize;
+    sub.n = count;
+    sub.inv_norm = index->inv_norm ? index->inv_norm + start : nullptr;
+    tt_status st = tt_score_topk_ex(&sub, queries, q_dtype, b, mask, tau, k, out_ids, out_scores, s, nullptr);
+    tt_index keep = *index;  // the handle keeps its own view of the corpus
+    *index = sub;
+    index->rows = keep.rows;
+    index->n = keep.n;
+    index->inv_norm = keep.inv_norm;
     if (st != TT_OK) return st;
     cudaError_t e = launch_offset_ids(out_ids, (int64_t)b * k, start, s);
     if (e != cudaSuccess) return cuda_fail(e, "id offset");
@@ -1129,6 +1234,72 @@ tt_status tt_score_topk(tt_index* index, const void* queries, tt_dtype q_dtype, 
                         float* out_scores, void* stream) {
     return tt_score_topk_ex(index, queries, q_dtype, b, exclude_bits, tau, k, out_ids, out_scores,
                             stream, nullptr);
+}
+
+// Host memory of the process (pageable or pinned), never device memory.
+static bool host_memory(const void* p) {
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();
+        return true;  // not known to CUDA: ordinary pageable memory
+    }
+    return attr.type == cudaMemoryTypeUnregistered || attr.type == cudaMemoryTypeHost;
+}
+
+tt_status tt_score_topk_host(tt_index* index, const void* host_queries, tt_dtype q_dtype, int32_t b,
+                             int32_t normalize, tt_dtype norm_dtype, const uint32_t* exclude_bits, float tau,
+                             int32_t k, int32_t* host_ids, float* host_scores, void* stream) {
+    // ---------------- host-side validation ----------------
+    if (!index || b < 0 || k <= 0) return TT_ERR_INVALID_ARG;
+    if (k > TT_MAX_K) return TT_ERR_UNSUPPORTED;
+    if (!valid_dtype(q_dtype)) return TT_ERR_INVALID_ARG;
+    if (normalize && !valid_dtype(norm_dtype)) return TT_ERR_INVALID_ARG;
+    if (!(tau > 0.0f) || !isfinite(tau)) return TT_ERR_INVALID_ARG;
+    if (b > 0 && (host_queries == nullptr || host_ids == nullptr || host_scores == nullptr))
+        return TT_ERR_INVALID_ARG;
+    if (b == 0) return TT_OK;
+    if (!host_memory(host_queries) || !host_memory(host_ids) || !host_memory(host_scores)) {
+        snprintf(g_last_error, sizeof g_last_error, "tt_score_topk_host takes host buffers");
+        return TT_ERR_INVALID_ARG;
+    }
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev != index->device) {
+        snprintf(g_last_error, sizeof g_last_error, "index was made on device %d, current is %d",
+                 index->device, dev);
+        return TT_ERR_INVALID_ARG;
+    }
+    tt_status st = report_pending(index);
+    if (st != TT_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int d = index->d;
+    const size_t q_bytes = (size_t)b * d * (q_dtype == TT_F32 ? 4 : 2);
+    const size_t n_bytes = normalize ? (size_t)b * d * (norm_dtype == TT_F32 ? 4 : 2) : 0;
+    const size_t o_bytes = (size_t)b * k * 4;
+    const size_t o_q = 0, o_n = align_up(q_bytes, 256), o_ids = align_up(o_n + n_bytes, 256),
+                 o_sc = align_up(o_ids + o_bytes, 256), total = align_up(o_sc + o_bytes, 256);
+    if ((st = grow_block(index, &index->io, &index->io_bytes, total, s, "host staging allocation")) != TT_OK)
+        return st;
+    uint8_t* io = static_cast<uint8_t*>(index->io);
+    TT_CUDA(cudaMemcpyAsync(io + o_q, host_queries, q_bytes, cudaMemcpyHostToDevice, s), "queries to device");
+    const void* q_dev = io + o_q;
+    tt_dtype q_dt = q_dtype;
+    if (normalize) {
+        // the model normalises the user vector before retrieval (RecsysTwoTowerModel.__call__)
+        cudaError_t e = launch_normalize(io + o_q, q_dtype, b, d, io + o_n, norm_dtype, TT_NORM_STORE, s);
+        if (e != cudaSuccess) return cuda_fail(e, "query normalize");
+        q_dev = io + o_n;
+        q_dt = norm_dtype;
+    }
+    int32_t* d_ids = reinterpret_cast<int32_t*>(io + o_ids);
+    float* d_scores = reinterpret_cast<float*>(io + o_sc);
+    st = score_core(index, q_dev, q_dt, b, exclude_bits, tau, k, d_ids, d_scores, stream, nullptr, nullptr, 0,
+                    nullptr);
+    if (st != TT_OK) return st;
+    TT_CUDA(cudaMemcpyAsync(host_ids, d_ids, o_bytes, cudaMemcpyDeviceToHost, s), "ids to host");
+    TT_CUDA(cudaMemcpyAsync(host_scores, d_scores, o_bytes, cudaMemcpyDeviceToHost, s), "scores to host");
+    TT_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+    return report_pending(index);  // this search's own expired wait, if any
 }
 
 }  // extern "C"

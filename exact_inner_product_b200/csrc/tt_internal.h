@@ -76,13 +76,56 @@ cudaError_t launch_init(uint32_t* count, uint64_t* theta, float* thf, uint64_t t
 // fewer than r keys were kept; counts reset to 0.
 cudaError_t launch_select_threshold(const uint64_t* keys, uint32_t* count, int cap, int b, int r,
                                     uint64_t* theta_next, float* thf_next, cudaStream_t s);
-// Final mode: writes the sorted top-k (ids, scores) of queries whose pass was
-// exact; otherwise marks status[q] = 1, sets flags[0] and leaves the next
-// threshold in theta[q]. In a repair round (repair != 0) queries whose
-// status is 0 are skipped.
+// Final mode: writes the sorted top-k (ids, scores) of lists whose pass was
+// exact; any other list goes to flagged[atomicAdd(flags[0], 1)], with a valid
+// lower bound on its k-th best key left in theta, for the exact fallback.
+// Skips everything when flags[1] (a device wait expired) is set.
 cudaError_t launch_select_final(const uint64_t* keys, uint32_t* count, int cap, int b, int k,
-                                uint64_t* theta, float* thf, int32_t* status, int* flags,
-                                int repair, int32_t* out_ids, float* out_scores, cudaStream_t s);
+                                uint64_t* theta, float* thf, int32_t* flagged, int* flags,
+                                int32_t* out_ids, float* out_scores, cudaStream_t s);
+
+// Written by the device at the end of every search (host-mapped memory of an
+// index handle): the error code of an expired device wait (only written when
+// there is one; the host clears it once reported), the number of lists the
+// exact fallback recomputed, and the sequence number of the call.
+struct HostStatus {
+    volatile int32_t err;
+    volatile int32_t repaired;
+    volatile int64_t seq;
+};
+
+// The exact fallback scan (k_exact.cu), launched at the end of every search.
+struct ExactArgs {
+    const void* rows;          // corpus [n, d] (row stride d)
+    int dtype;                 // TT_F32 / TT_BF16 / TT_I8
+    int64_t n;
+    int d;
+    const float* inv_norm;     // [n] or null (int8: the per-row scales)
+    const uint32_t* exclude;   // [ceil(n/32)] or null
+    float inv_tau;
+    const void* queries;       // [b, d] as the main passes read them (int8: codes)
+    int q_dtype;
+    const float* qscale;       // int8: query scales [b]
+    int b;                     // queries
+    int V;                     // lists (b, or sets * b)
+    const uint8_t* types;      // several result sets by type, else null
+    const int8_t* set_of;
+    uint64_t* keys;            // [V * cap] work keys
+    int cap;
+    int k;
+    const uint64_t* theta;     // [V] lower bounds left by the final select
+    uint32_t* done;            // [V] chunk counters, zero on entry
+    const int32_t* flagged;    // lists to recompute (flags[0] of them)
+    const int* flags;          // [0] flagged lists, [1] error word
+    int32_t* out_ids;          // [V, k]
+    float* out_scores;
+    HostStatus* status;        // device view of the handle's status block, or null
+    int64_t seq;
+    int chunks;                // corpus chunks per list (exact_chunks)
+};
+int exact_chunks(int64_t n, int k, int cap);
+cudaError_t launch_exact(const ExactArgs& a, cudaStream_t s, int sm_count);
+
 // Merge per-shard top-k lists (see k4_merge); id_offset_host: host array of
 // `parts` global-id offsets; scratch: b * parts * k_in keys when parts * k_in
 // exceeds merge_smem_keys(), else unused (may be null).
@@ -90,10 +133,6 @@ cudaError_t launch_merge(const int32_t* ids, const float* scores, int parts, int
                          const int64_t* id_offset_host, int k_out, uint64_t* scratch, int32_t* out_ids,
                          float* out_scores, cudaStream_t s);
 int merge_smem_keys();
-// Before a repair round: theta[q] = KEY_MAX where status[q] == 0; flags[0] = 0.
-cudaError_t launch_prepare_repair(uint64_t* theta, float* thf, const int32_t* status, int b,
-                                  int* flags, cudaStream_t s);
-
 // Tensor maps (built on the host through the driver entry point).
 // Tensor-core pass: bf16 boxes of 64 elements x box_rows rows, 128-byte swizzle.
 bool bf16_tile_tensor_map(const void* base, int64_t rows, int d, int64_t row_pitch_elems,

@@ -21,7 +21,11 @@
 //   - the array keeps whatever the last call left in it; every call first
 //     resets the counters and thresholds it relies on;
 //   - the first call on each GPU looks up the array's device address (with
-//     that GPU current); make that first call before any stream capture.
+//     that GPU current); make that first call before any stream capture;
+//   - like tt_score_topk the call only enqueues its work on the stream and
+//     returns; it has no handle to report a device-side timeout through, so
+//     a search whose bounded wait expired leaves id -1 and score NaN in every
+//     output entry.
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -130,8 +134,8 @@ tt_status tt_score_topk_noalloc(const void* rows, tt_dtype dtype, int64_t n, int
     const size_t o_count = up256(o_keys + (size_t)b * cap * 8);
     const size_t o_theta = up256(o_count + (size_t)b_pad * 4);
     const size_t o_thf = up256(o_theta + (size_t)b_pad * 8);
-    const size_t o_status = up256(o_thf + (size_t)b_pad * 4);
-    const size_t o_flags = up256(o_status + (size_t)b_pad * 4);
+    const size_t o_flagged = up256(o_thf + (size_t)b_pad * 4);
+    const size_t o_flags = up256(o_flagged + (size_t)b_pad * 4);
     const size_t o_q = up256(o_flags + 64);
     const size_t total = up256(o_q + (need_qcast ? (size_t)b * d * 2 : 0));
     if (total > (size_t)TT_NOALLOC_SCRATCH_BYTES) {
@@ -147,7 +151,11 @@ tt_status tt_score_topk_noalloc(const void* rows, tt_dtype dtype, int64_t n, int
 
     // ---- device ----
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return TT_ERR_CUDA;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        noalloc_error("tt_score_topk_noalloc: no current CUDA device");
+        return TT_ERR_CUDA;
+    }
     if (!on_device(rows, dev) || !on_device(inv_norm, dev) || !on_device(queries, dev) ||
         !on_device(exclude_bits, dev) || !on_device(out_ids, dev) || !on_device(out_scores, dev)) {
         noalloc_error("tt_score_topk_noalloc: every pointer must be device memory of the current GPU");
@@ -160,14 +168,20 @@ tt_status tt_score_topk_noalloc(const void* rows, tt_dtype dtype, int64_t n, int
     uint32_t* count = reinterpret_cast<uint32_t*>(base + o_count);
     uint64_t* theta = reinterpret_cast<uint64_t*>(base + o_theta);
     float* thf = reinterpret_cast<float*>(base + o_thf);
-    int32_t* status = reinterpret_cast<int32_t*>(base + o_status);
+    int32_t* flagged = reinterpret_cast<int32_t*>(base + o_flagged);
     int* flags = reinterpret_cast<int*>(base + o_flags);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
+    auto launch_failed = [](const char* what, cudaError_t err) {
+        char msg[200];
+        snprintf(msg, sizeof msg, "tt_score_topk_noalloc %s: %s", what, cudaGetErrorString(err));
+        noalloc_error(msg);
+        return TT_ERR_CUDA;
+    };
 
     if (n == 0) {
         e = launch_pad(out_ids, out_scores, (int64_t)b * k, s);
-        return e == cudaSuccess ? TT_OK : TT_ERR_CUDA;
+        return e == cudaSuccess ? TT_OK : launch_failed("padding", e);
     }
     int sms = 148;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -180,14 +194,18 @@ tt_status tt_score_topk_noalloc(const void* rows, tt_dtype dtype, int64_t n, int
         if (need_qcast) {
             __nv_bfloat16* qc = reinterpret_cast<__nv_bfloat16*>(base + o_q);
             e = launch_cast_bf16(static_cast<const float*>(queries), (int64_t)b * d, qc, s);
-            if (e != cudaSuccess) return TT_ERR_CUDA;
+            if (e != cudaSuccess) return launch_failed("query cast", e);
             q_use = qc;
             q_dt_use = TT_BF16;
         }
-        if (!bf16_tile_tensor_map(q_use, b, d, d, nq, &tm_q)) return TT_ERR_CUDA;
+        if (!bf16_tile_tensor_map(q_use, b, d, d, nq, &tm_q)) {
+            noalloc_error("tt_score_topk_noalloc: query tensor map could not be encoded");
+            return TT_ERR_CUDA;
+        }
     }
     auto pass = [&](int lv) -> cudaError_t {
         PassArgs a;
+        memset(&a, 0, sizeof a);
         a.rows = rows;
         a.dtype = dtype;
         a.n_rows = lrows[lv];
@@ -198,11 +216,6 @@ tt_status tt_score_topk_noalloc(const void* rows, tt_dtype dtype, int64_t n, int
         a.inv_tau = inv_tau;
         a.queries = q_use;
         a.q_dtype = q_dt_use;
-        a.qscale = nullptr;
-        a.withhold_copy = 0;
-        a.types = nullptr;
-        a.set_of = nullptr;
-        a.theta_v = nullptr;
         a.b = b;
         a.theta = theta;
         a.thf = thf;
@@ -219,35 +232,46 @@ tt_status tt_score_topk_noalloc(const void* rows, tt_dtype dtype, int64_t n, int
         return launch_stream_pass(a, s, sms);
     };
 
-    // the array holds the previous call's leftovers: reset counters, thresholds, flags
+    // The array holds the previous call's leftovers: counters, thresholds and
+    // flags are reset first, in the stream, before anything reads them.
     e = launch_init(count, theta, thf, KEY_MIN, b, b_pad, flags, s);
-    for (int lv = levels - 1; lv >= 0 && e == cudaSuccess; --lv) {
+    if (e != cudaSuccess) return launch_failed("init", e);
+    for (int lv = levels - 1; lv >= 0; --lv) {
         e = pass(lv);
-        if (e != cudaSuccess) break;
+        if (e != cudaSuccess) return launch_failed("scoring pass", e);
         e = lv > 0 ? launch_select_threshold(keys, count, cap, b, ranks[lv], theta, thf, s)
-                   : launch_select_final(keys, count, cap, b, k, theta, thf, status, flags, 0,
-                                         out_ids, out_scores, s);
+                   : launch_select_final(keys, count, cap, b, k, theta, thf, flagged, flags, out_ids,
+                                         out_scores, s);
+        if (e != cudaSuccess) return launch_failed("select", e);
     }
-    if (e != cudaSuccess) {
-        char msg[160];
-        snprintf(msg, sizeof msg, "tt_score_topk_noalloc launch: %s", cudaGetErrorString(e));
-        noalloc_error(msg);
-        return TT_ERR_CUDA;
-    }
-    for (int rescans = 0;; ++rescans) {
-        int h[2] = {0, 0};
-        if (cudaStreamSynchronize(s) != cudaSuccess) return TT_ERR_CUDA;
-        if (cudaMemcpy(h, flags, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess) return TT_ERR_CUDA;
-        if (h[1] != 0) return TT_ERR_TIMEOUT;
-        if (h[0] == 0) return TT_OK;
-        if (rescans >= 64) return TT_ERR_INTERNAL;
-        e = launch_prepare_repair(theta, thf, status, b, flags, s);
-        if (e == cudaSuccess) e = pass(0);
-        if (e == cudaSuccess)
-            e = launch_select_final(keys, count, cap, b, k, theta, thf, status, flags, 1, out_ids,
-                                    out_scores, s);
-        if (e != cudaSuccess) return TT_ERR_CUDA;
-    }
+    // lists the final select could not prove exact are recomputed on the device
+    ExactArgs ea;
+    memset(&ea, 0, sizeof ea);
+    ea.rows = rows;
+    ea.dtype = dtype;
+    ea.n = n;
+    ea.d = d;
+    ea.inv_norm = inv_norm;
+    ea.exclude = exclude_bits;
+    ea.inv_tau = inv_tau;
+    ea.queries = q_use;
+    ea.q_dtype = q_dt_use;
+    ea.b = b;
+    ea.V = b;
+    ea.keys = keys;
+    ea.cap = cap;
+    ea.k = k;
+    ea.theta = theta;
+    ea.done = count;
+    ea.flagged = flagged;
+    ea.flags = flags;
+    ea.out_ids = out_ids;
+    ea.out_scores = out_scores;
+    ea.status = nullptr;  // no handle: an expired device wait shows as NaN scores
+    ea.chunks = exact_chunks(n, k, cap);
+    e = launch_exact(ea, s, sms);
+    if (e != cudaSuccess) return launch_failed("exact fallback", e);
+    return TT_OK;
 }
 
 }  // extern "C"

@@ -17,7 +17,8 @@
  *   - Data pointers are DEVICE pointers (cudaMalloc'd or torch CUDA tensors)
  *     owned by the caller, 16-byte aligned, rows contiguous (row-major
  *     [rows, d], row stride d elements). Host pointers are rejected with
- *     TT_ERR_INVALID_ARG.
+ *     TT_ERR_INVALID_ARG (except by tt_score_topk_host, which takes host
+ *     buffers for the queries and results).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream). Work is enqueued on it in order.
  *   - Arguments are validated on the host before any device work; a rejected
@@ -48,7 +49,7 @@ typedef enum tt_status {
     TT_ERR_CUDA = 3,        /* a CUDA call failed; tt_last_error() has the message */
     TT_ERR_NO_MEMORY = 4,   /* device or pinned-host allocation failed */
     TT_ERR_TIMEOUT = 5,     /* a bounded device-side wait expired; outputs are not valid */
-    TT_ERR_INTERNAL = 6     /* the exactness check could not be satisfied (not expected) */
+    TT_ERR_INTERNAL = 6     /* reserved (not returned: the exact fallback has no failure mode) */
 } tt_status;
 
 typedef enum tt_dtype {
@@ -164,8 +165,10 @@ TT_API tt_status tt_index_wrap(const void* rows, tt_dtype dtype, int64_t n, int3
  *  local_top_k with k_actual = min(k, N); TwoTower.score divides by tau.)
  *
  * The result is exact: the kernels keep fp32 scores and select by a total
- * order on (score, id), and the call verifies on the device that no
- * candidate of the true top-k was filtered out, rescanning when needed.
+ * order on (score, id). The filtered passes are checked on the device; a
+ * list they cannot prove exact is recomputed, still on the device and in the
+ * same stream, by an exact scan with no capacity limit (launched at the end
+ * of every search; it returns at once when nothing needs it).
  *
  * index        handle from tt_normalize_candidates or tt_index_wrap
  * queries      device [b, d], q_dtype. Queries are used as given (normalise
@@ -182,9 +185,15 @@ TT_API tt_status tt_index_wrap(const void* rows, tt_dtype dtype, int64_t n, int3
  * out_scores   device [b, k] f32
  * stream       cudaStream_t
  *
- * The call returns once the results are complete on `stream` (it
- * synchronises with the stream to read the device-side exactness check).
- * TT_ERR_TIMEOUT: a device-side wait gave up; outputs undefined.
+ * Asynchronous: TT_OK means the arguments were valid and the whole search
+ * is enqueued on `stream`; the outputs are complete when the stream reaches
+ * that point. The host never waits for the device here. Calls on one handle
+ * must be issued on one stream (or ordered by the caller), because they
+ * share the handle's work memory.
+ * Device-side timeouts: if a bounded wait of the search expires (a correct
+ * run never does), every entry of its outputs becomes (id -1, score NaN), and
+ * the next call on the handle, or tt_index_check, returns TT_ERR_TIMEOUT
+ * (once, without enqueueing anything).
  */
 TT_API tt_status tt_score_topk(tt_index* index, const void* queries, tt_dtype q_dtype, int32_t b,
                         const uint32_t* exclude_bits, float tau, int32_t k, int32_t* out_ids,
@@ -215,7 +224,8 @@ TT_API tt_status tt_score_topk_ex(tt_index* index, const void* queries, tt_dtype
 typedef struct tt_stats {
     int32_t path;            /* 1 streaming, 2 tensor core, 3 tensor core on SM pairs */
     int32_t levels;          /* scoring passes in the plan (1 = single pass) */
-    int32_t rescans;         /* extra full passes made to restore exactness */
+    int32_t rescans;         /* lists the exact fallback recomputed; -1 while the
+                                search's work has not completed yet */
     int32_t launches;        /* kernels launched by the call */
     int64_t level_rows[4];   /* rows scanned per level, finest first */
     int64_t level_stride[4]; /* corpus-row stride per level */
@@ -224,6 +234,36 @@ typedef struct tt_stats {
 } tt_stats;
 
 TT_API tt_status tt_last_stats(const tt_index* index, tt_stats* out);
+
+/*
+ * tt_index_check - wait for the work enqueued on `stream` and report whether
+ * a device-side wait of a search on this handle expired (TT_ERR_TIMEOUT,
+ * reported once; that search's outputs hold id -1 and score NaN) or not
+ * (TT_OK). TT_ERR_CUDA if the stream itself failed.
+ */
+TT_API tt_status tt_index_check(tt_index* index, void* stream);
+
+/*
+ * tt_score_topk_host - the search from host buffers to host buffers: copies
+ * the b x d queries to the device, optionally L2-normalises them there
+ * (normalize != 0, into norm_dtype, as the model normalises the user vector in
+ * RecsysTwoTowerModel.__call__), runs tt_score_topk against the index resident
+ * in device memory, and copies (ids, scores) back. Synchronous: it returns
+ * once host_ids and host_scores hold the result.
+ *
+ * host_queries  HOST [b, d] q_dtype (pinned memory makes the copy faster;
+ *               pageable memory works)
+ * normalize     0: score the queries as given; else normalise them first
+ * norm_dtype    TT_F32 or TT_BF16: the dtype the normalised queries are kept in
+ * exclude_bits  DEVICE mask words as in tt_score_topk, or NULL
+ * host_ids      HOST [b, k] int32; host_scores HOST [b, k] f32
+ * The device staging buffers belong to the handle (grown on demand).
+ * Errors as tt_score_topk; TT_ERR_TIMEOUT when this search's own device
+ * wait expired.
+ */
+TT_API tt_status tt_score_topk_host(tt_index* index, const void* host_queries, tt_dtype q_dtype, int32_t b,
+                                    int32_t normalize, tt_dtype norm_dtype, const uint32_t* exclude_bits,
+                                    float tau, int32_t k, int32_t* host_ids, float* host_scores, void* stream);
 
 /*
  * tt_plan - the scan plan tt_score_topk would use for a corpus of n rows and
@@ -284,8 +324,8 @@ TT_API tt_status tt_merge_topk(const int32_t* ids, const float* scores, int32_t 
  * ranges    HOST int64 [n_ranges * 2]: 0 <= start <= end <= n
  * n_ranges  1 <= n_ranges <= TT_MAX_PARTS
  * out_ids, out_scores  device [n_ranges, b, k]
- * other arguments, the exactness and the errors as tt_score_topk; the call
- * returns once the results are complete on `stream`.
+ * other arguments, the exactness, the errors and the asynchronous
+ * completion as tt_score_topk.
  */
 TT_API tt_status tt_score_topk_ranges(tt_index* index, const void* queries, tt_dtype q_dtype, int32_t b,
                                       const uint32_t* exclude_bits, float tau, int32_t k, int32_t n_ranges,
@@ -311,7 +351,8 @@ TT_API tt_status tt_score_topk_ranges(tt_index* index, const void* queries, tt_d
  * set_types  HOST int32 [n_sets], each 0..255
  * n_sets     1 <= n_sets <= TT_MAX_PARTS, and n_sets * b <= TT_MAX_SET_LISTS
  * out_ids, out_scores  device [n_sets, b, k]
- * other arguments, the exactness and the errors as tt_score_topk.
+ * other arguments, the exactness, the errors and the asynchronous
+ * completion as tt_score_topk.
  */
 TT_API tt_status tt_score_topk_types(tt_index* index, const void* queries, tt_dtype q_dtype, int32_t b,
                                      const uint32_t* exclude_bits, float tau, int32_t k, const uint8_t* types,
@@ -368,10 +409,10 @@ TT_API tt_status tt_inbatch_softmax(const void* users, const void* items, tt_dty
  * and report TT_OK or TT_ERR_TIMEOUT. */
 TT_API tt_status tt_inbatch_softmax_check(const void* workspace, void* stream);
 
-/* Release a handle. Its scratch memory returns to a per-device pool that
- * later handles reuse (it is not returned to CUDA before the process exits).
- * NULL is a no-op. Must not be called while work using the handle is still
- * running on a stream. */
+/* Release a handle. Its work memory returns to a per-device pool that later
+ * handles reuse (it is not returned to CUDA before the process exits); a
+ * later user's stream first waits for the work this handle had enqueued, so
+ * tt_free may be called while that work is still running. NULL is a no-op. */
 TT_API void tt_free(tt_index* index);
 
 /*
@@ -386,12 +427,11 @@ TT_API void tt_free(tt_index* index);
  * index handle and grows them with cudaMalloc; this entry point calls no
  * allocator at all (no cudaMalloc, cudaFree, pinned host memory or handle):
  * its work buffers are one fixed array of TT_NOALLOC_SCRATCH_BYTES that the
- * library declares in device memory, reserved on every GPU where the library
- * is loaded until the process exits.
+ * library declares in device memory.
  *
  * Arguments: the corpus directly (rows: device [n, d] dtype; inv_norm:
- * device [n] f32 for a raw corpus, else NULL), then as tt_score_topk. Result
- * and exactness as tt_score_topk.
+ * device [n] f32 for a raw corpus, else NULL), then as tt_score_topk. Result,
+ * exactness and asynchronous completion as tt_score_topk.
  *
  * Limits and rules:
  *   - b is limited by the array: about 128 KiB of work memory per query, so
@@ -402,8 +442,15 @@ TT_API void tt_free(tt_index* index);
  *     results, so callers must serialise them;
  *   - the array keeps the previous call's contents; each call resets what it
  *     relies on before use;
- *   - the first call on each GPU looks up the array's device address with
- *     that GPU current; make this first call before any stream capture.
+ *   - when the array's memory is taken: CUDA loads a module's device memory
+ *     when it is first used (lazy module loading, the default since CUDA
+ *     12.2), so the 32 MiB of a GPU are committed by the first call on that
+ *     GPU, which looks up the array's address with that GPU current; from then
+ *     on it stays reserved until the process exits. Make one warm-up call per
+ *     GPU at start-up, before any stream capture; later calls allocate nothing;
+ *   - there is no handle to report a device-side timeout through: a search
+ *     whose bounded wait expired leaves id -1 and score NaN in every output
+ *     entry.
  */
 #define TT_NOALLOC_SCRATCH_BYTES (32 * 1024 * 1024)
 

@@ -203,7 +203,8 @@ def test_edge_cases():
                                   {"rank_scale_pct": 3, "path": 3}, {"cap": 256, "path": 3}])
 def test_rescans_stay_exact(opts):
     """Thresholds deliberately mis-estimated (tiny ranks, tiny buffers): the
-    exactness check must trigger rescans and the answer must not change."""
+    on-device exactness check must hand the lists to the exact fallback scan,
+    and the answer must still match the oracle."""
     _cuda()
     k = 60 if "cap" in opts else 200
     w = W.workload("small_batch", n=200_003, b=24, k=k)
@@ -235,22 +236,95 @@ def test_repeat_runs_are_bitwise_identical():
 
 def test_bounded_wait_expiry_is_reported():
     """The tensor-core pass is told (test hook) to withhold its first corpus
-    copy: the wait for it gives up after its time limit, every role of the
-    kernel drains and exits, and the call reports TT_ERR_TIMEOUT. The device
-    and the handle stay usable: the next call gives the earlier answer."""
+    copy: the wait for it gives up after its time limit and every role of the
+    kernel drains and exits. The search was only enqueued (the call returned
+    TT_OK); its outputs become (id -1, score NaN), and the expiry is reported
+    once, as TT_ERR_TIMEOUT, by tt_index_check or else by the next call on the
+    handle. The device and the handle stay usable: the next search gives the
+    earlier answer."""
     import time
     _cuda()
     w = W.workload("small_batch", n=100_003, b=40, k=50)
     raw_c, raw_q = W.corpus(w, "cuda"), W.queries(w, "cuda")
     index, qn = parity.gpu_prepare(w, raw_c, raw_q)
-    good = tt.tt_score_topk(index, qn, w.k, path=2)
+    good = [t.clone() for t in tt.tt_score_topk(index, qn, w.k, path=2)]
+    torch.cuda.synchronize()
     t0 = time.time()
+    bad_ids, bad_scores = tt.tt_score_topk(index, qn, w.k, path=2, force_levels=1, withhold_copy=1)
     with pytest.raises(tt.TTError) as e:
-        tt.tt_score_topk(index, qn, w.k, path=2, force_levels=1, withhold_copy=1)
+        tt.tt_index_check(index)
     assert e.value.status == tt.TT_ERR_TIMEOUT
     assert time.time() - t0 < 60
+    assert (bad_ids == -1).all() and torch.isnan(bad_scores).all()
+    tt.tt_index_check(index)  # reported once
     again = tt.tt_score_topk(index, qn, w.k, path=2)
+    torch.cuda.synchronize()
     assert torch.equal(good[0], again[0]) and torch.equal(good[1], again[1])
+    # unchecked: the next call reports it, without enqueueing anything
+    tt.tt_score_topk(index, qn, w.k, path=2, force_levels=1, withhold_copy=1)
+    torch.cuda.synchronize()
+    with pytest.raises(tt.TTError) as e:
+        tt.tt_score_topk(index, qn, w.k, path=2)
+    assert e.value.status == tt.TT_ERR_TIMEOUT
+    again = tt.tt_score_topk(index, qn, w.k, path=2)
+    tt.tt_index_check(index)
+    assert torch.equal(good[0], again[0]) and torch.equal(good[1], again[1])
+
+
+def test_search_is_asynchronous():
+    """tt_score_topk only enqueues: two searches issued back to back return
+    before the stream has finished the first, and both results are right."""
+    import time
+    _cuda()
+    n, d, k = 8_000_000, 128, 100
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    rows = torch.randn(n, d, device="cuda", generator=g).to(torch.bfloat16)
+    q = torch.randn(1024, d, device="cuda", generator=g).to(torch.bfloat16)
+    index = tt.tt_index_wrap(rows)
+    ref = [t.clone() for t in tt.tt_score_topk(index, q, k)]  # warm-up: grows the work memory
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    t0 = time.perf_counter()
+    first = tt.tt_score_topk(index, q, k)
+    second = tt.tt_score_topk(index, q[:512].contiguous(), k)
+    t_calls = time.perf_counter() - t0
+    pending = not stream.query()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    tt.tt_score_topk(index, q, k)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    assert pending, "the calls waited for their own work"
+    assert t_calls * 1e3 < 2 * e0.elapsed_time(e1), (t_calls, e0.elapsed_time(e1))
+    assert torch.equal(first[0], ref[0]) and torch.equal(first[1], ref[1])
+    assert torch.equal(second[0], ref[0][:512]) and torch.equal(second[1], ref[1][:512])
+    tt.tt_index_check(index)
+
+
+def test_host_buffer_entry_point():
+    """tt_score_topk_host (host queries in, host results out, queries
+    normalised on the device) equals the device-buffer call."""
+    _cuda()
+    w = W.workload("small_batch", n=200_003, b=40, k=100)
+    raw_c, raw_q = W.corpus(w, "cuda"), W.queries(w, "cuda")
+    index, qn = parity.gpu_prepare(w, raw_c, raw_q)
+    ids, scores = tt.tt_score_topk(index, qn, w.k, tau=w.tau)
+    torch.cuda.synchronize()
+    hid, hsc = tt.tt_score_topk_host(index, raw_q.cpu().pin_memory(), w.k, tau=w.tau, normalize=True,
+                                     norm_dtype=torch.bfloat16)
+    assert not hid.is_cuda
+    assert torch.equal(hid, ids.cpu()) and torch.equal(hsc, scores.cpu())
+    # pageable memory, queries already normalised
+    hid, hsc = tt.tt_score_topk_host(index, qn.cpu(), w.k, tau=w.tau, normalize=False)
+    assert torch.equal(hid, ids.cpu()) and torch.equal(hsc, scores.cpu())
+    # the streaming scorer with an fp32 query
+    w1 = W.workload("stream_b1", n=150_001)
+    raw_c, raw_q = W.corpus(w1, "cuda"), W.queries(w1, "cuda")
+    index, qn = parity.gpu_prepare(w1, raw_c, raw_q)
+    ids, scores = tt.tt_score_topk(index, qn, w1.k)
+    hid, hsc = tt.tt_score_topk_host(index, raw_q.cpu(), w1.k, normalize=True, norm_dtype=torch.float32)
+    assert torch.equal(hid, ids.cpu()) and torch.equal(hsc, scores.cpu())
 
 
 def test_rejects_host_pointers_and_bad_args():

@@ -1,8 +1,11 @@
 """Corpus sharding on one GPU: the corpus is split into row shards, each shard
-is scored as its own index, and tt_merge_topk combines the lists. The result
-must equal the single-corpus call bit for bit (ids and scores), on every
-scorer path, with masks, per-row norms, k larger than a shard and lists too
-long for the merge's shared-memory staging. (GPU)"""
+is scored as its own index, and tt_merge_topk combines the lists. The merged
+result is checked against the fp64 oracle's top-k of the whole corpus (the
+comparison rule of the parity tests), and must also equal the single-corpus
+call bit for bit (ids and scores), on every scorer path, with masks, per-row
+norms, k larger than a shard and lists too long for the merge's
+shared-memory staging. (GPU)"""
+import numpy as np
 import pytest
 import torch
 
@@ -50,6 +53,12 @@ def test_sharded_equals_single(name, over, parts):
     want_ids, want_scores = tt.tt_score_topk(index, qn, w.k, tau=w.tau, exclude=excl)
     path = tt.tt_last_stats(index)["path"]
     got_ids, got_scores = _shard_and_merge(index, qn, w.k, w.tau, excl, parts)
+    # the merged lists against the oracle's top-k of the whole corpus
+    qids = W.oracle_query_ids(w)
+    side = parity.OracleSide(w, W.to_numpy_rows(raw_c), raw_q.cpu().numpy(),
+                             None if excl is None else excl.cpu().numpy().view(np.uint32), qids)
+    res = parity.compare(got_ids.cpu().numpy()[qids], got_scores.cpu().numpy()[qids], side, w.k, w.tolerance)
+    assert res["max_abs_err"] <= w.tolerance and res.get("sure_checked", 0) > 0, res
     assert torch.equal(got_ids, want_ids), name
     assert torch.equal(got_scores, want_scores), name
     if name == "masked_fused":  # the SM-pair kernel too, forced on every shard and on the whole

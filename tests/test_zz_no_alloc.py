@@ -4,10 +4,12 @@ pool reserved the GPU at start-up, where a late cudaMalloc would fail or
 stall the device). It works in a fixed array the library reserves on each
 GPU instead of buffers grown with cudaMalloc.
 
-The test calls it through the C ABI, twice in a row on the same inputs (the
-array keeps the first call's leftovers, which the second call must not see),
-and checks both results against the regular tt_score_topk within the score
-tolerance of the other parity tests. It sits in a file of its own that
+The test calls it through the C ABI, twice on the same inputs with a
+different call between them (the array keeps each call's leftovers, which
+the next call must not see), and checks every result against the regular
+tt_score_topk within the score tolerance of the other parity tests. Another
+test checks that calls after the first leave the device's free memory
+unchanged. It sits in a file of its own that
 pytest collects last, and passes alone in a fresh process as well as after
 the other tests.
 """
@@ -43,6 +45,10 @@ CASES = [
 
 @pytest.mark.parametrize("name,over", CASES, ids=[c[0] for c in CASES])
 def test_noalloc_matches_regular_entry_point(name, over):
+    """Two calls with the same arguments, with a different call between them
+    (more queries, a larger k, another tau, no mask), which leaves larger
+    counts and looser thresholds in the shared array: every call must still
+    equal tt_score_topk."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     w = W.workload(name, **over)
@@ -51,17 +57,55 @@ def test_noalloc_matches_regular_entry_point(name, over):
     excl = W.exclusion_bits(w, "cuda")
     index, qn = parity.gpu_prepare(w, raw_c, raw_q)
     ref_ids, ref_scores = tt.tt_score_topk(index, qn, w.k, tau=w.tau, exclude=excl)
+    # the call in between: twice the queries (repeated), k * 3, tau 0.5, no mask
+    q2 = torch.cat([qn, qn.flip(0)]).contiguous()
+    k2 = min(3 * w.k, 2048)
+    ref2_ids, ref2_scores = tt.tt_score_topk(index, q2, k2, tau=0.5)
     torch.cuda.synchronize()
-    for _ in range(2):
+
+    def check(ids, scores, want_ids, want_scores, tol):
+        assert torch.equal(ids, want_ids)
+        pad = torch.isinf(want_scores)
+        assert torch.equal(pad, torch.isinf(scores))
+        assert (scores[~pad] - want_scores[~pad]).abs().max().item() <= tol
+
+    for step in range(3):
+        if step == 1:
+            ids = torch.full((q2.shape[0], k2), -7, dtype=torch.int32, device="cuda")
+            scores = torch.full((q2.shape[0], k2), math.nan, dtype=torch.float32, device="cuda")
+            st = _noalloc(index.rows, index.inv_norm, q2, k2, 0.5, None, ids, scores)
+            assert st == tt.TT_OK, tt._lib.tt_last_error().decode()
+            torch.cuda.synchronize()
+            check(ids, scores, ref2_ids, ref2_scores, 2 * w.tolerance)
+            continue
         ids = torch.full((w.b, w.k), -7, dtype=torch.int32, device="cuda")
         scores = torch.full((w.b, w.k), math.nan, dtype=torch.float32, device="cuda")
         st = _noalloc(index.rows, index.inv_norm, qn, w.k, w.tau, excl, ids, scores)
         assert st == tt.TT_OK, tt._lib.tt_last_error().decode()
         torch.cuda.synchronize()
-        assert torch.equal(ids, ref_ids)
-        pad = torch.isinf(ref_scores)
-        assert torch.equal(pad, torch.isinf(scores))
-        assert (scores[~pad] - ref_scores[~pad]).abs().max().item() <= w.tolerance
+        check(ids, scores, ref_ids, ref_scores, w.tolerance)
+
+
+def test_noalloc_allocates_nothing_after_the_first_call():
+    """After one warm-up call on the GPU (which may commit the fixed array:
+    CUDA loads a module's device memory when first used), further calls leave
+    the device's free memory unchanged."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    w = W.workload("small_batch", n=150_001, b=40, k=300)
+    raw_c = W.corpus(w, "cuda")
+    raw_q = W.queries(w, "cuda")
+    index, qn = parity.gpu_prepare(w, raw_c, raw_q)
+    ids = torch.empty((w.b, w.k), dtype=torch.int32, device="cuda")
+    scores = torch.empty((w.b, w.k), dtype=torch.float32, device="cuda")
+    assert _noalloc(index.rows, None, qn, w.k, w.tau, None, ids, scores) == tt.TT_OK
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        assert _noalloc(index.rows, None, qn, w.k, w.tau, None, ids, scores) == tt.TT_OK
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, (free0, free1)
 
 
 def test_noalloc_rejects_batches_beyond_its_array():

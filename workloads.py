@@ -133,18 +133,25 @@ def _centres(w: Workload, g: torch.Generator, device) -> torch.Tensor:
     return (signs.to(torch.float32) * 2.0 - 1.0) * (1.0 / math.sqrt(w.d))
 
 
-def _cluster_rows(centres, assign, sigma, d, g, device, out, row0):
-    """out[row0 + i] = centres[assign[i]] + sigma * N(0, I)."""
-    for s in range(0, assign.numel(), CHUNK_ROWS):
+def _cluster_rows(centres, assign, sigma, d, g, device, out, row0, limit=None):
+    """out[row0 + i] = centres[assign[i]] + sigma * N(0, I), for i < limit
+    (default: every row). Noise is drawn in whole chunks, so a prefix holds
+    the same numbers as the full draw."""
+    limit = assign.numel() if limit is None else limit
+    for s in range(0, limit, CHUNK_ROWS):
         a = assign[s:s + CHUNK_ROWS]
         noise = torch.randn((a.numel(), d), generator=g, device=device, dtype=torch.float32)
-        out[row0 + s:row0 + s + a.numel()] = (centres[a] + sigma * noise).to(out.dtype)
+        m = min(a.numel(), limit - s)
+        out[row0 + s:row0 + s + m] = (centres[a[:m]] + sigma * noise[:m]).to(out.dtype)
 
 
-def corpus(w: Workload, device="cpu") -> torch.Tensor:
-    """Raw candidate rows [n, d] in ``w.raw_dtype``."""
+def corpus(w: Workload, device="cpu", rows: int | None = None) -> torch.Tensor:
+    """Raw candidate rows [n, d] in ``w.raw_dtype``; with ``rows``, only the
+    first ``rows`` of them (the same numbers as the full corpus holds there,
+    without drawing the rest)."""
     g = _gen(w.seed, device)
-    out = torch.empty((w.n, w.d), dtype=_torch_dtype(w.raw_dtype), device=device)
+    m_out = w.n if rows is None else max(0, min(int(rows), w.n))
+    out = torch.empty((m_out, w.d), dtype=_torch_dtype(w.raw_dtype), device=device)
     if w.recipe == "clusters":
         centres = _centres(w, g, device)
         if w.zipf:
@@ -153,17 +160,20 @@ def corpus(w: Workload, device="cpu") -> torch.Tensor:
             assign = assign[torch.randperm(w.n, generator=g, device=device)]
         else:
             assign = torch.randint(0, w.n_clusters, (w.n,), generator=g, device=device)
-        _cluster_rows(centres, assign, w.sigma, w.d, g, device, out, 0)
+        _cluster_rows(centres, assign, w.sigma, w.d, g, device, out, 0, limit=m_out)
     elif w.recipe == "gaussian":
-        for s in range(0, w.n, CHUNK_ROWS):
+        for s in range(0, m_out, CHUNK_ROWS):
             m = min(CHUNK_ROWS, w.n - s)
-            out[s:s + m] = torch.randn((m, w.d), generator=g, device=device).to(out.dtype)
+            x = torch.randn((m, w.d), generator=g, device=device)
+            keep = min(m, m_out - s)
+            out[s:s + keep] = x[:keep].to(out.dtype)
     elif w.recipe == "lognormal_rows":
-        for s in range(0, w.n, CHUNK_ROWS):
+        for s in range(0, m_out, CHUNK_ROWS):
             m = min(CHUNK_ROWS, w.n - s)
             x = torch.randn((m, w.d), generator=g, device=device)
             z = torch.randn((m, 1), generator=g, device=device)
-            out[s:s + m] = (x * torch.exp(0.5 * z)).to(out.dtype)
+            keep = min(m, m_out - s)
+            out[s:s + keep] = (x[:keep] * torch.exp(0.5 * z[:keep])).to(out.dtype)
     else:
         raise ValueError(w.recipe)
     return out
