@@ -19,8 +19,15 @@
 //   - gives every epilogue thread one query, so its threshold stays in
 //     registers and the fast test is one compare per score with no
 //     shared-memory traffic (with per-row norms the row scales are read once
-//     per tile from shared memory);
-//   - appends each survivor to the thread's own query buffer.
+//     per tile from shared memory).
+//
+// The epilogue reads its 128 accumulator columns with one TMEM round trip
+// (four loads, one wait) and hands the accumulator back to the MMA issuer
+// before testing anything: with d = 128 a tile is only eight MMAs long, and
+// the hand-off is on the MMAs' critical path. A survivor of the exact test is
+// staged in shared memory by its lane; the warp appends every lane's staged
+// keys with one atomic instruction, so the lanes' round trips to the counters
+// overlap instead of stalling the warp once per survivor.
 //
 // Roles (320 threads per CTA): warp 0 issues this CTA's TMA loads; warp 1
 // allocates tensor memory (both CTAs) and, in the even CTA, issues the MMAs;
@@ -58,6 +65,9 @@ constexpr int KP_TMEM_COLS = 512;
 constexpr int KP_ACC_COLS = 256;
 constexpr int KP_WARP_COLS = 128;              // columns (corpus rows) one epilogue warp reads
 constexpr int KP_SMEM_BUDGET = 227 * 1024;
+// Survivors a lane keeps in shared memory before the warp appends them to
+// the global lists with one atomic instruction for all its lanes.
+constexpr int KP_STAGED = 8;
 
 struct KPCtl {
     uint64_t full[KP_MAX_STAGES];    // even CTA: both CTAs' halves of the stage landed
@@ -70,6 +80,8 @@ struct KPCtl {
     int abort;
     // per-row score scales (rows with norms), read as float4
     alignas(16) float cvals[KP_EPI_WARPS][KP_WARP_COLS];
+    // per epilogue lane: survivors waiting for their append ([slot][lane])
+    uint64_t staged[KP_EPI_WARPS][KP_STAGED][32];
 };
 static_assert(offsetof(KPCtl, cvals) % 16 == 0, "float4 reads of cvals need 16-byte alignment");
 
@@ -97,6 +109,9 @@ __device__ __forceinline__ void raise_abort(KPCtl* ctl, uint32_t peer) {
     st_cluster_u32(mapa_shared(&ctl->abort, peer), 1u);
 }
 
+// NORMS: per-row score scales (raw rows with norms); MASK: an exclusion
+// bitmask; TYPES: several result sets by candidate type.
+template <bool NORMS, bool MASK, bool TYPES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
     k3_pair(const __grid_constant__ CUtensorMap tm_rows, const __grid_constant__ CUtensorMap tm_q,
             const KPParams p) {
@@ -250,8 +265,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
         const int quarter = warp & 3;
         const int half = ew >> 2;
         const PassArgs& a = p.a;
-        const bool uniform_c = a.inv_norm == nullptr;
         float* cw = ctl->cvals[ew];
+        uint64_t* staged = &ctl->staged[ew][0][lane];
         const uint32_t r_tempty0 = mapa_shared(&ctl->tempty[0], 0);
         const uint32_t r_tempty1 = mapa_shared(&ctl->tempty[1], 0);
         uint32_t tc = 0;
@@ -268,7 +283,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
             // With no per-row norms the score scale is the same for every row,
             // and the raw accumulator is compared with th / c, lowered by a
             // relative 2^-20 so that fl(v * c) >= th implies v >= t_fast.
-            if (uniform_c && t_fast != INFINITY && t_fast != -INFINITY) {
+            if (!NORMS && t_fast != INFINITY && t_fast != -INFINITY) {
                 const float r = t_fast / a.inv_tau;
                 t_fast = r - fabsf(r) * 0x1p-20f - 1e-30f;
             }
@@ -277,10 +292,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
             // v*c - t_low, and t_low sits below t_fast by more than the rounding
             // of fl(v*c), so fl(v*c) >= t_fast implies a non-negative result.
             float neg_t_low = -t_fast;
-            if (!uniform_c && t_fast != INFINITY && t_fast != -INFINITY)
+            if (NORMS && t_fast != INFINITY && t_fast != -INFINITY)
                 neg_t_low = -(t_fast - fabsf(t_fast) * 0x1p-20f - 0x1p-140f);
             uint32_t* cnt = a.count + q;
             uint64_t* qkeys = a.keys + (int64_t)q * a.cap;
+            // Survivors are staged per lane and appended by the whole warp at
+            // once: one atomic instruction reserves every lane's slots, so the
+            // round trips of the 32 lanes overlap instead of stalling the warp
+            // once per survivor.
+            int n_staged = 0;
+            auto flush = [&]() {
+                const uint32_t base = n_staged > 0 ? atomicAdd(cnt, (uint32_t)n_staged) : 0u;
+                for (int j = 0; j < n_staged; ++j)
+                    if (base + j < (uint32_t)a.cap) qkeys[base + j] = staged[j * 32];
+                n_staged = 0;
+            };
             // Per-row data of this warp's 128 columns of a tile, fetched one
             // tile ahead: lane l holds rows l, l+32, l+64, l+96 - the inverse
             // norm (rows with norms; 0 past the last row), the mask word
@@ -293,134 +319,138 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
                     const int64_t r = tile * KP_TILE + half * KP_WARP_COLS + lane + 32 * j;
                     const bool valid = r < a.n_rows;
                     // raw values: nothing waits for these loads until the next tile
-                    if (!uniform_c) cl[j] = valid ? __ldg(a.inv_norm + r * a.stride) : 0.0f;
-                    if (a.exclude) {
+                    if (NORMS) cl[j] = valid ? __ldg(a.inv_norm + r * a.stride) : 0.0f;
+                    if (MASK) {
                         xl[j] = valid ? __ldg(a.exclude + ((r * a.stride) >> 5)) : 0u;
                         xs[j] = (uint32_t)((r * a.stride) & 31);
                     }
                 }
             };
-            if (!uniform_c || a.exclude) fetch_rows(t0);
+            if (NORMS || MASK) fetch_rows(t0);
             for (int64_t t = t0; t < t1; ++t, ++tc) {
                 const int buf = tc & 1;
                 const int64_t row0 = t * KP_TILE + half * KP_WARP_COLS;  // level row of column 0
                 // bit i of skip[j]: row row0 + 32j + i is excluded or past the end
-                uint32_t skip[4];
+                uint32_t skip[4] = {0u, 0u, 0u, 0u};
+                if (MASK || row0 + KP_WARP_COLS > a.n_rows) {  // warp-uniform
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    bool bad = row0 + lane + 32 * j >= a.n_rows;
-                    if (a.exclude) bad |= ((xl[j] >> xs[j]) & 1u) != 0u;
-                    skip[j] = __ballot_sync(0xFFFFFFFFu, bad);
+                    for (int j = 0; j < 4; ++j) {
+                        bool bad = row0 + lane + 32 * j >= a.n_rows;
+                        if (MASK) bad |= ((xl[j] >> xs[j]) & 1u) != 0u;
+                        skip[j] = __ballot_sync(0xFFFFFFFFu, bad);
+                    }
                 }
-                if (!uniform_c) {
+                if (NORMS) {
                     __syncwarp();  // the previous tile's reads of cw are done
 #pragma unroll
                     for (int j = 0; j < 4; ++j) cw[lane + 32 * j] = cl[j] * a.inv_tau;
                     __syncwarp();
                 }
-                if ((!uniform_c || a.exclude) && t + 1 < t1) fetch_rows(t + 1);
-                if (!mbar_wait(&ctl->tfull[buf], (tc >> 1) & 1, abort)) {
+                if ((NORMS || MASK) && t + 1 < t1) fetch_rows(t + 1);
+                // the warp decides together, so that it stays converged
+                if (!__all_sync(0xFFFFFFFFu, mbar_wait(&ctl->tfull[buf], (tc >> 1) & 1, abort))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) +
                                        (uint32_t)(buf * KP_ACC_COLS + half * KP_WARP_COLS);
+                // One round trip: the warp's 128 columns into registers, then
+                // the accumulator goes back to the MMA issuer before any test.
+                Cols32 v[4];
 #pragma unroll
-                for (int pair = 0; pair < 2; ++pair) {
-                    Cols32 v[2];
-                    tmem_ld_32cols(tbase + (uint32_t)(pair * 64), v[0].x);
-                    tmem_ld_32cols(tbase + (uint32_t)(pair * 64 + 32), v[1].x);
-                    tmem_ld_wait();
-                    if (pair == 1) {
-                        // values are in registers: release the accumulator
-                        tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) {
-                            if (even)
-                                mbar_arrive(&ctl->tempty[buf]);
-                            else
-                                mbar_arrive_cluster_relaxed(buf ? r_tempty1 : r_tempty0);
+                for (int h = 0; h < 4; ++h) tmem_ld_32cols(tbase + (uint32_t)(h * 32), v[h].x);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (even)
+                        mbar_arrive(&ctl->tempty[buf]);
+                    else
+                        mbar_arrive_cluster_relaxed(buf ? r_tempty1 : r_tempty0);
+                }
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const int col0 = h * 32;  // within this warp's 128 columns
+                    // Fast test. One threshold per thread: compare the maximum
+                    // of the 32 scores (four chains of three-input max, half an
+                    // instruction per score).
+                    bool pass;
+                    float gmax[4];
+                    if (!NORMS) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {  // chain j: scores 8j .. 8j+7
+                            const float* x = v[h].x + 8 * j;
+                            gmax[j] = fmaxf(max3f(max3f(max3f(x[0], x[1], x[2]), x[3], x[4]), x[5], x[6]), x[7]);
+                        }
+                        pass = fmaxf(max3f(gmax[0], gmax[1], gmax[2]), gmax[3]) >= t_fast;
+                    } else {
+                        // all-negative test: AND of the sign words
+                        const float4* c4 = reinterpret_cast<const float4*>(cw + col0);
+                        uint32_t n0 = ~0u, n1 = ~0u;
+#pragma unroll
+                        for (int i4 = 0; i4 < 8; ++i4) {
+                            const float4 c = c4[i4];
+                            n0 &= __float_as_uint(fmaf(v[h].x[4 * i4 + 0], c.x, neg_t_low)) &
+                                  __float_as_uint(fmaf(v[h].x[4 * i4 + 1], c.y, neg_t_low));
+                            n1 &= __float_as_uint(fmaf(v[h].x[4 * i4 + 2], c.z, neg_t_low)) &
+                                  __float_as_uint(fmaf(v[h].x[4 * i4 + 3], c.w, neg_t_low));
+                        }
+                        pass = ((n0 & n1) >> 31) == 0u;
+                    }
+                    if (!pass) continue;
+                    // Rare: this thread's exact survivors among the 32 rows.
+                    uint32_t m = 0;
+                    if (!NORMS) {
+                        // only the groups of eight whose maximum passed
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            if (gmax[j] >= t_fast) {
+#pragma unroll
+                                for (int i = 8 * j; i < 8 * j + 8; ++i) m |= (v[h].x[i] >= t_fast) ? (1u << i) : 0u;
+                            }
+                        }
+                    } else {
+                        const float4* c4 = reinterpret_cast<const float4*>(cw + col0);
+#pragma unroll
+                        for (int i4 = 0; i4 < 8; ++i4) {
+                            const float4 c = c4[i4];
+                            m |= (v[h].x[4 * i4 + 0] * c.x >= t_fast) ? (1u << (4 * i4 + 0)) : 0u;
+                            m |= (v[h].x[4 * i4 + 1] * c.y >= t_fast) ? (1u << (4 * i4 + 1)) : 0u;
+                            m |= (v[h].x[4 * i4 + 2] * c.z >= t_fast) ? (1u << (4 * i4 + 2)) : 0u;
+                            m |= (v[h].x[4 * i4 + 3] * c.w >= t_fast) ? (1u << (4 * i4 + 3)) : 0u;
                         }
                     }
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int col0 = (2 * pair + h) * 32;  // within this warp's 128 columns
-                        // Fast test. One threshold per thread: compare the
-                        // maximum of the 32 scores (four chains of
-                        // three-input max, half an instruction per score).
-                        bool h0 = false, h1 = false, h2 = false, h3 = false;
-                        float gmax[4];
-                        if (uniform_c) {
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {  // chain j: scores 8j .. 8j+7
-                                const float* x = v[h].x + 8 * j;
-                                gmax[j] = fmaxf(max3f(max3f(max3f(x[0], x[1], x[2]), x[3], x[4]), x[5], x[6]), x[7]);
-                            }
-                            h0 = fmaxf(max3f(gmax[0], gmax[1], gmax[2]), gmax[3]) >= t_fast;
-                        } else {
-                            // all-negative test: AND of the sign words
-                            const float4* c4 = reinterpret_cast<const float4*>(cw + col0);
-                            uint32_t n0 = ~0u, n1 = ~0u;
-#pragma unroll
-                            for (int i4 = 0; i4 < 8; ++i4) {
-                                const float4 c = c4[i4];
-                                n0 &= __float_as_uint(fmaf(v[h].x[4 * i4 + 0], c.x, neg_t_low)) &
-                                      __float_as_uint(fmaf(v[h].x[4 * i4 + 1], c.y, neg_t_low));
-                                n1 &= __float_as_uint(fmaf(v[h].x[4 * i4 + 2], c.z, neg_t_low)) &
-                                      __float_as_uint(fmaf(v[h].x[4 * i4 + 3], c.w, neg_t_low));
-                            }
-                            h0 = ((n0 & n1) >> 31) == 0u;
-                        }
-                        // Rare: this thread's exact survivors among the 32 rows.
-                        if (h0 | h1 | h2 | h3) {
-                            uint32_t m = 0;
-                            if (uniform_c) {
-                                // only the groups of eight whose maximum passed
-#pragma unroll
-                                for (int j = 0; j < 4; ++j) {
-                                    if (gmax[j] >= t_fast) {
-#pragma unroll
-                                        for (int i = 8 * j; i < 8 * j + 8; ++i)
-                                            m |= (v[h].x[i] >= t_fast) ? (1u << i) : 0u;
-                                    }
-                                }
-                            } else {
-                                const float4* c4 = reinterpret_cast<const float4*>(cw + col0);
-#pragma unroll
-                                for (int i4 = 0; i4 < 8; ++i4) {
-                                    const float4 c = c4[i4];
-                                    m |= (v[h].x[4 * i4 + 0] * c.x >= t_fast) ? (1u << (4 * i4 + 0)) : 0u;
-                                    m |= (v[h].x[4 * i4 + 1] * c.y >= t_fast) ? (1u << (4 * i4 + 1)) : 0u;
-                                    m |= (v[h].x[4 * i4 + 2] * c.z >= t_fast) ? (1u << (4 * i4 + 2)) : 0u;
-                                    m |= (v[h].x[4 * i4 + 3] * c.w >= t_fast) ? (1u << (4 * i4 + 3)) : 0u;
+                    m &= ~skip[h];
+                    while (m) {
+                        const int i = __ffs(m) - 1;
+                        m &= m - 1;
+                        const int64_t id = (row0 + col0 + i) * a.stride;
+                        const float c = NORMS ? cw[col0 + i] : a.inv_tau;
+                        const uint64_t key = make_key(select32(v[h], i) * c, (uint32_t)id);
+                        if (TYPES) {  // several result sets: the row's set, appended at once
+                            const int rset = a.set_of[a.types[id]];
+                            if (rset >= 0 && q < a.b) {
+                                const int64_t vq = (int64_t)rset * a.b + q;
+                                if (key > a.theta_v[vq]) {
+                                    const uint32_t slot = atomicAdd(a.count + vq, 1u);
+                                    if (slot < (uint32_t)a.cap) a.keys[vq * a.cap + slot] = key;
                                 }
                             }
-                            m &= ~skip[2 * pair + h];
-                            while (m) {
-                                const int i = __ffs(m) - 1;
-                                m &= m - 1;
-                                const int64_t id = (row0 + col0 + i) * a.stride;
-                                const float c = uniform_c ? a.inv_tau : cw[col0 + i];
-                                const uint64_t key = make_key(select32(v[h], i) * c, (uint32_t)id);
-                                if (a.types) {  // several result sets: the row's set
-                                    const int rset = a.set_of[a.types[id]];
-                                    if (rset >= 0 && q < a.b) {
-                                        const int64_t vq = (int64_t)rset * a.b + q;
-                                        if (key > a.theta_v[vq]) {
-                                            const uint32_t slot = atomicAdd(a.count + vq, 1u);
-                                            if (slot < (uint32_t)a.cap) a.keys[vq * a.cap + slot] = key;
-                                        }
-                                    }
-                                } else if (key > th_key) {
-                                    const uint32_t slot = atomicAdd(cnt, 1u);
-                                    if (slot < (uint32_t)a.cap) qkeys[slot] = key;
-                                }
+                        } else if (key > th_key) {
+                            if (n_staged < KP_STAGED) {
+                                staged[n_staged * 32] = key;
+                                ++n_staged;
+                            } else {  // this lane's staging is full: append on its own
+                                const uint32_t slot = atomicAdd(cnt, 1u);
+                                if (slot < (uint32_t)a.cap) qkeys[slot] = key;
                             }
                         }
                     }
                 }
+                if (!TYPES && __any_sync(0xFFFFFFFFu, n_staged >= KP_STAGED / 2)) flush();
             }
+            if (!TYPES && __any_sync(0xFFFFFFFFu, n_staged > 0)) flush();
         }
         if (!ok) {
             atomicExch(a.err, ERR_TIMEOUT_EPI);
@@ -447,26 +477,11 @@ int pair_stages(int d) {
     return stages;
 }
 
-}  // namespace
-
-int tensor_pair_smem_bytes(int d) {
-    const int kchunks = (d + KP_KC - 1) / KP_KC;
-    const int stages = pair_stages(d);
-    if (stages < 2) return -1;
-    return 1024 + kchunks * KP_QCHUNK_BYTES + (int)sizeof(KPCtl) + stages * KP_STAGE_BYTES;
-}
-
-cudaError_t launch_tensor_pair_pass(const PassArgs& a, const CUtensorMap& tm_rows,
-                                    const CUtensorMap& tm_queries, cudaStream_t s, int sm_count) {
-    if (a.n_rows == 0 || a.b == 0) return cudaSuccess;
-    const int smem = tensor_pair_smem_bytes(a.d);
-    if (smem <= 0) return cudaErrorInvalidValue;
-    KPParams p;
-    p.a = a;
-    p.q_tiles = (a.b + 2 * KP_QROWS - 1) / (2 * KP_QROWS);
-    p.kchunks = (a.d + KP_KC - 1) / KP_KC;
-    p.stages = pair_stages(a.d);
-    p.tiles = (a.n_rows + KP_TILE - 1) / KP_TILE;
+template <bool NORMS, bool MASK, bool TYPES>
+cudaError_t launch_variant(const KPParams& base, const CUtensorMap& tm_rows, const CUtensorMap& tm_queries,
+                           int smem, cudaStream_t s, int sm_count) {
+    auto kern = k3_pair<NORMS, MASK, TYPES>;
+    KPParams p = base;
     // Pairs that can be resident at once (clusters must fit inside a GPC).
     int pairs = sm_count / 2 > 0 ? sm_count / 2 : 1;
     {
@@ -475,9 +490,9 @@ cudaError_t launch_tensor_pair_pass(const PassArgs& a, const CUtensorMap& tm_row
         cfg.blockDim = dim3(KP_THREADS);
         cfg.dynamicSmemBytes = (size_t)smem;
         int max_clusters = 0;
-        cudaError_t e = cudaFuncSetAttribute(k3_pair, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        if (cudaOccupancyMaxActiveClusters(&max_clusters, k3_pair, &cfg) == cudaSuccess) {
+        if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) == cudaSuccess) {
             if (max_clusters > 0 && max_clusters < pairs) pairs = max_clusters;
         } else {
             cudaGetLastError();
@@ -492,13 +507,51 @@ cudaError_t launch_tensor_pair_pass(const PassArgs& a, const CUtensorMap& tm_row
     if (chunks < 1) chunks = 1;
     if (chunks > p.tiles) chunks = (int)p.tiles;
     p.chunks = chunks;
-    p.idesc = umma_idesc_bf16(2 * KP_QROWS, KP_TILE);
     const int n_units = p.q_tiles * p.chunks;
     const int clusters = n_units < pairs ? n_units : pairs;
     note_launch_begin(TT_KIND_TENSOR, s);
-    k3_pair<<<2 * clusters, KP_THREADS, smem, s>>>(tm_rows, tm_queries, p);
+    kern<<<2 * clusters, KP_THREADS, smem, s>>>(tm_rows, tm_queries, p);
     note_launch_end(TT_KIND_TENSOR, s);
     return cudaGetLastError();
+}
+
+}  // namespace
+
+int tensor_pair_box_rows(int) { return KP_ROWS; }
+
+int tensor_pair_smem_bytes(int d) {
+    if (d % KP_KC != 0 || d > TT_MAX_D) return -1;
+    const int kchunks = (d + KP_KC - 1) / KP_KC;
+    const int stages = pair_stages(d);
+    if (stages < 2) return -1;
+    return 1024 + kchunks * KP_QCHUNK_BYTES + (int)sizeof(KPCtl) + stages * KP_STAGE_BYTES;
+}
+
+cudaError_t launch_tensor_pair_pass(const PassArgs& a, const CUtensorMap& tm_rows, cudaStream_t s, int sm_count) {
+    if (a.n_rows == 0 || a.b == 0) return cudaSuccess;
+    if (a.q_dtype != TT_BF16) return cudaErrorInvalidValue;
+    const int smem = tensor_pair_smem_bytes(a.d);
+    if (smem <= 0) return cudaErrorInvalidValue;
+    CUtensorMap tm_queries;
+    if (!bf16_tile_tensor_map(a.queries, a.b, a.d, a.d, KP_QROWS, &tm_queries)) return cudaErrorInvalidValue;
+    KPParams p;
+    p.a = a;
+    p.q_tiles = (a.b + 2 * KP_QROWS - 1) / (2 * KP_QROWS);
+    p.kchunks = (a.d + KP_KC - 1) / KP_KC;
+    p.stages = pair_stages(a.d);
+    p.tiles = (a.n_rows + KP_TILE - 1) / KP_TILE;
+    p.chunks = 1;
+    p.idesc = umma_idesc_bf16(2 * KP_QROWS, KP_TILE);
+    const bool norms = a.inv_norm != nullptr, mask = a.exclude != nullptr, types = a.types != nullptr;
+    if (types) {
+        return norms ? launch_variant<true, true, true>(p, tm_rows, tm_queries, smem, s, sm_count)
+                     : launch_variant<false, true, true>(p, tm_rows, tm_queries, smem, s, sm_count);
+    }
+    if (norms)
+        return mask ? launch_variant<true, true, false>(p, tm_rows, tm_queries, smem, s, sm_count)
+                    : launch_variant<true, false, false>(p, tm_rows, tm_queries, smem, s, sm_count);
+    return mask ? launch_variant<false, true, false>(p, tm_rows, tm_queries, smem, s, sm_count)
+                : launch_variant<false, false, false>(p, tm_rows, tm_queries, smem, s, sm_count);
 }
 
 }  // namespace tt

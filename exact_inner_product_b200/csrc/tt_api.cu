@@ -588,9 +588,10 @@ static tt_status run_pass(const tt_index* ix, const PathCfg& pc, const Plan& pla
         e = launch_tensor_pass(a, tm_rows, pc.tm_q, pc.nq, s, sms);
     } else if (pc.path == 3) {
         CUtensorMap tm_rows;
-        if (!bf16_tile_tensor_map(ix->rows, a.n_rows, ix->d, a.stride * ix->d, 128, &tm_rows))
+        if (!bf16_tile_tensor_map(ix->rows, a.n_rows, ix->d, a.stride * ix->d, tensor_pair_box_rows(ix->d),
+                                  &tm_rows))
             return TT_ERR_CUDA;
-        e = launch_tensor_pair_pass(a, tm_rows, pc.tm_q, s, sms);
+        e = launch_tensor_pair_pass(a, tm_rows, s, sms);
     } else {
         e = launch_stream_pass(a, s, sms);
     }
@@ -941,8 +942,9 @@ static tt_status score_core(tt_index* index, const void* queries, tt_dtype q_dty
             pc.q_dtype = TT_BF16;
         }
         pc.nq = path == 2 ? nq : 256;
-        // single-CTA kernel: boxes of nq queries; pairs: each CTA loads 128
-        if (!tile_tensor_map(pc.q_dtype, pc.queries, b, index->d, index->d, path == 2 ? nq : 128, &pc.tm_q))
+        // single-CTA kernel: the query tile by TMA, boxes of nq queries (the
+        // SM-pair kernel reads its queries into tensor memory directly)
+        if (path == 2 && !tile_tensor_map(pc.q_dtype, pc.queries, b, index->d, index->d, nq, &pc.tm_q))
             return TT_ERR_CUDA;
     }
 

@@ -64,10 +64,11 @@ cudaError_t launch_stream_pass(const PassArgs& a, cudaStream_t s, int sm_count);
 cudaError_t launch_tensor_pass(const PassArgs& a, const CUtensorMap& tm_rows,
                                const CUtensorMap& tm_queries, int nq_tile, cudaStream_t s,
                                int sm_count);
-// Tensor-core pass on SM pairs (b >= 1; queries in tiles of 256, tm_queries
-// with boxes of 128 rows).
-cudaError_t launch_tensor_pair_pass(const PassArgs& a, const CUtensorMap& tm_rows,
-                                    const CUtensorMap& tm_queries, cudaStream_t s, int sm_count);
+// Tensor-core pass on SM pairs (b >= 1, bf16 queries in tiles of 256, d a
+// multiple of 64; tm_rows with boxes of tensor_pair_box_rows(d) rows).
+cudaError_t launch_tensor_pair_pass(const PassArgs& a, const CUtensorMap& tm_rows, cudaStream_t s,
+                                    int sm_count);
+int tensor_pair_box_rows(int d);
 // count[0..b) = 0; theta/thf[0..b) = theta_value; [b, b_pad) = KEY_MAX / +inf;
 // flags[0..2) = 0.
 cudaError_t launch_init(uint32_t* count, uint64_t* theta, float* thf, uint64_t theta_value, int b,
