@@ -64,16 +64,16 @@ PATH_NAMES = {1: "streaming", 2: "tensor-core", 3: "tensor-core (SM pairs)"}
 # K1 bytes per corpus row; K3 bytes per level row scanned (level-0 capture,
 # applied to every level of a step, like `achieved`).
 TRAFFIC = {
-    # ncu --set full -k regex:k1_normalize -s 5 -c 1 on `python bench.py --steps 50 --warmup 3
+    # ncu --set full --clock-control none -k regex:k1_normalize -s 5 -c 1 on `python bench.py --steps 50 --warmup 3
     # --no-e2e --no-cpu-baseline`: 512.019 MB read + 200.806 MB written for 1,000,000 rows
     ("k1_normalize", "stream_b1"): {"bytes_per_row": 712.825, "src": "exact_inner_product_b200/csrc/k_normalize.cu",
                                     "sha": "4273a9f8869b74ec01b8762c20eb598dc6f0b1597fcd3e5f8ad9afde664127f4"},
-    # ncu --set full -k regex:k3_pair -s 5 -c 1 on `python bench.py --workload large_batch --n 4000000
+    # ncu --set full --clock-control none -k regex:k3_pair -s 5 -c 1 on `python bench.py --workload large_batch --n 4000000
     # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 1592.981 MB read
     # + 28.070 MB written; scaled to the full corpus by rows scanned
     ("k3_pair", "large_batch"): {"bytes_per_row": 405.263, "src": "exact_inner_product_b200/csrc/k_tensor_pair.cu",
                                  "sha": "6f303eca084c883abd77d28ff639f8375a1558b5412efecc66fc5478f0e084eb"},
-    # ncu --set full -k regex:k3_tensor -s 5 -c 1 on `python bench.py --workload masked_fused --n 4000000
+    # ncu --set full --clock-control none -k regex:k3_tensor -s 5 -c 1 on `python bench.py --workload masked_fused --n 4000000
     # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 4385.550 MB read
     # + 66.286 MB written; scaled to the full corpus by rows scanned
     ("k3_tensor", "masked_fused"): {"bytes_per_row": 1112.959, "src": "exact_inner_product_b200/csrc/k_tensor.cu",
@@ -380,7 +380,10 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize(dev)
     tt.tt_index_check(index)  # raises if a device-side wait expired in the warm-up
     stats = tt.tt_last_stats(index)
-    plan = tt.tt_plan(w.n, w.k)
+    # the plan the searches ran: scored levels, and the sample of the estimate
+    # when the small-batch plan replaced the coarse levels with it
+    plan = {"rows": stats["level_rows"][:1] if stats["sampled"] else stats["level_rows"],
+            "sample_rows": stats["level_rows"][1] if stats["sampled"] else 0}
 
     clocks = ClockSampler(local)
     clocks.start()
@@ -534,6 +537,7 @@ def run_ours(args, world, rank, local):
                    "queries": w.query_dtype, "mask_rate": w.mask_rate, "l2": l2_note,
                    "step": "normalise the raw queries + tt_score_topk on the index (built once)",
                    "path": PATH_NAMES[stats["path"]], "levels": plan["rows"],
+                   "estimate_sample_rows": plan["sample_rows"],
                    "parallelism": (f"corpus shards x{world} (all-gather of [b, k] lists + merge)" if sharded
                                    else f"replicas x{world}")},
         "topk_queries_per_s": qps,

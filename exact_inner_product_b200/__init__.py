@@ -38,7 +38,7 @@ TT_NORM_FUSED = 1
 TT_MAX_D = 512
 TT_MAX_K = 2048
 
-KIND_NAMES = ("normalize", "cast", "stream", "tensor", "select", "aux", "softmax")
+KIND_NAMES = ("normalize", "cast", "stream", "tensor", "select", "aux", "softmax", "estimate")
 TT_NUM_KINDS = len(KIND_NAMES)
 
 if not os.path.exists(LIB_PATH):
@@ -56,7 +56,7 @@ class tt_stats(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int32), ("levels", ctypes.c_int32), ("rescans", ctypes.c_int32),
                 ("launches", ctypes.c_int32), ("level_rows", ctypes.c_int64 * 4),
                 ("level_stride", ctypes.c_int64 * 4), ("cap", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("sampled", ctypes.c_int32)]
 
 
 _lib = ctypes.CDLL(LIB_PATH)
@@ -469,7 +469,7 @@ def tt_last_stats(index: Index) -> dict:
     _check(_lib.tt_last_stats(index.handle, ctypes.byref(s)), "tt_last_stats")
     return {"path": s.path, "levels": s.levels, "rescans": s.rescans, "launches": s.launches,
             "level_rows": list(s.level_rows[:s.levels]), "level_stride": list(s.level_stride[:s.levels]),
-            "cap": s.cap}
+            "cap": s.cap, "sampled": bool(s.sampled)}
 
 
 def tt_plan(n: int, k: int, **options) -> dict:

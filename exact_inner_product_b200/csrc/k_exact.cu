@@ -36,6 +36,7 @@
 
 #include "tt_device.cuh"
 #include "tt_internal.h"
+#include "tt_rowdot.cuh"
 #include "tt_select.cuh"
 
 namespace tt {
@@ -46,60 +47,11 @@ constexpr int KX_BUF = K4_SMEM_KEYS;  // keys a block keeps between compactions
 
 __device__ __forceinline__ int ld_volatile(const int* p) { return *reinterpret_cast<const volatile int*>(p); }
 
-// fp32 / bf16 rows: the streaming scorer's dot product (element order, fmaf).
-__device__ __forceinline__ float dot_bf16(const __nv_bfloat16* row, const float* qf, int d) {
-    const uint4* p = reinterpret_cast<const uint4*>(row);
-    float acc = 0.f;
-    for (int i = 0; i < d / 8; ++i) {
-        const uint4 r = __ldcs(p + i);
-        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            acc = fmaf(__uint_as_float(w[j] << 16), qf[8 * i + 2 * j], acc);
-            acc = fmaf(__uint_as_float(w[j] & 0xFFFF0000u), qf[8 * i + 2 * j + 1], acc);
-        }
-    }
-    return acc;
-}
-
-__device__ __forceinline__ float dot_f32(const float* row, const float* qf, int d) {
-    const float4* p = reinterpret_cast<const float4*>(row);
-    float acc = 0.f;
-    for (int i = 0; i < d / 4; ++i) {
-        const float4 r = __ldcs(p + i);
-        acc = fmaf(r.x, qf[4 * i + 0], acc);
-        acc = fmaf(r.y, qf[4 * i + 1], acc);
-        acc = fmaf(r.z, qf[4 * i + 2], acc);
-        acc = fmaf(r.w, qf[4 * i + 3], acc);
-    }
-    return acc;
-}
-
-// int8 rows: exact int32 sum of code products (d % 32 == 0).
-__device__ __forceinline__ int dot_i8(const int8_t* row, const int* qw, int d) {
-    const int4* p = reinterpret_cast<const int4*>(row);
-    int acc = 0;
-    for (int i = 0; i < d / 16; ++i) {
-        const int4 r = __ldcs(p + i);
-        acc = __dp4a(r.x, qw[4 * i + 0], acc);
-        acc = __dp4a(r.y, qw[4 * i + 1], acc);
-        acc = __dp4a(r.z, qw[4 * i + 2], acc);
-        acc = __dp4a(r.w, qw[4 * i + 3], acc);
-    }
-    return acc;
-}
-
 // Keep the k best of the block's n buffered keys (n > k): they move to the
 // front of the buffer; returns the k-th best.
 __device__ uint64_t compact_to_k(K4Smem& sm, int n, int k, uint32_t* s_count) {
     const uint64_t kth = block_kth_largest(sm.keys, n, k, sm);
-    if (threadIdx.x == 0) sm.n_collected = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < n; i += KX_THREADS) {
-        const uint64_t key = sm.keys[i];
-        if (key >= kth) sm.sorted[atomicAdd(&sm.n_collected, 1u)] = key;  // exactly k (keys are distinct)
-    }
-    __syncthreads();
+    gather_above(sm.keys, n, kth - 1, (uint32_t)k, sm);  // exactly k (keys are distinct and above KEY_MIN)
     for (int i = threadIdx.x; i < k; i += KX_THREADS) sm.keys[i] = sm.sorted[i];
     if (threadIdx.x == 0) *s_count = (uint32_t)k;
     __syncthreads();
@@ -114,13 +66,15 @@ __global__ void __launch_bounds__(KX_THREADS) k4_exact(const ExactArgs a) {
     __shared__ uint64_t s_th;
     __shared__ int s_last;
     const int tid = threadIdx.x;
+    pdl_wait();  // launched behind the final select
     const int err = ld_volatile(a.flags + 1);
     const int n_flagged = ld_volatile(a.flags);
     if (blockIdx.x == 0 && tid == 0 && a.status != nullptr) {
-        if (err != 0) a.status->err = err;
-        a.status->repaired = err != 0 ? 0 : n_flagged;
-        __threadfence_system();
-        a.status->seq = a.seq;
+        if (err != 0) {
+            a.status->err = err;
+            __threadfence_system();  // the error is visible no later than the sequence number
+        }
+        a.status->seq_repaired = ((uint64_t)(uint32_t)a.seq << 32) | (uint32_t)(err != 0 ? 0 : n_flagged);
     }
     if (err != 0) {
         const int64_t total = (int64_t)a.V * a.k;
@@ -144,16 +98,7 @@ __global__ void __launch_bounds__(KX_THREADS) k4_exact(const ExactArgs a) {
         const int set = v / a.b;
         // the list's query, as the main passes saw it
         __syncthreads();  // the previous unit is done with qf and the buffer
-        if (a.dtype == TT_I8) {
-            const int* qw = reinterpret_cast<const int*>(a.queries) + (int64_t)q * (d / 4);
-            for (int i = tid; i < d / 4; i += KX_THREADS) reinterpret_cast<int*>(qf)[i] = qw[i];
-        } else {
-            for (int i = tid; i < d; i += KX_THREADS) {
-                const int64_t off = (int64_t)q * d + i;
-                qf[i] = a.q_dtype == TT_F32 ? static_cast<const float*>(a.queries)[off]
-                                            : __bfloat162float(static_cast<const __nv_bfloat16*>(a.queries)[off]);
-            }
-        }
+        stage_query(a.dtype, a.queries, a.q_dtype, q, d, qf);
         if (tid == 0) {
             s_count = 0;
             s_th = a.theta[v];
@@ -169,19 +114,7 @@ __global__ void __launch_bounds__(KX_THREADS) k4_exact(const ExactArgs a) {
                 if (a.exclude) ok = !((a.exclude[r >> 5] >> (r & 31)) & 1u);
                 if (ok && a.types) ok = a.set_of[a.types[r]] == set;
                 if (ok) {
-                    float s;
-                    if (a.dtype == TT_I8) {
-                        const int acc = dot_i8(static_cast<const int8_t*>(a.rows) + r * d,
-                                               reinterpret_cast<const int*>(qf), d);
-                        const float cj = a.inv_norm[r] * a.inv_tau;
-                        s = (float)acc * us * cj;
-                    } else {
-                        const float acc = a.dtype == TT_F32
-                                              ? dot_f32(static_cast<const float*>(a.rows) + r * d, qf, d)
-                                              : dot_bf16(static_cast<const __nv_bfloat16*>(a.rows) + r * d, qf, d);
-                        const float cj = a.inv_norm ? a.inv_norm[r] * a.inv_tau : a.inv_tau;
-                        s = acc * cj;
-                    }
+                    const float s = score_row(a.dtype, a.rows, r, d, qf, a.inv_norm, a.inv_tau, us);
                     const uint64_t key = make_key(s, (uint32_t)r);
                     if (key > th) sm.keys[atomicAdd(&s_count, 1u)] = key;
                 }
@@ -242,14 +175,16 @@ cudaError_t launch_exact(const ExactArgs& a, cudaStream_t s, int sm_count) {
     const size_t smem = sizeof(K4Smem) + (size_t)a.d * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(k4_exact, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    // one block per SM at most: a search that needs no repair launches few
+    // blocks, each of which returns at once
     int64_t grid = (int64_t)a.V * a.chunks;
-    const int64_t max_grid = (int64_t)sm_count * 3;
+    const int64_t max_grid = sm_count;
     if (grid > max_grid) grid = max_grid;
     if (grid < 1) grid = 1;
     note_launch_begin(TT_KIND_AUX, s);
-    k4_exact<<<(unsigned)grid, KX_THREADS, smem, s>>>(a);
+    e = launch_pdl(k4_exact, dim3((unsigned)grid), dim3(KX_THREADS), smem, s, a);
     note_launch_end(TT_KIND_AUX, s);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace tt

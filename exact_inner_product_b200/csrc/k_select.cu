@@ -71,12 +71,15 @@ __global__ void __launch_bounds__(K4_THREADS)
                         int r, uint64_t* __restrict__ theta_next, float* __restrict__ thf_next) {
     extern __shared__ __align__(16) uint8_t k4_smem_raw[];
     K4Smem& sm = *reinterpret_cast<K4Smem*>(k4_smem_raw);
+    pdl_trigger();
+    pdl_wait();  // the pass that kept the keys is done
     const int q = blockIdx.x;
     const uint32_t c = count[q];
     const int n = c < (uint32_t)cap ? (int)c : cap;
     uint64_t th = KEY_MIN;
     if (n >= r && r > 0) {
-        const uint64_t* qkeys = stage_keys(keys + (int64_t)q * cap, n, sm);
+        // the register top-r reads every key once: no staging for it
+        const uint64_t* qkeys = r <= K4_TOP_MAX ? keys + (int64_t)q * cap : stage_keys(keys + (int64_t)q * cap, n, sm);
         th = block_kth_largest(qkeys, n, r, sm) - 1;
     }
     __syncthreads();
@@ -98,13 +101,15 @@ __global__ void __launch_bounds__(K4_THREADS)
                     int* __restrict__ flags, int32_t* __restrict__ out_ids, float* __restrict__ out_scores) {
     extern __shared__ __align__(16) uint8_t k4_smem_raw[];
     K4Smem& sm = *reinterpret_cast<K4Smem*>(k4_smem_raw);
+    pdl_trigger();
+    pdl_wait();  // the pass that kept the keys is done
     const int q = blockIdx.x;
     const int tid = threadIdx.x;
     if (flags[1] != 0) return;  // a device wait expired earlier in this call: nothing is valid
     const uint32_t c = count[q];
     const int n = c < (uint32_t)cap ? (int)c : cap;
     const uint64_t th = theta[q];
-    const uint64_t* qkeys = stage_keys(keys + (int64_t)q * cap, n, sm);
+    const uint64_t* qkeys = k <= K4_TOP_MAX ? keys + (int64_t)q * cap : stage_keys(keys + (int64_t)q * cap, n, sm);
     const bool exact = (c <= (uint32_t)cap) && (c >= (uint32_t)k || th == KEY_MIN);
     if (exact) {
         write_sorted_topk(qkeys, n, n, k, sm, out_ids + (int64_t)q * k, out_scores + (int64_t)q * k);
@@ -125,6 +130,8 @@ __global__ void __launch_bounds__(K4_THREADS)
 
 __global__ void k4_init(uint32_t* count, uint64_t* theta, float* thf, uint64_t th0, int b, int b_pad,
                         int* flags) {
+    pdl_trigger();
+    pdl_wait();  // the previous search on this work memory is done with it
     const float f0 = key_floor(th0), fmax = key_floor(KEY_MAX);
     for (int q = blockIdx.x * blockDim.x + threadIdx.x; q < b_pad; q += gridDim.x * blockDim.x) {
         if (q < b) {
@@ -136,7 +143,7 @@ __global__ void k4_init(uint32_t* count, uint64_t* theta, float* thf, uint64_t t
             thf[q] = fmax;
         }
     }
-    if (blockIdx.x == 0 && threadIdx.x < 2) flags[threadIdx.x] = 0;
+    if (blockIdx.x == 0 && threadIdx.x < 16) flags[threadIdx.x] = 0;
 }
 
 __global__ void k4_pad(int32_t* out_ids, float* out_scores, int64_t count) {
@@ -190,9 +197,10 @@ unsigned small_grid(int64_t n) {
 cudaError_t launch_init(uint32_t* count, uint64_t* theta, float* thf, uint64_t theta_value, int b,
                         int b_pad, int* flags, cudaStream_t s) {
     note_launch_begin(TT_KIND_AUX, s);
-    k4_init<<<small_grid(b_pad), 256, 0, s>>>(count, theta, thf, theta_value, b, b_pad, flags);
+    const cudaError_t e = launch_pdl(k4_init, dim3(small_grid(b_pad)), dim3(256), 0, s, count, theta, thf,
+                                     theta_value, b, b_pad, flags);
     note_launch_end(TT_KIND_AUX, s);
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_select_threshold(const uint64_t* keys, uint32_t* count, int cap, int b, int r,
@@ -201,9 +209,10 @@ cudaError_t launch_select_threshold(const uint64_t* keys, uint32_t* count, int c
     const int smem = (int)sizeof(K4Smem);
     cudaFuncSetAttribute(k4_select_threshold, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     note_launch_begin(TT_KIND_SELECT, s);
-    k4_select_threshold<<<b, K4_THREADS, smem, s>>>(keys, count, cap, r, theta_next, thf_next);
+    const cudaError_t e = launch_pdl(k4_select_threshold, dim3(b), dim3(K4_THREADS), smem, s, keys, count, cap, r,
+                                     theta_next, thf_next);
     note_launch_end(TT_KIND_SELECT, s);
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_select_final(const uint64_t* keys, uint32_t* count, int cap, int b, int k,
@@ -213,10 +222,10 @@ cudaError_t launch_select_final(const uint64_t* keys, uint32_t* count, int cap, 
     const int smem = (int)sizeof(K4Smem);
     cudaFuncSetAttribute(k4_select_final, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     note_launch_begin(TT_KIND_SELECT, s);
-    k4_select_final<<<b, K4_THREADS, smem, s>>>(keys, count, cap, k, theta, thf, flagged, flags, out_ids,
-                                                out_scores);
+    const cudaError_t e = launch_pdl(k4_select_final, dim3(b), dim3(K4_THREADS), smem, s, keys, count, cap, k,
+                                     theta, thf, flagged, flags, out_ids, out_scores);
     note_launch_end(TT_KIND_SELECT, s);
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_merge(const int32_t* ids, const float* scores, int parts, int b, int k_in,

@@ -520,7 +520,7 @@ cudaError_t launch_variant(const KPParams& base, const CUtensorMap& tm_rows, con
 int tensor_pair_box_rows(int) { return KP_ROWS; }
 
 int tensor_pair_smem_bytes(int d) {
-    if (d % KP_KC != 0 || d > TT_MAX_D) return -1;
+    if (d > TT_MAX_D) return -1;
     const int kchunks = (d + KP_KC - 1) / KP_KC;
     const int stages = pair_stages(d);
     if (stages < 2) return -1;

@@ -248,7 +248,6 @@ constexpr int MAX_DEEPEST_ROWS = 4096;  // the deepest level keeps every key
 // fewer keys kept per pass.
 constexpr int MIN_RANK = 32;
 constexpr int MIN_RANK_DEEP = 10;
-constexpr int MAX_LEVELS = 4;
 // Batches at least this large, on a corpus stored normalised, go to the
 // tensor-core kernel on SM pairs (queries in tiles of 256 on TMEM lanes);
 // the rest to the single-SM kernel (queries in tiles of up to 256 on TMEM
@@ -258,15 +257,62 @@ constexpr int MAX_LEVELS = 4;
 // corpora with per-row norms stay on the single-SM kernel.
 constexpr int PAIR_MIN_BATCH = 256;
 
-struct Plan {
-    int levels;
-    int64_t stride[MAX_LEVELS];
-    int64_t rows[MAX_LEVELS];
-    int rank[MAX_LEVELS];  // rank[i] (i >= 1): r-th best key of level i sets theta of level i-1
-    int cap;
-};
+// P(X >= r) for X ~ Poisson(lambda), r >= 1 (small when lambda < r).
+static double poisson_upper(double lambda, int r) {
+    if (lambda <= 0.0) return 0.0;
+    if (lambda >= r) return 1.0;
+    double t = exp(-lambda + r * log(lambda) - lgamma(r + 1.0)), sum = 0.0;
+    for (int i = r; i < r + 2000 && t > sum * 1e-17; ++i) {
+        sum += t;
+        t *= lambda / (i + 1);
+    }
+    return sum;
+}
 
-static tt_status make_plan(int64_t n, int32_t k, const tt_options* opt, Plan* p) {
+// P(X < r) for X ~ Poisson(mu).
+static double poisson_lower(double mu, int r) {
+    double sum = 0.0;
+    for (int i = 0; i < r; ++i) sum += exp(-mu + i * log(mu) - lgamma(i + 1.0));
+    return sum;
+}
+
+// The sampled plan of a small batch: one sample of about SAMPLE_ROWS rows
+// (every S-th row, S odd, so that masks repeating every 2, 4, 8 ... rows are
+// sampled evenly), reduced to the threshold in one launch. The rank r is the
+// smallest for which the true top-k misses the filter with probability at
+// most PLAN_FAIL_P (more than r - 1 sample rows among the true top k - 1, a
+// Poisson(k / S) count), and the filter must also keep at most `cap` rows with
+// that probability (fewer than r sample rows among the best cap, a
+// Poisson(cap / S) count). Returns false when no such plan exists.
+constexpr int64_t SAMPLE_ROWS = 16384;
+constexpr double PLAN_FAIL_P = 1e-9;
+
+static bool sampled_plan(int64_t n, int32_t k, int cap, int scale, Plan* p) {
+    if (n <= 2 * SAMPLE_ROWS) return false;
+    int64_t S = n / SAMPLE_ROWS;
+    if ((S & 1) == 0) ++S;
+    const int64_t ns = (n + S - 1) / S;
+    const double f = (double)ns / (double)n;
+    int r = 1;
+    while (r <= 256 && poisson_upper(k * f, r) > PLAN_FAIL_P) ++r;
+    if (r > 256 || poisson_lower(cap * f, r) > PLAN_FAIL_P) return false;
+    r = (int)((int64_t)r * scale / 100);
+    if (r < 1) r = 1;
+    if (r > ESTIMATE_MAX_RANK) return false;
+    const int64_t blocks = (ns + ESTIMATE_BLOCK_ROWS - 1) / ESTIMATE_BLOCK_ROWS;
+    if (blocks * r > 4096 || blocks * r > cap) return false;  // the blocks' lists are merged in shared memory
+    p->levels = 2;
+    p->sampled = true;
+    p->stride[0] = 1;
+    p->rows[0] = n;
+    p->rank[0] = k;
+    p->stride[1] = S;
+    p->rows[1] = ns;
+    p->rank[1] = r;
+    return true;
+}
+
+tt_status make_plan(int64_t n, int32_t k, const tt_options* opt, bool small_batch, Plan* p) {
     int cap = (opt && opt->cap) ? opt->cap : DEFAULT_CAP;
     if (cap < 256 || cap > DEFAULT_CAP || (cap & (cap - 1)) != 0) return TT_ERR_INVALID_ARG;
     if (cap < 2 * k) return TT_ERR_INVALID_ARG;
@@ -275,6 +321,8 @@ static tt_status make_plan(int64_t n, int32_t k, const tt_options* opt, Plan* p)
     const int forced = opt ? opt->force_levels : 0;
     if (forced < 0 || forced > MAX_LEVELS) return TT_ERR_INVALID_ARG;
     p->cap = cap;
+    p->sampled = false;
+    if (small_batch && forced == 0 && sampled_plan(n, k, cap, scale, p)) return TT_OK;
     int L = 0;
     int64_t s = 1;
     if (forced > 0) {
@@ -530,8 +578,7 @@ static tt_status get_scratch(tt_index* ix, int b, int b_pad, int vq, int vpad, i
         }
         ix->dstat = static_cast<HostStatus*>(dp);
         ix->hstat->err = 0;
-        ix->hstat->repaired = 0;
-        ix->hstat->seq = 0;
+        ix->hstat->seq_repaired = 0;
     }
     return TT_OK;
 }
@@ -692,7 +739,7 @@ tt_status tt_plan(int64_t n, int32_t k, const tt_options* options, int32_t* leve
     if (k <= 0) return TT_ERR_INVALID_ARG;
     if (k > TT_MAX_K) return TT_ERR_UNSUPPORTED;
     Plan p;
-    tt_status st = make_plan(n, k, options, &p);
+    tt_status st = make_plan(n, k, options, false, &p);
     if (st != TT_OK) return st;
     if (levels) *levels = p.levels;
     if (cap) *cap = p.cap;
@@ -799,8 +846,12 @@ void tt_free(tt_index* index) {
 tt_status tt_last_stats(const tt_index* index, tt_stats* out) {
     if (!index || !out) return TT_ERR_INVALID_ARG;
     *out = index->last;
-    if (index->last_pending != 0)  // known once the call's last kernel has run
-        out->rescans = (index->hstat && index->hstat->seq == index->last_pending) ? index->hstat->repaired : -1;
+    if (index->last_pending != 0 && index->hstat) {  // known once the call's last kernel has run
+        const uint64_t w = index->hstat->seq_repaired;
+        out->rescans = (uint32_t)(w >> 32) == (uint32_t)index->last_pending ? (int32_t)(uint32_t)w : -1;
+    } else if (index->last_pending != 0) {
+        out->rescans = -1;
+    }
     return TT_OK;
 }
 
@@ -832,9 +883,7 @@ static tt_status score_core(tt_index* index, const void* queries, tt_dtype q_dty
         return TT_ERR_INVALID_ARG;
     const int path_req = options ? options->path : 0;
     if (path_req < 0 || path_req > 3) return TT_ERR_INVALID_ARG;
-    Plan plan;
-    tt_status st = make_plan(index->n, k, options, &plan);
-    if (st != TT_OK) return st;
+    tt_status st;
     if (index->dtype == TT_F32 && index->d > 256) return TT_ERR_UNSUPPORTED;
     const bool i8 = index->dtype == TT_I8;
     // int8 rows are read in 32-byte pieces by the streaming scorer
@@ -851,6 +900,9 @@ static tt_status score_core(tt_index* index, const void* queries, tt_dtype q_dty
     }
     if (path == 2 && !tc_possible) return TT_ERR_UNSUPPORTED;
     if (path == 3 && !pair_possible) return TT_ERR_UNSUPPORTED;
+    // a few queries on the streaming scorer: one sample sets the threshold
+    Plan plan;
+    if ((st = make_plan(index->n, k, options, path == 1 && types == nullptr && b <= 8, &plan)) != TT_OK) return st;
     if (b == 0) return TT_OK;
     const int V = types ? n_sets * b : b;  // lists kept: one per (set, query)
 
@@ -874,6 +926,7 @@ static tt_status score_core(tt_index* index, const void* queries, tt_dtype q_dty
     stats.path = path;
     stats.levels = plan.levels;
     stats.cap = plan.cap;
+    stats.sampled = plan.sampled ? 1 : 0;
     for (int i = 0; i < plan.levels; ++i) {
         stats.level_rows[i] = plan.rows[i];
         stats.level_stride[i] = plan.stride[i];
@@ -951,7 +1004,30 @@ static tt_status score_core(tt_index* index, const void* queries, tt_dtype q_dty
     cudaError_t e = launch_init(sc.count, sc.theta, sc.thf, KEY_MIN, V, v_pad, sc.flags, s);
     if (e == cudaSuccess) e = sets_min();
     if (e != cudaSuccess) return cuda_fail(e, "init");
-    for (int lv = plan.levels - 1; lv >= 0; --lv) {
+    if (plan.sampled) {
+        EstimateArgs es;
+        memset(&es, 0, sizeof es);
+        es.rows = index->rows;
+        es.dtype = index->dtype;
+        es.d = index->d;
+        es.inv_norm = index->inv_norm;
+        es.exclude = exclude_bits;
+        es.inv_tau = inv_tau;
+        es.queries = pc.queries;
+        es.q_dtype = pc.q_dtype;
+        es.qscale = pc.qscale;
+        es.b = b;
+        es.stride = plan.stride[1];
+        es.n_sample = plan.rows[1];
+        es.rank = plan.rank[1];
+        es.keys = sc.keys;
+        es.cap = plan.cap;
+        es.theta = sc.theta;
+        es.thf = sc.thf;
+        es.tickets = sc.flags + 4;
+        if ((e = launch_estimate(es, s)) != cudaSuccess) return cuda_fail(e, "threshold estimate");
+    }
+    for (int lv = plan.sampled ? 0 : plan.levels - 1; lv >= 0; --lv) {
         if ((st = run_pass(index, pc, plan, lv, sc, exclude_bits, inv_tau, b, s, sms)) != TT_OK) return st;
         if (lv > 0) {
             e = launch_select_threshold(sc.keys, sc.count, plan.cap, V, plan.rank[lv], sc.theta,

@@ -45,6 +45,41 @@ struct PassArgs {
     const uint64_t* theta_v;   // [n_sets * b]
 };
 
+// Launch `kernel` with programmatic stream serialization: it may start while
+// the stream's previous kernel still runs (the kernel then orders its memory
+// accesses with pdl_wait(), see tt_device.cuh).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
+// The scan plan of a search (tt_api.cu). Level i scans every stride[i]-th
+// row; rank[i] (i >= 1): the r-th best key of level i, minus one, is the
+// filter threshold of level i - 1. A sampled plan (small batches on the
+// streaming scorer: small_batch) has two levels, and its level 1 is scored
+// and reduced to the threshold by one launch (launch_estimate).
+constexpr int MAX_LEVELS = 4;
+struct Plan {
+    int levels;
+    int64_t stride[MAX_LEVELS];
+    int64_t rows[MAX_LEVELS];
+    int rank[MAX_LEVELS];
+    int cap;
+    bool sampled;
+};
+tt_status make_plan(int64_t n, int32_t k, const tt_options* opt, bool small_batch, Plan* p);
+
 // Set the text tt_last_error() returns on the calling thread.
 void set_last_error_message(const char* msg);
 
@@ -64,15 +99,45 @@ cudaError_t launch_stream_pass(const PassArgs& a, cudaStream_t s, int sm_count);
 cudaError_t launch_tensor_pass(const PassArgs& a, const CUtensorMap& tm_rows,
                                const CUtensorMap& tm_queries, int nq_tile, cudaStream_t s,
                                int sm_count);
-// Tensor-core pass on SM pairs (b >= 1, bf16 queries in tiles of 256, d a
-// multiple of 64; tm_rows with boxes of tensor_pair_box_rows(d) rows).
+// Tensor-core pass on SM pairs (b >= 1, bf16 queries in tiles of 256;
+// tm_rows with boxes of tensor_pair_box_rows(d) rows).
 cudaError_t launch_tensor_pair_pass(const PassArgs& a, const CUtensorMap& tm_rows, cudaStream_t s,
                                     int sm_count);
 int tensor_pair_box_rows(int d);
 // count[0..b) = 0; theta/thf[0..b) = theta_value; [b, b_pad) = KEY_MAX / +inf;
-// flags[0..2) = 0.
+// flags[0..16) = 0 (flagged lists, error word, estimate tickets).
 cudaError_t launch_init(uint32_t* count, uint64_t* theta, float* thf, uint64_t theta_value, int b,
                         int b_pad, int* flags, cudaStream_t s);
+// The threshold of a small batch from one sample of the corpus, in one
+// launch (k_estimate.cu): level row j = corpus row j * stride (j < n_sample)
+// is scored for every query with the streaming scorer's arithmetic; blocks of
+// 256 sample rows keep their best `rank` keys per query (in keys[q * cap...]),
+// and the last block of each query sets theta[q] = (rank-th best key) - 1, or
+// KEY_MIN when fewer were eligible. tickets: [b] counters, zero on entry.
+struct EstimateArgs {
+    const void* rows;
+    int dtype;
+    int d;
+    const float* inv_norm;
+    const uint32_t* exclude;
+    float inv_tau;
+    const void* queries;  // as the streaming pass reads them (int8: codes)
+    int q_dtype;
+    const float* qscale;  // int8: query scales
+    int b;
+    int64_t stride;
+    int64_t n_sample;
+    int rank;
+    uint64_t* keys;       // work keys [b * cap]; blocks' lists at keys[q * cap + g * rank]
+    int cap;
+    uint64_t* theta;
+    float* thf;
+    int* tickets;
+};
+constexpr int ESTIMATE_BLOCK_ROWS = 256;  // sample rows per block: one per thread
+constexpr int ESTIMATE_MAX_RANK = 256;    // the sample rank a plan may ask of the estimate
+cudaError_t launch_estimate(const EstimateArgs& a, cudaStream_t s);
+
 // Threshold mode: theta_next[q] = (r-th best kept key) - 1, or KEY_MIN when
 // fewer than r keys were kept; counts reset to 0.
 cudaError_t launch_select_threshold(const uint64_t* keys, uint32_t* count, int cap, int b, int r,
@@ -87,12 +152,14 @@ cudaError_t launch_select_final(const uint64_t* keys, uint32_t* count, int cap, 
 
 // Written by the device at the end of every search (host-mapped memory of an
 // index handle): the error code of an expired device wait (only written when
-// there is one; the host clears it once reported), the number of lists the
-// exact fallback recomputed, and the sequence number of the call.
+// there is one; the host clears it once reported), and the number of lists the
+// exact fallback recomputed with the sequence number of the call.
 struct HostStatus {
     volatile int32_t err;
-    volatile int32_t repaired;
-    volatile int64_t seq;
+    int32_t reserved;
+    // low 32 bits of the call's sequence number << 32 | lists recomputed, in
+    // one store (the host can never see one half of it without the other)
+    volatile uint64_t seq_repaired;
 };
 
 // The exact fallback scan (k_exact.cu), launched at the end of every search.

@@ -114,12 +114,12 @@ tt_status tt_score_topk_noalloc(const void* rows, tt_dtype dtype, int64_t n, int
         (uintptr_t)out_scores % 4 || (uintptr_t)exclude_bits % 4 || (uintptr_t)inv_norm % 4)
         return TT_ERR_INVALID_ARG;
     if (dtype == TT_F32 && d > 256) return TT_ERR_UNSUPPORTED;
-    int32_t levels = 0, cap = 0, ranks[4] = {0};
-    int64_t lrows[4] = {0}, lstride[4] = {0};
-    tt_status st = tt_plan(n, k, nullptr, &levels, lrows, lstride, ranks, &cap);
-    if (st != TT_OK) return st;
     const bool tc_possible = dtype == TT_BF16 && d >= 64 && tensor_pass_max_nq(d, 2) > 0;
     const int path = (tc_possible && b > 8) ? 2 : 1;
+    Plan plan;
+    tt_status st = make_plan(n, k, nullptr, path == 1 && b <= 8, &plan);
+    if (st != TT_OK) return st;
+    const int cap = plan.cap;
     int nq = 0, q_tiles = 1;
     if (path == 2) {
         const int max_nq = tensor_pass_max_nq(d, 2);
@@ -208,8 +208,8 @@ tt_status tt_score_topk_noalloc(const void* rows, tt_dtype dtype, int64_t n, int
         memset(&a, 0, sizeof a);
         a.rows = rows;
         a.dtype = dtype;
-        a.n_rows = lrows[lv];
-        a.stride = lstride[lv];
+        a.n_rows = plan.rows[lv];
+        a.stride = plan.stride[lv];
         a.d = d;
         a.inv_norm = inv_norm;
         a.exclude = exclude_bits;
@@ -236,10 +236,33 @@ tt_status tt_score_topk_noalloc(const void* rows, tt_dtype dtype, int64_t n, int
     // flags are reset first, in the stream, before anything reads them.
     e = launch_init(count, theta, thf, KEY_MIN, b, b_pad, flags, s);
     if (e != cudaSuccess) return launch_failed("init", e);
-    for (int lv = levels - 1; lv >= 0; --lv) {
+    if (plan.sampled) {
+        EstimateArgs es;
+        memset(&es, 0, sizeof es);
+        es.rows = rows;
+        es.dtype = dtype;
+        es.d = d;
+        es.inv_norm = inv_norm;
+        es.exclude = exclude_bits;
+        es.inv_tau = inv_tau;
+        es.queries = q_use;
+        es.q_dtype = q_dt_use;
+        es.b = b;
+        es.stride = plan.stride[1];
+        es.n_sample = plan.rows[1];
+        es.rank = plan.rank[1];
+        es.keys = keys;
+        es.cap = cap;
+        es.theta = theta;
+        es.thf = thf;
+        es.tickets = flags + 4;
+        e = launch_estimate(es, s);
+        if (e != cudaSuccess) return launch_failed("threshold estimate", e);
+    }
+    for (int lv = plan.sampled ? 0 : plan.levels - 1; lv >= 0; --lv) {
         e = pass(lv);
         if (e != cudaSuccess) return launch_failed("scoring pass", e);
-        e = lv > 0 ? launch_select_threshold(keys, count, cap, b, ranks[lv], theta, thf, s)
+        e = lv > 0 ? launch_select_threshold(keys, count, cap, b, plan.rank[lv], theta, thf, s)
                    : launch_select_final(keys, count, cap, b, k, theta, thf, flagged, flags, out_ids,
                                          out_scores, s);
         if (e != cudaSuccess) return launch_failed("select", e);

@@ -1,7 +1,9 @@
 // tt_select.cuh - block-wide selection over 64-bit candidate keys, shared
 // by the select kernels (K4) and the exact fallback scan.
 //
-// One CTA of K4_THREADS threads works on one list of distinct keys. The r-th
+// One CTA of K4_THREADS threads works on one list of distinct keys. For
+// r <= K4_TOP_MAX the best r keys are kept sorted in registers (bitonic
+// networks, below). For larger r the r-th
 // largest key is found by a most-significant-digit radix select (digits of
 // 11/11/10/11/11/10 bits, a 2048-bin shared-memory histogram per digit)
 // until at most K4_THREADS keys share the selected prefix; those are ranked
@@ -43,31 +45,266 @@ __device__ __forceinline__ const uint64_t* stage_keys(const uint64_t* __restrict
     return sm.keys;
 }
 
+// ---------------------------------------------------------------------------
+// Top-r in registers (r <= K4_TOP_MAX). A warp holds 32 * KPL keys, element
+// e = lane * KPL + j in register j of its lane. Bitonic networks (Batcher's
+// sorting network) sort such a list with compare-exchanges inside a lane's
+// registers (partner distance below KPL) or across lanes through shuffles.
+// Two lists A and B sorted descending give the best 32 * KPL keys of their
+// union as max(A[e], B[N - 1 - e]), a bitonic sequence that one cleaning
+// cascade sorts. Every warp folds its chunks of the input into its own list
+// this way; the warps' lists are then folded pairwise through shared memory.
+// No shared-memory atomics and log2(8) block barriers, whatever the keys.
+// ---------------------------------------------------------------------------
+constexpr int K4_TOP_MAX = 256;
+
+// One compare-exchange step of a bitonic network over the warp's list:
+// elements e and e ^ D (D < KPL: both in this lane's registers), the larger
+// first where (e & size) == 0.
+template <int KPL, int D>
+__device__ __forceinline__ void bitonic_in_lane(uint64_t (&v)[KPL], int size) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+        if (j & D) continue;
+        const bool desc = ((lane * KPL + j) & size) == 0;
+        const uint64_t x = v[j], y = v[j | D];
+        const bool swap = desc ? x < y : x > y;
+        v[j] = swap ? y : x;
+        v[j | D] = swap ? x : y;
+    }
+}
+
+// The same step for d >= KPL: the partner element sits in register j of lane
+// lane ^ (d / KPL).
+template <int KPL>
+__device__ __forceinline__ void bitonic_across(uint64_t (&v)[KPL], int size, int d) {
+    const int lane = threadIdx.x & 31;
+    const int ld = d / KPL;
+    const bool lower = (lane & ld) == 0;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+        const uint64_t o = __shfl_xor_sync(0xFFFFFFFFu, v[j], ld);
+        const bool desc = ((lane * KPL + j) & size) == 0;
+        const uint64_t hi = v[j] > o ? v[j] : o, lo = v[j] > o ? o : v[j];
+        v[j] = desc == lower ? hi : lo;
+    }
+}
+
+template <int KPL>
+__device__ __forceinline__ void warp_bitonic_step(uint64_t (&v)[KPL], int size, int d) {
+    if (d >= KPL)
+        bitonic_across<KPL>(v, size, d);
+    else if (d == 1)
+        bitonic_in_lane<KPL, 1>(v, size);
+    else if (d == 2)
+        bitonic_in_lane<KPL, (KPL > 2 ? 2 : 1)>(v, size);  // (d == 2 only when KPL > 2)
+    else
+        bitonic_in_lane<KPL, (KPL > 4 ? 4 : 1)>(v, size);  // (d == 4 only when KPL > 4)
+}
+
+// The loops over the network's stages stay rolled: these kernels run once per
+// search on a few SMs, often with their code evicted from L2, and a fully
+// unrolled network is tens of KB of straight-line code to fetch.
+
+// Sort the warp's 32 * KPL keys descending.
+template <int KPL>
+__device__ __forceinline__ void warp_sort_list(uint64_t (&v)[KPL]) {
+#pragma unroll 1
+    for (int size = 2; size <= 32 * KPL; size <<= 1) {
+#pragma unroll 1
+        for (int d = size >> 1; d > 0; d >>= 1) warp_bitonic_step<KPL>(v, size, d);
+    }
+}
+
+// a <- the best 32 * KPL keys of a and b (both sorted descending), sorted descending.
+template <int KPL>
+__device__ __forceinline__ void warp_fold_list(uint64_t (&a)[KPL], const uint64_t (&b)[KPL]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) {
+        const uint64_t o = __shfl_sync(0xFFFFFFFFu, b[KPL - 1 - j], 31 - lane);  // b[N - 1 - e]
+        a[j] = a[j] > o ? a[j] : o;
+    }
+#pragma unroll 1
+    for (int d = 16 * KPL; d > 0; d >>= 1) warp_bitonic_step<KPL>(a, 64 * KPL, d);  // all descending
+}
+
+template <int KPL>
+__device__ __noinline__ void block_top_sorted_impl(const uint64_t* keys, int n, K4Smem& sm) {
+    constexpr int N = 32 * KPL;
+    constexpr int W = K4_THREADS / 32;
+    static_assert(W * N <= K4_SORT_MAX, "the warps' lists are folded in sm.sorted");
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint64_t a[KPL];
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) a[j] = KEY_MIN;
+    for (int base = warp * N; base < n; base += W * N) {
+        uint64_t b[KPL];
+        bool any = false;
+        const uint64_t least = __shfl_sync(0xFFFFFFFFu, a[KPL - 1], 31);  // the list's last key
+#pragma unroll
+        for (int j = 0; j < KPL; ++j) {
+            const int i = base + j * 32 + lane;  // coalesced; the order within a chunk is irrelevant
+            b[j] = i < n ? keys[i] : KEY_MIN;
+            any |= b[j] > least;
+        }
+        if (!__any_sync(0xFFFFFFFFu, any)) continue;  // nothing here enters the list
+        warp_sort_list<KPL>(b);
+        warp_fold_list<KPL>(a, b);
+    }
+    __syncthreads();  // callers may still read sm.sorted before this call
+#pragma unroll
+    for (int j = 0; j < KPL; ++j) sm.sorted[warp * N + lane * KPL + j] = a[j];
+    __syncthreads();
+#pragma unroll
+    for (int half = W / 2; half >= 1; half >>= 1) {
+        if (warp < half) {
+            uint64_t b[KPL];
+#pragma unroll
+            for (int j = 0; j < KPL; ++j) b[j] = sm.sorted[(warp + half) * N + lane * KPL + j];
+            warp_fold_list<KPL>(a, b);
+#pragma unroll
+            for (int j = 0; j < KPL; ++j) sm.sorted[warp * N + lane * KPL + j] = a[j];
+        }
+        __syncthreads();
+    }
+}
+
+// The min(r, n) largest of n keys, sorted descending, in sm.sorted[0 .. r)
+// (KEY_MIN past the n-th); 1 <= r <= K4_TOP_MAX. Block-wide.
+__device__ inline void block_top_sorted(const uint64_t* keys, int n, int r, K4Smem& sm) {
+    if (r <= 32)
+        block_top_sorted_impl<1>(keys, n, sm);
+    else if (r <= 64)
+        block_top_sorted_impl<2>(keys, n, sm);
+    else if (r <= 128)
+        block_top_sorted_impl<4>(keys, n, sm);
+    else
+        block_top_sorted_impl<8>(keys, n, sm);
+}
+
+// Keys with this prefix, appended to sm.sorted (warp-aggregated: one
+// shared-memory atomic per warp and pass). Block-wide; returns their number.
+__device__ __forceinline__ uint32_t gather_prefix(const uint64_t* keys, int n, uint64_t mask, uint64_t prefix,
+                                                  K4Smem& sm) {
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) sm.n_collected = 0;
+    __syncthreads();
+    for (int base = 0; base < n; base += K4_THREADS) {
+        const int i = base + threadIdx.x;
+        uint64_t key = 0;
+        bool in = false;
+        if (i < n) {
+            key = keys[i];
+            in = (key & mask) == prefix;
+        }
+        const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, in);
+        if (ballot) {
+            const int leader = __ffs(ballot) - 1;
+            uint32_t slot0 = 0;
+            if (lane == leader) slot0 = atomicAdd(&sm.n_collected, (uint32_t)__popc(ballot));
+            slot0 = __shfl_sync(0xFFFFFFFFu, slot0, leader);
+            if (in) sm.sorted[slot0 + __popc(ballot & lanemask_lt())] = key;
+        }
+    }
+    __syncthreads();
+    return sm.n_collected;
+}
+
+// r-th largest of the `count` keys in sm.sorted (1-based, counting repeats),
+// by counting; count <= K4_THREADS. Block-wide.
+__device__ __forceinline__ uint64_t rank_select(uint32_t count, uint32_t r, K4Smem& sm) {
+    const int tid = threadIdx.x;
+    if (tid < (int)count) {
+        const uint64_t mine = sm.sorted[tid];
+        uint32_t above_me = 0, equal = 0;
+        for (uint32_t j = 0; j < count; ++j) {
+            above_me += sm.sorted[j] > mine;
+            equal += sm.sorted[j] == mine;
+        }
+        if (above_me < r && r <= above_me + equal) sm.result = mine;
+    }
+    __syncthreads();
+    const uint64_t res = sm.result;
+    __syncthreads();  // callers may reuse sm.sorted and sm.result at once
+    return res;
+}
+
 // r-th largest (1-based, counting repeats) of n keys; 1 <= r <= n. Block-wide.
-// Radix passes narrow the candidates to a digit prefix; once at most
-// K4_THREADS keys share the prefix they are gathered and ranked directly.
+// Lists of at most K4_THREADS keys are ranked directly. Otherwise the bits
+// all keys share (from the block's minimum and maximum) are skipped, and
+// radix passes over the remaining bits, most significant digit first (11 bits
+// at a time, a 2048-bin shared-memory histogram), narrow the candidates to a
+// prefix until at most K4_THREADS keys share it; those are ranked directly.
+// Kept keys cluster (they are the best scores of one query), so histogram
+// increments are combined per warp for lanes that hit the same bin.
 __device__ inline uint64_t block_kth_largest(const uint64_t* keys, int n, int r, K4Smem& sm) {
     const int tid = threadIdx.x;
-    // digits, most significant first: widths 11, 11, 10, 11, 11, 10
-    uint64_t prefix = 0, mask = 0;
+    const int lane = tid & 31, warp = tid >> 5;
+    if (r <= K4_TOP_MAX) {
+        block_top_sorted(keys, n, r, sm);
+        const uint64_t res = sm.sorted[r - 1];
+        __syncthreads();  // callers may reuse sm.sorted at once
+        return res;
+    }
+    if (n <= K4_THREADS) return rank_select(gather_prefix(keys, n, 0ull, 0ull, sm), (uint32_t)r, sm);
+    // bits common to every key
+    uint64_t lo = ~0ull, hi = 0ull;
+    for (int i = tid; i < n; i += K4_THREADS) {
+        const uint64_t key = keys[i];
+        lo = key < lo ? key : lo;
+        hi = key > hi ? key : hi;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const uint64_t l2 = __shfl_xor_sync(0xFFFFFFFFu, lo, off), h2 = __shfl_xor_sync(0xFFFFFFFFu, hi, off);
+        lo = l2 < lo ? l2 : lo;
+        hi = h2 > hi ? h2 : hi;
+    }
+    if (lane == 0) {
+        sm.sorted[warp] = lo;
+        sm.sorted[K4_THREADS / 32 + warp] = hi;
+    }
+    __syncthreads();
+    lo = sm.sorted[0];
+    hi = sm.sorted[K4_THREADS / 32];
+    for (int w = 1; w < K4_THREADS / 32; ++w) {
+        lo = sm.sorted[w] < lo ? sm.sorted[w] : lo;
+        hi = sm.sorted[K4_THREADS / 32 + w] > hi ? sm.sorted[K4_THREADS / 32 + w] : hi;
+    }
+    __syncthreads();
+    if (lo == hi) return lo;  // every key equal
+    int shift = 64 - __clzll((long long)(lo ^ hi));  // bits [shift, 64) are common
+    uint64_t mask = shift >= 64 ? 0ull : ~((1ull << shift) - 1ull);
+    uint64_t prefix = hi & mask;
     uint32_t remaining = (uint32_t)r;
-    int shift = 64;
 #pragma unroll 1
-    for (int pass = 0; pass < 6; ++pass) {
-        const int w = (pass == 2 || pass == 5) ? 10 : 11;
+    while (shift > 0) {
+        const int w = shift >= 11 ? 11 : shift;
         shift -= w;
         const int nb = 1 << w;
+        const int per = (nb + K4_THREADS - 1) / K4_THREADS;  // bins thread t sums: [t*per, t*per + per)
         for (int i = tid; i < nb; i += K4_THREADS) sm.hist[i] = 0;
         __syncthreads();
-        for (int i = tid; i < n; i += K4_THREADS) {
-            const uint64_t key = keys[i];
-            if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & (uint64_t)(nb - 1)], 1u);
+        for (int base = 0; base < n; base += K4_THREADS) {
+            const int i = base + tid;
+            bool in = false;
+            uint32_t bin = 0;
+            if (i < n) {
+                const uint64_t key = keys[i];
+                in = (key & mask) == prefix;
+                bin = (uint32_t)(key >> shift) & (uint32_t)(nb - 1);
+            }
+            // lanes outside the prefix get tags no other lane has
+            const uint32_t peers = __match_any_sync(0xFFFFFFFFu, in ? bin : (0x80000000u | (uint32_t)lane));
+            if (in && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[bin], (uint32_t)__popc(peers));
         }
         __syncthreads();
         // Thread t owns bins [t*per, (t+1)*per); above[t] = count in higher bins.
-        const int per = nb / K4_THREADS;
         uint32_t local = 0;
-        for (int i = 0; i < per; ++i) local += sm.hist[tid * per + i];
+        for (int i = 0; i < per; ++i)
+            if (tid * per + i < nb) local += sm.hist[tid * per + i];
         sm.part[tid] = local;
         __syncthreads();
         if (tid < 32) {
@@ -88,9 +325,10 @@ __device__ inline uint64_t block_kth_largest(const uint64_t* keys, int n, int r,
         }
         __syncthreads();
         const uint32_t above = sm.above[tid];
-        if (above < remaining && remaining <= above + local) {
+        if (local > 0 && above < remaining && remaining <= above + local) {
             uint32_t run = above;
             for (int i = per - 1; i >= 0; --i) {
+                if (tid * per + i >= nb) continue;
                 const uint32_t c = sm.hist[tid * per + i];
                 if (remaining <= run + c) {
                     sm.found_prefix = (uint64_t)(tid * per + i);
@@ -107,29 +345,38 @@ __device__ inline uint64_t block_kth_largest(const uint64_t* keys, int n, int r,
         remaining = sm.found_remaining;
         const uint32_t count = sm.found_count;
         __syncthreads();
-        if (count <= (uint32_t)K4_THREADS) {
-            // gather the keys with this prefix and rank them by counting
-            if (tid == 0) sm.n_collected = 0;
-            __syncthreads();
-            for (int i = tid; i < n; i += K4_THREADS) {
-                const uint64_t key = keys[i];
-                if ((key & mask) == prefix) sm.sorted[atomicAdd(&sm.n_collected, 1u)] = key;
-            }
-            __syncthreads();
-            if (tid < (int)count) {
-                const uint64_t mine = sm.sorted[tid];
-                uint32_t above_me = 0, equal = 0;
-                for (uint32_t j = 0; j < count; ++j) {
-                    above_me += sm.sorted[j] > mine;
-                    equal += sm.sorted[j] == mine;
-                }
-                if (above_me < remaining && remaining <= above_me + equal) sm.result = mine;
-            }
-            __syncthreads();
-            return sm.result;
-        }
+        if (count <= (uint32_t)K4_THREADS) return rank_select(gather_prefix(keys, n, mask, prefix, sm), remaining, sm);
     }
     return prefix;
+}
+
+// Keys greater than `th`, appended to sm.sorted (warp-aggregated), at most
+// `limit` of them stored. Block-wide; returns their number (may exceed limit).
+__device__ __forceinline__ uint32_t gather_above(const uint64_t* keys, int n, uint64_t th, uint32_t limit,
+                                                 K4Smem& sm) {
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) sm.n_collected = 0;
+    __syncthreads();
+    for (int base = 0; base < n; base += K4_THREADS) {
+        const int i = base + threadIdx.x;
+        uint64_t key = 0;
+        bool in = false;
+        if (i < n) {
+            key = keys[i];
+            in = key > th;
+        }
+        const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, in);
+        if (ballot) {
+            const int leader = __ffs(ballot) - 1;
+            uint32_t slot0 = 0;
+            if (lane == leader) slot0 = atomicAdd(&sm.n_collected, (uint32_t)__popc(ballot));
+            slot0 = __shfl_sync(0xFFFFFFFFu, slot0, leader);
+            const uint32_t slot = slot0 + __popc(ballot & lanemask_lt());
+            if (in && slot < limit) sm.sorted[slot] = key;
+        }
+    }
+    __syncthreads();
+    return sm.n_collected;
 }
 
 // The min(n_valid, k) largest of n keys, sorted descending, written as
@@ -140,55 +387,65 @@ __device__ inline void write_sorted_topk(const uint64_t* keys, int n, int n_vali
                                          int32_t* out_ids, float* out_scores) {
     const int tid = threadIdx.x;
     const int r = n_valid < k ? n_valid : k;
-    if (r > 0) {
-        const uint64_t kth = block_kth_largest(keys, n, r, sm);
-        if (tid == 0) sm.n_collected = 0;
-        __syncthreads();
-        // fewer than r keys are above the r-th largest; the rest of the r
-        // slots hold it (one copy when keys are distinct)
-        for (int i = tid; i < n; i += K4_THREADS) {
-            const uint64_t key = keys[i];
-            if (key > kth) {
-                const uint32_t slot = atomicAdd(&sm.n_collected, 1u);
-                if (slot < (uint32_t)r) sm.sorted[slot] = key;
-            }
+    for (int i = r + tid; i < k; i += K4_THREADS) {
+        out_ids[i] = -1;
+        out_scores[i] = -INFINITY;
+    }
+    if (r == 0) return;
+    if (r <= K4_TOP_MAX) {
+        block_top_sorted(keys, n, r, sm);
+        for (int i = tid; i < r; i += K4_THREADS) {
+            out_ids[i] = (int32_t)key_id(sm.sorted[i]);
+            out_scores[i] = key_score(sm.sorted[i]);
         }
         __syncthreads();
-        const int above = (int)sm.n_collected < r ? (int)sm.n_collected : r;
-        for (int i = above + tid; i < r; i += K4_THREADS) sm.sorted[i] = kth;
+        return;
+    }
+    const uint64_t kth = block_kth_largest(keys, n, r, sm);
+    // the r best: the keys above the r-th largest (r - 1 of them when keys
+    // are distinct), then the r-th largest in the remaining slots
+    uint32_t above = gather_above(keys, n, kth, (uint32_t)r, sm);
+    if (above > (uint32_t)r) above = (uint32_t)r;
+    for (int i = (int)above + tid; i < r; i += K4_THREADS) sm.sorted[i] = kth;
+    __syncthreads();
+    if (r <= 2 * K4_THREADS) {
+        // sort by rank: a key's place is the number of keys above it
+        for (int i = tid; i < r; i += K4_THREADS) {
+            const uint64_t mine = sm.sorted[i];
+            int place = 0;
+            for (int j = 0; j < r; ++j) place += sm.sorted[j] > mine || (sm.sorted[j] == mine && j < i);
+            out_ids[place] = (int32_t)key_id(mine);
+            out_scores[place] = key_score(mine);
+        }
         __syncthreads();
-        int P = 1;
-        while (P < r) P <<= 1;
-        for (int i = r + tid; i < P; i += K4_THREADS) sm.sorted[i] = KEY_MIN;
-        __syncthreads();
-        // bitonic sort, descending
-        for (int size = 2; size <= P; size <<= 1) {
-            for (int stride = size >> 1; stride > 0; stride >>= 1) {
-                for (int i = tid; i < P; i += K4_THREADS) {
-                    const int j = i ^ stride;
-                    if (j > i) {
-                        const uint64_t x = sm.sorted[i], y = sm.sorted[j];
-                        const bool desc = (i & size) == 0;
-                        if (desc ? (x < y) : (x > y)) {
-                            sm.sorted[i] = y;
-                            sm.sorted[j] = x;
-                        }
+        return;
+    }
+    int P = 1;
+    while (P < r) P <<= 1;
+    for (int i = r + tid; i < P; i += K4_THREADS) sm.sorted[i] = KEY_MIN;
+    __syncthreads();
+    // bitonic sort, descending
+    for (int size = 2; size <= P; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int i = tid; i < P; i += K4_THREADS) {
+                const int j = i ^ stride;
+                if (j > i) {
+                    const uint64_t x = sm.sorted[i], y = sm.sorted[j];
+                    const bool desc = (i & size) == 0;
+                    if (desc ? (x < y) : (x > y)) {
+                        sm.sorted[i] = y;
+                        sm.sorted[j] = x;
                     }
                 }
-                __syncthreads();
             }
+            __syncthreads();
         }
     }
-    for (int i = tid; i < k; i += K4_THREADS) {
-        int32_t id = -1;
-        float sc = -INFINITY;
-        if (i < r) {
-            id = (int32_t)key_id(sm.sorted[i]);
-            sc = key_score(sm.sorted[i]);
-        }
-        out_ids[i] = id;
-        out_scores[i] = sc;
+    for (int i = tid; i < r; i += K4_THREADS) {
+        out_ids[i] = (int32_t)key_id(sm.sorted[i]);
+        out_scores[i] = key_score(sm.sorted[i]);
     }
+    __syncthreads();
 }
 
 }  // namespace tt

@@ -230,7 +230,9 @@ typedef struct tt_stats {
     int64_t level_rows[4];   /* rows scanned per level, finest first */
     int64_t level_stride[4]; /* corpus-row stride per level */
     int32_t cap;             /* candidate buffer per query */
-    int32_t reserved;
+    int32_t sampled;         /* 1: level 1 is a one-launch sample estimate of the
+                                threshold (small batches on the streaming scorer),
+                                not a filtered pass; 0 otherwise */
 } tt_stats;
 
 TT_API tt_status tt_last_stats(const tt_index* index, tt_stats* out);
@@ -466,8 +468,9 @@ TT_API tt_status tt_score_topk_noalloc(const void* rows, tt_dtype dtype, int64_t
 #define TT_KIND_TENSOR 3
 #define TT_KIND_SELECT 4
 #define TT_KIND_AUX 5
-#define TT_KIND_SOFTMAX 6 /* tt_inbatch_softmax */
-#define TT_NUM_KINDS 7
+#define TT_KIND_SOFTMAX 6  /* tt_inbatch_softmax */
+#define TT_KIND_ESTIMATE 7 /* the sampled threshold estimate of a small batch */
+#define TT_NUM_KINDS 8
 
 /* Total kernels this library has launched in the process. */
 TT_API int64_t tt_launch_count(void);

@@ -345,3 +345,54 @@ def test_rejects_host_pointers_and_bad_args():
     with pytest.raises(tt.TTError) as e:
         tt.tt_score_topk(index, q, 4096)
     assert e.value.status == tt.TT_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("name,over,opts", [
+    ("stream_b1", {"n": 300_007, "k": 100}, {}),
+    ("stream_b1", {"n": 250_013, "b": 6, "k": 333}, {}),
+    ("masked_fused", {"n": 180_017, "b": 2, "k": 64, "oracle_queries": 0}, {}),
+    ("stream_b1", {"n": 200_003, "b": 3, "k": 100}, {"rank_scale_pct": 3}),
+])
+def test_sampled_plan_small_batches(name, over, opts):
+    """A few queries on the streaming scorer: one sample of the corpus sets
+    the threshold in one launch (a two-level plan whose level 1 is every S-th
+    row, S odd). The result matches the oracle; with the rank scaled down the
+    filter keeps too few candidates and the exact fallback restores the
+    answer."""
+    _cuda()
+    w = W.workload(name, **over)
+    res, st = parity.run_case(w, **opts)
+    assert st["path"] == 1 and st["levels"] == 2 and st["sampled"], st
+    stride = st["level_stride"][1]
+    assert stride % 2 == 1 and st["level_rows"][1] == -(-w.n // stride)
+    assert res["max_abs_err"] <= w.tolerance
+    if opts:
+        assert st["rescans"] >= 1, st
+    else:
+        assert st["rescans"] == 0, st
+
+
+def test_sampled_plan_int8_and_f32_rows():
+    """The sample is scored with each row type's own arithmetic."""
+    _cuda()
+    w = W.workload("stream_b1", n=120_011, b=4, k=50)
+    res, st = parity.run_case_q8(w)
+    assert st["path"] == 1 and st["levels"] == 2 and st["rescans"] == 0, st
+    w = W.workload("tiny_f32", n=90_001, d=64, b=3, k=40, oracle_queries=0)
+    res, st = parity.run_case(w)
+    assert st["path"] == 1 and st["levels"] == 2 and st["rescans"] == 0, st
+    assert res["max_abs_err"] <= w.tolerance
+
+
+@pytest.mark.parametrize("k", [1, 31, 32, 33, 64, 65, 128, 129, 256, 257])
+@pytest.mark.parametrize("path,b", [(1, 2), (2, 24), (3, 256)])
+def test_select_widths(path, b, k):
+    """The selects keep the best r <= 256 keys sorted in registers, 32, 64,
+    128 or 256 per warp, and use the radix select above that; k on both sides
+    of each width, on every scorer (on the streaming scorer the sample
+    estimate's rank varies with k too)."""
+    _cuda()
+    w = W.workload("small_batch", n=60_013, b=b, k=k, tau=1.0, oracle_queries=6)
+    res, st = parity.run_case(w, path=path)
+    assert st["path"] == path and st["rescans"] == 0, st
+    assert res["max_abs_err"] <= w.tolerance and res["set_checked"] + res["rank_checked"] > 0, res
