@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(KE_THREADS) k2_estimate(const EstimateArgs a) 
     __syncthreads();
     // this block's best R keys, sorted (KEY_MIN past the block's eligible rows)
     uint64_t* out = a.keys + (int64_t)q * a.cap + (int64_t)g * R;
-    block_top_sorted(sm.keys, KE_ROWS, R, sm);
+    block_top(sm.keys, KE_ROWS, R, sm);  // R <= K4_TOP_MAX: always decides
     for (int i = tid; i < R; i += KE_THREADS) out[i] = sm.sorted[i];
     __threadfence();
     __syncthreads();
@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(KE_THREADS) k2_estimate(const EstimateArgs a) 
     const int m = G * R;
     for (int i = tid; i < m; i += KE_THREADS) sm.keys[i] = __ldcg(lk + i);
     __syncthreads();
-    block_top_sorted(sm.keys, m, R, sm);
+    block_top(sm.keys, m, R, sm);
     const uint64_t kth = sm.sorted[R - 1];  // KEY_MIN when fewer than R rows were eligible
     const uint64_t th = kth == KEY_MIN ? KEY_MIN : kth - 1;
     if (tid == 0) {

@@ -1,9 +1,10 @@
 // tt_select.cuh - block-wide selection over 64-bit candidate keys, shared
 // by the select kernels (K4) and the exact fallback scan.
 //
-// One CTA of K4_THREADS threads works on one list of distinct keys. For
-// r <= K4_TOP_MAX the best r keys are kept sorted in registers (bitonic
-// networks, below). For larger r the r-th
+// One CTA of K4_THREADS threads works on one list of distinct keys. Up to
+// 4096 keys and r <= 512: a bucket select over linear score bins (below);
+// where that cannot decide, for r <= K4_TOP_MAX, the best r keys kept sorted
+// in registers (bitonic networks, below). Otherwise the r-th
 // largest key is found by a most-significant-digit radix select (digits of
 // 11/11/10/11/11/10 bits, a 2048-bin shared-memory histogram per digit)
 // until at most K4_THREADS keys share the selected prefix; those are ranked
@@ -184,6 +185,149 @@ __device__ inline void block_top_sorted(const uint64_t* keys, int n, int r, K4Sm
         block_top_sorted_impl<8>(keys, n, sm);
 }
 
+// ---------------------------------------------------------------------------
+// Bucket select (n <= K4_BUCKET_N keys, r <= K4_BUCKET_R): the keys stay in
+// registers (K4_BUCKET_PT per thread); the score part of each key, ord(score),
+// is binned linearly over the block's own [min, max] range into K4_BINS bins
+// (a monotone map, so a higher bin holds only greater keys). One histogram, a
+// suffix scan over the bins and the boundary bin B (the bin holding the r-th
+// best key) give every candidate (bin >= B) its place: the keys in higher
+// bins, plus the keys of its own bin that beat it. Six block barriers; the
+// only comparisons are within a bin. Gives up (returns false, before writing
+// any output) when the boundary bin or the candidate set is too large to rank
+// this way, e.g. many equal scores.
+// ---------------------------------------------------------------------------
+constexpr int K4_BUCKET_PT = 16;
+constexpr int K4_BUCKET_N = K4_BUCKET_PT * K4_THREADS;  // 4096
+constexpr int K4_BUCKET_R = 512;
+constexpr int K4_BUCKET_M = 1024;          // candidates, held in sm.sorted[1024 ..)
+constexpr int K4_BUCKET_BIN_MAX = 256;     // keys in the boundary bin
+static_assert(K4_BINS == 8 * K4_THREADS, "each thread owns eight bins in the scan");
+static_assert(K4_BUCKET_R + K4_BUCKET_M <= K4_SORT_MAX, "outputs and candidates share sm.sorted");
+
+__device__ __forceinline__ uint32_t bucket_of(uint64_t key, uint32_t lo, float scale) {
+    const uint32_t b = (uint32_t)((float)((uint32_t)(key >> 32) - lo) * scale);
+    return b < (uint32_t)K4_BINS ? b : (uint32_t)K4_BINS - 1;
+}
+
+// The best min(r, valid) keys sorted descending in sm.sorted[0 .. r), KEY_MIN
+// after them (KEY_MIN entries of the input are not keys). Block-wide; every
+// thread gets the same return value.
+__device__ inline bool block_top_bucket(const uint64_t* keys, int n, int r, K4Smem& sm) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int W = K4_THREADS / 32;
+    uint64_t kv[K4_BUCKET_PT];
+    uint32_t lo = 0xFFFFFFFFu, hi = 0, valid = 0;
+#pragma unroll
+    for (int j = 0; j < K4_BUCKET_PT; ++j) {
+        const int i = tid + j * K4_THREADS;
+        kv[j] = i < n ? keys[i] : KEY_MIN;
+        if (kv[j] != KEY_MIN) {
+            const uint32_t o = (uint32_t)(kv[j] >> 32);
+            lo = o < lo ? o : lo;
+            hi = o > hi ? o : hi;
+            ++valid;
+        }
+    }
+    for (int b = tid; b < K4_BINS; b += K4_THREADS) sm.hist[b] = 0;
+    if (tid == 0) sm.n_collected = 0;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const uint32_t l2 = __shfl_xor_sync(0xFFFFFFFFu, lo, off), h2 = __shfl_xor_sync(0xFFFFFFFFu, hi, off);
+        lo = l2 < lo ? l2 : lo;
+        hi = h2 > hi ? h2 : hi;
+        valid += __shfl_xor_sync(0xFFFFFFFFu, valid, off);
+    }
+    if (lane == 0) {
+        sm.part[warp] = lo;
+        sm.part[W + warp] = hi;
+        sm.part[2 * W + warp] = valid;
+    }
+    __syncthreads();  // (1)
+    lo = sm.part[0];
+    hi = sm.part[W];
+    valid = sm.part[2 * W];
+#pragma unroll
+    for (int w = 1; w < W; ++w) {
+        lo = sm.part[w] < lo ? sm.part[w] : lo;
+        hi = sm.part[W + w] > hi ? sm.part[W + w] : hi;
+        valid += sm.part[2 * W + w];
+    }
+    const float scale = (float)K4_BINS / ((float)(hi - lo) + 1.0f);
+#pragma unroll
+    for (int j = 0; j < K4_BUCKET_PT; ++j)
+        if (kv[j] != KEY_MIN) atomicAdd(&sm.hist[bucket_of(kv[j], lo, scale)], 1u);
+    __syncthreads();  // (2)
+    // thread t owns bins [8t, 8t + 8); count the keys in higher bins
+    uint32_t c[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        c[i] = sm.hist[8 * tid + i];
+        sum += c[i];
+    }
+    uint32_t incl = sum;  // suffix sum over the warp's lanes >= lane
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t v = __shfl_down_sync(0xFFFFFFFFu, incl, off);
+        if (lane + off < 32) incl += v;
+    }
+    if (lane == 0) sm.part[3 * W + warp] = incl;  // the warp's total
+    __syncthreads();  // (3)
+    uint32_t run = incl - sum;
+    for (int w = warp + 1; w < W; ++w) run += sm.part[3 * W + w];
+    const uint32_t want = (uint32_t)r < valid ? (uint32_t)r : valid;  // keys to output
+    // start of each bin's region (bins in descending order); the boundary bin
+#pragma unroll
+    for (int i = 7; i >= 0; --i) {
+        if (want > 0 && run < want && want <= run + c[i]) {
+            sm.found_prefix = (uint64_t)(8 * tid + i);
+            sm.found_count = run + c[i];  // candidates: every key in bins >= B
+            sm.found_remaining = c[i];
+        }
+        sm.hist[8 * tid + i] = run;
+        run += c[i];
+    }
+    if (want == 0 && tid == 0) {
+        sm.found_prefix = (uint64_t)K4_BINS;  // no candidates
+        sm.found_count = 0;
+        sm.found_remaining = 0;
+    }
+    __syncthreads();  // (4)
+    const uint32_t B = (uint32_t)sm.found_prefix;
+    const uint32_t m = sm.found_count;
+    if (m > (uint32_t)K4_BUCKET_M || sm.found_remaining > (uint32_t)K4_BUCKET_BIN_MAX) return false;
+    uint64_t* cand = sm.sorted + K4_BUCKET_R;
+#pragma unroll
+    for (int j = 0; j < K4_BUCKET_PT; ++j) {
+        if (kv[j] == KEY_MIN) continue;
+        const uint32_t b = bucket_of(kv[j], lo, scale);
+        if (b >= B) cand[atomicAdd(&sm.hist[b], 1u)] = kv[j];
+    }
+    __syncthreads();  // (5)
+    // sm.hist[b] is now the end of bin b's region, and its start the end of bin b + 1's
+    for (uint32_t i = tid; i < m; i += K4_THREADS) {
+        const uint64_t key = cand[i];
+        const uint32_t b = bucket_of(key, lo, scale);
+        const uint32_t start = b + 1 < (uint32_t)K4_BINS ? sm.hist[b + 1] : 0u, end = sm.hist[b];
+        uint32_t place = start;
+        for (uint32_t p = start; p < end; ++p) place += cand[p] > key;
+        if (place < want) sm.sorted[place] = key;
+    }
+    for (int i = (int)want + tid; i < r; i += K4_THREADS) sm.sorted[i] = KEY_MIN;
+    __syncthreads();  // (6)
+    return true;
+}
+
+// The best r keys sorted descending in sm.sorted[0 .. r) (KEY_MIN after the
+// valid ones) by the bucket select, or by the register top-r where that gives
+// up; false (nothing written) when neither applies. Block-wide.
+__device__ inline bool block_top(const uint64_t* keys, int n, int r, K4Smem& sm) {
+    if (r <= K4_BUCKET_R && n <= K4_BUCKET_N && block_top_bucket(keys, n, r, sm)) return true;
+    if (r > K4_TOP_MAX) return false;
+    block_top_sorted(keys, n, r, sm);
+    return true;
+}
+
 // Keys with this prefix, appended to sm.sorted (warp-aggregated: one
 // shared-memory atomic per warp and pass). Block-wide; returns their number.
 __device__ __forceinline__ uint32_t gather_prefix(const uint64_t* keys, int n, uint64_t mask, uint64_t prefix,
@@ -242,8 +386,7 @@ __device__ __forceinline__ uint64_t rank_select(uint32_t count, uint32_t r, K4Sm
 __device__ inline uint64_t block_kth_largest(const uint64_t* keys, int n, int r, K4Smem& sm) {
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
-    if (r <= K4_TOP_MAX) {
-        block_top_sorted(keys, n, r, sm);
+    if (block_top(keys, n, r, sm)) {
         const uint64_t res = sm.sorted[r - 1];
         __syncthreads();  // callers may reuse sm.sorted at once
         return res;
@@ -392,8 +535,7 @@ __device__ inline void write_sorted_topk(const uint64_t* keys, int n, int n_vali
         out_scores[i] = -INFINITY;
     }
     if (r == 0) return;
-    if (r <= K4_TOP_MAX) {
-        block_top_sorted(keys, n, r, sm);
+    if (block_top(keys, n, r, sm)) {
         for (int i = tid; i < r; i += K4_THREADS) {
             out_ids[i] = (int32_t)key_id(sm.sorted[i]);
             out_scores[i] = key_score(sm.sorted[i]);
