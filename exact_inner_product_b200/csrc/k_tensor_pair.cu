@@ -82,6 +82,10 @@ struct KPCtl {
     alignas(16) float cvals[KP_EPI_WARPS][KP_WARP_COLS];
     // per epilogue lane: survivors waiting for their append ([slot][lane])
     uint64_t staged[KP_EPI_WARPS][KP_STAGED][32];
+    // int8: per epilogue thread, its query's scale and score floor (kept out
+    // of registers: ten warps leave 168 registers per thread)
+    float q_us[KP_EPI_WARPS][32];
+    float q_t[KP_EPI_WARPS][32];
 };
 static_assert(offsetof(KPCtl, cvals) % 16 == 0, "float4 reads of cvals need 16-byte alignment");
 
@@ -110,11 +114,14 @@ __device__ __forceinline__ void raise_abort(KPCtl* ctl, uint32_t peer) {
 }
 
 // NORMS: per-row score scales (raw rows with norms); MASK: an exclusion
-// bitmask; TYPES: several result sets by candidate type.
-template <bool NORMS, bool MASK, bool TYPES>
+// bitmask; TYPES: several result sets by candidate type; I8: int8 codes
+// (kind::i8, int32 accumulators) with per-row and per-query scales.
+template <bool NORMS, bool MASK, bool TYPES, bool I8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
     k3_pair(const __grid_constant__ CUtensorMap tm_rows, const __grid_constant__ CUtensorMap tm_q,
             const KPParams p) {
+    static_assert(!(I8 && (NORMS || TYPES)), "int8 rows carry their scales themselves");
+    constexpr int KC = I8 ? 128 : KP_KC;  // elements per 128-byte swizzle row
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -175,7 +182,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
                 q_issued = uc;
                 if (even) mbar_arrive_expect_tx(&ctl->qfull, (uint32_t)(2 * p.kchunks * KP_QCHUNK_BYTES));
                 for (int kc = 0; kc < p.kchunks; ++kc)
-                    tma_load_2d_pair(qsm + (size_t)kc * KP_QCHUNK_BYTES, &tm_q, qfull0, kc * KP_KC,
+                    tma_load_2d_pair(qsm + (size_t)kc * KP_QCHUNK_BYTES, &tm_q, qfull0, kc * KC,
                                      qt * (2 * KP_QROWS) + (int)rank * KP_QROWS);
                 for (int64_t t = t0; ok && t < t1; ++t) {
                     for (int kc = 0; kc < p.kchunks; ++kc, ++it) {
@@ -186,7 +193,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
                         }
                         if (even) mbar_arrive_expect_tx(&ctl->full[s], 2 * KP_STAGE_BYTES);
                         tma_load_2d_pair(ring + (size_t)s * KP_STAGE_BYTES, &tm_rows,
-                                         mapa_shared(&ctl->full[s], 0), kc * KP_KC,
+                                         mapa_shared(&ctl->full[s], 0), kc * KC,
                                          (int32_t)(t * KP_TILE + (int64_t)rank * KP_ROWS));
                     }
                 }
@@ -238,10 +245,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
                         const uint32_t a_addr = qbase + (uint32_t)(kc * KP_QCHUNK_BYTES);
                         const uint32_t b_addr = rbase + (uint32_t)(s * KP_STAGE_BYTES);
 #pragma unroll
-                        for (int kk = 0; kk < KP_KC / 16; ++kk) {
-                            umma_bf16_pair(d_tmem, umma_desc_kmajor_sw128(a_addr + kk * 32),
-                                           umma_desc_kmajor_sw128(b_addr + kk * 32), p.idesc,
-                                           (kc | kk) != 0 ? 1u : 0u);
+                        for (int kk = 0; kk < 4; ++kk) {  // 32 bytes of K per instruction
+                            if constexpr (I8)
+                                umma_i8_pair(d_tmem, umma_desc_kmajor_sw128(a_addr + kk * 32),
+                                             umma_desc_kmajor_sw128(b_addr + kk * 32), p.idesc,
+                                             (kc | kk) != 0 ? 1u : 0u);
+                            else
+                                umma_bf16_pair(d_tmem, umma_desc_kmajor_sw128(a_addr + kk * 32),
+                                               umma_desc_kmajor_sw128(b_addr + kk * 32), p.idesc,
+                                               (kc | kk) != 0 ? 1u : 0u);
                         }
                         umma_commit_pair_mc(&ctl->empty[s], 0x3);  // stage free in both CTAs
                     }
@@ -280,17 +292,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
             const int q = qt * (2 * KP_QROWS) + (int)rank * KP_QROWS + quarter * 32 + lane;
             const uint64_t th_key = __ldg(a.theta + q);
             float t_fast = __ldg(a.thf + q);
-            // With no per-row norms the score scale is the same for every row,
-            // and the raw accumulator is compared with th / c, lowered by a
-            // relative 2^-20 so that fl(v * c) >= th implies v >= t_fast.
-            if (!NORMS && t_fast != INFINITY && t_fast != -INFINITY) {
-                const float r = t_fast / a.inv_tau;
-                t_fast = r - fabsf(r) * 0x1p-20f - 1e-30f;
+            // int8: score = fl(fl(acc * us) * c_row); us is this thread's query scale
+            if (I8) {
+                // int8 fast test: a non-negative int32 accumulator below 2^23
+                // (|code| <= 127, d <= 512), read as float bits, is the
+                // subnormal acc * 2^-149, exactly; times c_row * 2^64 it gives
+                // acc * c_row * 2^-85 with one rounding, a normal float for
+                // scores near any threshold. A score fl(fl(acc * us) * c_row)
+                // >= t > 0 needs acc * c_row >= t / us * (1 - 2^-23), so
+                // t_fast = (t / us) * 2^-85 lowered by a relative 2^-20 (and
+                // an absolute 2^-148 for the subnormal range) keeps every such
+                // row. Negative accumulators read as negative floats or NaN,
+                // and never reach a positive threshold. Without a positive
+                // floor every score takes the exact test (t_fast = -inf, and
+                // the test passes NaN maxima).
+                const float us = q < a.b ? __ldg(a.qscale + q) : 1.0f;
+                ctl->q_us[ew][lane] = us;
+                ctl->q_t[ew][lane] = t_fast;
+                if (!(t_fast > 0.0f)) {
+                    t_fast = -INFINITY;
+                } else if (t_fast != INFINITY) {
+                    const float r = (t_fast / us) * 0x1p-85f;
+                    t_fast = r - r * 0x1p-20f - 0x1p-148f;
+                }
             }
-            // With per-row scales the fast test is the sign of fma(v, c, -t_low):
-            // the fma is exact before its one rounding, which keeps the sign of
-            // v*c - t_low, and t_low sits below t_fast by more than the rounding
-            // of fl(v*c), so fl(v*c) >= t_fast implies a non-negative result.
             float neg_t_low = -t_fast;
             if (NORMS && t_fast != INFINITY && t_fast != -INFINITY)
                 neg_t_low = -(t_fast - fabsf(t_fast) * 0x1p-20f - 0x1p-140f);
@@ -319,14 +344,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
                     const int64_t r = tile * KP_TILE + half * KP_WARP_COLS + lane + 32 * j;
                     const bool valid = r < a.n_rows;
                     // raw values: nothing waits for these loads until the next tile
-                    if (NORMS) cl[j] = valid ? __ldg(a.inv_norm + r * a.stride) : 0.0f;
+                    if (NORMS || I8) cl[j] = valid ? __ldg(a.inv_norm + r * a.stride) : 0.0f;
                     if (MASK) {
                         xl[j] = valid ? __ldg(a.exclude + ((r * a.stride) >> 5)) : 0u;
                         xs[j] = (uint32_t)((r * a.stride) & 31);
                     }
                 }
             };
-            if (NORMS || MASK) fetch_rows(t0);
+            if (NORMS || MASK || I8) fetch_rows(t0);
             for (int64_t t = t0; t < t1; ++t, ++tc) {
                 const int buf = tc & 1;
                 const int64_t row0 = t * KP_TILE + half * KP_WARP_COLS;  // level row of column 0
@@ -340,13 +365,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
                         skip[j] = __ballot_sync(0xFFFFFFFFu, bad);
                     }
                 }
-                if (NORMS) {
+                if (NORMS || I8) {
                     __syncwarp();  // the previous tile's reads of cw are done
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) cw[lane + 32 * j] = cl[j] * a.inv_tau;
+                    for (int j = 0; j < 4; ++j)
+                        cw[lane + 32 * j] = I8 ? (cl[j] * a.inv_tau) * 0x1p64f : cl[j] * a.inv_tau;
                     __syncwarp();
                 }
-                if ((NORMS || MASK) && t + 1 < t1) fetch_rows(t + 1);
+                if ((NORMS || MASK || I8) && t + 1 < t1) fetch_rows(t + 1);
                 // the warp decides together, so that it stays converged
                 if (!__all_sync(0xFFFFFFFFu, mbar_wait(&ctl->tfull[buf], (tc >> 1) & 1, abort))) {
                     ok = false;
@@ -357,27 +383,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
                                        (uint32_t)(buf * KP_ACC_COLS + half * KP_WARP_COLS);
                 // One round trip: the warp's 128 columns into registers, then
                 // the accumulator goes back to the MMA issuer before any test.
-                Cols32 v[4];
+                // (int8: two round trips of 64 columns, the accumulator going
+                // back after the second; its fast test needs the registers.)
+                constexpr int NV = I8 ? 2 : 4;  // 32-column chunks held at once
 #pragma unroll
-                for (int h = 0; h < 4; ++h) tmem_ld_32cols(tbase + (uint32_t)(h * 32), v[h].x);
+                for (int part = 0; part < 4 / NV; ++part) {
+                Cols32 v[NV];
+#pragma unroll
+                for (int h = 0; h < NV; ++h) tmem_ld_32cols(tbase + (uint32_t)((part * NV + h) * 32), v[h].x);
                 tmem_ld_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-                    if (even)
-                        mbar_arrive(&ctl->tempty[buf]);
-                    else
-                        mbar_arrive_cluster_relaxed(buf ? r_tempty1 : r_tempty0);
+                if (part == 4 / NV - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (even)
+                            mbar_arrive(&ctl->tempty[buf]);
+                        else
+                            mbar_arrive_cluster_relaxed(buf ? r_tempty1 : r_tempty0);
+                    }
                 }
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                    const int col0 = h * 32;  // within this warp's 128 columns
+                for (int h = 0; h < NV; ++h) {
+                    const int hc = part * NV + h;  // chunk of the warp's 128 columns
+                    const int col0 = hc * 32;      // within this warp's 128 columns
                     // Fast test. One threshold per thread: compare the maximum
                     // of the 32 scores (four chains of three-input max, half an
                     // instruction per score).
                     bool pass;
                     float gmax[4];
-                    if (!NORMS) {
+                    if (I8) {
+                        const float* cc = cw + col0;  // c_row * 2^64 (one broadcast read per score)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {  // chain j: scores 8j .. 8j+7
+                            const float* x = v[h].x + 8 * j;
+                            const float* c = cc + 8 * j;
+                            gmax[j] = fmaxf(max3f(max3f(max3f(x[0] * c[0], x[1] * c[1], x[2] * c[2]), x[3] * c[3],
+                                                        x[4] * c[4]),
+                                                  x[5] * c[5], x[6] * c[6]),
+                                            x[7] * c[7]);
+                        }
+                        pass = !(fmaxf(max3f(gmax[0], gmax[1], gmax[2]), gmax[3]) < t_fast);
+                    } else if (!NORMS) {
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {  // chain j: scores 8j .. 8j+7
                             const float* x = v[h].x + 8 * j;
@@ -401,7 +447,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
                     if (!pass) continue;
                     // Rare: this thread's exact survivors among the 32 rows.
                     uint32_t m = 0;
-                    if (!NORMS) {
+                    if (I8) {
+                        // exact scores, only in the groups of eight whose
+                        // maximum passed (acc is exact in fp32: |acc| < 2^24)
+                        const float us = ctl->q_us[ew][lane], t_exact = ctl->q_t[ew][lane];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            if (!(gmax[j] < t_fast)) {
+#pragma unroll
+                                for (int i = 8 * j; i < 8 * j + 8; ++i)
+                                    m |= ((float)__float_as_int(v[h].x[i]) * us * (cw[col0 + i] * 0x1p-64f) >= t_exact)
+                                             ? (1u << i) : 0u;
+                            }
+                        }
+                    } else if (!NORMS) {
                         // only the groups of eight whose maximum passed
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
@@ -421,13 +480,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
                             m |= (v[h].x[4 * i4 + 3] * c.w >= t_fast) ? (1u << (4 * i4 + 3)) : 0u;
                         }
                     }
-                    m &= ~skip[h];
+                    m &= ~skip[hc];
                     while (m) {
                         const int i = __ffs(m) - 1;
                         m &= m - 1;
                         const int64_t id = (row0 + col0 + i) * a.stride;
                         const float c = NORMS ? cw[col0 + i] : a.inv_tau;
-                        const uint64_t key = make_key(select32(v[h], i) * c, (uint32_t)id);
+                        const float sc = I8 ? (float)__float_as_int(select32(v[h], i)) * ctl->q_us[ew][lane] *
+                                                  (cw[col0 + i] * 0x1p-64f)
+                                            : select32(v[h], i) * c;
+                        const uint64_t key = make_key(sc, (uint32_t)id);
                         if (TYPES) {  // several result sets: the row's set, appended at once
                             const int rset = a.set_of[a.types[id]];
                             if (rset >= 0 && q < a.b) {
@@ -448,6 +510,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
                         }
                     }
                 }
+                }  // part
                 if (!TYPES && __any_sync(0xFFFFFFFFu, n_staged >= KP_STAGED / 2)) flush();
             }
             if (!TYPES && __any_sync(0xFFFFFFFFu, n_staged > 0)) flush();
@@ -469,18 +532,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
     }
 }
 
-int pair_stages(int d) {
-    const int kchunks = (d + KP_KC - 1) / KP_KC;
+// K chunks of 128 bytes per row: 64 bf16 or 128 int8 elements each.
+int pair_kchunks(int d, int esize) { return (d * esize + 127) / 128; }
+
+int pair_stages(int d, int esize) {
+    const int kchunks = pair_kchunks(d, esize);
     const int fixed = 1024 + kchunks * KP_QCHUNK_BYTES + (int)sizeof(KPCtl);
     int stages = (KP_SMEM_BUDGET - fixed) / KP_STAGE_BYTES;
     if (stages > KP_MAX_STAGES) stages = KP_MAX_STAGES;
     return stages;
 }
 
-template <bool NORMS, bool MASK, bool TYPES>
+template <bool NORMS, bool MASK, bool TYPES, bool I8 = false>
 cudaError_t launch_variant(const KPParams& base, const CUtensorMap& tm_rows, const CUtensorMap& tm_queries,
                            int smem, cudaStream_t s, int sm_count) {
-    auto kern = k3_pair<NORMS, MASK, TYPES>;
+    auto kern = k3_pair<NORMS, MASK, TYPES, I8>;
     KPParams p = base;
     // Pairs that can be resident at once (clusters must fit inside a GPC).
     int pairs = sm_count / 2 > 0 ? sm_count / 2 : 1;
@@ -519,30 +585,38 @@ cudaError_t launch_variant(const KPParams& base, const CUtensorMap& tm_rows, con
 
 int tensor_pair_box_rows(int) { return KP_ROWS; }
 
-int tensor_pair_smem_bytes(int d) {
+int tensor_pair_smem_bytes(int d, int esize) {
     if (d > TT_MAX_D) return -1;
-    const int kchunks = (d + KP_KC - 1) / KP_KC;
-    const int stages = pair_stages(d);
+    const int kchunks = pair_kchunks(d, esize);
+    const int stages = pair_stages(d, esize);
     if (stages < 2) return -1;
     return 1024 + kchunks * KP_QCHUNK_BYTES + (int)sizeof(KPCtl) + stages * KP_STAGE_BYTES;
 }
 
 cudaError_t launch_tensor_pair_pass(const PassArgs& a, const CUtensorMap& tm_rows, cudaStream_t s, int sm_count) {
     if (a.n_rows == 0 || a.b == 0) return cudaSuccess;
-    if (a.q_dtype != TT_BF16) return cudaErrorInvalidValue;
-    const int smem = tensor_pair_smem_bytes(a.d);
+    const bool i8 = a.dtype == TT_I8;
+    if (a.q_dtype != (i8 ? TT_I8 : TT_BF16)) return cudaErrorInvalidValue;
+    if (i8 && (a.types != nullptr || a.inv_norm == nullptr || a.qscale == nullptr)) return cudaErrorInvalidValue;
+    const int esize = i8 ? 1 : 2;
+    const int smem = tensor_pair_smem_bytes(a.d, esize);
     if (smem <= 0) return cudaErrorInvalidValue;
     CUtensorMap tm_queries;
-    if (!bf16_tile_tensor_map(a.queries, a.b, a.d, a.d, KP_QROWS, &tm_queries)) return cudaErrorInvalidValue;
+    const bool mapped = i8 ? i8_tile_tensor_map(a.queries, a.b, a.d, a.d, KP_QROWS, &tm_queries)
+                           : bf16_tile_tensor_map(a.queries, a.b, a.d, a.d, KP_QROWS, &tm_queries);
+    if (!mapped) return cudaErrorInvalidValue;
     KPParams p;
     p.a = a;
     p.q_tiles = (a.b + 2 * KP_QROWS - 1) / (2 * KP_QROWS);
-    p.kchunks = (a.d + KP_KC - 1) / KP_KC;
-    p.stages = pair_stages(a.d);
+    p.kchunks = pair_kchunks(a.d, esize);
+    p.stages = pair_stages(a.d, esize);
     p.tiles = (a.n_rows + KP_TILE - 1) / KP_TILE;
     p.chunks = 1;
-    p.idesc = umma_idesc_bf16(2 * KP_QROWS, KP_TILE);
+    p.idesc = i8 ? umma_idesc_s8(2 * KP_QROWS, KP_TILE) : umma_idesc_bf16(2 * KP_QROWS, KP_TILE);
     const bool norms = a.inv_norm != nullptr, mask = a.exclude != nullptr, types = a.types != nullptr;
+    if (i8)  // the row scales go through the int8 epilogue, not the norms one
+        return mask ? launch_variant<false, true, false, true>(p, tm_rows, tm_queries, smem, s, sm_count)
+                    : launch_variant<false, false, false, true>(p, tm_rows, tm_queries, smem, s, sm_count);
     if (types) {
         return norms ? launch_variant<true, true, true>(p, tm_rows, tm_queries, smem, s, sm_count)
                      : launch_variant<false, true, true>(p, tm_rows, tm_queries, smem, s, sm_count);

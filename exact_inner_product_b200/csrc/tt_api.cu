@@ -173,8 +173,8 @@ bool bf16_tile_tensor_map(const void* base, int64_t rows, int d, int64_t row_pit
 }
 
 // int8 rows: boxes of 128 codes (one 128-byte swizzle row) x box_rows rows.
-static bool i8_tile_tensor_map(const void* base, int64_t rows, int d, int64_t row_pitch_elems,
-                               int box_rows, CUtensorMap* tm) {
+bool i8_tile_tensor_map(const void* base, int64_t rows, int d, int64_t row_pitch_elems,
+                        int box_rows, CUtensorMap* tm) {
     return encode_2d(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, base, (uint64_t)d, (uint64_t)rows,
                      (uint64_t)row_pitch_elems, 128, (uint32_t)box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
@@ -635,8 +635,8 @@ static tt_status run_pass(const tt_index* ix, const PathCfg& pc, const Plan& pla
         e = launch_tensor_pass(a, tm_rows, pc.tm_q, pc.nq, s, sms);
     } else if (pc.path == 3) {
         CUtensorMap tm_rows;
-        if (!bf16_tile_tensor_map(ix->rows, a.n_rows, ix->d, a.stride * ix->d, tensor_pair_box_rows(ix->d),
-                                  &tm_rows))
+        if (!tile_tensor_map(ix->dtype, ix->rows, a.n_rows, ix->d, a.stride * ix->d, tensor_pair_box_rows(ix->d),
+                             &tm_rows))
             return TT_ERR_CUDA;
         e = launch_tensor_pair_pass(a, tm_rows, s, sms);
     } else {
@@ -891,12 +891,16 @@ static tt_status score_core(tt_index* index, const void* queries, tt_dtype q_dty
     const int esize = i8 ? 1 : 2;
     const bool tc_possible = (index->dtype == TT_BF16 || i8) && index->d >= 64 &&
                              tensor_pass_max_nq(index->d, esize) > 0;
-    const bool pair_possible = index->dtype == TT_BF16 && index->d >= 64 && tensor_pair_smem_bytes(index->d) > 0;
+    // SM pairs: bf16 rows, or int8 codes (not with several result sets)
+    const bool pair_possible = (index->dtype == TT_BF16 || (i8 && types == nullptr)) && index->d >= 64 &&
+                               tensor_pair_smem_bytes(index->d, esize) > 0;
     int path = path_req;
     if (path == 0) {
         path = 1;
         if (tc_possible && b > 8) path = 2;
-        if (pair_possible && b >= PAIR_MIN_BATCH && index->inv_norm == nullptr) path = 3;
+        // rows with norms stay on the single-SM kernel (measured faster there);
+        // int8 scales take the pair kernel's integer fast test
+        if (pair_possible && b >= PAIR_MIN_BATCH && (index->inv_norm == nullptr || i8)) path = 3;
     }
     if (path == 2 && !tc_possible) return TT_ERR_UNSUPPORTED;
     if (path == 3 && !pair_possible) return TT_ERR_UNSUPPORTED;

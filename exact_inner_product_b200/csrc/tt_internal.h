@@ -205,6 +205,9 @@ int merge_smem_keys();
 // Tensor-core pass: bf16 boxes of 64 elements x box_rows rows, 128-byte swizzle.
 bool bf16_tile_tensor_map(const void* base, int64_t rows, int d, int64_t row_pitch_elems,
                           int box_rows, CUtensorMap* tm);
+// int8 codes: boxes of 128 codes (one 128-byte swizzle row) x box_rows rows.
+bool i8_tile_tensor_map(const void* base, int64_t rows, int d, int64_t row_pitch_elems, int box_rows,
+                        CUtensorMap* tm);
 cudaError_t launch_pad(int32_t* out_ids, float* out_scores, int64_t count, cudaStream_t s);
 // Exclusion words for rows [start, start + count) of a mask (null: none),
 // optionally also excluding rows whose types[j] != want (types null: none).
@@ -237,6 +240,6 @@ cudaError_t launch_offset_ids(int32_t* ids, int64_t count, int64_t offset, cudaS
 // esize: bytes per element of the rows (2 bf16, 1 int8).
 int tensor_pass_smem_bytes(int d, int nq_tile, int esize);
 int tensor_pass_max_nq(int d, int esize);
-int tensor_pair_smem_bytes(int d);  // -1 when d does not fit
+int tensor_pair_smem_bytes(int d, int esize);  // -1 when d does not fit (esize: 2 bf16, 1 int8)
 
 }  // namespace tt

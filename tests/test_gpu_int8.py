@@ -45,8 +45,9 @@ CASES = [
     ("stream_b1", {"n": 150_001, "b": 5, "k": 64}, 1),
     ("small_batch", {"n": 300_077, "tau": 1.0}, 2),
     ("small_batch", {"n": 100_003, "b": 9, "k": 17}, 2),
-    ("large_batch", {"n": 400_005, "b": 300, "k": 1000, "oracle_queries": 12}, 2),
-    ("masked_fused", {"n": 200_099, "b": 260, "oracle_queries": 12}, 2),
+    ("large_batch", {"n": 400_005, "b": 300, "k": 1000, "oracle_queries": 12}, 3),
+    ("large_batch", {"n": 250_001, "b": 200, "k": 300, "oracle_queries": 12}, 2),
+    ("masked_fused", {"n": 200_099, "b": 260, "oracle_queries": 12}, 3),
     ("masked_fused", {"n": 120_031, "b": 3, "k": 256}, 1),
 ]
 
@@ -62,8 +63,9 @@ def test_int8_parity(name, over, path):
 
 
 def test_int8_both_scorers_agree():
-    """The dp4a streaming scorer and the kind::i8 tensor-core scorer compute
-    the same exact integer sums, so their results are identical."""
+    """The dp4a streaming scorer, the kind::i8 tensor-core scorer and its
+    SM-pair form compute the same exact integer sums and the same score
+    arithmetic, so their results are identical."""
     _cuda()
     w = W.workload("small_batch", n=70_001, b=40, k=100, tau=1.0)
     raw_c, raw_q = W.corpus(w, "cuda"), W.queries(w, "cuda")
@@ -72,7 +74,10 @@ def test_int8_both_scorers_agree():
     assert tt.tt_last_stats(index)["path"] == 1
     b = tt.tt_score_topk(index, qn, w.k, path=2)
     assert tt.tt_last_stats(index)["path"] == 2
+    c = tt.tt_score_topk(index, qn, w.k, path=3)
+    assert tt.tt_last_stats(index)["path"] == 3
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    assert torch.equal(a[0], c[0]) and torch.equal(a[1], c[1])
     res, _ = parity.run_case_q8(w, path=1)
     assert res["max_abs_err"] <= parity.q8_tolerance(w)
 
@@ -86,7 +91,7 @@ def test_int8_ties_and_edges():
     codes = torch.empty((5000, d), dtype=torch.int8, device="cuda")
     scales = torch.empty((5000,), dtype=torch.float32, device="cuda")
     index = tt.tt_quantize_candidates(raw, codes, scales)
-    for path, b in ((1, 2), (2, 40)):
+    for path, b in ((1, 2), (2, 40), (3, 260)):
         q = torch.randn(b, d, device="cuda")
         ids, sc = tt.tt_score_topk(index, q, 300, path=path)
         assert (ids.cpu() == torch.arange(300, dtype=torch.int32)[None, :]).all()
@@ -99,7 +104,7 @@ def test_int8_ties_and_edges():
     excl = torch.full((2,), -1, dtype=torch.int32, device="cuda")
     ids, _ = tt.tt_score_topk(small, q, 5, exclude=excl)
     assert (ids == -1).all()
-    # int8 rows need the scales, d % 32 == 0, and no SM-pair kernel
+    # int8 rows need the scales and d % 32 == 0
     with pytest.raises(tt.TTError) as e:
         tt.tt_index_wrap(codes)
     assert e.value.status == tt.TT_ERR_INVALID_ARG
@@ -108,6 +113,25 @@ def test_int8_ties_and_edges():
     with pytest.raises(tt.TTError) as e:
         tt.tt_score_topk(ix48, torch.randn(2, 48, device="cuda"), 3)
     assert e.value.status == tt.TT_ERR_UNSUPPORTED
-    with pytest.raises(tt.TTError) as e:
-        tt.tt_score_topk(index, torch.randn(300, d, device="cuda"), 3, path=3)
-    assert e.value.status == tt.TT_ERR_UNSUPPORTED
+    # several result sets by type stay on the single-SM kernel for int8 rows
+    types = torch.zeros(5000, dtype=torch.uint8, device="cuda")
+    ids_t, _ = tt.tt_score_topk_types(index, torch.randn(300, d, device="cuda"), 3, types, [0])
+    assert tt.tt_last_stats(index)["path"] == 2 and (ids_t[0] == torch.arange(3, dtype=torch.int32, device="cuda")).all()
+
+
+def test_int8_pair_negative_thresholds():
+    """k close to n: the k-th best score is negative, so the integer fast test
+    of the SM-pair kernel (which needs a positive threshold) is bypassed and
+    every score takes the exact test; the result still equals the other
+    scorers' and the oracle's."""
+    _cuda()
+    w = W.workload("large_batch", n=3_001, b=270, k=2048, oracle_queries=6)
+    raw_c, raw_q = W.corpus(w, "cuda"), W.queries(w, "cuda")
+    index, qn = parity.gpu_prepare_q8(w, raw_c, raw_q)
+    a = tt.tt_score_topk(index, qn, w.k, path=2)
+    c = tt.tt_score_topk(index, qn, w.k, path=3)
+    assert tt.tt_last_stats(index)["path"] == 3
+    assert torch.equal(a[0], c[0]) and torch.equal(a[1], c[1])
+    assert (c[1][:, -1] < 0).float().mean() > 0.5  # mostly negative k-th scores
+    res, _ = parity.run_case_q8(w, path=3)
+    assert res["max_abs_err"] <= parity.q8_tolerance(w)
