@@ -89,20 +89,27 @@ def test_noalloc_matches_regular_entry_point(name, over):
 def test_noalloc_allocates_nothing_after_the_first_call():
     """After one warm-up call on the GPU (which may commit the fixed array:
     CUDA loads a module's device memory when first used), further calls leave
-    the device's free memory unchanged."""
+    the device's free memory unchanged: the single-SM tensor-core plan, the
+    one-sample plan of a few queries on the streaming scorer and a wider
+    batch, each called several times."""
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
-    w = W.workload("small_batch", n=150_001, b=40, k=300)
+    w = W.workload("small_batch", n=150_001, b=200, k=300)
     raw_c = W.corpus(w, "cuda")
     raw_q = W.queries(w, "cuda")
     index, qn = parity.gpu_prepare(w, raw_c, raw_q)
-    ids = torch.empty((w.b, w.k), dtype=torch.int32, device="cuda")
-    scores = torch.empty((w.b, w.k), dtype=torch.float32, device="cuda")
-    assert _noalloc(index.rows, None, qn, w.k, w.tau, None, ids, scores) == tt.TT_OK
+    calls = []
+    for b in (40, 4, 200):  # tensor-core levels, one sample (b <= 8), a wider batch
+        ids = torch.empty((b, w.k), dtype=torch.int32, device="cuda")
+        scores = torch.empty((b, w.k), dtype=torch.float32, device="cuda")
+        calls.append((qn[:b].contiguous(), ids, scores))
+    for q, ids, scores in calls:  # warm-up
+        assert _noalloc(index.rows, None, q, w.k, w.tau, None, ids, scores) == tt.TT_OK
     torch.cuda.synchronize()
     free0, _ = torch.cuda.mem_get_info()
     for _ in range(3):
-        assert _noalloc(index.rows, None, qn, w.k, w.tau, None, ids, scores) == tt.TT_OK
+        for q, ids, scores in calls:
+            assert _noalloc(index.rows, None, q, w.k, w.tau, None, ids, scores) == tt.TT_OK
     torch.cuda.synchronize()
     free1, _ = torch.cuda.mem_get_info()
     assert free1 == free0, (free0, free1)
