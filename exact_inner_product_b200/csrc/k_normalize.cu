@@ -105,6 +105,13 @@ __device__ __forceinline__ void store_codes<8>(int8_t* row_out, int e0, const in
     *reinterpret_cast<uint2*>(row_out + e0) = make_uint2(w[0], w[1]);
 }
 
+// The int8 coding quotient as the page writes it, fl(fl(v / norm) / scale)
+// (norm == 0: v taken as given); the rare elements near a rounding boundary.
+__device__ __noinline__ float ieee_code_quotient(float v, float norm, float scale) {
+    const float w = norm != 0.0f ? __fdiv_rn(v, norm) : v;
+    return __fdiv_rn(w, scale);
+}
+
 // MODE 0: out rows = v / norm (Tout). MODE 1: inv_norm[j] = 1 / norm.
 // MODE 2: w = v / norm, then int8 codes of w to out (Tout = int8_t) and the
 // row's scale to inv_norm. MODE 3: the same coding of v as given (queries).
@@ -179,46 +186,58 @@ __global__ void __launch_bounds__(K1_THREADS)
         }
         if constexpr (MODE >= 2) {
             // int8 coding (recsys_two_tower_model.py `compute_top_k_int8`):
-            // scale = max(max|w| / 127, 1e-12), code = clip(round(w / scale)),
-            // round half to even, in fp32 as written there.
-            // The row values w are computed once (one IEEE division each when
-            // normalising) and kept in registers for the coding pass.
-            float mx[U];
-            float wv[U][CPL][E];
+            // w = fl(v / norm) (MODE 2; MODE 3: w = v), scale = max(fl(max|w|
+            // / 127), 1e-12), code = clip(round_half_even(fl(w / scale))),
+            // every step an IEEE fp32 operation as written there. Two
+            // divisions per element are not needed for that result:
+            //  - dividing by a positive norm is monotone, so max|w| =
+            //    fl(max|v| / norm): one division per row gives the scale;
+            //  - y = fl(fl(v * fl(1/norm)) * fl(1/scale)) differs from the
+            //    IEEE quotient fl(w / scale) by at most four relative
+            //    roundings, |y| * 2^-21 in all, so round(y) is the exact code
+            //    unless y lies within that distance of a half-integer; such
+            //    rare elements (the margin below is four times wider) take
+            //    the two IEEE divisions.
+            float mv[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                const float norm = MODE == 2 ? __fsqrt_rn(fmaxf(ss[u], 1e-12f)) : 1.0f;
-                mx[u] = 0.f;
+                mv[u] = 0.f;
 #pragma unroll
                 for (int i = 0; i < CPL; ++i) {
                     float x[E];
                     Elem<Tin>::unpack(raw[u][i], x);
 #pragma unroll
-                    for (int e = 0; e < E; ++e) {
-                        wv[u][i][e] = MODE == 2 ? __fdiv_rn(x[e], norm) : x[e];
-                        mx[u] = fmaxf(mx[u], fabsf(wv[u][i][e]));
-                    }
+                    for (int e = 0; e < E; ++e) mv[u] = fmaxf(mv[u], fabsf(x[e]));
                 }
             }
 #pragma unroll
             for (int off = L / 2; off > 0; off >>= 1) {
 #pragma unroll
-                for (int u = 0; u < U; ++u) mx[u] = fmaxf(mx[u], __shfl_xor_sync(0xFFFFFFFFu, mx[u], off));
+                for (int u = 0; u < U; ++u) mv[u] = fmaxf(mv[u], __shfl_xor_sync(0xFFFFFFFFu, mv[u], off));
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 if (row[u] >= n) continue;
-                const float scale = fmaxf(__fdiv_rn(mx[u], 127.0f), 1e-12f);
+                const float norm = MODE == 2 ? __fsqrt_rn(fmaxf(ss[u], 1e-12f)) : 1.0f;
+                const float mx = MODE == 2 ? __fdiv_rn(mv[u], norm) : mv[u];  // max_i |fl(v_i / norm)|
+                const float scale = fmaxf(__fdiv_rn(mx, 127.0f), 1e-12f);
+                const float rn = MODE == 2 ? __frcp_rn(norm) : 1.0f;
+                const float rs = __frcp_rn(scale);
                 if (sub == 0) inv_norm[row[u]] = scale;
 #pragma unroll
                 for (int i = 0; i < CPL; ++i) {
                     const int c = sub + i * L;
                     if (c < chunks) {
+                        float x[E];
+                        Elem<Tin>::unpack(raw[u][i], x);
                         int q[E];
 #pragma unroll
                         for (int e = 0; e < E; ++e) {
-                            const float r = fminf(fmaxf(rintf(__fdiv_rn(wv[u][i][e], scale)), -127.f), 127.f);
-                            q[e] = (int)r;
+                            float y = (MODE == 2 ? x[e] * rn : x[e]) * rs;
+                            const float to_int = fabsf(y - rintf(y));  // distance to the nearest integer
+                            if (!(0.5f - to_int > fabsf(y) * 0x1p-19f + 0x1p-19f))
+                                y = ieee_code_quotient(x[e], MODE == 2 ? norm : 0.0f, scale);
+                            q[e] = (int)fminf(fmaxf(rintf(y), -127.f), 127.f);
                         }
                         store_codes<E>(reinterpret_cast<int8_t*>(out) + row[u] * d, c * E, q);
                     }
@@ -263,6 +282,15 @@ cudaError_t dispatch_lanes(const void* in, int64_t n, int d, void* out, cudaStre
     const int chunks = d / E;
     int L = 32;
     while (L > chunks) L >>= 1;
+    if (MODE >= 2) {
+        // int8 coding does per-row work (a square root, two divisions, two
+        // reciprocals, two reductions) that every lane of a row repeats:
+        // fewer lanes per row (up to four chunks each) spread it over
+        // several rows at once. (32 lanes per 512-byte row ran at 0.41 of
+        // HBM; plain normalisation, with less per-row work, at 0.94.)
+        L = 4;
+        while (L < 32 && L * 4 < chunks) L <<= 1;
+    }
     const int cpl = (chunks + L - 1) / L;
     const int unroll = (L == 32 && cpl == 1) ? 4 : 2;
     const int rows_per_block = (K1_THREADS / 32) * unroll * (32 / L);
@@ -278,7 +306,12 @@ cudaError_t dispatch_lanes(const void* in, int64_t n, int d, void* out, cudaStre
     float* pinv = MODE == 1 ? static_cast<float*>(out) : static_cast<float*>(aux);
     note_launch_begin(TT_KIND_NORMALIZE, s);
     const dim3 g((unsigned)blocks), t(K1_THREADS);
-    if (L == 32 && cpl == 1) k1_normalize<Tin, Tout, MODE, 32, 1, 4><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
+    if (MODE >= 2) {
+        if (L == 4) k1_normalize<Tin, Tout, MODE, 4, 4, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
+        else if (L == 8) k1_normalize<Tin, Tout, MODE, 8, 4, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
+        else if (L == 16) k1_normalize<Tin, Tout, MODE, 16, 4, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
+        else k1_normalize<Tin, Tout, MODE, 32, 4, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
+    } else if (L == 32 && cpl == 1) k1_normalize<Tin, Tout, MODE, 32, 1, 4><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
     else if (L == 32 && cpl == 2) k1_normalize<Tin, Tout, MODE, 32, 2, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
     else if (L == 32) k1_normalize<Tin, Tout, MODE, 32, 4, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);
     else if (L == 16) k1_normalize<Tin, Tout, MODE, 16, 2, 2><<<g, t, 0, s>>>(pin, n, d, pout, pinv);

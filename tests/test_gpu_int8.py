@@ -39,6 +39,46 @@ def test_coding_matches_oracle(name, n):
     assert np.abs(codes.cpu().numpy().astype(np.int32)).max() <= 127
 
 
+@pytest.mark.parametrize("dtype,d", [(torch.float32, 128), (torch.bfloat16, 256), (torch.float32, 64)])
+def test_coding_is_the_ieee_fp32_formula_bitwise(dtype, d):
+    """The coding of tt_quantize_candidates is the page's formula in IEEE fp32
+    (w = fl(v / norm), scale = max(fl(max|w| / 127), 1e-12), code =
+    round_half_even(fl(w / scale)), clipped), bit for bit, although the kernel
+    divides once per row: torch's fp32 operations (IEEE division and square
+    root on the GPU) evaluate the formula as written. Rows of small integers
+    make the sum of squares exact, so the norm does not depend on the order
+    of the sum; rows with a value on a half step of the code grid test the
+    kernel's near-tie fallback."""
+    _cuda()
+    g = torch.Generator(device="cpu").manual_seed(11)
+    n = 60_000
+    v = torch.randint(-40, 41, (n, d), generator=g).to(torch.float32)
+    v[::7, 0] = 0.0
+    v[1::97] = 0.0                                   # zero rows: scale 1e-12, codes 0
+    # rows whose values sit on code half steps: max|v| = 254 puts v = 1 at code 0.5
+    v[2::11, 0] = 254.0
+    v[2::11, 1:6] = torch.tensor([1.0, 3.0, -5.0, 127.0, -253.0])
+    x = v.to(dtype).cuda()
+    codes = torch.empty((n, d), dtype=torch.int8, device="cuda")
+    scales = torch.empty((n,), dtype=torch.float32, device="cuda")
+    tt.tt_quantize_candidates(x, codes, scales, make_index=False)
+    xf = x.float()
+    ss = (xf * xf).sum(1)                            # exact: small integers
+    norm = torch.sqrt(torch.clamp(ss, min=1e-12))
+    # every division tensor by tensor: a Python-scalar divisor may be turned
+    # into a multiply by its reciprocal, which is not the IEEE quotient
+    w = xf / norm[:, None]
+    sc = torch.clamp(w.abs().amax(1) / torch.full_like(ss, 127.0), min=1e-12)
+    want = torch.clamp(torch.round(w / sc[:, None]), -127, 127).to(torch.int8)
+    bad = (scales != sc).nonzero()
+    assert bad.numel() == 0, (bad.numel(), bad[:3].tolist(), scales[bad[:3, 0]].tolist(), sc[bad[:3, 0]].tolist())
+    bad = (codes != want).nonzero()
+    assert bad.numel() == 0, (bad.numel(), bad[:3].tolist())
+    # quotients within the kernel's margin of a half step occurred (v = +-1, +-3, ... -> code +-0.5, +-1.5, ...)
+    q = (w / sc[:, None])[2::11, 1:6]
+    assert ((q - q.floor() - 0.5).abs() < 1e-5).float().mean() > 0.5
+
+
 CASES = [
     # name, overrides, expected path
     ("stream_b1", {"n": 200_037}, 1),
