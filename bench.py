@@ -68,11 +68,11 @@ TRAFFIC = {
     # --no-e2e --no-cpu-baseline`: 512.019 MB read + 200.806 MB written for 1,000,000 rows
     ("k1_normalize", "stream_b1"): {"bytes_per_row": 712.825, "src": "exact_inner_product_b200/csrc/k_normalize.cu",
                                     "sha": "4273a9f8869b74ec01b8762c20eb598dc6f0b1597fcd3e5f8ad9afde664127f4"},
-    # ncu --set full --clock-control none -k regex:k3_pair -s 5 -c 1 on `python bench.py --workload large_batch --n 4000000
-    # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 1592.981 MB read
-    # + 28.070 MB written; scaled to the full corpus by rows scanned
-    ("k3_pair", "large_batch"): {"bytes_per_row": 405.263, "src": "exact_inner_product_b200/csrc/k_tensor_pair.cu",
-                                 "sha": "6f303eca084c883abd77d28ff639f8375a1558b5412efecc66fc5478f0e084eb"},
+    # ncu --set full --import-source no --clock-control none -k regex:k3_pair -s 8 -c 1 on `python bench.py
+    # --workload large_batch --n 4000000 --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass,
+    # 4,000,000 rows): 1092.787 MB read + 29.671 MB written; scaled to the full corpus by rows scanned
+    ("k3_pair", "large_batch"): {"bytes_per_row": 280.615, "src": "exact_inner_product_b200/csrc/k_tensor_pair.cu",
+                                 "sha": "9c6e8b8b844010494e6a9b58ec46d9018dadaf82caa4fcd975a7e92590a5471f"},
     # ncu --set full --clock-control none -k regex:k3_tensor -s 5 -c 1 on `python bench.py --workload masked_fused --n 4000000
     # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 4385.550 MB read
     # + 66.286 MB written; scaled to the full corpus by rows scanned
