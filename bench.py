@@ -288,8 +288,11 @@ def workload_from_args(args) -> W.Workload:
 # times a bounded prefix of the corpus, never the whole of a large one).
 CPU_SAMPLE_ROWS = 4_000_000
 # Corpora smaller than this are scored with an L2 flush before every step
-# (the 126 MB L2 could otherwise hold part of them between steps).
-FLUSH_BELOW_BYTES = 1 << 30
+# (the 126 MB L2 could otherwise hold part of them between steps); a corpus of
+# at least twice the L2 size, streamed front to back every step, leaves no
+# reusable lines behind (ncu: the one-query pass reads its whole 256 MB from
+# DRAM in back-to-back steps), and runs without one.
+FLUSH_BELOW_BYTES = 2 * 126_000_000
 K1_REPS = 3
 
 

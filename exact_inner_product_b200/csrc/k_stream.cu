@@ -38,6 +38,7 @@ namespace {
 constexpr int K2_THREADS = 256;
 constexpr int K2_BATCH = 8;  // 32-byte loads in flight per thread
 constexpr int K2_MAX_QB = 8;
+constexpr int K2_DEFER = 4;  // rows per thread scored before the threshold is known
 
 struct Raw32 {
     uint32_t w[8];
@@ -86,19 +87,41 @@ __device__ __forceinline__ void append_set(const PassArgs& a, int q, int rset, b
     }
 }
 
+// Kept keys of one warp appended to query q's buffer (warp-aggregated).
+__device__ __forceinline__ void append_warp(const PassArgs& a, int q, bool keep, uint64_t key, int lane) {
+    const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, keep);
+    if (ballot) {
+        const int leader = __ffs(ballot) - 1;
+        uint32_t slot0 = 0;
+        if (lane == leader) slot0 = atomicAdd(a.count + q, (uint32_t)__popc(ballot));
+        slot0 = __shfl_sync(0xFFFFFFFFu, slot0, leader);
+        if (keep) {
+            const uint32_t slot = slot0 + __popc(ballot & lanemask_lt());
+            if (slot < (uint32_t)a.cap) a.keys[(int64_t)q * a.cap + slot] = key;
+        }
+    }
+}
+
 // T: corpus element type. QB: queries per block (blockIdx.y selects the
 // group). V8: rows start on 32-byte boundaries. PF: the whole row fits one
 // batch of loads, and the next row's loads are issued before the current
 // row is scored (used when every thread streams many rows: on 10^7 rows of
 // 256 bytes it raised the pass from 5.5 to 6.1 TB/s; with only three or four
 // rows per thread, as on 10^6 rows, it was slower).
-template <typename T, int QB, bool V8, bool PF>
+// DEFER > 0: the pass follows the one-sample estimate of its threshold. Each
+// thread scores its first DEFER rows before it waits for that kernel, keeps
+// their keys in registers and filters them once the threshold is known, so
+// the first blocks stream rows while the estimate runs. Reading the rows and
+// the queries before the wait is safe: no kernel that writes them signals its
+// dependents early, so the search's first kernel, and with it every later
+// one, starts only after those writes completed.
+template <typename T, int QB, bool V8, bool PF, int DEFER>
 __global__ void __launch_bounds__(K2_THREADS)
     k2_stream(const PassArgs a) {
     constexpr int E = 32 / (int)sizeof(T);  // elements per 32-byte piece
     extern __shared__ __align__(16) float qs[];  // [QB][d]
     pdl_trigger();
-    pdl_wait();  // queries, thresholds and counters come from earlier kernels
+    if (DEFER == 0) pdl_wait();  // queries, thresholds and counters come from earlier kernels
     const int lane = threadIdx.x & 31;
     const int q0 = blockIdx.y * QB;
     const int d = a.d;
@@ -114,24 +137,77 @@ __global__ void __launch_bounds__(K2_THREADS)
         }
         qs[i] = v;
     }
-    uint64_t th[QB];
-#pragma unroll
-    for (int qb = 0; qb < QB; ++qb) th[qb] = (q0 + qb < a.b) ? a.theta[q0 + qb] : KEY_MAX;
     __syncthreads();
 
     const int64_t pitch = (int64_t)a.stride * d * (int)sizeof(T);
     const uint8_t* base = static_cast<const uint8_t*>(a.rows);
     const int64_t n_threads = (int64_t)gridDim.x * blockDim.x;
+    int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    uint64_t th[QB];
+    if constexpr (DEFER > 0) {
+        uint64_t kb[DEFER][QB];  // keys of the first DEFER rows (KEY_MIN: no row, or excluded)
+#pragma unroll
+        for (int i = 0; i < DEFER; ++i, r += n_threads) {
+            const bool valid = r < a.n_rows;
+            const uint8_t* row = base + (valid ? r : 0) * pitch;
+            float acc[QB];
+#pragma unroll
+            for (int qb = 0; qb < QB; ++qb) acc[qb] = 0.f;
+            for (int p0 = 0; p0 < pieces; p0 += K2_BATCH) {
+                Raw32 raw[K2_BATCH];
+#pragma unroll
+                for (int j = 0; j < K2_BATCH; ++j)
+                    if (p0 + j < pieces && valid) raw[j] = ld32<V8>(row + (int64_t)(p0 + j) * 32);
+#pragma unroll
+                for (int j = 0; j < K2_BATCH; ++j) {
+                    if (p0 + j >= pieces) break;
+                    float x[E];
+                    unpack32(raw[j], x, T());
+                    const int e0 = (p0 + j) * E;
+#pragma unroll
+                    for (int qb = 0; qb < QB; ++qb) {
+                        const float4* qv = reinterpret_cast<const float4*>(qs + qb * d + e0);
+#pragma unroll
+                        for (int v4 = 0; v4 < E / 4; ++v4) {
+                            const float4 q = qv[v4];
+                            acc[qb] = fmaf(x[4 * v4 + 0], q.x, acc[qb]);
+                            acc[qb] = fmaf(x[4 * v4 + 1], q.y, acc[qb]);
+                            acc[qb] = fmaf(x[4 * v4 + 2], q.z, acc[qb]);
+                            acc[qb] = fmaf(x[4 * v4 + 3], q.w, acc[qb]);
+                        }
+                    }
+                }
+            }
+            const int64_t id = r * a.stride;
+            bool row_ok = valid;
+            float c = a.inv_tau;
+            if (valid) {
+                if (a.exclude) row_ok = !((a.exclude[id >> 5] >> (id & 31)) & 1u);
+                if (a.inv_norm) c = a.inv_norm[id] * a.inv_tau;
+            }
+#pragma unroll
+            for (int qb = 0; qb < QB; ++qb) kb[i][qb] = row_ok ? make_key(acc[qb] * c, (uint32_t)id) : KEY_MIN;
+        }
+        pdl_wait();  // this pass's thresholds
+#pragma unroll
+        for (int qb = 0; qb < QB; ++qb) th[qb] = (q0 + qb < a.b) ? a.theta[q0 + qb] : KEY_MAX;
+#pragma unroll
+        for (int i = 0; i < DEFER; ++i)
+#pragma unroll
+            for (int qb = 0; qb < QB; ++qb) append_warp(a, q0 + qb, kb[i][qb] > th[qb], kb[i][qb], lane);
+    } else {
+#pragma unroll
+        for (int qb = 0; qb < QB; ++qb) th[qb] = (q0 + qb < a.b) ? a.theta[q0 + qb] : KEY_MAX;
+    }
     // whole warps step together so the ballots below see every lane
     Raw32 nxt[PF ? K2_BATCH : 1];
     if (PF) {
-        const int64_t r0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-        if (r0 < a.n_rows)
+        if (r < a.n_rows)
 #pragma unroll
             for (int j = 0; j < K2_BATCH; ++j)
-                if (j < pieces) nxt[j] = ld32<V8>(base + r0 * pitch + (int64_t)j * 32);
+                if (j < pieces) nxt[j] = ld32<V8>(base + r * pitch + (int64_t)j * 32);
     }
-    for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r - lane < a.n_rows; r += n_threads) {
+    for (; r - lane < a.n_rows; r += n_threads) {
         const bool valid = r < a.n_rows;
         const uint8_t* row = base + (valid ? r : 0) * pitch;
         float acc[QB];
@@ -195,34 +271,7 @@ __global__ void __launch_bounds__(K2_THREADS)
 #pragma unroll
         for (int qb = 0; qb < QB; ++qb) {
             const uint64_t key = make_key(acc[qb] * c, (uint32_t)id);
-            const bool keep = row_ok && key > th[qb];
-            const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, keep);
-            if (ballot) {
-                const int q = q0 + qb;
-                const int leader = __ffs(ballot) - 1;
-                uint32_t slot0 = 0;
-                if (lane == leader) slot0 = atomicAdd(a.count + q, (uint32_t)__popc(ballot));
-                slot0 = __shfl_sync(0xFFFFFFFFu, slot0, leader);
-                if (keep) {
-                    const uint32_t slot = slot0 + __popc(ballot & lanemask_lt());
-                    if (slot < (uint32_t)a.cap) a.keys[(int64_t)q * a.cap + slot] = key;
-                }
-            }
-        }
-    }
-}
-
-// Kept keys of one warp appended to query q's buffer (warp-aggregated).
-__device__ __forceinline__ void append_warp(const PassArgs& a, int q, bool keep, uint64_t key, int lane) {
-    const uint32_t ballot = __ballot_sync(0xFFFFFFFFu, keep);
-    if (ballot) {
-        const int leader = __ffs(ballot) - 1;
-        uint32_t slot0 = 0;
-        if (lane == leader) slot0 = atomicAdd(a.count + q, (uint32_t)__popc(ballot));
-        slot0 = __shfl_sync(0xFFFFFFFFu, slot0, leader);
-        if (keep) {
-            const uint32_t slot = slot0 + __popc(ballot & lanemask_lt());
-            if (slot < (uint32_t)a.cap) a.keys[(int64_t)q * a.cap + slot] = key;
+            append_warp(a, q0 + qb, row_ok && key > th[qb], key, lane);
         }
     }
 }
@@ -315,7 +364,8 @@ __global__ void __launch_bounds__(K2_THREADS)
 }
 
 // Grid of a streaming pass: one block per 256 rows, at most eight blocks per
-// SM (blocks loop over their rows). Measured on the 10^6-row pass: a grid of
+// Grid: one block per 256 rows, at most 8 blocks of 256 threads per SM
+// (blocks loop over their rows). Measured on the 10^6-row pass: a grid of
 // exactly the resident blocks (each looping ~13 times) took 53 us against 47
 // us for this one, which runs in about four waves of resident blocks.
 template <typename K>
@@ -329,13 +379,18 @@ dim3 stream_grid(K, const PassArgs& a, int gy, size_t, int sm_count) {
 
 template <typename T, int QB, bool V8>
 cudaError_t launch_qbv(const PassArgs& a, int gy, size_t smem, cudaStream_t s, int sms) {
-    const dim3 grid = stream_grid(k2_stream<T, QB, V8, false>, a, gy, smem, sms);
+    const dim3 grid = stream_grid(k2_stream<T, QB, V8, false, 0>, a, gy, smem, sms);
     constexpr int E = 32 / (int)sizeof(T);
     const bool one_batch = a.d / E <= K2_BATCH;
     const int64_t rows_per_thread = a.n_rows / ((int64_t)grid.x * K2_THREADS);
     if (one_batch && rows_per_thread >= 8)
-        return launch_pdl(k2_stream<T, QB, V8, true>, grid, dim3(K2_THREADS), smem, s, a);
-    return launch_pdl(k2_stream<T, QB, V8, false>, grid, dim3(K2_THREADS), smem, s, a);
+        return launch_pdl(k2_stream<T, QB, V8, true, 0>, grid, dim3(K2_THREADS), smem, s, a);
+    // after the one-sample estimate: the first rows are scored while it runs
+    if constexpr (QB <= 2) {
+        if (a.defer && a.types == nullptr)
+            return launch_pdl(k2_stream<T, QB, V8, false, K2_DEFER>, grid, dim3(K2_THREADS), smem, s, a);
+    }
+    return launch_pdl(k2_stream<T, QB, V8, false, 0>, grid, dim3(K2_THREADS), smem, s, a);
 }
 
 template <typename T, int QB>

@@ -622,6 +622,7 @@ static tt_status run_pass(const tt_index* ix, const PathCfg& pc, const Plan& pla
     a.err = sc.flags + 1;
     a.types = pc.types;
     a.set_of = pc.types ? sc.set_of : nullptr;
+    a.defer = (plan.sampled && level == 0) ? 1 : 0;  // the pass right after the one-sample estimate
     a.theta_v = pc.types ? sc.theta : nullptr;
     if (pc.types) {  // first tests against each query's loosest set threshold
         a.theta = sc.theta_min;

@@ -43,6 +43,7 @@ struct PassArgs {
     const uint8_t* types;      // [n] or null
     const int8_t* set_of;      // [256]
     const uint64_t* theta_v;   // [n_sets * b]
+    int defer;                 // streaming pass right after the one-sample estimate (its thresholds)
 };
 
 // Launch `kernel` with programmatic stream serialization: it may start while

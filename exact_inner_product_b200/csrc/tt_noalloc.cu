@@ -223,6 +223,7 @@ tt_status tt_score_topk_noalloc(const void* rows, tt_dtype dtype, int64_t n, int
         a.keys = keys;
         a.cap = cap;
         a.err = flags + 1;
+        a.defer = (plan.sampled && lv == 0) ? 1 : 0;  // the pass right after the one-sample estimate
         if (path == 2) {
             CUtensorMap tm_rows;
             if (!bf16_tile_tensor_map(rows, a.n_rows, d, a.stride * d, 128, &tm_rows))
