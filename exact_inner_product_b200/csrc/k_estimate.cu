@@ -46,6 +46,8 @@ __global__ void __launch_bounds__(KE_THREADS) k2_estimate(const EstimateArgs a) 
     const int R = a.rank;
     pdl_trigger();  // the streaming pass may launch and wait behind this kernel
     pdl_wait();     // the queries and the work memory are ready
+    if (g == 0 && tid == 0 && a.count != nullptr) a.count[q] = 0;
+    if (g == 0 && q == 0 && tid < 4 && a.flags != nullptr) a.flags[tid] = 0;
     stage_query(a.dtype, a.queries, a.q_dtype, q, a.d, qf);
     __syncthreads();
     const float us = a.dtype == TT_I8 ? a.qscale[q] : 1.0f;

@@ -53,6 +53,9 @@ struct tt_index {
     int64_t seq;            // calls issued on the handle
     int64_t last_pending;   // seq of the last search whose status block reports it (0: none)
     tt_stats last;
+    // the flag block of the last search: its estimate tickets are zero there
+    // (cleared by the init kernel, or reset by the estimate that used them)
+    int* tickets_zero_at;
 };
 
 namespace tt {
@@ -1006,7 +1009,12 @@ static tt_status score_core(tt_index* index, const void* queries, tt_dtype q_dty
             return TT_ERR_CUDA;
     }
 
-    cudaError_t e = launch_init(sc.count, sc.theta, sc.thf, KEY_MIN, V, v_pad, sc.flags, s);
+    // With one sample the estimate is the first kernel and clears the counters
+    // and flags itself, when its tickets are known to be zero: the last search
+    // on this handle used the same flag block (the block moves with b and k).
+    const bool estimate_clears = plan.sampled && sc.flags == index->tickets_zero_at;
+    cudaError_t e = estimate_clears ? cudaSuccess
+                                    : launch_init(sc.count, sc.theta, sc.thf, KEY_MIN, V, v_pad, sc.flags, s);
     if (e == cudaSuccess) e = sets_min();
     if (e != cudaSuccess) return cuda_fail(e, "init");
     if (plan.sampled) {
@@ -1030,6 +1038,8 @@ static tt_status score_core(tt_index* index, const void* queries, tt_dtype q_dty
         es.theta = sc.theta;
         es.thf = sc.thf;
         es.tickets = sc.flags + 4;
+        es.count = estimate_clears ? sc.count : nullptr;
+        es.flags = estimate_clears ? sc.flags : nullptr;
         if ((e = launch_estimate(es, s)) != cudaSuccess) return cuda_fail(e, "threshold estimate");
     }
     for (int lv = plan.sampled ? 0 : plan.levels - 1; lv >= 0; --lv) {
@@ -1076,6 +1086,7 @@ static tt_status score_core(tt_index* index, const void* queries, tt_dtype q_dty
     ea.chunks = exact_chunks(index->n, k, plan.cap);
     e = launch_exact(ea, s, sms);
     if (e != cudaSuccess) return cuda_fail(e, "exact fallback");
+    index->tickets_zero_at = sc.flags;
     stats.rescans = -1;  // known once the work has run (tt_last_stats)
     stats.launches = (int)(g_launches.load() - launches0);
     index->last = stats;

@@ -134,6 +134,11 @@ struct EstimateArgs {
     uint64_t* theta;
     float* thf;
     int* tickets;
+    // As the search's first kernel, the estimate clears the work memory a
+    // separate init kernel clears otherwise: count[q] and flags[0..4)
+    // (null: not cleared here). The tickets clear themselves.
+    uint32_t* count;
+    int* flags;
 };
 constexpr int ESTIMATE_BLOCK_ROWS = 256;  // sample rows per block: one per thread
 constexpr int ESTIMATE_MAX_RANK = 256;    // the sample rank a plan may ask of the estimate

@@ -396,3 +396,21 @@ def test_select_widths(path, b, k):
     res, st = parity.run_case(w, path=path)
     assert st["path"] == path and st["rescans"] == 0, st
     assert res["max_abs_err"] <= w.tolerance and res["set_checked"] + res["rank_checked"] > 0, res
+
+
+@pytest.mark.parametrize("name,over", [
+    ("tiny_f32", {"n": 200_003, "d": 64, "b": 1, "k": 50, "oracle_queries": 0}),   # fp32 rows
+    ("stream_b1", {"n": 1_500_007, "b": 1, "k": 100}),                            # rows after the deferred four
+    ("masked_fused", {"n": 400_009, "b": 2, "k": 64, "oracle_queries": 0}),       # two queries, mask, norms
+])
+def test_pass_scores_rows_before_the_threshold(name, over):
+    """After the one-sample estimate the streaming pass scores each thread's
+    first rows before waiting for the threshold and filters them afterwards
+    (one or two queries per block). Every form of that pass matches the
+    oracle: fp32 rows, a corpus with more rows per thread than are deferred,
+    and a masked raw corpus with norms."""
+    _cuda()
+    w = W.workload(name, **over)
+    res, st = parity.run_case(w)
+    assert st["path"] == 1 and st["sampled"] and st["rescans"] == 0, st
+    assert res["max_abs_err"] <= w.tolerance
