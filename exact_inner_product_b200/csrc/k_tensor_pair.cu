@@ -93,6 +93,7 @@ struct KPParams {
     PassArgs a;
     int q_tiles;    // ceil(b / 256)
     int kchunks;    // ceil(d / 64)
+    int kps;        // K chunks per ring stage
     int stages;
     int64_t tiles;  // corpus tiles of 256 rows in this level
     int chunks;     // corpus chunks (units = q_tiles * chunks)
@@ -127,7 +128,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* qsm = smem;                                          // [kchunks][128 x 128 B]
     uint8_t* ring = smem + (size_t)p.kchunks * KP_QCHUNK_BYTES;   // [stages][16 KB]
-    KPCtl* ctl = reinterpret_cast<KPCtl*>(ring + (size_t)p.stages * KP_STAGE_BYTES);
+    KPCtl* ctl = reinterpret_cast<KPCtl*>(ring + (size_t)p.stages * p.kps * KP_STAGE_BYTES);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -185,16 +186,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
                     tma_load_2d_pair(qsm + (size_t)kc * KP_QCHUNK_BYTES, &tm_q, qfull0, kc * KC,
                                      qt * (2 * KP_QROWS) + (int)rank * KP_QROWS);
                 for (int64_t t = t0; ok && t < t1; ++t) {
-                    for (int kc = 0; kc < p.kchunks; ++kc, ++it) {
+                    for (int kg = 0; kg < p.kchunks; kg += p.kps, ++it) {
                         const int s = it % p.stages;
                         if (!mbar_wait(&ctl->empty[s], ((it / p.stages) & 1) ^ 1, abort)) {
                             ok = false;
                             break;
                         }
-                        if (even) mbar_arrive_expect_tx(&ctl->full[s], 2 * KP_STAGE_BYTES);
-                        tma_load_2d_pair(ring + (size_t)s * KP_STAGE_BYTES, &tm_rows,
-                                         mapa_shared(&ctl->full[s], 0), kc * KC,
-                                         (int32_t)(t * KP_TILE + (int64_t)rank * KP_ROWS));
+                        if (even) mbar_arrive_expect_tx(&ctl->full[s], (uint32_t)(2 * p.kps * KP_STAGE_BYTES));
+                        for (int j = 0; j < p.kps; ++j)
+                            tma_load_2d_pair(ring + ((size_t)s * p.kps + j) * KP_STAGE_BYTES, &tm_rows,
+                                             mapa_shared(&ctl->full[s], 0), (kg + j) * KC,
+                                             (int32_t)(t * KP_TILE + (int64_t)rank * KP_ROWS));
                     }
                 }
             }
@@ -237,23 +239,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
                     }
                     tc_fence_after();
                     const uint32_t d_tmem = tmem_base + (uint32_t)(buf * KP_ACC_COLS);
-                    for (int kc = 0; kc < p.kchunks; ++kc, ++it) {
+                    for (int kg = 0; kg < p.kchunks; kg += p.kps, ++it) {
                         const int s = it % p.stages;
                         const uint32_t par = (it / p.stages) & 1;
                         if (!mbar_wait_cluster(&ctl->full[s], par, abort)) { ok = false; break; }
                         tc_fence_after();
-                        const uint32_t a_addr = qbase + (uint32_t)(kc * KP_QCHUNK_BYTES);
-                        const uint32_t b_addr = rbase + (uint32_t)(s * KP_STAGE_BYTES);
+                        for (int j = 0; j < p.kps; ++j) {
+                            const int kc = kg + j;
+                            const uint32_t a_addr = qbase + (uint32_t)(kc * KP_QCHUNK_BYTES);
+                            const uint32_t b_addr = rbase + (uint32_t)((s * p.kps + j) * KP_STAGE_BYTES);
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {  // 32 bytes of K per instruction
-                            if constexpr (I8)
-                                umma_i8_pair(d_tmem, umma_desc_kmajor_sw128(a_addr + kk * 32),
-                                             umma_desc_kmajor_sw128(b_addr + kk * 32), p.idesc,
-                                             (kc | kk) != 0 ? 1u : 0u);
-                            else
-                                umma_bf16_pair(d_tmem, umma_desc_kmajor_sw128(a_addr + kk * 32),
-                                               umma_desc_kmajor_sw128(b_addr + kk * 32), p.idesc,
-                                               (kc | kk) != 0 ? 1u : 0u);
+                            for (int kk = 0; kk < 4; ++kk) {  // 32 bytes of K per instruction
+                                if constexpr (I8)
+                                    umma_i8_pair(d_tmem, umma_desc_kmajor_sw128(a_addr + kk * 32),
+                                                 umma_desc_kmajor_sw128(b_addr + kk * 32), p.idesc,
+                                                 (kc | kk) != 0 ? 1u : 0u);
+                                else
+                                    umma_bf16_pair(d_tmem, umma_desc_kmajor_sw128(a_addr + kk * 32),
+                                                   umma_desc_kmajor_sw128(b_addr + kk * 32), p.idesc,
+                                                   (kc | kk) != 0 ? 1u : 0u);
+                            }
                         }
                         umma_commit_pair_mc(&ctl->empty[s], 0x3);  // stage free in both CTAs
                     }
@@ -535,10 +540,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
 // K chunks of 128 bytes per row: 64 bf16 or 128 int8 elements each.
 int pair_kchunks(int d, int esize) { return (d * esize + 127) / 128; }
 
+// K chunks per ring stage: two when the row has an even number of them (one
+// barrier handshake and one commit per two chunks).
+int pair_kps(int kchunks) { return kchunks % 2 == 0 ? 2 : 1; }
+
 int pair_stages(int d, int esize) {
     const int kchunks = pair_kchunks(d, esize);
     const int fixed = 1024 + kchunks * KP_QCHUNK_BYTES + (int)sizeof(KPCtl);
-    int stages = (KP_SMEM_BUDGET - fixed) / KP_STAGE_BYTES;
+    int stages = (KP_SMEM_BUDGET - fixed) / (pair_kps(kchunks) * KP_STAGE_BYTES);
     if (stages > KP_MAX_STAGES) stages = KP_MAX_STAGES;
     return stages;
 }
@@ -590,7 +599,7 @@ int tensor_pair_smem_bytes(int d, int esize) {
     const int kchunks = pair_kchunks(d, esize);
     const int stages = pair_stages(d, esize);
     if (stages < 2) return -1;
-    return 1024 + kchunks * KP_QCHUNK_BYTES + (int)sizeof(KPCtl) + stages * KP_STAGE_BYTES;
+    return 1024 + kchunks * KP_QCHUNK_BYTES + (int)sizeof(KPCtl) + stages * pair_kps(kchunks) * KP_STAGE_BYTES;
 }
 
 cudaError_t launch_tensor_pair_pass(const PassArgs& a, const CUtensorMap& tm_rows, cudaStream_t s, int sm_count) {
@@ -609,6 +618,7 @@ cudaError_t launch_tensor_pair_pass(const PassArgs& a, const CUtensorMap& tm_row
     p.a = a;
     p.q_tiles = (a.b + 2 * KP_QROWS - 1) / (2 * KP_QROWS);
     p.kchunks = pair_kchunks(a.d, esize);
+    p.kps = pair_kps(p.kchunks);
     p.stages = pair_stages(a.d, esize);
     p.tiles = (a.n_rows + KP_TILE - 1) / KP_TILE;
     p.chunks = 1;
