@@ -12,7 +12,8 @@
 // Layout of one MMA: M = 128 corpus rows (TMEM lanes), N = NQ <= 256
 // queries (TMEM columns), K = 16. A query tile (NQ x d, bf16) stays resident
 // in shared memory for a whole work unit; corpus tiles stream through a ring
-// of 16 KB stages (128 rows x 64 elements, 128-byte swizzle). Two TMEM
+// of stages of one or two 16 KB K chunks (128 rows x 64 elements each,
+// 128-byte swizzle; two when d has an even number of chunks). Two TMEM
 // accumulators (columns 0 and 256) let the epilogue drain tile t while the
 // tensor cores work on tile t + 1.
 //
@@ -74,6 +75,7 @@ struct K3Params {
     int nq;          // queries per tile (multiple of 32, <= 256)
     int q_tiles;     // ceil(b / nq)
     int kchunks;     // 128-byte chunks of K: ceil(d * element size / 128)
+    int kps;         // K chunks per ring stage
     int stages;
     int64_t tiles;   // corpus tiles of 128 rows in this level
     int chunks;      // corpus chunks (units = q_tiles * chunks)
@@ -90,7 +92,7 @@ __device__ __forceinline__ void unit_range(const K3Params& p, int u, int* qt, in
 
 // I8: int8 codes (kind::i8, int32 accumulators; recsys_two_tower_model.py
 // `compute_top_k_int8`), else bf16 (kind::f16, fp32 accumulators).
-template <bool I8>
+template <bool I8, int KPS>
 __global__ void __launch_bounds__(K3_THREADS, 1)
     k3_tensor(const __grid_constant__ CUtensorMap tm_rows, const __grid_constant__ CUtensorMap tm_q,
               const K3Params p) {
@@ -101,7 +103,7 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
     const int q_chunk_bytes = p.nq * 128;
     uint8_t* qsm = smem;                                           // [kchunks][nq x 128 B]
     uint8_t* ring = smem + (size_t)p.kchunks * q_chunk_bytes;      // [stages][16 KB]
-    K3Ctl* ctl = reinterpret_cast<K3Ctl*>(ring + (size_t)p.stages * K3_STAGE_BYTES);
+    K3Ctl* ctl = reinterpret_cast<K3Ctl*>(ring + (size_t)p.stages * KPS * K3_STAGE_BYTES);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -158,16 +160,18 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
                     tma_load_2d(qsm + (size_t)kc * q_chunk_bytes, &tm_q, &ctl->qfull, kc * KC,
                                 qt * p.nq);
                 for (int64_t t = t0; ok && t < t1; ++t) {
-                    for (int kc = 0; kc < p.kchunks; ++kc, ++it) {
+                    for (int kg = 0; kg < p.kchunks; kg += KPS, ++it) {
                         const int s = it % p.stages;
                         if (!mbar_wait(&ctl->empty[s], ((it / p.stages) & 1) ^ 1, abort)) {
                             ok = false;
                             break;
                         }
                         if (p.a.withhold_copy && it == 0) continue;  // test hook: never lands
-                        mbar_arrive_expect_tx(&ctl->full[s], K3_STAGE_BYTES);
-                        tma_load_2d(ring + (size_t)s * K3_STAGE_BYTES, &tm_rows, &ctl->full[s],
-                                    kc * KC, (int32_t)(t * K3_M));
+                        mbar_arrive_expect_tx(&ctl->full[s], (uint32_t)(KPS * K3_STAGE_BYTES));
+#pragma unroll
+                        for (int j = 0; j < KPS; ++j)
+                            tma_load_2d(ring + ((size_t)s * KPS + j) * K3_STAGE_BYTES, &tm_rows, &ctl->full[s],
+                                        (kg + j) * KC, (int32_t)(t * K3_M));
                     }
                 }
             }
@@ -200,22 +204,26 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
                     if (!mbar_wait(&ctl->tempty[buf], ((tc >> 1) & 1) ^ 1, abort)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t d_tmem = tmem_base + (uint32_t)(buf * K3_ACC_COLS);
-                    for (int kc = 0; kc < p.kchunks; ++kc, ++it) {
+                    for (int kg = 0; kg < p.kchunks; kg += KPS, ++it) {
                         const int s = it % p.stages;
                         if (!mbar_wait(&ctl->full[s], (it / p.stages) & 1, abort)) { ok = false; break; }
                         tc_fence_after();
-                        const uint32_t a_addr = rbase + (uint32_t)(s * K3_STAGE_BYTES);
-                        const uint32_t b_addr = qbase + (uint32_t)(kc * q_chunk_bytes);
 #pragma unroll
-                        for (int kk = 0; kk < K3_ROW_BYTES / 32; ++kk) {  // 32 bytes of K per MMA
-                            if constexpr (I8)
-                                umma_i8(d_tmem, umma_desc_kmajor_sw128(a_addr + kk * 32),
-                                        umma_desc_kmajor_sw128(b_addr + kk * 32), p.idesc,
-                                        (kc | kk) != 0 ? 1u : 0u);
-                            else
-                                umma_bf16(d_tmem, umma_desc_kmajor_sw128(a_addr + kk * 32),
-                                          umma_desc_kmajor_sw128(b_addr + kk * 32), p.idesc,
-                                          (kc | kk) != 0 ? 1u : 0u);
+                        for (int j = 0; j < KPS; ++j) {
+                            const int kc = kg + j;
+                            const uint32_t a_addr = rbase + (uint32_t)((s * KPS + j) * K3_STAGE_BYTES);
+                            const uint32_t b_addr = qbase + (uint32_t)(kc * q_chunk_bytes);
+#pragma unroll
+                            for (int kk = 0; kk < K3_ROW_BYTES / 32; ++kk) {  // 32 bytes of K per MMA
+                                if constexpr (I8)
+                                    umma_i8(d_tmem, umma_desc_kmajor_sw128(a_addr + kk * 32),
+                                            umma_desc_kmajor_sw128(b_addr + kk * 32), p.idesc,
+                                            (kc | kk) != 0 ? 1u : 0u);
+                                else
+                                    umma_bf16(d_tmem, umma_desc_kmajor_sw128(a_addr + kk * 32),
+                                              umma_desc_kmajor_sw128(b_addr + kk * 32), p.idesc,
+                                              (kc | kk) != 0 ? 1u : 0u);
+                            }
                         }
                         umma_commit(&ctl->empty[s]);  // stage free once these MMAs finish
                     }
@@ -406,14 +414,23 @@ __global__ void __launch_bounds__(K3_THREADS, 1)
 
 }  // namespace
 
+// K chunks per ring stage: two for rows of two chunks (one barrier handshake
+// and one commit per tile: the 10^7 x 128, 32-query pass went from 0.56 to
+// 0.53 ms), else one (rows of four chunks, 2*10^7 x 256 with 4096 queries,
+// measured 8 % slower with two).
+static int k3_kps(int kchunks, int fixed) {
+    return (kchunks == 2 && (K3_SMEM_BUDGET - fixed) / (2 * K3_STAGE_BYTES) >= 3) ? 2 : 1;
+}
+
 int tensor_pass_smem_bytes(int d, int nq, int esize) {
     const int kchunks = (d * esize + K3_ROW_BYTES - 1) / K3_ROW_BYTES;
     const int q_bytes = kchunks * nq * 128;
     const int fixed = 1024 + q_bytes + (int)sizeof(K3Ctl);
-    int stages = (K3_SMEM_BUDGET - fixed) / K3_STAGE_BYTES;
+    const int kps = k3_kps(kchunks, fixed);
+    int stages = (K3_SMEM_BUDGET - fixed) / (kps * K3_STAGE_BYTES);
     if (stages > K3_MAX_STAGES) stages = K3_MAX_STAGES;
     if (stages < 2) return -1;
-    return fixed + stages * K3_STAGE_BYTES;
+    return fixed + stages * kps * K3_STAGE_BYTES;
 }
 
 int tensor_pass_max_nq(int d, int esize) {
@@ -438,7 +455,8 @@ cudaError_t launch_tensor_pass(const PassArgs& a, const CUtensorMap& tm_rows,
     const int smem = tensor_pass_smem_bytes(a.d, nq, esize);
     if (smem <= 0) return cudaErrorInvalidValue;
     const int fixed = 1024 + p.kchunks * nq * 128 + (int)sizeof(K3Ctl);
-    p.stages = (smem - fixed) / K3_STAGE_BYTES;
+    p.kps = k3_kps(p.kchunks, fixed);
+    p.stages = (smem - fixed) / (p.kps * K3_STAGE_BYTES);
     p.tiles = (a.n_rows + K3_M - 1) / K3_M;
     // Corpus chunks: make q_tiles * chunks a multiple of the SM count when
     // possible (every CTA gets the same number of units), with at least one
@@ -453,14 +471,12 @@ cudaError_t launch_tensor_pass(const PassArgs& a, const CUtensorMap& tm_rows,
     p.idesc = i8 ? umma_idesc_s8(K3_M, nq) : umma_idesc_bf16(K3_M, nq);
     const int n_units = p.q_tiles * p.chunks;
     const int grid = n_units < sm_count ? n_units : sm_count;
-    cudaError_t e = i8 ? cudaFuncSetAttribute(k3_tensor<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
-                       : cudaFuncSetAttribute(k3_tensor<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    auto kern = i8 ? (p.kps == 2 ? k3_tensor<true, 2> : k3_tensor<true, 1>)
+                   : (p.kps == 2 ? k3_tensor<false, 2> : k3_tensor<false, 1>);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     note_launch_begin(TT_KIND_TENSOR, s);
-    if (i8)
-        k3_tensor<true><<<grid, K3_THREADS, smem, s>>>(tm_rows, tm_queries, p);
-    else
-        k3_tensor<false><<<grid, K3_THREADS, smem, s>>>(tm_rows, tm_queries, p);
+    kern<<<grid, K3_THREADS, smem, s>>>(tm_rows, tm_queries, p);
     note_launch_end(TT_KIND_TENSOR, s);
     return cudaGetLastError();
 }

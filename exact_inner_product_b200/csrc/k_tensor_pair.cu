@@ -117,7 +117,7 @@ __device__ __forceinline__ void raise_abort(KPCtl* ctl, uint32_t peer) {
 // NORMS: per-row score scales (raw rows with norms); MASK: an exclusion
 // bitmask; TYPES: several result sets by candidate type; I8: int8 codes
 // (kind::i8, int32 accumulators) with per-row and per-query scales.
-template <bool NORMS, bool MASK, bool TYPES, bool I8>
+template <bool NORMS, bool MASK, bool TYPES, bool I8, int KPS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
     k3_pair(const __grid_constant__ CUtensorMap tm_rows, const __grid_constant__ CUtensorMap tm_q,
             const KPParams p) {
@@ -128,7 +128,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* qsm = smem;                                          // [kchunks][128 x 128 B]
     uint8_t* ring = smem + (size_t)p.kchunks * KP_QCHUNK_BYTES;   // [stages][16 KB]
-    KPCtl* ctl = reinterpret_cast<KPCtl*>(ring + (size_t)p.stages * p.kps * KP_STAGE_BYTES);
+    KPCtl* ctl = reinterpret_cast<KPCtl*>(ring + (size_t)p.stages * KPS * KP_STAGE_BYTES);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -186,15 +186,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
                     tma_load_2d_pair(qsm + (size_t)kc * KP_QCHUNK_BYTES, &tm_q, qfull0, kc * KC,
                                      qt * (2 * KP_QROWS) + (int)rank * KP_QROWS);
                 for (int64_t t = t0; ok && t < t1; ++t) {
-                    for (int kg = 0; kg < p.kchunks; kg += p.kps, ++it) {
+                    for (int kg = 0; kg < p.kchunks; kg += KPS, ++it) {
                         const int s = it % p.stages;
                         if (!mbar_wait(&ctl->empty[s], ((it / p.stages) & 1) ^ 1, abort)) {
                             ok = false;
                             break;
                         }
-                        if (even) mbar_arrive_expect_tx(&ctl->full[s], (uint32_t)(2 * p.kps * KP_STAGE_BYTES));
-                        for (int j = 0; j < p.kps; ++j)
-                            tma_load_2d_pair(ring + ((size_t)s * p.kps + j) * KP_STAGE_BYTES, &tm_rows,
+                        if (even) mbar_arrive_expect_tx(&ctl->full[s], (uint32_t)(2 * KPS * KP_STAGE_BYTES));
+#pragma unroll
+                        for (int j = 0; j < KPS; ++j)
+                            tma_load_2d_pair(ring + ((size_t)s * KPS + j) * KP_STAGE_BYTES, &tm_rows,
                                              mapa_shared(&ctl->full[s], 0), (kg + j) * KC,
                                              (int32_t)(t * KP_TILE + (int64_t)rank * KP_ROWS));
                     }
@@ -239,15 +240,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
                     }
                     tc_fence_after();
                     const uint32_t d_tmem = tmem_base + (uint32_t)(buf * KP_ACC_COLS);
-                    for (int kg = 0; kg < p.kchunks; kg += p.kps, ++it) {
+                    for (int kg = 0; kg < p.kchunks; kg += KPS, ++it) {
                         const int s = it % p.stages;
                         const uint32_t par = (it / p.stages) & 1;
                         if (!mbar_wait_cluster(&ctl->full[s], par, abort)) { ok = false; break; }
                         tc_fence_after();
-                        for (int j = 0; j < p.kps; ++j) {
+#pragma unroll
+                        for (int j = 0; j < KPS; ++j) {
                             const int kc = kg + j;
                             const uint32_t a_addr = qbase + (uint32_t)(kc * KP_QCHUNK_BYTES);
-                            const uint32_t b_addr = rbase + (uint32_t)((s * p.kps + j) * KP_STAGE_BYTES);
+                            const uint32_t b_addr = rbase + (uint32_t)((s * KPS + j) * KP_STAGE_BYTES);
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk) {  // 32 bytes of K per instruction
                                 if constexpr (I8)
@@ -540,9 +542,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
 // K chunks of 128 bytes per row: 64 bf16 or 128 int8 elements each.
 int pair_kchunks(int d, int esize) { return (d * esize + 127) / 128; }
 
-// K chunks per ring stage: two when the row has an even number of them (one
-// barrier handshake and one commit per two chunks).
-int pair_kps(int kchunks) { return kchunks % 2 == 0 ? 2 : 1; }
+// K chunks per ring stage: two for rows of two chunks (d = 128 bf16: one
+// barrier handshake and one commit per tile), else one (the single-SM kernel
+// measured slower with two on rows of four chunks).
+int pair_kps(int kchunks) { return kchunks == 2 ? 2 : 1; }
 
 int pair_stages(int d, int esize) {
     const int kchunks = pair_kchunks(d, esize);
@@ -555,7 +558,9 @@ int pair_stages(int d, int esize) {
 template <bool NORMS, bool MASK, bool TYPES, bool I8 = false>
 cudaError_t launch_variant(const KPParams& base, const CUtensorMap& tm_rows, const CUtensorMap& tm_queries,
                            int smem, cudaStream_t s, int sm_count) {
-    auto kern = k3_pair<NORMS, MASK, TYPES, I8>;
+    // the stage grouping is a compile-time constant: a run-time bound on the
+    // MMA issuer's inner loop cost the single-SM kernel 8 % on 2*10^7 x 256 rows
+    auto kern = base.kps == 2 ? k3_pair<NORMS, MASK, TYPES, I8, 2> : k3_pair<NORMS, MASK, TYPES, I8, 1>;
     KPParams p = base;
     // Pairs that can be resident at once (clusters must fit inside a GPC).
     int pairs = sm_count / 2 > 0 ? sm_count / 2 : 1;
