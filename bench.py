@@ -70,14 +70,14 @@ TRAFFIC = {
                                     "sha": "4273a9f8869b74ec01b8762c20eb598dc6f0b1597fcd3e5f8ad9afde664127f4"},
     # ncu --set full --import-source no --clock-control none -k regex:k3_pair -s 8 -c 1 on `python bench.py
     # --workload large_batch --n 4000000 --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass,
-    # 4,000,000 rows): 1092.787 MB read + 29.671 MB written; scaled to the full corpus by rows scanned
-    ("k3_pair", "large_batch"): {"bytes_per_row": 280.615, "src": "exact_inner_product_b200/csrc/k_tensor_pair.cu",
-                                 "sha": "9c6e8b8b844010494e6a9b58ec46d9018dadaf82caa4fcd975a7e92590a5471f"},
-    # ncu --set full --clock-control none -k regex:k3_tensor -s 5 -c 1 on `python bench.py --workload masked_fused --n 4000000
-    # --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass, 4,000,000 rows): 4385.550 MB read
-    # + 66.286 MB written; scaled to the full corpus by rows scanned
-    ("k3_tensor", "masked_fused"): {"bytes_per_row": 1112.959, "src": "exact_inner_product_b200/csrc/k_tensor.cu",
-                                    "sha": "dcfd00e71e06c525df0eb6aac897f7ad09d53050bd7abde0b4238ef405fb3486"},
+    # 4,000,000 rows): 1066.455 MB read + 27.004 MB written; scaled to the full corpus by rows scanned
+    ("k3_pair", "large_batch"): {"bytes_per_row": 273.365, "src": "exact_inner_product_b200/csrc/k_tensor_pair.cu",
+                                 "sha": "fe96c9c80fcef016851e2cc5569f9b9b67b3d7bfb3929d40c4bfb96d4e0d64d5"},
+    # ncu --set full --import-source no --clock-control none -k regex:k3_tensor -s 8 -c 1 on `python bench.py
+    # --workload masked_fused --n 4000000 --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass,
+    # 4,000,000 rows): 4145.305 MB read + 66.409 MB written; scaled to the full corpus by rows scanned
+    ("k3_tensor", "masked_fused"): {"bytes_per_row": 1052.929, "src": "exact_inner_product_b200/csrc/k_tensor.cu",
+                                    "sha": "d8167680c49f9dea7eb98c71503e446b913a57b8dae7e637926c337aee2309ab"},
 }
 
 
