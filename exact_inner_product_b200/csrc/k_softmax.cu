@@ -20,17 +20,28 @@
 //   k5_columns      per column: bias nb_j = -log q_j * log2(e) (-inf for an
 //                   invalid column) and item group g_j (the table slot of its
 //                   id, so equal ids <=> equal groups); zero the error word
+//   k5_sort_count,  (with item ids) a stable counting sort of the rows and of
+//   k5_sort_scan,   the columns by a 256-bin hash of the item id (rows and the
+//   k5_sort_scatter first b columns by one permutation, the shared negatives
+//   k5_permute      by another), then copies of the users, the items and the
+//                   column data in that order, so that a row's hits can only lie
+//                   in its bins' column ranges
 //   k5_softmax      tcgen05 MMAs of 128 users x 192 candidates into TMEM;
 //                   the epilogue turns each accumulator row into running
 //                   (max, sum of 2^(x - max)) pairs, x = acc * log2(e)/tau + nb_j,
 //                   so the exponentials never leave registers
 //   k5_merge        per row: combine the partial pairs (and, with item ids,
-//                   the diagonal term the group test left out), lse, loss,
-//                   and the mean over valid rows in a fixed order
+//                   the diagonal term the group test left out), lse, loss
+//                   (written at the row's own index), and the mean over valid
+//                   rows in a fixed order
 //
 // The epilogue runs in base-2 units so that each term is one ex2.approx
 // (MUFU) instruction; that unit, 16 results per clock per SM, bounds the
-// kernel at d <= 128, not the tensor cores.
+// kernel at d <= 128, not the tensor cores. With item ids, the hit test (a
+// compare and a select per logit) would cost as much issue time as the
+// exponential itself; in the bin order, an epilogue warp's 32 rows fall in a
+// few bins, so one warp-uniform range test per 32-column chunk tells where a
+// hit is possible at all and only those chunks (a few percent) run the test.
 //
 // Every wait is bounded; on expiry the kernel records an error code, the
 // merge writes NaN to every output, and the host check reports a timeout.
@@ -68,6 +79,10 @@ constexpr float K5_LOG2E = 1.4426950408889634f;
 constexpr float K5_LN2 = 0.6931471805599453f;
 constexpr unsigned long long K5_EMPTY = 0x8000000000000000ull;  // free table slot
 constexpr int K5_MERGE_THREADS = 256;
+constexpr int K5_BINS = 256;                 // sort bins: the top 8 bits of the id's hash
+constexpr int K5_SORT_THREADS = 256;         // one element per thread and round
+constexpr int K5_SORT_WARPS = K5_SORT_THREADS / 32;
+constexpr int K5_SCAN_THREADS = 1024;
 
 struct alignas(8) ColInfo {
     float nb;  // -log q_j * log2(e), or -inf when the column is invalid or past nc
@@ -85,12 +100,18 @@ struct K5Ctl {
     // per epilogue warp: biases and groups of its columns, for two tiles in flight
     alignas(16) float nb[K5_EPI_WARPS][2][K5_WARP_COLS];
     alignas(16) int grp[K5_EPI_WARPS][2][K5_WARP_COLS];
+    // per epilogue warp, with item ids: the column ranges [lo0, hi0) and
+    // [lo1, hi1) where its rows can have hits (kept here, not in registers)
+    alignas(16) int hit_cols[K5_EPI_WARPS][4];
 };
 static_assert(offsetof(K5Ctl, nb) % 16 == 0 && offsetof(K5Ctl, grp) % 16 == 0,
               "float4 / int4 reads of the column data need 16-byte alignment");
 
 struct K5Params {
-    const ColInfo* col;  // [nc]
+    const ColInfo* col;  // [nc] (with item ids: in the bin order)
+    const uint8_t* sbin; // with item ids: [b] bin of each row in the bin order, else null
+    const int* bstart;   // with item ids: [2][K5_BINS + 1] first column of each bin, in-batch
+                         // columns then shared negatives (the last entry: the part's end)
     float* numer;        // [b] diagonal logit, base-2 units
     float2* part;        // [chunks * K5_COL_GROUPS][b] (running max, sum)
     int* err;
@@ -205,6 +226,164 @@ __global__ void k5_columns(const float* __restrict__ logq, const uint8_t* __rest
         }
     }
     col[j] = c;
+}
+
+// ---------------------------------------------------------------------------
+// the bin order (item ids only)
+//
+// A stable counting sort, done separately on the two parts of the columns:
+// part 0 = [0, b) (the rows use the same permutation, so row r's positive
+// stays column r) and part 1 = [b, nc) (the shared negatives). The key of
+// column j is bin(id_j); equal ids share a bin, so the columns that can be
+// hits of row r lie in the column ranges of bin(r) in both parts. Stable
+// ranks make the order, and with it every sum, the same on every run.
+//
+// Part p is cut into tiles of `tile` elements; hist holds, part after part,
+// bin-major, the count of each (bin, tile); its exclusive prefix is the
+// sorted position of the first element of each (bin, tile).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int k5_bin(long long id) {
+    return (int)(((unsigned long long)id * 0x9E3779B97F4A7C15ull) >> 56);
+}
+
+struct SortShape {
+    int b, nc, tile, tiles0, tiles1;
+    __device__ __forceinline__ void block_part(int blk, int* part, int* t, int* lo, int* hi) const {
+        *part = blk < tiles0 ? 0 : 1;
+        *t = *part == 0 ? blk : blk - tiles0;
+        const int base = *part == 0 ? 0 : b;
+        const int end = *part == 0 ? b : nc;
+        *lo = base + *t * tile;
+        *hi = *lo + tile < end ? *lo + tile : end;
+    }
+    __device__ __forceinline__ int64_t hist_at(int part, int bin, int t) const {
+        return part == 0 ? (int64_t)bin * tiles0 + t : (int64_t)K5_BINS * tiles0 + (int64_t)bin * tiles1 + t;
+    }
+};
+
+__global__ void __launch_bounds__(K5_SORT_THREADS)
+    k5_sort_count(const int64_t* __restrict__ item_ids, SortShape sh, int* __restrict__ hist) {
+    __shared__ int h[K5_BINS];
+    int part, t, lo, hi;
+    sh.block_part(blockIdx.x, &part, &t, &lo, &hi);
+    h[threadIdx.x] = 0;
+    __syncthreads();
+    for (int j = lo + threadIdx.x; j < hi; j += K5_SORT_THREADS) atomicAdd(&h[k5_bin(item_ids[j])], 1);
+    __syncthreads();
+    hist[sh.hist_at(part, threadIdx.x, t)] = h[threadIdx.x];
+}
+
+// One block: exclusive prefix of hist in place, then the bin starts. hist
+// has a multiple of 256 entries; each thread scans a slice of whole int4s.
+__global__ void __launch_bounds__(K5_SCAN_THREADS)
+    k5_sort_scan(SortShape sh, int* __restrict__ hist, int* __restrict__ bstart) {
+    __shared__ int warp_tot[K5_SCAN_THREADS / 32];
+    const int64_t len4 = (int64_t)K5_BINS / 4 * (sh.tiles0 + sh.tiles1);
+    const int64_t per4 = (len4 + K5_SCAN_THREADS - 1) / K5_SCAN_THREADS;
+    const int64_t a = threadIdx.x * per4;
+    const int64_t e = a + per4 < len4 ? a + per4 : len4;
+    int4* h4 = reinterpret_cast<int4*>(hist);
+    int mine = 0;
+#pragma unroll 4
+    for (int64_t q = a; q < e; ++q) {
+        const int4 v = h4[q];
+        mine += v.x + v.y + v.z + v.w;
+    }
+    // block exclusive scan of the per-thread totals
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int inc = mine;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+    }
+    if (lane == 31) warp_tot[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        int w = warp_tot[lane];
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        warp_tot[lane] = w;  // inclusive
+    }
+    __syncthreads();
+    int run = inc - mine + (warp > 0 ? warp_tot[warp - 1] : 0);
+#pragma unroll 4
+    for (int64_t q = a; q < e; ++q) {
+        const int4 v = h4[q];
+        int4 o;
+        o.x = run;
+        o.y = o.x + v.x;
+        o.z = o.y + v.y;
+        o.w = o.z + v.z;
+        run = o.w + v.w;
+        h4[q] = o;
+    }
+    __syncthreads();
+    for (int k = threadIdx.x; k < 2 * (K5_BINS + 1); k += K5_SCAN_THREADS) {
+        const int part = k / (K5_BINS + 1), bin = k % (K5_BINS + 1);
+        const int tiles = part == 0 ? sh.tiles0 : sh.tiles1;
+        const int end = part == 0 ? sh.b : sh.nc;
+        bstart[k] = (bin < K5_BINS && tiles > 0) ? hist[sh.hist_at(part, bin, 0)] : end;
+    }
+}
+
+// Element j of a tile goes to hist[(bin, tile)] + (elements of its bin
+// before it in the tile); the tile is walked in rounds of 256 in index order.
+__global__ void __launch_bounds__(K5_SORT_THREADS)
+    k5_sort_scatter(const int64_t* __restrict__ item_ids, SortShape sh, const int* __restrict__ hist,
+                    int* __restrict__ perm, uint8_t* __restrict__ sbin) {
+    __shared__ int run[K5_BINS];
+    __shared__ int wcnt[K5_SORT_WARPS][K5_BINS];
+    int part, t, lo, hi;
+    sh.block_part(blockIdx.x, &part, &t, &lo, &hi);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    run[threadIdx.x] = 0;
+    for (int w = 0; w < K5_SORT_WARPS; ++w) wcnt[w][threadIdx.x] = 0;
+    __syncthreads();
+    for (int r0 = lo; r0 < hi; r0 += K5_SORT_THREADS) {
+        const int j = r0 + threadIdx.x;
+        const bool in = j < hi;
+        const int bin = in ? k5_bin(item_ids[j]) : K5_BINS;  // K5_BINS: no element
+        const unsigned peers = __match_any_sync(0xffffffffu, bin);
+        const int lrank = __popc(peers & ((1u << lane) - 1u));
+        if (in && lrank == 0) wcnt[warp][bin] = __popc(peers);
+        __syncthreads();
+        if (in) {
+            int pos = hist[sh.hist_at(part, bin, t)] + run[bin] + lrank;
+            for (int w = 0; w < warp; ++w) pos += wcnt[w][bin];
+            perm[pos] = j;
+            if (part == 0) sbin[pos] = (uint8_t)bin;
+        }
+        __syncthreads();
+        int add = 0;
+        for (int w = 0; w < K5_SORT_WARPS; ++w) {
+            add += wcnt[w][threadIdx.x];
+            wcnt[w][threadIdx.x] = 0;
+        }
+        run[threadIdx.x] += add;
+        __syncthreads();
+    }
+}
+
+// Sorted position q takes original row perm[q]: items (and, for q < b,
+// users) in 16-byte pieces, and the column data.
+__global__ void k5_permute(const int* __restrict__ perm, int b, int nc, int vpr, const uint4* __restrict__ users,
+                           const uint4* __restrict__ items, const ColInfo* __restrict__ col, uint4* __restrict__ users_s,
+                           uint4* __restrict__ items_s, ColInfo* __restrict__ col_s, int* err) {
+    const int64_t total = (int64_t)nc * vpr;
+    for (int64_t v = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; v < total; v += (int64_t)gridDim.x * blockDim.x) {
+        const int q = (int)(v / vpr);
+        const int piece = (int)(v - (int64_t)q * vpr);
+        const int src = perm[q];
+        if ((unsigned)src >= (unsigned)(q < b ? b : nc)) {  // never, for a permutation of each part
+            atomicExch(err, ERR_BAD_ORDER);
+            continue;
+        }
+        items_s[v] = items[(int64_t)src * vpr + piece];
+        if (q < b) users_s[v] = users[(int64_t)src * vpr + piece];
+        if (piece == 0) col_s[q] = col[src];
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -361,6 +540,23 @@ __global__ void __launch_bounds__(K5_THREADS, 1)
             const int i = ut * K5_M + quarter * 32 + lane;  // this thread's user
             const bool row_ok = i < p.b;
             const int my_g = (HITS && row_ok) ? p.col[i].g : -1;
+            // Columns where this warp's rows can have hits: the ranges of the
+            // bins from its first row's to its last row's, in both parts.
+            if constexpr (HITS) {
+                __syncwarp();  // the previous unit's reads are done
+                if (lane == 0) {
+                    int4 r = make_int4(0, 0, 0, 0);
+                    const int r0 = ut * K5_M + quarter * 32;
+                    if (r0 < p.b) {
+                        const int rl = r0 + 31 < p.b ? r0 + 31 : p.b - 1;
+                        const int k0 = p.sbin[r0], k1 = p.sbin[rl];
+                        r = make_int4(p.bstart[k0], p.bstart[k1 + 1], p.bstart[K5_BINS + 1 + k0],
+                                      p.bstart[K5_BINS + 1 + k1 + 1]);
+                    }
+                    *reinterpret_cast<int4*>(ctl->hit_cols[ew]) = r;
+                }
+                __syncwarp();
+            }
             // Running max m (base-2 units) and sum of 2^(x - m). m is raised
             // only when a chunk's sum leaves [0, 2^64] (terms up to 2^64 are
             // exact enough and far from overflow), so the common path needs
@@ -393,7 +589,15 @@ __global__ void __launch_bounds__(K5_THREADS, 1)
                     for (int e = 0; e < 32; ++e) tmp.x[e] = x[e];
                     p.numer[i] = select32(tmp, i - col0);
                 }
+                bool maybe_hit = false;
                 if constexpr (HITS) {
+                    int lo0, hi0, lo1, hi1;
+                    asm volatile("ld.shared.v4.s32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(lo0), "=r"(hi0), "=r"(lo1), "=r"(hi1)
+                                 : "r"(smem_u32(ctl->hit_cols[ew])));
+                    maybe_hit = (col0 < hi0 && col0 + 32 > lo0) || (col0 < hi1 && col0 + 32 > lo1);
+                }
+                if (maybe_hit) {  // warp-uniform
                     const int4* g4 = reinterpret_cast<const int4*>(g_s + c * 32);
 #pragma unroll
                     for (int e4 = 0; e4 < 8; ++e4) {
@@ -546,8 +750,8 @@ __global__ void __launch_bounds__(K5_THREADS, 1)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(K5_MERGE_THREADS)
     k5_merge(const float2* __restrict__ part, int parts, const float* __restrict__ numer,
-             const uint8_t* __restrict__ valid, int b, int hits, const int* err, float* lse, float* loss,
-             float* mean, double* block_sum, int* block_rows, unsigned* ticket) {
+             const uint8_t* __restrict__ valid, const int* __restrict__ perm, int b, int hits, const int* err,
+             float* lse, float* loss, float* mean, double* block_sum, int* block_rows, unsigned* ticket) {
     __shared__ double red_s[K5_MERGE_THREADS / 32];
     __shared__ int red_n[K5_MERGE_THREADS / 32];
     __shared__ bool last;
@@ -565,12 +769,16 @@ __global__ void __launch_bounds__(K5_MERGE_THREADS)
             sum += pq.y * exp2f(pq.x - mx);
         }
         const float l2 = sum > 0.0f ? mx + log2f(sum) : -INFINITY;
-        const bool row_valid = valid ? valid[i] != 0 : true;
+        const int o = perm ? perm[i] : i;  // the row's own index
+        const bool o_ok = (unsigned)o < (unsigned)b;  // always, k5_permute checked it
+        const bool row_valid = o_ok && (valid ? valid[o] != 0 : true);
         float li = row_valid ? (l2 - num) * K5_LN2 : 0.0f;
         float le = l2 * K5_LN2;
         if (failed) li = le = NAN;
-        lse[i] = le;
-        loss[i] = li;
+        if (o_ok) {
+            lse[o] = le;
+            loss[o] = li;
+        }
         if (row_valid) {
             my_loss = (double)li;
             my_rows = 1;
@@ -599,15 +807,32 @@ __global__ void __launch_bounds__(K5_MERGE_THREADS)
         last = atomicAdd(ticket, 1u) == gridDim.x - 1;
     }
     __syncthreads();
-    if (last && threadIdx.x == 0) {  // the last block adds the block sums in block order
+    if (last) {  // the last block adds the block sums: a fixed-shape tree, the same on every run
         __threadfence();
         double s = 0.0;
-        long long n = 0;
-        for (unsigned blk = 0; blk < gridDim.x; ++blk) {
+        int n = 0;
+        for (unsigned blk = threadIdx.x; blk < gridDim.x; blk += K5_MERGE_THREADS) {
             s += ((volatile double*)block_sum)[blk];
             n += ((volatile int*)block_rows)[blk];
         }
-        *mean = failed ? NAN : (n > 0 ? (float)(s / (double)n) : 0.0f);
+        for (int o = 16; o > 0; o >>= 1) {
+            s += __shfl_xor_sync(0xffffffffu, s, o);
+            n += __shfl_xor_sync(0xffffffffu, n, o);
+        }
+        if ((threadIdx.x & 31) == 0) {
+            red_s[threadIdx.x >> 5] = s;
+            red_n[threadIdx.x >> 5] = n;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            double tot = 0.0;
+            long long rows = 0;
+            for (int w = 0; w < K5_MERGE_THREADS / 32; ++w) {
+                tot += red_s[w];
+                rows += red_n[w];
+            }
+            *mean = failed ? NAN : (rows > 0 ? (float)(tot / (double)rows) : 0.0f);
+        }
     }
 }
 
@@ -649,6 +874,11 @@ SoftmaxPlan softmax_plan(int b, int nc, int d, bool item_ids, int sm_count) {
     pl.chunks = chunks;
     pl.log2_slots = item_ids ? log2_ceil(2 * (int64_t)(nc > 32 ? nc : 32)) : 0;
     pl.merge_blocks = (b + K5_MERGE_THREADS - 1) / K5_MERGE_THREADS;
+    // bin order: tiles of a multiple of 1024 elements, at most 1024 tiles per part
+    pl.sort_tile = 1024 * (int)(((int64_t)nc + (1 << 20) - 1) >> 20);
+    if (pl.sort_tile < 1024) pl.sort_tile = 1024;
+    pl.sort_tiles0 = item_ids ? (b + pl.sort_tile - 1) / pl.sort_tile : 0;
+    pl.sort_tiles1 = item_ids ? (nc - b + pl.sort_tile - 1) / pl.sort_tile : 0;
     // workspace: every region starts on a 256-byte boundary
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -664,6 +894,14 @@ SoftmaxPlan softmax_plan(int b, int nc, int d, bool item_ids, int sm_count) {
     pl.off_keys = take(item_ids ? ((size_t)1 << pl.log2_slots) * sizeof(unsigned long long) : 0);
     pl.off_block_sum = take((size_t)(pl.merge_blocks > 0 ? pl.merge_blocks : 1) * sizeof(double));
     pl.off_block_rows = take((size_t)(pl.merge_blocks > 0 ? pl.merge_blocks : 1) * sizeof(int));
+    const size_t row_bytes = (size_t)d * 2;  // bf16
+    pl.off_perm = take(item_ids ? (size_t)nc * sizeof(int) : 0);
+    pl.off_sbin = take(item_ids ? (size_t)b : 0);
+    pl.off_hist = take(item_ids ? (size_t)K5_BINS * (pl.sort_tiles0 + pl.sort_tiles1) * sizeof(int) : 0);
+    pl.off_bstart = take(item_ids ? (size_t)2 * (K5_BINS + 1) * sizeof(int) : 0);
+    pl.off_col_s = take(item_ids ? (size_t)nc * sizeof(ColInfo) : 0);
+    pl.off_users_s = take(item_ids ? (size_t)b * row_bytes : 0);
+    pl.off_items_s = take(item_ids ? (size_t)nc * row_bytes : 0);
     pl.bytes = off;
     return pl;
 }
@@ -672,9 +910,9 @@ SoftmaxPlan softmax_plan(int b, int nc, int d, bool item_ids, int sm_count) {
 bool softmax_supported(int d) { return d >= 64 && d <= 512 && softmax_stages(d) >= 2; }
 
 cudaError_t launch_softmax(const SoftmaxPlan& pl, const CUtensorMap& tm_users, const CUtensorMap& tm_items,
-                           int b, int nc, int d, float tau, const float* logq, const int64_t* item_ids,
-                           const uint8_t* valid, float* lse, float* loss, float* mean, void* workspace,
-                           cudaStream_t s, int sm_count) {
+                           const void* users, const void* items, int b, int nc, int d, float tau, const float* logq,
+                           const int64_t* item_ids, const uint8_t* valid, float* lse, float* loss, float* mean,
+                           void* workspace, cudaStream_t s, int sm_count) {
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     ColInfo* col = reinterpret_cast<ColInfo*>(ws + pl.off_col);
     float* numer = reinterpret_cast<float*>(ws + pl.off_numer);
@@ -701,8 +939,49 @@ cudaError_t launch_softmax(const SoftmaxPlan& pl, const CUtensorMap& tm_users, c
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (b == 0) return cudaMemsetAsync(mean, 0, sizeof(float), s);
 
+    int* perm = nullptr;
+    if (hits) {
+        SortShape sh;
+        sh.b = b;
+        sh.nc = nc;
+        sh.tile = pl.sort_tile;
+        sh.tiles0 = pl.sort_tiles0;
+        sh.tiles1 = pl.sort_tiles1;
+        perm = reinterpret_cast<int*>(ws + pl.off_perm);
+        uint8_t* sbin = ws + pl.off_sbin;
+        int* hist = reinterpret_cast<int*>(ws + pl.off_hist);
+        int* bstart = reinterpret_cast<int*>(ws + pl.off_bstart);
+        ColInfo* col_s = reinterpret_cast<ColInfo*>(ws + pl.off_col_s);
+        const int sort_blocks = sh.tiles0 + sh.tiles1;
+        note_launch_begin(TT_KIND_SOFTMAX, s);
+        k5_sort_count<<<sort_blocks, K5_SORT_THREADS, 0, s>>>(item_ids, sh, hist);
+        note_launch_end(TT_KIND_SOFTMAX, s);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        note_launch_begin(TT_KIND_SOFTMAX, s);
+        k5_sort_scan<<<1, K5_SCAN_THREADS, 0, s>>>(sh, hist, bstart);
+        note_launch_end(TT_KIND_SOFTMAX, s);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        note_launch_begin(TT_KIND_SOFTMAX, s);
+        k5_sort_scatter<<<sort_blocks, K5_SORT_THREADS, 0, s>>>(item_ids, sh, hist, perm, sbin);
+        note_launch_end(TT_KIND_SOFTMAX, s);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        const int vpr = d / 8;  // 16-byte pieces of a bf16 row
+        const int64_t pieces = (int64_t)nc * vpr;
+        const int pblocks = (int)((pieces + 255) / 256 < 8 * sm_count ? (pieces + 255) / 256 : 8 * sm_count);
+        note_launch_begin(TT_KIND_SOFTMAX, s);
+        k5_permute<<<pblocks, 256, 0, s>>>(perm, b, nc, vpr, static_cast<const uint4*>(users),
+                                           static_cast<const uint4*>(items), col,
+                                           reinterpret_cast<uint4*>(ws + pl.off_users_s),
+                                           reinterpret_cast<uint4*>(ws + pl.off_items_s), col_s, err);
+        note_launch_end(TT_KIND_SOFTMAX, s);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        col = col_s;
+    }
+
     K5Params p;
     p.col = col;
+    p.sbin = hits ? ws + pl.off_sbin : nullptr;
+    p.bstart = hits ? reinterpret_cast<const int*>(ws + pl.off_bstart) : nullptr;
     p.numer = numer;
     p.part = part;
     p.err = err;
@@ -730,8 +1009,9 @@ cudaError_t launch_softmax(const SoftmaxPlan& pl, const CUtensorMap& tm_users, c
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     note_launch_begin(TT_KIND_SOFTMAX, s);
-    k5_merge<<<pl.merge_blocks, K5_MERGE_THREADS, 0, s>>>(part, pl.chunks * K5_COL_GROUPS, numer, valid, b, hits ? 1 : 0,
-                                                           err, lse, loss, mean, block_sum, block_rows, ticket);
+    k5_merge<<<pl.merge_blocks, K5_MERGE_THREADS, 0, s>>>(part, pl.chunks * K5_COL_GROUPS, numer, valid, perm, b,
+                                                           hits ? 1 : 0, err, lse, loss, mean, block_sum, block_rows,
+                                                           ticket);
     note_launch_end(TT_KIND_SOFTMAX, s);
     return cudaGetLastError();
 }

@@ -1189,11 +1189,14 @@ tt_status tt_inbatch_softmax(const void* users, const void* items, tt_dtype dtyp
     memset(&tm_users, 0, sizeof tm_users);
     memset(&tm_items, 0, sizeof tm_items);
     if (b > 0) {
-        if (!bf16_tile_tensor_map(users, b, d, d, 128, &tm_users)) return TT_ERR_CUDA;
-        if (!bf16_tile_tensor_map(items, nc, d, d, pl.tile_cols, &tm_items)) return TT_ERR_CUDA;
+        // with item ids the tensor cores read the bin-order copies in the workspace
+        const void* u_src = item_ids ? static_cast<const uint8_t*>(workspace) + pl.off_users_s : users;
+        const void* v_src = item_ids ? static_cast<const uint8_t*>(workspace) + pl.off_items_s : items;
+        if (!bf16_tile_tensor_map(u_src, b, d, d, 128, &tm_users)) return TT_ERR_CUDA;
+        if (!bf16_tile_tensor_map(v_src, nc, d, d, pl.tile_cols, &tm_items)) return TT_ERR_CUDA;
     }
-    cudaError_t e = launch_softmax(pl, tm_users, tm_items, b, nc, d, tau, logq, item_ids, valid, lse, loss, mean,
-                                   workspace, static_cast<cudaStream_t>(stream), sms);
+    cudaError_t e = launch_softmax(pl, tm_users, tm_items, users, items, b, nc, d, tau, logq, item_ids, valid, lse,
+                                   loss, mean, workspace, static_cast<cudaStream_t>(stream), sms);
     if (e != cudaSuccess) return cuda_fail(e, "in-batch softmax");
     return TT_OK;
 }
@@ -1207,7 +1210,7 @@ tt_status tt_inbatch_softmax_check(const void* workspace, void* stream) {
     TT_CUDA(cudaMemcpyAsync(&err, workspace, sizeof err, cudaMemcpyDeviceToHost, s), "error word readback");
     TT_CUDA(cudaStreamSynchronize(s), "stream synchronize");
     if (err != 0) {
-        snprintf(g_last_error, sizeof g_last_error, "device wait expired (code %d)", err);
+        snprintf(g_last_error, sizeof g_last_error, "device-side wait expired or check failed (code %d)", err);
         return TT_ERR_TIMEOUT;
     }
     return TT_OK;

@@ -57,6 +57,7 @@ constexpr int ERR_TIMEOUT_TMA = 1;
 constexpr int ERR_TIMEOUT_MMA = 2;
 constexpr int ERR_TIMEOUT_EPI = 3;
 constexpr int ERR_TIMEOUT_STREAM = 4;
+constexpr int ERR_BAD_ORDER = 5;  // a permutation entry out of range (the access is skipped)
 constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;  // 2 s
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {

@@ -225,17 +225,21 @@ cudaError_t launch_mask_slice(const uint32_t* in, int64_t start, int64_t count, 
 struct SoftmaxPlan {
     int tile_cols;  // candidates per tile (rows of one items box)
     int u_tiles, c_tiles, chunks, stages, log2_slots, merge_blocks;
+    int sort_tile, sort_tiles0, sort_tiles1;  // bin order (item ids only)
     size_t off_err, off_ticket, off_col, off_numer, off_part, off_keys, off_block_sum, off_block_rows;
+    size_t off_perm, off_sbin, off_hist, off_bstart, off_col_s, off_users_s, off_items_s;
     size_t bytes;
 };
 SoftmaxPlan softmax_plan(int b, int nc, int d, bool item_ids, int sm_count);
 bool softmax_supported(int d);
-// users [b, d] and items [nc, d] bf16 through tm_users (boxes of 64 x 128)
-// and tm_items (boxes of 64 x tile_cols).
+// users [b, d] and items [nc, d] bf16 (16-byte aligned). The tensor cores
+// read them through tm_users (boxes of 64 x 128) and tm_items (boxes of
+// 64 x tile_cols), which must map, with item ids, the bin-order copies in the
+// workspace at off_users_s / off_items_s, else users and items themselves.
 cudaError_t launch_softmax(const SoftmaxPlan& pl, const CUtensorMap& tm_users, const CUtensorMap& tm_items,
-                           int b, int nc, int d, float tau, const float* logq, const int64_t* item_ids,
-                           const uint8_t* valid, float* lse, float* loss, float* mean, void* workspace,
-                           cudaStream_t s, int sm_count);
+                           const void* users, const void* items, int b, int nc, int d, float tau, const float* logq,
+                           const int64_t* item_ids, const uint8_t* valid, float* lse, float* loss, float* mean,
+                           void* workspace, cudaStream_t s, int sm_count);
 // Per query, the minimum over n_sets of the virtual thresholds (v = s * b + q):
 // theta_min[q], thf_min[q] for q < b; KEY_MAX / +inf for b <= q < b_pad.
 cudaError_t launch_sets_min(const uint64_t* theta_v, const float* thf_v, int n_sets, int b, int b_pad,

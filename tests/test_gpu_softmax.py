@@ -97,6 +97,10 @@ FULL = ("logq", "ids", "valid")
     ({"b": 200, "nc": 700, "d": 512, "catalogue": 400}, FULL),  # widest rows: two pipeline stages
     ({"b": 640, "nc": 2000, "d": 64, "tau": 1.0}, ("logq",)),
     ({"b": 512, "nc": 512, "d": 64, "pad_rate": 0.3}, ("ids", "valid")),
+    # twenty items: groups of hundreds of rows, hits in every chunk of every warp
+    ({"b": 4096, "nc": 6000, "d": 64, "catalogue": 20}, FULL),
+    # uniform ids from a large catalogue: almost every row's only hit is its own positive
+    ({"b": 3000, "nc": 3500, "d": 64, "zipf_s": 0.0}, FULL),
 ])
 def test_small_batches_every_row(over, use):
     _cuda()
@@ -115,6 +119,16 @@ def test_full_size_sampled_rows(name):
     # the same call again gives the same bits
     lse2, loss2, mean2 = _run(inp, w.tau, FULL)
     assert torch.equal(lse, lse2) and torch.equal(loss, loss2) and torch.equal(mean, mean2)
+
+
+def test_many_columns_sampled_rows():
+    """More than 2^20 columns: the bin order cuts each part into tiles of
+    2048 elements."""
+    _cuda()
+    w = W.batch("inbatch_b8192_d64", b=700, nc=(1 << 20) + 3000, catalogue=5000)
+    inp = W.batch_inputs(w, "cuda")
+    rows = np.array([0, 1, 31, 32, 255, 256, 511, 600, 699], dtype=np.int64)
+    _compare(inp, w.tau, FULL, rows)
 
 
 def test_edge_cases():
