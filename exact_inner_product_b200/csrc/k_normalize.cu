@@ -86,24 +86,25 @@ __device__ __forceinline__ void store_chunk<__nv_bfloat16, 8>(__nv_bfloat16* row
                    pack_bf16x2(y[6], y[7]));
 }
 
-// Store E int8 codes at element offset e0 of the row.
+// Store E int8 codes at element offset e0 of the row; the code of element e
+// is the low byte of qb[e] (two's complement).
+__device__ __forceinline__ uint32_t pack_low_bytes(const uint32_t* qb) {
+    const uint32_t lo = __byte_perm(qb[0], qb[1], 0x0040);  // bytes: qb0.b0, qb1.b0
+    const uint32_t hi = __byte_perm(qb[2], qb[3], 0x0040);
+    return __byte_perm(lo, hi, 0x5410);
+}
 template <int E>
-__device__ __forceinline__ void store_codes(int8_t* row_out, int e0, const int* q);
+__device__ __forceinline__ void store_codes(int8_t* row_out, int e0, const uint32_t* qb);
 template <>
-__device__ __forceinline__ void store_codes<4>(int8_t* row_out, int e0, const int* q) {
-    const uint32_t w = (uint32_t)(q[0] & 0xFF) | ((uint32_t)(q[1] & 0xFF) << 8) |
-                       ((uint32_t)(q[2] & 0xFF) << 16) | ((uint32_t)(q[3] & 0xFF) << 24);
-    *reinterpret_cast<uint32_t*>(row_out + e0) = w;
+__device__ __forceinline__ void store_codes<4>(int8_t* row_out, int e0, const uint32_t* qb) {
+    *reinterpret_cast<uint32_t*>(row_out + e0) = pack_low_bytes(qb);
 }
 template <>
-__device__ __forceinline__ void store_codes<8>(int8_t* row_out, int e0, const int* q) {
-    uint32_t w[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h)
-        w[h] = (uint32_t)(q[4 * h] & 0xFF) | ((uint32_t)(q[4 * h + 1] & 0xFF) << 8) |
-               ((uint32_t)(q[4 * h + 2] & 0xFF) << 16) | ((uint32_t)(q[4 * h + 3] & 0xFF) << 24);
-    *reinterpret_cast<uint2*>(row_out + e0) = make_uint2(w[0], w[1]);
+__device__ __forceinline__ void store_codes<8>(int8_t* row_out, int e0, const uint32_t* qb) {
+    *reinterpret_cast<uint2*>(row_out + e0) = make_uint2(pack_low_bytes(qb), pack_low_bytes(qb + 4));
 }
+
+constexpr float K1_ROUND = 0x1.8p23f;
 
 // The int8 coding quotient as the page writes it, fl(fl(v / norm) / scale)
 // (norm == 0: v taken as given); the rare elements near a rounding boundary.
@@ -230,16 +231,26 @@ __global__ void __launch_bounds__(K1_THREADS)
                     if (c < chunks) {
                         float x[E];
                         Elem<Tin>::unpack(raw[u][i], x);
-                        int q[E];
+                        uint32_t qb[E];
 #pragma unroll
                         for (int e = 0; e < E; ++e) {
                             float y = (MODE == 2 ? x[e] * rn : x[e]) * rs;
-                            const float to_int = fabsf(y - rintf(y));  // distance to the nearest integer
-                            if (!(0.5f - to_int > fabsf(y) * 0x1p-19f + 0x1p-19f))
+                            // Adding 1.5 * 2^23 rounds y to an integer, ties to
+                            // even, and leaves it in the low mantissa bits of t
+                            // (|y| < 2^22); subtracting it back gives rint(y).
+                            float t = __fadd_rn(y, K1_ROUND);
+                            const float to_int = fabsf(__fadd_rn(y, -__fadd_rn(t, -K1_ROUND)));
+                            if (!(0.5f - to_int > fabsf(y) * 0x1p-19f + 0x1p-19f)) {
                                 y = ieee_code_quotient(x[e], MODE == 2 ? norm : 0.0f, scale);
-                            q[e] = (int)fminf(fmaxf(rintf(y), -127.f), 127.f);
+                                t = __fadd_rn(y, K1_ROUND);
+                            }
+                            // |y| <= 127 (1 + 2^-20) < 127.5 because scale >=
+                            // max|w| / 127 up to one rounding, so the page's clip
+                            // to [-127, 127] never changes a code; the low byte
+                            // of t is the code in two's complement.
+                            qb[e] = __float_as_uint(t);
                         }
-                        store_codes<E>(reinterpret_cast<int8_t*>(out) + row[u] * d, c * E, q);
+                        store_codes<E>(reinterpret_cast<int8_t*>(out) + row[u] * d, c * E, qb);
                     }
                 }
             }
