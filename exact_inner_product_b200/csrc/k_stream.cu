@@ -281,12 +281,15 @@ __global__ void __launch_bounds__(K2_THREADS)
 // flight per thread.
 constexpr int K2_BATCH_I8 = 4;
 
-template <int QB, bool V8>
+template <int QB, bool V8, int DEFER>
 __global__ void __launch_bounds__(K2_THREADS)
     k2_stream_i8(const PassArgs a) {
     extern __shared__ __align__(16) int qw[];  // [QB][d / 4] packed codes
     pdl_trigger();
-    pdl_wait();  // query codes, thresholds and counters come from earlier kernels
+    // DEFER > 0: as in k2_stream, the first DEFER rows of each thread are
+    // scored before the wait (the query codes and scales are written by the
+    // query coding, which completes before the search's next kernel starts)
+    if (DEFER == 0) pdl_wait();  // query codes, thresholds and counters come from earlier kernels
     const int lane = threadIdx.x & 31;
     const int q0 = blockIdx.y * QB;
     const int d = a.d;
@@ -297,22 +300,17 @@ __global__ void __launch_bounds__(K2_THREADS)
         const int q = q0 + qb;
         qw[i] = q < a.b ? reinterpret_cast<const int*>(a.queries)[(int64_t)q * dw + w] : 0;
     }
-    uint64_t th[QB];
     float us[QB];
 #pragma unroll
-    for (int qb = 0; qb < QB; ++qb) {
-        th[qb] = (q0 + qb < a.b) ? a.theta[q0 + qb] : KEY_MAX;
-        us[qb] = (q0 + qb < a.b) ? a.qscale[q0 + qb] : 1.0f;
-    }
+    for (int qb = 0; qb < QB; ++qb) us[qb] = (q0 + qb < a.b) ? a.qscale[q0 + qb] : 1.0f;
     __syncthreads();
 
     const int64_t pitch = (int64_t)a.stride * d;
     const uint8_t* base = static_cast<const uint8_t*>(a.rows);
     const int64_t n_threads = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r - lane < a.n_rows; r += n_threads) {
-        const bool valid = r < a.n_rows;
+    // the int32 dot products of row r with this block's query codes
+    auto dots = [&](int64_t r, bool valid, int* acc) {
         const uint8_t* row = base + (valid ? r : 0) * pitch;
-        int acc[QB];
 #pragma unroll
         for (int qb = 0; qb < QB; ++qb) acc[qb] = 0;
         for (int p0 = 0; p0 < pieces; p0 += K2_BATCH_I8) {
@@ -339,6 +337,43 @@ __global__ void __launch_bounds__(K2_THREADS)
                 }
             }
         }
+    };
+    int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    uint64_t th[QB];
+    if constexpr (DEFER > 0) {
+        uint64_t kb[DEFER][QB];  // keys of the first DEFER rows (KEY_MIN: no row, or excluded)
+#pragma unroll
+        for (int i = 0; i < DEFER; ++i, r += n_threads) {
+            const bool valid = r < a.n_rows;
+            int acc[QB];
+            dots(r, valid, acc);
+            const int64_t id = r * a.stride;
+            bool row_ok = valid;
+            float c = a.inv_tau;
+            if (valid) {
+                if (a.exclude) row_ok = !((a.exclude[id >> 5] >> (id & 31)) & 1u);
+                c = a.inv_norm[id] * a.inv_tau;
+            }
+#pragma unroll
+            for (int qb = 0; qb < QB; ++qb)
+                kb[i][qb] = row_ok ? make_key((float)acc[qb] * us[qb] * c, (uint32_t)id) : KEY_MIN;
+        }
+        pdl_wait();  // this pass's thresholds
+#pragma unroll
+        for (int qb = 0; qb < QB; ++qb) th[qb] = (q0 + qb < a.b) ? a.theta[q0 + qb] : KEY_MAX;
+#pragma unroll
+        for (int i = 0; i < DEFER; ++i)
+#pragma unroll
+            for (int qb = 0; qb < QB; ++qb) append_warp(a, q0 + qb, kb[i][qb] > th[qb], kb[i][qb], lane);
+    } else {
+#pragma unroll
+        for (int qb = 0; qb < QB; ++qb) th[qb] = (q0 + qb < a.b) ? a.theta[q0 + qb] : KEY_MAX;
+    }
+
+    for (; r - lane < a.n_rows; r += n_threads) {
+        const bool valid = r < a.n_rows;
+        int acc[QB];
+        dots(r, valid, acc);
         const int64_t id = r * a.stride;
         bool row_ok = valid;
         float c = a.inv_tau;
@@ -363,8 +398,7 @@ __global__ void __launch_bounds__(K2_THREADS)
     }
 }
 
-// Grid of a streaming pass: one block per 256 rows, at most eight blocks per
-// Grid: one block per 256 rows, at most 8 blocks of 256 threads per SM
+// Grid of a streaming pass: one block per 256 rows, at most 8 blocks of 256 threads per SM
 // (blocks loop over their rows). Measured on the 10^6-row pass: a grid of
 // exactly the resident blocks (each looping ~13 times) took 53 us against 47
 // us for this one, which runs in about four waves of resident blocks.
@@ -398,14 +432,20 @@ cudaError_t launch_qb(const PassArgs& a, int gy, size_t smem, bool v8, cudaStrea
     return v8 ? launch_qbv<T, QB, true>(a, gy, smem, s, sms) : launch_qbv<T, QB, false>(a, gy, smem, s, sms);
 }
 
+template <int QB, bool V8>
+cudaError_t launch_i8_qbv(const PassArgs& a, int gy, size_t smem, cudaStream_t s, int sms) {
+    const dim3 grid = stream_grid(k2_stream_i8<QB, V8, 0>, a, gy, smem, sms);
+    // after the one-sample estimate: the first rows are scored while it runs
+    if constexpr (QB <= 2) {
+        if (a.defer && a.types == nullptr)
+            return launch_pdl(k2_stream_i8<QB, V8, K2_DEFER>, grid, dim3(K2_THREADS), smem, s, a);
+    }
+    return launch_pdl(k2_stream_i8<QB, V8, 0>, grid, dim3(K2_THREADS), smem, s, a);
+}
+
 template <int QB>
 cudaError_t launch_i8_qb(const PassArgs& a, int gy, size_t smem, bool v8, cudaStream_t s, int sms) {
-    if (v8) {
-        auto k = k2_stream_i8<QB, true>;
-        return launch_pdl(k, stream_grid(k, a, gy, smem, sms), dim3(K2_THREADS), smem, s, a);
-    }
-    auto k = k2_stream_i8<QB, false>;
-    return launch_pdl(k, stream_grid(k, a, gy, smem, sms), dim3(K2_THREADS), smem, s, a);
+    return v8 ? launch_i8_qbv<QB, true>(a, gy, smem, s, sms) : launch_i8_qbv<QB, false>(a, gy, smem, s, sms);
 }
 
 cudaError_t launch_i8(const PassArgs& a, int qb, int gy, size_t smem, bool v8, cudaStream_t s, int sms) {
