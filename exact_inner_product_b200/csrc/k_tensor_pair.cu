@@ -390,9 +390,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(KP_THREADS, 1)
                                        (uint32_t)(buf * KP_ACC_COLS + half * KP_WARP_COLS);
                 // One round trip: the warp's 128 columns into registers, then
                 // the accumulator goes back to the MMA issuer before any test.
-                // (int8: two round trips of 64 columns, the accumulator going
-                // back after the second; its fast test needs the registers.)
-                constexpr int NV = I8 ? 2 : 4;  // 32-column chunks held at once
+                // (int8 and rows with norms: two round trips of 64 columns, the
+                // accumulator going back after the second; their fast tests
+                // need the registers - with four chunks held the norms variant
+                // spilled and ran 45 % slower.)
+                constexpr int NV = (I8 || NORMS) ? 2 : 4;  // 32-column chunks held at once
 #pragma unroll
                 for (int part = 0; part < 4 / NV; ++part) {
                 Cols32 v[NV];
