@@ -70,9 +70,9 @@ TRAFFIC = {
                                     "sha": "4273a9f8869b74ec01b8762c20eb598dc6f0b1597fcd3e5f8ad9afde664127f4"},
     # ncu --set full --import-source no --clock-control none -k regex:k3_pair -s 8 -c 1 on `python bench.py
     # --workload large_batch --n 4000000 --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass,
-    # 4,000,000 rows): 1066.455 MB read + 27.004 MB written; scaled to the full corpus by rows scanned
-    ("k3_pair", "large_batch"): {"bytes_per_row": 273.365, "src": "exact_inner_product_b200/csrc/k_tensor_pair.cu",
-                                 "sha": "fe96c9c80fcef016851e2cc5569f9b9b67b3d7bfb3929d40c4bfb96d4e0d64d5"},
+    # 4,000,000 rows): 1056.253 MB read + 27.411 MB written; scaled to the full corpus by rows scanned
+    ("k3_pair", "large_batch"): {"bytes_per_row": 270.916, "src": "exact_inner_product_b200/csrc/k_tensor_pair.cu",
+                                 "sha": "8651752c99e9b667e5bf49f551f1fe48623ddfd247f4338868a4988d77e9c7bf"},
     # ncu --set full --import-source no --clock-control none -k regex:k3_tensor -s 8 -c 1 on `python bench.py
     # --workload masked_fused --n 4000000 --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass,
     # 4,000,000 rows): 4145.305 MB read + 66.409 MB written; scaled to the full corpus by rows scanned
