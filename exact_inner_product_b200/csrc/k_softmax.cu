@@ -83,6 +83,8 @@ constexpr int K5_BINS = 256;                 // sort bins: the top 8 bits of the
 constexpr int K5_SORT_THREADS = 256;         // one element per thread and round
 constexpr int K5_SORT_WARPS = K5_SORT_THREADS / 32;
 constexpr int K5_SCAN_THREADS = 1024;
+static_assert(K5_SORT_THREADS == K5_BINS, "the bin-order kernels give each thread one bin");
+static_assert(K5_SORT_THREADS % 32 == 0, "whole warps: the scatter matches bins across all 32 lanes");
 
 struct alignas(8) ColInfo {
     float nb;  // -log q_j * log2(e), or -inf when the column is invalid or past nc
