@@ -395,7 +395,9 @@ TT_API tt_status tt_score_topk_types(tt_index* index, const void* queries, tt_dt
  * lse, loss device f32 [b]; mean device f32 [1]
  * workspace device memory of at least tt_inbatch_softmax_workspace bytes,
  *           256-byte aligned, owned by the caller, not shared with another
- *           call in flight
+ *           call in flight (with item ids it also holds copies of users and
+ *           items in an order grouped by a hash of the id: about 2·d bytes
+ *           per user and per candidate; the results do not depend on it)
  *
  * Asynchronous: the work is enqueued on `stream` and the call returns. If a
  * bounded device-side wait expires (which a correct run never does), every
