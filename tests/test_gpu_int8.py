@@ -89,6 +89,11 @@ CASES = [
     ("large_batch", {"n": 250_001, "b": 200, "k": 300, "oracle_queries": 12}, 2),
     ("masked_fused", {"n": 200_099, "b": 260, "oracle_queries": 12}, 3),
     ("masked_fused", {"n": 120_031, "b": 3, "k": 256}, 1),
+    # the pass after the one-sample estimate scores its first rows before the
+    # threshold lands: two queries per block with a mask, and a corpus with
+    # more rows per thread than are deferred
+    ("masked_fused", {"n": 150_011, "b": 2, "k": 64}, 1),
+    ("stream_b1", {"n": 1_500_007, "k": 100}, 1),
 ]
 
 
