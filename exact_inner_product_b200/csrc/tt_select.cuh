@@ -2,7 +2,7 @@
 // by the select kernels (K4) and the exact fallback scan.
 //
 // One CTA of K4_THREADS threads works on one list of distinct keys. Up to
-// 4096 keys and r <= 512: a bucket select over linear score bins (below);
+// 4096 keys and r <= 1024: a bucket select over linear score bins (below);
 // where that cannot decide, for r <= K4_TOP_MAX, the best r keys kept sorted
 // in registers (bitonic networks, below). Otherwise the r-th
 // largest key is found by a most-significant-digit radix select (digits of
@@ -199,7 +199,7 @@ __device__ inline void block_top_sorted(const uint64_t* keys, int n, int r, K4Sm
 // ---------------------------------------------------------------------------
 constexpr int K4_BUCKET_PT = 16;
 constexpr int K4_BUCKET_N = K4_BUCKET_PT * K4_THREADS;  // 4096
-constexpr int K4_BUCKET_R = 512;
+constexpr int K4_BUCKET_R = 1024;          // outputs, in sm.sorted[0 .. 1024)
 constexpr int K4_BUCKET_M = 1024;          // candidates, held in sm.sorted[1024 ..)
 constexpr int K4_BUCKET_BIN_MAX = 256;     // keys in the boundary bin
 static_assert(K4_BINS == 8 * K4_THREADS, "each thread owns eight bins in the scan");

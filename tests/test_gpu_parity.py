@@ -384,13 +384,14 @@ def test_sampled_plan_int8_and_f32_rows():
     assert res["max_abs_err"] <= w.tolerance
 
 
-@pytest.mark.parametrize("k", [1, 31, 32, 33, 64, 65, 128, 129, 256, 257])
+@pytest.mark.parametrize("k", [1, 31, 32, 33, 64, 65, 128, 129, 256, 257, 513, 1000, 1024])
 @pytest.mark.parametrize("path,b", [(1, 2), (2, 24), (3, 256)])
 def test_select_widths(path, b, k):
-    """The selects keep the best r <= 256 keys sorted in registers, 32, 64,
-    128 or 256 per warp, and use the radix select above that; k on both sides
-    of each width, on every scorer (on the streaming scorer the sample
-    estimate's rank varies with k too)."""
+    """The selects rank up to 4096 kept keys by buckets (r <= 1024), keep
+    the best r <= 256 keys sorted in registers (32, 64, 128 or 256 per warp)
+    where the buckets cannot decide, and use the radix select beyond that; k
+    on both sides of each width, on every scorer (on the streaming scorer
+    the sample estimate's rank varies with k too)."""
     _cuda()
     w = W.workload("small_batch", n=60_013, b=b, k=k, tau=1.0, oracle_queries=6)
     res, st = parity.run_case(w, path=path)
