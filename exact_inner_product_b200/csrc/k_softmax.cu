@@ -236,7 +236,8 @@ __global__ void k5_columns(const float* __restrict__ logq, const uint8_t* __rest
 // A stable counting sort, done separately on the two parts of the columns:
 // part 0 = [0, b) (the rows use the same permutation, so row r's positive
 // stays column r) and part 1 = [b, nc) (the shared negatives). The key of
-// column j is bin(id_j); equal ids share a bin, so the columns that can be
+// column j is bin(id_j), the top 8 bits of the id's Fibonacci hash (as in
+// k5_hash); equal ids share a bin, so the columns that can be
 // hits of row r lie in the column ranges of bin(r) in both parts. Stable
 // ranks make the order, and with it every sum, the same on every run.
 //
