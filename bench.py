@@ -61,13 +61,9 @@ PATH_NAMES = {1: "streaming", 2: "tensor-core", 3: "tensor-core (SM pairs)"}
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per unit of work
 # from ncu captures of a kernel, with the sha256 of the kernel's source file at
 # capture time; `traffic` is reported only while that file is unchanged. Units:
-# K1 bytes per corpus row; K3 bytes per level row scanned (level-0 capture,
-# applied to every level of a step, like `achieved`).
+# bytes per level row scanned (level-0 capture, applied to every level of a
+# step, like `achieved`).
 TRAFFIC = {
-    # ncu --set full --clock-control none -k regex:k1_normalize -s 5 -c 1 on `python bench.py --steps 50 --warmup 3
-    # --no-e2e --no-cpu-baseline`: 512.019 MB read + 200.806 MB written for 1,000,000 rows
-    ("k1_normalize", "stream_b1"): {"bytes_per_row": 712.825, "src": "exact_inner_product_b200/csrc/k_normalize.cu",
-                                    "sha": "4273a9f8869b74ec01b8762c20eb598dc6f0b1597fcd3e5f8ad9afde664127f4"},
     # ncu --set full --import-source no --clock-control none -k regex:k3_pair -s 8 -c 1 on `python bench.py
     # --workload large_batch --n 4000000 --steps 3 --warmup 3 --no-e2e --no-cpu-baseline` (level-0 pass,
     # 4,000,000 rows): 1056.253 MB read + 27.411 MB written; scaled to the full corpus by rows scanned
